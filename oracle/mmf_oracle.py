@@ -1,0 +1,390 @@
+"""Plain CPU oracle for the MatMul-free block forward (FusedBitLinear + MLGRU + GLU).
+
+TEST INFRASTRUCTURE ONLY. This module is the slow, obviously-correct
+definition that the CUDA library is checked against. Only the test suite,
+``__graft_entry__.smoke()`` and the CPU-baseline / reference legs of
+``bench.py`` may import it. The library never calls it, and it shares no code
+with the CUDA path (no kernels, headers, tables or helpers): only the seeded
+input generators in ``synth`` feed both sides.
+
+Sources (web pages on "Scalable MatMul-free Language Modeling", arXiv 2406.02528):
+  [DC]  "MatMul-free language models", DataCamp blog (Chinese edition);
+        sections "Replacing MatMul with ternary operations" and
+        "Core components: MLGRU and GLU" (incl. the overview figure's panels
+        "MatMul vs. scaled ternary accumulation" and "RMS Norm").
+  [HL]  hysenlabs project review of ridgerchu/matmulfreellm; sections
+        "FusedBitLinear: how ternary weights save the multiplications" and
+        "HGRN attention: gated recurrence instead of softmax".
+  [AX]  arXiv abstract page of 2406.02528.
+
+Where the pages are silent the plainest reading is taken and stated at the
+function. Numerics: fp64 unless a step decides an integer (a quantised code),
+where the decision is taken in fp32 exactly as the kernels take it, so that
+both sides can agree bit for bit:
+  * weight codes: gamma is an fp64 mean cast to fp32, the division W/(gamma+eps)
+    is one IEEE fp32 division, rounding is half-to-even;
+  * activation codes: the mean square is an fp64 sum cast to fp32, then
+    r = sqrt(ms + eps), 1/r, x*(1/r), *gain, 127/max|x^|, x^*s and the rounding
+    are single IEEE fp32 operations in that order.
+
+Pins: every function below is checked in tests/test_oracle_pins.py against
+closed forms, hand-built cases, brute force or library routines. The
+composition ``block_forward`` / ``stack_forward`` is pinned only through its
+stages plus the zero-weight identity and the prefill == decode invariant.
+"""
+from __future__ import annotations
+
+import dataclasses
+from typing import Optional
+
+import numpy as np
+
+EPS_W = 1e-5      # weight ternarisation epsilon: W / (gamma + EPS_W)
+Q_FLOOR = 1e-5    # floor on max|x^| before 127/max|x^|
+Q_MAX = 127       # int8 activation code range [-127, 127] (-128 is never produced)
+EPS_NORM = 1e-6   # default RMSNorm epsilon (the pages give none)
+
+# ---------------------------------------------------------------------------
+# Storage rounding
+# ---------------------------------------------------------------------------
+
+
+def round_f32(x) -> np.ndarray:
+    """Round to the nearest fp32 (IEEE, half-to-even); returned as fp64 values."""
+    return np.asarray(x, dtype=np.float64).astype(np.float32).astype(np.float64)
+
+
+def round_bf16(x) -> np.ndarray:
+    """Round fp64 values to the nearest bfloat16 (8-bit significand), ties to even.
+
+    Written from the format's definition: a normal bf16 number is m * 2^(e-8)
+    with an integer 128 <= |m| < 256; below 2^-126 the spacing is fixed at 2^-133.
+    Scaling by powers of two is exact in fp64, so the only rounding is np.rint.
+    """
+    x = np.asarray(x, dtype=np.float64)
+    mant, expo = np.frexp(x)                 # x = mant * 2^expo, 0.5 <= |mant| < 1
+    normal = np.ldexp(np.rint(np.ldexp(mant, 8)), expo - 8)
+    sub = np.ldexp(np.rint(np.ldexp(x, 133)), -133)
+    out = np.where(np.abs(x) < 2.0 ** -126, sub, normal)
+    return out
+
+
+def store(x, dtype: str) -> np.ndarray:
+    """Round to the run's storage type ("f32" or "bf16")."""
+    if dtype == "f32":
+        return round_f32(x)
+    if dtype == "bf16":
+        return round_bf16(x)
+    raise ValueError(dtype)
+
+
+# ---------------------------------------------------------------------------
+# Weights: absmean ternarisation and the 2-bit packed format
+# ---------------------------------------------------------------------------
+
+
+def ternarize(W, gamma: Optional[np.float32] = None):
+    """Absmean ternarisation of one latent weight matrix.
+
+    [DC] "Replacing MatMul with ternary operations": the weights are scaled by
+    the mean of the absolute values of the matrix's elements and each element
+    is rounded to the nearest of -1, 0, 1. Reading: one gamma per whole matrix,
+    codes = clip(round(W / (gamma + 1e-5)), -1, 1), ties to even.
+
+    If ``gamma`` is given it is used instead of the matrix's own mean (used to
+    compare codes given another implementation's gamma).
+    Returns (gamma as np.float32, codes as int8 array of W's shape).
+    """
+    W32 = np.asarray(W, dtype=np.float32)
+    if W32.size == 0:
+        raise ValueError("empty weight matrix")
+    if gamma is None:
+        total = np.sum(np.abs(W32.astype(np.float64)))
+        gamma = np.float32(total / W32.size)
+    gamma = np.float32(gamma)
+    denom = np.float32(gamma + np.float32(EPS_W))       # one fp32 addition
+    t = W32 / denom                                      # one IEEE fp32 division
+    codes = np.clip(np.rint(t), -1, 1).astype(np.int8)
+    return gamma, codes
+
+
+def pack_codes(codes) -> np.ndarray:
+    """Pack ternary codes {-1,0,1} [N, K] (K % 16 == 0) into uint32 [N, K/16].
+
+    Storage format of this library (not from the pages): the stored 2-bit value
+    is code + 1 in {0, 1, 2}; the code for column k = 16*j + 4*i + b sits in
+    word j at bits [8*b + 2*i, 8*b + 2*i + 2).
+    """
+    codes = np.asarray(codes)
+    N, K = codes.shape
+    if K % 16 != 0:
+        raise ValueError("K must be a multiple of 16")
+    if codes.size and (codes.min() < -1 or codes.max() > 1):
+        raise ValueError("codes must be in {-1,0,1}")
+    v = (codes.astype(np.int64) + 1).reshape(N, K // 16, 4, 4)   # [n, j, i, b]
+    words = np.zeros((N, K // 16), dtype=np.int64)
+    for i in range(4):
+        for b in range(4):
+            words |= v[:, :, i, b] << (8 * b + 2 * i)
+    return words.astype(np.uint32)
+
+
+def unpack_codes(packed, K: int) -> np.ndarray:
+    """Inverse of pack_codes: uint32 [N, K/16] -> int8 codes [N, K]."""
+    packed = np.asarray(packed, dtype=np.uint32).astype(np.int64)
+    N = packed.shape[0]
+    out = np.zeros((N, K // 16, 4, 4), dtype=np.int64)
+    for i in range(4):
+        for b in range(4):
+            out[:, :, i, b] = (packed >> (8 * b + 2 * i)) & 3
+    if np.any(out == 3):
+        raise ValueError("invalid 2-bit field 3 in packed weights")
+    return (out.reshape(N, K) - 1).astype(np.int8)
+
+
+@dataclasses.dataclass
+class TLinear:
+    """A ternary BitLinear: codes [N,K] int8, per-matrix gamma, optional gain [K] / bias [N]."""
+    codes: np.ndarray
+    gamma: np.float32
+    gain: Optional[np.ndarray] = None
+    bias: Optional[np.ndarray] = None
+
+    @property
+    def N(self) -> int:
+        return self.codes.shape[0]
+
+    @property
+    def K(self) -> int:
+        return self.codes.shape[1]
+
+
+def make_tlinear(W_latent, gain=None, bias=None) -> TLinear:
+    gamma, codes = ternarize(W_latent)
+    g = None if gain is None else np.asarray(gain, dtype=np.float32)
+    b = None if bias is None else np.asarray(bias, dtype=np.float64)
+    return TLinear(codes, gamma, g, b)
+
+
+# ---------------------------------------------------------------------------
+# Activations: RMSNorm, per-token absmax int8 quantisation
+# ---------------------------------------------------------------------------
+
+
+def rmsnorm(x, gain=None, eps: float = EPS_NORM) -> np.ndarray:
+    """RMSNorm over the last axis, in the fp32 steps listed in the module docstring.
+
+    [DC] overview figure, "RMS Norm" panel: activations are normalised before
+    quantisation. [HL] "FusedBitLinear": RMSNorm on the input, then the fused
+    bit-op kernel. x^ = x / sqrt(mean(x^2) + eps) * gain. Returns fp32.
+    """
+    x32 = np.asarray(x, dtype=np.float32)
+    K = x32.shape[-1]
+    ss = np.sum(np.square(x32.astype(np.float64)), axis=-1)
+    ms = (ss / K).astype(np.float32)
+    r = np.sqrt(ms + np.float32(eps))
+    rinv = (np.float32(1.0) / r).astype(np.float32)
+    xhat = x32 * rinv[..., None]
+    if gain is not None:
+        xhat = xhat * np.asarray(gain, dtype=np.float32)
+    return xhat.astype(np.float32)
+
+
+def absmax_quantize(xhat):
+    """Per-token absmax int8 quantisation of normalised activations.
+
+    The pages only say the activations are normalised before quantisation
+    ([DC] "RMS Norm" panel); the per-token absmax rule is the reading taken:
+    s = 127 / max(max|x^|, 1e-5), q = clip(round_half_even(x^ * s), -128, 127).
+    Returns (q int8, s fp32 per token).
+    """
+    xh = np.asarray(xhat, dtype=np.float32)
+    a = np.max(np.abs(xh), axis=-1)
+    s = (np.float32(Q_MAX) / np.maximum(a, np.float32(Q_FLOOR))).astype(np.float32)
+    q = np.clip(np.rint(xh * s[..., None]), -128, 127).astype(np.int8)
+    return q, s
+
+
+def ternary_accumulate(q, codes) -> np.ndarray:
+    """acc[m, n] = sum over k of q[m,k] * w[n,k] with w in {-1,0,1}, done as add/subtract.
+
+    [DC] "Replacing MatMul with ternary operations": multiplying by -1 negates,
+    by 0 drops, by 1 keeps. So acc = (sum of q where w = +1) - (sum of q where
+    w = -1). The two masked sums use an fp64 matrix product as a library step;
+    every partial sum is an integer below 2^53, so the result is exact.
+    """
+    q64 = np.asarray(q, dtype=np.float64)
+    c = np.asarray(codes)
+    plus = (c == 1).astype(np.float64)
+    minus = (c == -1).astype(np.float64)
+    acc = q64 @ plus.T - q64 @ minus.T
+    return np.rint(acc).astype(np.int64)
+
+
+def rescale(acc, gamma, s, bias=None) -> np.ndarray:
+    """Scaled ternary accumulation: y = acc * gamma / s (+ bias), fp64.
+
+    [DC] overview figure panel "MatMul vs. scaled ternary accumulation".
+    """
+    y = np.asarray(acc, dtype=np.float64) * np.float64(gamma) / np.asarray(s, dtype=np.float64)[..., None]
+    if bias is not None:
+        y = y + np.asarray(bias, dtype=np.float64)
+    return y
+
+
+def bitlinear(x, lin: TLinear, eps: float = EPS_NORM, parts: bool = False):
+    """FusedBitLinear forward: RMSNorm -> absmax int8 quant -> ternary accumulate -> rescale.
+
+    [HL] "FusedBitLinear": RMSNorm, quantisation and accumulation against
+    ternary weights in one layer. x: [..., K] -> y: [..., N] fp64.
+    """
+    x = np.asarray(x)
+    lead = x.shape[:-1]
+    x2 = x.reshape(-1, x.shape[-1])
+    xhat = rmsnorm(x2, lin.gain, eps)
+    q, s = absmax_quantize(xhat)
+    acc = ternary_accumulate(q, lin.codes)
+    y = rescale(acc, lin.gamma, s, lin.bias)
+    y = y.reshape(*lead, lin.N)
+    if parts:
+        return y, dict(xhat=xhat, q=q, s=s, acc=acc)
+    return y
+
+
+# ---------------------------------------------------------------------------
+# MLGRU token mixer
+# ---------------------------------------------------------------------------
+
+
+def sigmoid(z) -> np.ndarray:
+    z = np.asarray(z, dtype=np.float64)
+    with np.errstate(over="ignore"):
+        return 1.0 / (1.0 + np.exp(-z))
+
+
+def silu(z) -> np.ndarray:
+    z = np.asarray(z, dtype=np.float64)
+    return z * sigmoid(z)
+
+
+def mlgru_scan(pf, pc, pg, h0):
+    """MLGRU gates and recurrence over pre-activations [B, T, d] (fp64).
+
+    [DC] "Core components: MLGRU and GLU": the MLGRU walks the sequence token
+    by token, takes the current token and the previous hidden state, and
+    updates the state with element-wise operations and gates valued in [0,1].
+    [HL] "HGRN attention": forget-gate and candidate paths, recurrence that
+    depends only on the current token and the previous state. The pages print
+    no formula; the plainest reading used here:
+        f_t = sigmoid(f~_t), c_t = SiLU(c~_t), g_t = sigmoid(g~_t)
+        h_t = f_t * h_{t-1} + (1 - f_t) * c_t
+        o'_t = g_t * h_t
+    Returns (o' [B,T,d] fp64, h_T [B,d] fp64). h is carried in fp64 here.
+    """
+    pf = np.asarray(pf, dtype=np.float64)
+    pc = np.asarray(pc, dtype=np.float64)
+    pg = np.asarray(pg, dtype=np.float64)
+    h = np.array(h0, dtype=np.float64, copy=True)
+    T = pf.shape[1]
+    o = np.empty_like(pf)
+    for t in range(T):
+        f = sigmoid(pf[:, t])
+        c = silu(pc[:, t])
+        g = sigmoid(pg[:, t])
+        h = f * h + (1.0 - f) * c
+        o[:, t] = g * h
+    return o, h
+
+
+@dataclasses.dataclass
+class Block:
+    """Ternary weights of one MatMul-free block."""
+    f: TLinear
+    c: TLinear
+    g: TLinear
+    o: TLinear
+    gate: TLinear
+    up: TLinear
+    down: TLinear
+
+    @property
+    def d(self) -> int:
+        return self.f.K
+
+    @property
+    def inner(self) -> int:
+        return self.gate.N
+
+
+def make_block(latents: dict) -> Block:
+    """latents: dict of name -> fp32 latent [N, K] for f, c, g, o, gate, up, down."""
+    return Block(**{k: make_tlinear(latents[k]) for k in ("f", "c", "g", "o", "gate", "up", "down")})
+
+
+def mlgru_preacts(x, blk: Block, dtype: str, eps: float = EPS_NORM):
+    """f~, c~, g~ = BitLinear_{f,c,g}(x), each rounded to the storage type."""
+    pf = store(bitlinear(x, blk.f, eps), dtype)
+    pc = store(bitlinear(x, blk.c, eps), dtype)
+    pg = store(bitlinear(x, blk.g, eps), dtype)
+    return pf, pc, pg
+
+
+def mlgru(x, blk: Block, h0, dtype: str, eps: float = EPS_NORM, parts: bool = False):
+    """MLGRU token mixer on x [B,T,d]: projections, gated scan, output gate, o-projection.
+
+    Storage points (the kernels store these tensors): f~/c~/g~ and o' in the run
+    dtype, the state h in fp32. Returns (o [B,T,d] fp64 unrounded, h_T fp32 values).
+    """
+    pf, pc, pg = mlgru_preacts(x, blk, dtype, eps)
+    o_gate, hT = mlgru_scan(pf, pc, pg, h0)
+    o_gate = store(o_gate, dtype)
+    o = bitlinear(o_gate, blk.o, eps)
+    hT = round_f32(hT)
+    if parts:
+        return o, hT, dict(pf=pf, pc=pc, pg=pg, o_gate=o_gate)
+    return o, hT
+
+
+def glu(x, blk: Block, dtype: str, eps: float = EPS_NORM, parts: bool = False):
+    """MatMul-free GLU channel mixer.
+
+    [DC] "Core components: MLGRU and GLU": the input goes through two separate
+    BitLinear layers; one branch passes SiLU and is multiplied element-wise by
+    the other; a third BitLinear gives the output. Reading: the SiLU branch is
+    "gate", the other "up": p = SiLU(gate(x)) * up(x), stored in the run dtype;
+    returns down(p) in fp64.
+    """
+    u = bitlinear(x, blk.gate, eps)
+    v = bitlinear(x, blk.up, eps)
+    p = store(silu(u) * v, dtype)
+    y = bitlinear(p, blk.down, eps)
+    if parts:
+        return y, dict(u=u, v=v, p=p)
+    return y
+
+
+def block_forward(x, blk: Block, h0, dtype: str, eps: float = EPS_NORM, parts: bool = False):
+    """One MatMul-free block: y1 = x + MLGRU(x); y = y1 + GLU(y1).
+
+    [HL] "HGRN attention": the block input passes RMSNorm first; [DC] names
+    the token mixer (MLGRU) and channel mixer (GLU). Reading: pre-norm blocks
+    with residual connections; each BitLinear's own RMSNorm is the block norm.
+    x [B,T,d] in the run dtype -> (y [B,T,d] stored, h_T [B,d] fp32 values).
+    """
+    x = store(x, dtype)
+    o, hT, p1 = mlgru(x, blk, h0, dtype, eps, parts=True)
+    y1 = store(x + o, dtype)
+    g, p2 = glu(y1, blk, dtype, eps, parts=True)
+    y = store(y1 + g, dtype)
+    if parts:
+        return y, hT, dict(y1=y1, o=o, **p1, **p2)
+    return y, hT
+
+
+def stack_forward(x, blocks, h0s, dtype: str, eps: float = EPS_NORM):
+    """L blocks in sequence; h0s [L,B,d]. Returns (y, h_T [L,B,d])."""
+    hs = []
+    for l, blk in enumerate(blocks):
+        x, h = block_forward(x, blk, h0s[l], dtype, eps)
+        hs.append(h)
+    return x, np.stack(hs)

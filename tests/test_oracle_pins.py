@@ -1,0 +1,443 @@
+"""Pins for the CPU oracle: closed forms, hand-built cases, brute force, library routines.
+
+Each test pins an oracle function to something other than itself, chosen so
+that a plausible slip (dropped term, wrong sign or index, swapped operand)
+fails at least one of them. CPU only.
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+from scipy.stats import norm as _norm
+
+import oracle as O
+import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+def _load(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        return json.load(f)
+
+
+# ----------------------------------------------------------------- bf16 rounding
+
+def test_round_bf16_matches_torch_on_random_fp32():
+    g = torch.Generator().manual_seed(1)
+    x = torch.randn(200000, generator=g) * torch.exp(torch.randn(200000, generator=g) * 8)
+    ref = x.to(torch.bfloat16).to(torch.float64).numpy()
+    got = O.round_bf16(x.to(torch.float64).numpy())
+    np.testing.assert_array_equal(got, ref)
+
+
+def test_round_bf16_ties_to_even():
+    # 1 + 2^-8 is exactly halfway between 1 and 1 + 2^-7 -> even (1.0)
+    # 1 + 3*2^-8 is halfway between 1+2^-7 and 1+2^-6 -> even (1 + 2^-6)
+    x = np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, -(1 + 2 ** -8), 2 ** -130 * 1.5, 0.0])
+    want = np.array([1.0, 1 + 2 ** -6, -1.0, 2 ** -130 * 1.5, 0.0])
+    np.testing.assert_array_equal(O.round_bf16(x), want)
+    t = torch.tensor(x[:3], dtype=torch.float32).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(O.round_bf16(x[:3]), t)
+
+
+# ----------------------------------------------------------------- ternarisation
+
+def test_ternarize_worked_example():
+    gd = _load("ternarize_worked.json")
+    gamma, codes = O.ternarize(np.array(gd["W"]))
+    assert gamma == np.float32(gd["gamma"])
+    np.testing.assert_array_equal(codes, np.array(gd["codes"]))
+
+
+@pytest.mark.parametrize("c", [0.02, -0.5, 3.0, 1e-3])
+def test_ternarize_all_equal_gives_sign(c):
+    W = np.full((7, 32), c, dtype=np.float32)
+    gamma, codes = O.ternarize(W)
+    assert gamma == np.float32(abs(c))
+    assert np.all(codes == np.sign(c))
+
+
+def test_ternarize_all_equal_below_eps_gives_zero():
+    # |c| / (|c| + 1e-5) < 0.5 exactly when |c| < 1e-5: the epsilon wins
+    W = np.full((3, 16), 1e-6, dtype=np.float32)
+    _, codes = O.ternarize(W)
+    assert np.all(codes == 0)
+
+
+def test_ternarize_zero_matrix():
+    gamma, codes = O.ternarize(np.zeros((4, 16), np.float32))
+    assert gamma == 0 and np.all(codes == 0)
+
+
+def test_ternarize_gaussian_zero_fraction_closed_form():
+    # For W ~ N(0, s^2): mean|W| = s*sqrt(2/pi), and |W|/gamma < 1/2 has probability
+    # 2*Phi(sqrt(2/pi)/2) - 1 ~= 0.3101; +/-1 split evenly.
+    W = synth.latent_weight(7, 1024, 1024).numpy()
+    _, codes = O.ternarize(W)
+    p0 = 2 * _norm.cdf(0.5 * math.sqrt(2 / math.pi)) - 1
+    assert abs(p0 - 0.3101) < 1e-4
+    frac0 = np.mean(codes == 0)
+    assert abs(frac0 - p0) < 3e-3
+    assert abs(np.mean(codes == 1) - np.mean(codes == -1)) < 3e-3
+
+
+def test_ternarize_negation_and_permutation():
+    W = synth.latent_weight(8, 64, 128).numpy()
+    g1, c1 = O.ternarize(W)
+    g2, c2 = O.ternarize(-W)
+    assert g1 == g2
+    np.testing.assert_array_equal(c2, -c1)
+    perm = np.random.default_rng(0).permutation(W.size)
+    g3, c3 = O.ternarize(W.reshape(-1)[perm].reshape(W.shape))
+    assert g3 == g1 or abs(float(g3) - float(g1)) <= 1e-7 * float(g1)
+    np.testing.assert_array_equal(c3.reshape(-1), c1.reshape(-1)[perm])
+
+
+def test_ternarize_gamma_is_mean_abs_library():
+    W = synth.latent_weight(9, 100, 48).numpy()
+    gamma, _ = O.ternarize(W)
+    ref = math.fsum(abs(float(v)) for v in W.reshape(-1)) / W.size   # exactly rounded sum
+    assert gamma == np.float32(ref)
+
+
+# ----------------------------------------------------------------- packing
+
+def test_pack_golden_words():
+    gd = _load("packed_words.json")
+    for case in gd["cases"]:
+        codes = np.array([case["codes"]], dtype=np.int8)
+        w = O.pack_codes(codes)
+        assert w.shape == (1, 1)
+        assert int(w[0, 0]) == int(case["word"], 16), case["why"]
+        np.testing.assert_array_equal(O.unpack_codes(w, 16), codes)
+
+
+def test_pack_roundtrip_exhaustive_one_word():
+    # every one of the 3^16 code patterns of one uint32 round-trips; a left
+    # inverse also proves that no two patterns share a packed word
+    n = 3 ** 16
+    chunk = 3 ** 12
+    for start in range(0, n, chunk):
+        idx = np.arange(start, start + chunk, dtype=np.int64)
+        digits = np.empty((chunk, 16), dtype=np.int8)
+        v = idx.copy()
+        for k in range(16):
+            digits[:, k] = v % 3 - 1
+            v //= 3
+        words = O.pack_codes(digits)
+        np.testing.assert_array_equal(O.unpack_codes(words, 16), digits)
+
+
+def test_pack_multiword_layout():
+    rng = np.random.default_rng(3)
+    codes = rng.integers(-1, 2, size=(5, 64)).astype(np.int8)
+    words = O.pack_codes(codes)
+    assert words.shape == (5, 4)
+    # word j only depends on columns 16j..16j+15
+    for j in range(4):
+        np.testing.assert_array_equal(words[:, j], O.pack_codes(codes[:, 16 * j:16 * j + 16])[:, 0])
+
+
+# ----------------------------------------------------------------- RMSNorm + absmax quantisation
+
+def test_quant_constant_vector():
+    for c in (0.3, -2.0, 1e-3):
+        q, s = O.absmax_quantize(O.rmsnorm(np.full((1, 64), c, np.float32)))
+        assert np.all(q == 127 * np.sign(c))
+
+
+def test_quant_one_hot():
+    x = np.zeros((1, 128), np.float32)
+    x[0, 17] = -3.5
+    xhat = O.rmsnorm(x)
+    q, s = O.absmax_quantize(xhat)
+    assert q[0, 17] == -127 and np.count_nonzero(q) == 1
+    # x^ at the hot index = x / sqrt(x^2/K + eps) (~= -sqrt(K))
+    want = -3.5 / math.sqrt(3.5 ** 2 / 128 + O.EPS_NORM)
+    assert abs(xhat[0, 17] - want) < 1e-6 * abs(want)
+
+
+@pytest.mark.parametrize("a,b", [(2.0, 0.75), (-4.0, 1.1), (0.5, -0.2)])
+def test_quant_two_value_closed_form(a, b):
+    # x^ is proportional to x, so q_b = round(127 * b / |a|) * sign... and q_a = 127*sign(a)
+    x = np.zeros((1, 48), np.float32)
+    x[0, 0], x[0, 1] = a, b
+    xhat = O.rmsnorm(x)
+    q, s = O.absmax_quantize(xhat)
+    assert q[0, 0] == 127 * np.sign(a)
+    assert q[0, 1] == round(127 * b / abs(a))
+    assert np.count_nonzero(q) == 2
+    # s = 127 / max|x^| with x^ = x / sqrt(mean(x^2) + eps)
+    r = math.sqrt((a * a + b * b) / 48 + O.EPS_NORM)
+    assert abs(float(s[0]) - 127 * r / abs(a)) <= 1e-6 * 127 * r / abs(a)
+
+
+def test_quant_gain_closed_form():
+    gain = np.array([1.0, 0.5, -1.0, 0.25, 2.0, -0.1, 0.0, 1.5] * 4, np.float32)
+    q, _ = O.absmax_quantize(O.rmsnorm(np.ones((1, 32), np.float32), gain=gain))
+    np.testing.assert_array_equal(q[0], np.rint(127 * gain / 2.0).astype(np.int8))
+
+
+def test_quant_max_element_is_127_and_negation_symmetry():
+    x = synth.activations(11, 64, 256, outlier_p=0.01).numpy()
+    q, s = O.absmax_quantize(O.rmsnorm(x))
+    am = np.argmax(np.abs(x), axis=1)
+    np.testing.assert_array_equal(np.abs(q[np.arange(64), am]), 127)
+    assert np.all(np.abs(q) <= 127)
+    qn, sn = O.absmax_quantize(O.rmsnorm(-x))
+    np.testing.assert_array_equal(qn, -q)
+    np.testing.assert_array_equal(sn, s)
+
+
+def test_quant_error_bound():
+    # |q/s - x^| <= 1/(2s): the round-to-nearest bound
+    x = synth.activations(12, 32, 512).numpy()
+    xhat = O.rmsnorm(x)
+    q, s = O.absmax_quantize(xhat)
+    err = np.abs(q / s[:, None].astype(np.float64) - xhat.astype(np.float64))
+    assert np.all(err <= 0.5 / s[:, None] * (1 + 1e-6))
+
+
+def test_rmsnorm_textbook():
+    x = synth.activations(13, 16, 300).numpy().astype(np.float64)
+    ref = x / np.sqrt(np.mean(x * x, axis=1, keepdims=True) + O.EPS_NORM)
+    np.testing.assert_allclose(O.rmsnorm(x), ref, rtol=2e-7, atol=0)
+
+
+def test_quant_zero_row_is_degenerate_zero():
+    q, s = O.absmax_quantize(O.rmsnorm(np.zeros((2, 32), np.float32)))
+    assert np.all(q == 0)
+    assert np.all(s == np.float32(127) / np.float32(1e-5))
+
+
+# ----------------------------------------------------------------- ternary accumulation
+
+def test_accumulate_brute_force_all_ternary_rows():
+    # every ternary row of length 4 against every integer input in {-2..2}^4
+    rows = np.array(np.meshgrid(*[[-1, 0, 1]] * 4, indexing="ij")).reshape(4, -1).T.astype(np.int8)
+    qs = np.array(np.meshgrid(*[range(-2, 3)] * 4, indexing="ij")).reshape(4, -1).T.astype(np.int8)
+    acc = O.ternary_accumulate(qs, rows)
+    ref = qs.astype(np.float64) @ rows.astype(np.float64).T
+    np.testing.assert_array_equal(acc, ref.astype(np.int64))
+
+
+def test_accumulate_extremes_and_library_matmul():
+    rng = np.random.default_rng(5)
+    K = 6912
+    q = rng.integers(-127, 128, size=(3, K)).astype(np.int8)
+    codes = rng.integers(-1, 2, size=(9, K)).astype(np.int8)
+    q[0] = 127
+    codes[0] = 1
+    codes[1] = -1
+    acc = O.ternary_accumulate(q, codes)
+    ref = torch.tensor(q, dtype=torch.int64) @ torch.tensor(codes, dtype=torch.int64).T
+    np.testing.assert_array_equal(acc, ref.numpy())
+    assert acc[0, 0] == 127 * K and acc[0, 1] == -127 * K
+
+
+def test_accumulate_via_packed_words():
+    rng = np.random.default_rng(6)
+    codes = rng.integers(-1, 2, size=(33, 96)).astype(np.int8)
+    q = rng.integers(-127, 128, size=(5, 96)).astype(np.int8)
+    back = O.unpack_codes(O.pack_codes(codes), 96)
+    np.testing.assert_array_equal(O.ternary_accumulate(q, back), O.ternary_accumulate(q, codes))
+
+
+# ----------------------------------------------------------------- BitLinear
+
+def _lin(seed, n, k):
+    return O.make_tlinear(synth.latent_weight(seed, n, k).numpy())
+
+
+def test_bitlinear_identity_weights_closed_form():
+    K = 64
+    W = np.eye(K, dtype=np.float32) * 0.3
+    lin = O.make_tlinear(W)
+    np.testing.assert_array_equal(lin.codes, np.eye(K, dtype=np.int8))
+    assert lin.gamma == np.float32(0.3 / K)
+    x = synth.activations(21, 10, K).numpy()
+    y, p = O.bitlinear(x, lin, parts=True)
+    xhat = O.rmsnorm(x).astype(np.float64)
+    s = p["s"].astype(np.float64)[:, None]
+    np.testing.assert_allclose(y, float(lin.gamma) * p["q"] / s, rtol=1e-15)
+    assert np.all(np.abs(y - float(lin.gamma) * xhat) <= float(lin.gamma) * 0.5 / s * (1 + 1e-6))
+
+
+def test_bitlinear_sign_symmetries():
+    lin = _lin(22, 40, 128)
+    x = synth.activations(23, 7, 128).numpy()
+    y = O.bitlinear(x, lin)
+    np.testing.assert_array_equal(O.bitlinear(-x, lin), -y)
+    neg = O.TLinear(-lin.codes, lin.gamma)
+    np.testing.assert_array_equal(O.bitlinear(x, neg), -y)
+
+
+def test_bitlinear_scale_invariance():
+    lin = _lin(24, 64, 256)
+    x = synth.activations(25, 9, 256).numpy()
+    y = O.bitlinear(x, lin)
+    y2 = O.bitlinear(x * 4.0, lin)      # power of two: x^ changes only through eps
+    y3 = O.bitlinear(x * 3.7, lin)
+    scale = np.max(np.abs(y))
+    assert np.max(np.abs(y2 - y)) <= 1e-2 * scale
+    assert np.max(np.abs(y3 - y)) <= 1e-2 * scale
+
+
+def test_bitlinear_zero_input_gives_bias():
+    lin = _lin(26, 8, 32)
+    lin.bias = np.arange(8, dtype=np.float64)
+    np.testing.assert_array_equal(O.bitlinear(np.zeros((3, 32)), lin), np.tile(np.arange(8.0), (3, 1)))
+
+
+def test_bitlinear_approximates_dense_product():
+    # dequantised result is close to x^ @ (gamma*codes)^T: the quantisation error bound
+    lin = _lin(27, 50, 512)
+    x = synth.activations(28, 6, 512).numpy()
+    y, p = O.bitlinear(x, lin, parts=True)
+    dense = p["xhat"].astype(np.float64) @ (float(lin.gamma) * lin.codes.astype(np.float64)).T
+    bound = float(lin.gamma) * 0.5 / p["s"].astype(np.float64)[:, None] * np.sum(np.abs(lin.codes), axis=1)[None, :]
+    assert np.all(np.abs(y - dense) <= bound * (1 + 1e-9))
+
+
+# ----------------------------------------------------------------- MLGRU scan
+
+def test_sigmoid_silu_identities():
+    z = np.linspace(-30, 30, 601)
+    np.testing.assert_allclose(O.sigmoid(z) + O.sigmoid(-z), 1.0, rtol=0, atol=1e-15)
+    np.testing.assert_allclose(O.silu(z) - O.silu(-z), z, rtol=0, atol=1e-13)
+    assert O.sigmoid(0.0) == 0.5 and O.silu(0.0) == 0.0
+    assert O.sigmoid(-1e4) == 0.0 and O.sigmoid(1e4) == 1.0
+
+
+def _scan_inputs(seed, B=2, T=32, d=8):
+    p = synth.preacts(seed, B, T, d).numpy().astype(np.float64)
+    return p[:, :, 0], p[:, :, 1], p[:, :, 2]
+
+
+def test_scan_forget_zero_gives_candidate():
+    _, pc, pg = _scan_inputs(31)
+    pf = np.full_like(pc, -1e4)
+    h0 = np.ones(pc[:, 0].shape) * 5
+    o, hT = O.mlgru_scan(pf, pc, pg, h0)
+    np.testing.assert_allclose(o, O.sigmoid(pg) * O.silu(pc), rtol=1e-15)
+    np.testing.assert_allclose(hT, O.silu(pc[:, -1]), rtol=1e-15)
+
+
+def test_scan_forget_one_holds_state():
+    _, pc, pg = _scan_inputs(32)
+    pf = np.full_like(pc, 1e4)
+    h0 = synth.activations(33, 2, 8).numpy().astype(np.float64)
+    o, hT = O.mlgru_scan(pf, pc, pg, h0)
+    np.testing.assert_array_equal(hT, h0)
+    np.testing.assert_allclose(o, O.sigmoid(pg) * h0[:, None, :], rtol=1e-15)
+
+
+def test_scan_unrolled_closed_form():
+    pf, pc, pg = _scan_inputs(34, T=24)
+    h0 = synth.activations(35, 2, 8).numpy().astype(np.float64)
+    o, hT = O.mlgru_scan(pf, pc, pg, h0)
+    f, c, g = O.sigmoid(pf), O.silu(pc), O.sigmoid(pg)
+    T = pf.shape[1]
+    for t in range(T):
+        # h_t = (prod_{r<=t} f_r) h0 + sum_{s<=t} (prod_{s<r<=t} f_r) (1 - f_s) c_s
+        h = np.prod(f[:, :t + 1], axis=1) * h0
+        for s in range(t + 1):
+            h = h + np.prod(f[:, s + 1:t + 1], axis=1) * (1 - f[:, s]) * c[:, s]
+        np.testing.assert_allclose(o[:, t], g[:, t] * h, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(hT, h, rtol=1e-12)
+
+
+def test_scan_convex_bound_and_chunking_and_batch_independence():
+    pf, pc, pg = _scan_inputs(36, B=3, T=40, d=16)
+    h0 = synth.activations(37, 3, 16).numpy().astype(np.float64)
+    o, hT = O.mlgru_scan(pf, pc, pg, h0)
+    c = O.silu(pc)
+    # |h_t| <= max(|h0|, max_s |c_s|) because h_t is a convex combination
+    h = o / O.sigmoid(pg)
+    bound = np.maximum(np.abs(h0), np.max(np.abs(c), axis=1))
+    assert np.all(np.abs(h) <= bound[:, None, :] * (1 + 1e-12))
+    # split the sequence: scan(T) == scan(T1) then scan(T - T1) from its state
+    o1, h1 = O.mlgru_scan(pf[:, :13], pc[:, :13], pg[:, :13], h0)
+    o2, h2 = O.mlgru_scan(pf[:, 13:], pc[:, 13:], pg[:, 13:], h1)
+    np.testing.assert_array_equal(np.concatenate([o1, o2], axis=1), o)
+    np.testing.assert_array_equal(h2, hT)
+    # batch rows do not interact
+    ob, hb = O.mlgru_scan(pf[1:2], pc[1:2], pg[1:2], h0[1:2])
+    np.testing.assert_array_equal(ob[0], o[1])
+
+
+# ----------------------------------------------------------------- GLU and block
+
+def _block(seed, d, inner):
+    lat = {}
+    for i, name in enumerate(synth.PROJ_NAMES):
+        n, k = {"f": (d, d), "c": (d, d), "g": (d, d), "o": (d, d),
+                "gate": (inner, d), "up": (inner, d), "down": (d, inner)}[name]
+        lat[name] = synth.latent_weight(synth.sub_seed(seed, 0, i), n, k).numpy()
+    return O.make_block(lat)
+
+
+def test_glu_identity_weights_closed_form():
+    # gate = up = I: p = SiLU(gamma_g q/s) * (gamma_u q/s); swapping the SiLU branch changes it
+    d = 32
+    eye = O.make_tlinear(np.eye(d, dtype=np.float32) * d)            # gamma = 1
+    eye2 = O.make_tlinear(-np.eye(d, dtype=np.float32) * 2 * d)      # up = -I, gamma = 2
+    blk = _block(41, d, d)
+    blk.gate, blk.up = eye, eye2
+    x = synth.activations(42, 5, d).numpy()
+    _, parts = O.glu(x, blk, "f32", parts=True)
+    q, s = O.absmax_quantize(O.rmsnorm(x))
+    u = float(eye.gamma) * q / s[:, None].astype(np.float64)
+    v = -float(eye2.gamma) * q / s[:, None].astype(np.float64)
+    np.testing.assert_allclose(parts["p"], O.round_f32(O.silu(u) * v), rtol=1e-7)
+    swapped = O.silu(v) * u
+    assert np.max(np.abs(swapped - parts["p"])) > 0.1 * np.max(np.abs(parts["p"]))
+
+
+def test_block_zero_weights_is_identity():
+    d, inner, B, T = 32, 48, 2, 6
+    blk = _block(43, d, inner)
+    for name in ("f", "c", "g", "o", "gate", "up", "down"):
+        lin = getattr(blk, name)
+        setattr(blk, name, O.make_tlinear(np.zeros((lin.N, lin.K), np.float32)))
+    x = O.round_bf16(synth.activations(44, B * T, d).numpy().reshape(B, T, d))
+    h0 = synth.activations(45, B, d).numpy().astype(np.float64)
+    y, hT = O.block_forward(x, blk, h0, "bf16")
+    np.testing.assert_array_equal(y, x)
+    # f = sigmoid(0) = 1/2, c = SiLU(0) = 0: h_T = 2^-T h0
+    np.testing.assert_array_equal(hT, O.round_f32(h0 * 0.5 ** T))
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_block_prefill_equals_decode_steps(dtype):
+    d, inner, B, T = 32, 64, 2, 5
+    blk = _block(46, d, inner)
+    x = O.store(synth.activations(47, B * T, d).numpy().reshape(B, T, d), dtype)
+    h0 = np.zeros((B, d))
+    y, hT = O.block_forward(x, blk, h0, dtype)
+    h = h0
+    ys = []
+    for t in range(T):
+        yt, h = O.block_forward(x[:, t:t + 1], blk, h, dtype)
+        ys.append(yt)
+    yd = np.concatenate(ys, axis=1)
+    # state is stored in fp32 between decode calls, so agreement is to rounding
+    np.testing.assert_allclose(yd, y, rtol=0, atol=2e-2 * np.max(np.abs(y)))
+    np.testing.assert_allclose(h, hT, rtol=1e-5, atol=1e-6)
+
+
+def test_stack_composes_blocks():
+    d, inner, B, T = 16, 32, 1, 4
+    blocks = [_block(50 + l, d, inner) for l in range(3)]
+    x = O.round_f32(synth.activations(53, B * T, d).numpy().reshape(B, T, d))
+    h0s = np.zeros((3, B, d))
+    y, hs = O.stack_forward(x, blocks, h0s, "f32")
+    z = x
+    for l in range(3):
+        z, h = O.block_forward(z, blocks[l], h0s[l], "f32")
+        np.testing.assert_array_equal(h, hs[l])
+    np.testing.assert_array_equal(z, y)
