@@ -1,0 +1,372 @@
+#!/usr/bin/env python
+"""Benchmark of the MatMul-free block forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mmf|reference] [--workload NAME]
+
+One step = one pass of the whole hot path over one batch of synthetic input:
+for the default workload, the 370M-shaped stack prefill (24 MatMul-free blocks,
+d=1024, GLU inner 2816, batch 8 x 2048 tokens, bf16): per block the fused
+RMSNorm+absmax quantisation, the ternary contractions (f|c|g, o, gate|up, down),
+the MLGRU scan and the GLU, with the recurrent state reset to zero.
+
+Prints ONE JSON line (rank 0). `value` is whole-job tokens/s with the inputs
+already resident in HBM; `e2e` is the same metric through the public API with
+the step's input copied from pinned host memory and its output copied back
+inside the timed region. Under torchrun each rank runs an independent replica
+(sequences are independent: no collective on the data path) and the time is
+the max over ranks.
+
+`--impl reference` times the CPU oracle on a bounded sample of the same
+workload on this host's cores (the baseline arm; rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "BitLinear GB/s & int8 TOPS vs roofline; MMfree block tokens/sec on 1 B200"
+L2_BYTES = 126 * 1024 * 1024
+# int8 dense tensor peak = measured bf16 peak x (4.5 / 2.25), the nominal int8:bf16 ratio
+INT8_OVER_BF16 = 2.0
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["mmf", "reference"], default="mmf")
+    ap.add_argument("--workload", choices=["stack370m"], default="stack370m")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args(argv)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def dist_init(world):
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.idx = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+
+        def num(x):
+            try:
+                return float(x)
+            except ValueError:
+                return None
+        sm = [num(r[1]) for r in rows if num(r[1]) is not None]
+        mx = [num(r[2]) for r in rows if num(r[2]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- workload
+
+def stack_workload():
+    return synth.STACK_370M
+
+
+def gemm_ops_per_step(w) -> float:
+    """Algorithmic int8 ops (2 per weight per token) of one stack pass: 2*M*(3dd + dd + 2Id + dI) * L."""
+    M = w.batch * w.seq
+    per_layer = 3 * w.d * w.d + w.d * w.d + 2 * w.inner * w.d + w.d * w.inner
+    return 2.0 * M * per_layer * w.layers
+
+
+def build_stack(w, device):
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    shapes = {"f": (w.d, w.d), "c": (w.d, w.d), "g": (w.d, w.d), "o": (w.d, w.d),
+              "gate": (w.inner, w.d), "up": (w.inner, w.d), "down": (w.d, w.inner)}
+    blocks = []
+    for layer in range(w.layers):
+        lins = {}
+        for i, name in enumerate(synth.PROJ_NAMES):
+            W = synth.latent_weight(synth.sub_seed(w.seed, layer, i), *shapes[name], device=device)
+            lins[name] = mmf.quantize_weights(W)
+            del W
+        blocks.append(mmf.Block(lins))
+    torch.cuda.synchronize()
+    return blocks
+
+
+# ----------------------------------------------------------------------------- oracle timing
+
+def oracle_sample(w, tokens: int):
+    """Time the CPU oracle on one block over `tokens` tokens of one sequence; returns (seconds, threads)."""
+    import numpy as np
+    from threadpoolctl import threadpool_info
+
+    import oracle as O
+    shapes = {"f": (w.d, w.d), "c": (w.d, w.d), "g": (w.d, w.d), "o": (w.d, w.d),
+              "gate": (w.inner, w.d), "up": (w.inner, w.d), "down": (w.d, w.inner)}
+    lat = {n: synth.latent_weight(synth.sub_seed(w.seed, 0, i), *shapes[n]).numpy()
+           for i, n in enumerate(synth.PROJ_NAMES)}
+    blk = O.make_block(lat)
+    x = synth.activations(w.seed + synth.ACT_SEED_OFFSET, tokens, w.d, torch.bfloat16)
+    x = x.float().numpy().astype(np.float64).reshape(1, tokens, w.d)
+    t0 = time.perf_counter()
+    O.block_forward(x, blk, np.zeros((1, w.d)), w.dtype)
+    dt = time.perf_counter() - t0
+    threads = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+    return dt, threads
+
+
+def cpu_baseline_entry(w, tokens: int):
+    dt, threads = oracle_sample(w, tokens)
+    tps = tokens / (dt * w.layers)
+    return {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"1 of {w.layers} blocks on {tokens} tokens of 1 of {w.batch} sequences "
+                      f"({dt:.2f} s), extrapolated x{w.layers} blocks",
+            "host_cores_available": len(os.sched_getaffinity(0))}
+
+
+# ----------------------------------------------------------------------------- arms
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    w = stack_workload()
+    tokens = 512
+    times = []
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        dt, threads = oracle_sample(w, tokens)
+        if i >= args.warmup:
+            times.append(dt)
+    mean = sum(times) / len(times)
+    value = tokens / (mean * w.layers)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": mean * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "d": w.d, "inner": w.inner, "layers": w.layers, "batch": w.batch,
+                   "seq": w.seq, "global_batch": w.batch, "seq_len": w.seq, "parallelism": "none (CPU oracle)"},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"each step: 1 of {w.layers} blocks on {tokens} tokens of 1 sequence, "
+                                   f"extrapolated x{w.layers} blocks"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def run_mmf(args):
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist_init(world)
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    mmf.load()
+    dev = torch.device("cuda", local)
+    w = stack_workload()
+    peaks, peak_kind = load_peaks()
+
+    blocks = build_stack(w, dev)
+    st = mmf.State(w.layers, w.batch, w.d)
+    x_host = synth.activations(w.seed + synth.ACT_SEED_OFFSET + rank, w.batch * w.seq, w.d,
+                               torch.bfloat16).reshape(w.batch, w.seq, w.d)
+    x = x_host.to(dev)
+    y = torch.empty_like(x)
+    ws = torch.empty(mmf.stack_ws_size(blocks, w.batch, w.seq), dtype=torch.uint8, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(xin, yout):
+        st.reset()
+        mmf.stack_forward(blocks, st, xin, ws=ws, out=yout)
+
+    for _ in range(args.warmup):
+        step(x, y)
+    mmf.check()
+
+    # ------------------------------------------------------------ timed region (inputs resident)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    clocks = ClockSampler(local)
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()                     # L2 flush between timed steps, outside the step's events
+        starts[i].record(stream)
+        step(x, y)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    clk = clocks.stop()
+    mmf.prof_enable(False)
+    prof = mmf.prof_collect()
+    mmf.check()
+    step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = max_over_ranks(sum(step_ms), world)
+    ms_per_step = total_ms / args.steps
+    tokens_per_step = w.batch * w.seq
+    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+
+    # dominant kernel: the ternary contraction (tensor-bound)
+    gemm_names = [k for k in prof if k.startswith("tgemm")]
+    gemm_ms = sum(prof[k][1] for k in gemm_names)
+    gemm_launches = sum(prof[k][0] for k in gemm_names)
+    ops = gemm_ops_per_step(w) * args.steps
+    achieved = ops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
+    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_OVER_BF16
+    launches = sum(v[0] for v in prof.values())
+    roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                "frac": achieved / peak, "traffic": None,
+                "kernel": ",".join(gemm_names), "launches": gemm_launches,
+                "share_of_step": gemm_ms / sum(step_ms) if step_ms else None,
+                "peak_source": f"{peak_kind}: bf16 sustained x {INT8_OVER_BF16} (int8 dense : bf16 dense nominal)",
+                "per_kernel_ms": {k: round(v[1] / args.steps, 4) for k, v in prof.items()}}
+
+    # ------------------------------------------------------------ end to end through the public API
+    e2e = None
+    if not args.no_e2e:
+        x_pin = x_host.pin_memory()
+        y_pin = torch.empty_like(x_pin).pin_memory()
+        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        barrier(world)
+        torch.cuda.synchronize()
+        for i in range(args.steps):
+            flush.zero_()
+            e_s[i].record(stream)
+            x.copy_(x_pin, non_blocking=True)
+            step(x, y)
+            y_pin.copy_(y, non_blocking=True)
+            e_e[i].record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), world)
+        nbytes = x_pin.numel() * x_pin.element_size()
+        e2e = {"value": world * tokens_per_step * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+
+    cpu = None
+    if rank == 0 and world == 1:
+        cpu = cpu_baseline_entry(w, 2048)
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": w.name, "d": w.d, "inner": w.inner, "layers": w.layers, "batch": w.batch,
+                       "seq": w.seq, "global_batch": w.batch * world, "seq_len": w.seq,
+                       "parallelism": f"replicas x{world} (independent sequences)",
+                       "l2": "flushed between timed steps (256 MB write outside the step events)"},
+            "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": int(launches), "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+        dist.destroy_process_group()
+    return 0
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    if args.warmup < 3:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mmf(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

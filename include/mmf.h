@@ -1,0 +1,263 @@
+/*
+ * mmf.h - C ABI of the MatMul-free block forward on NVIDIA B200 (sm_100a).
+ *
+ * The operations follow the web pages on "Scalable MatMul-free Language
+ * Modeling" (arXiv 2406.02528):
+ *   [DC] "MatMul-free language models", DataCamp blog:
+ *        "Replacing MatMul with ternary operations" (absmean ternary weights,
+ *        multiply by -1/0/1 as negate/drop/keep) and "Core components: MLGRU
+ *        and GLU" (MLGRU token mixer, MatMul-free GLU, overview figure panels
+ *        "MatMul vs. scaled ternary accumulation" and "RMS Norm").
+ *   [HL] hysenlabs review of ridgerchu/matmulfreellm: "FusedBitLinear" (RMSNorm
+ *        then a fused quantise-and-accumulate kernel) and "HGRN attention"
+ *        (f/c/g projections, recurrence, o-projection).
+ *
+ * Conventions for every call below
+ *   - Pointers marked (device) are CUDA device addresses on the current
+ *     device; (host) are ordinary host addresses. The caller owns every buffer
+ *     it passes; the library never frees or keeps them past the call, except
+ *     the weight pointers remembered by mmf_block_create (see there).
+ *   - Tensors are dense and row-major (last index fastest). All device pointers
+ *     must be 16-byte aligned; row lengths K and d must be multiples of 16.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *     Compute calls are asynchronous on that stream and do not synchronise,
+ *     except mmf_state_get / mmf_state_set / mmf_check, which synchronise it.
+ *   - `ws` / `ws_bytes` is caller-owned device scratch; the matching *_ws_size
+ *     function gives the minimum size. Workspace contents need no initialisation
+ *     and are clobbered. Calls that share a workspace must not overlap in time.
+ *   - Every argument is validated on the host before any launch; on error the
+ *     call returns a non-zero mmf_status, launches nothing and sets a message
+ *     readable with mmf_last_error() (thread-local). No C++ exception, abort or
+ *     exit ever crosses this interface.
+ *   - Kernels never trap: a device-side fault condition (for example a bounded
+ *     wait that ran out) is recorded in a per-device status word which
+ *     mmf_check() returns and clears.
+ *   - Activation dtypes: MMF_F32 (float) or MMF_BF16 (bfloat16). Internal
+ *     arithmetic is int8 x ternary -> int32 for the accumulation and fp32
+ *     elsewhere; the recurrent state h is always fp32.
+ */
+#ifndef MMF_H_
+#define MMF_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum mmf_status {
+  MMF_OK = 0,
+  MMF_ERR_INVALID_ARG = 1,        /* null pointer, negative size, bad enum */
+  MMF_ERR_UNSUPPORTED_SHAPE = 2,  /* K or d not a multiple of 16, too large, gains differ */
+  MMF_ERR_MISALIGNED = 3,         /* a device pointer is not 16-byte aligned */
+  MMF_ERR_WORKSPACE = 4,          /* ws_bytes smaller than the *_ws_size answer */
+  MMF_ERR_CUDA = 5,               /* a CUDA runtime call failed (message has the CUDA error) */
+  MMF_ERR_TIMEOUT = 6,            /* a bounded device-side wait ran out (mmf_check) */
+  MMF_ERR_NOMEM = 7               /* host or device allocation inside the library failed */
+} mmf_status;
+
+typedef enum mmf_dtype { MMF_F32 = 0, MMF_BF16 = 1 } mmf_dtype;
+
+/* Library version string, e.g. "mmf 0.1.0 sm_100a". */
+const char* mmf_version(void);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* mmf_last_error(void);
+
+/* Synchronise `stream`, then return MMF_ERR_CUDA for a pending CUDA error or
+ * MMF_ERR_TIMEOUT if a kernel recorded a bounded-wait timeout since the last
+ * check (the status word is cleared), else MMF_OK. */
+mmf_status mmf_check(void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Ternary weights                                                            */
+/* ------------------------------------------------------------------------- */
+
+/* A ternary BitLinear layer y = BitLinear(x), x: [M, K] -> y: [M, N].
+ *   packed (device) uint32 [N, K/16]: 2-bit codes, K-contiguous. The stored
+ *          value is w + 1 in {0,1,2} for w in {-1,0,1}; the code of column
+ *          k = 16*j + 4*i + b is in word j at bits [8*b + 2*i, 8*b + 2*i + 2).
+ *          Field value 3 is invalid.
+ *   gamma  (device) one float: the absmean weight scale of the whole matrix.
+ *   gain   (device) float [K] RMSNorm gain, or NULL for all ones.
+ *   bias   (device) float [N], or NULL for all zeros.
+ * The struct itself is read during the call only. */
+typedef struct mmf_tlinear {
+  const uint32_t* packed;
+  const float* gamma;
+  const float* gain;
+  const float* bias;
+  int32_t N;
+  int32_t K;
+} mmf_tlinear;
+
+/* Scratch bytes mmf_quantize_weights needs for an N x K matrix. */
+size_t mmf_quantize_weights_ws_size(int32_t N, int32_t K);
+
+/* Absmean ternarisation and 2-bit packing of one latent weight matrix.
+ * [DC] "Replacing MatMul with ternary operations": the matrix is scaled by the
+ * mean absolute value of its elements and each element is rounded to the
+ * nearest of -1, 0, 1. Here gamma = (float)(sum |W| in fp64 / (N*K)) and
+ * w = clamp(round_half_even(W / (gamma + 1e-5f)), -1, 1) with one IEEE fp32
+ * division. The fp64 sum is reduced in a fixed order, so the result is
+ * deterministic for a given N, K.
+ *   W      (device) float [N, K] latent weights (read only)
+ *   packed (device) uint32 [N, K/16] output codes, format as in mmf_tlinear
+ *   gamma  (device) one float, output
+ * Errors: INVALID_ARG (null, N or K < 1), UNSUPPORTED_SHAPE (K % 16 != 0),
+ *         MISALIGNED, WORKSPACE. */
+mmf_status mmf_quantize_weights(const float* W, int32_t N, int32_t K, uint32_t* packed,
+                                float* gamma, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* FusedBitLinear                                                             */
+/* ------------------------------------------------------------------------- */
+
+/* Optional device outputs of mmf_bitlinear's intermediate steps (each may be NULL). */
+typedef struct mmf_bitlinear_debug {
+  int8_t* q;       /* [M, K] int8 activation codes */
+  float* scale;    /* [M] per-token quantisation scale s */
+  int32_t* acc;    /* [M, N] exact int32 accumulators sum_k q[m,k] * w[n,k] */
+} mmf_bitlinear_debug;
+
+/* Scratch bytes mmf_bitlinear needs for M tokens of length K. */
+size_t mmf_bitlinear_ws_size(int32_t M, int32_t K);
+
+/* FusedBitLinear forward. [HL] "FusedBitLinear": RMSNorm on the input, then
+ * quantisation and accumulation against ternary weights; [DC] "Replacing
+ * MatMul with ternary operations" and the overview figure's "MatMul vs. scaled
+ * ternary accumulation" panel. Per token m:
+ *   x^ = x * (1 / sqrt(mean(x^2) + eps)) * gain        (mean of squares summed in fp64)
+ *   s  = 127 / max(max|x^|, 1e-5),  q = clamp(round_half_even(x^ * s), -128, 127)
+ *   acc[n] = sum_k q[k] * w[n,k]   exactly, in int32
+ *   y[n] = acc[n] * gamma / s + bias[n]
+ *   lin (host) layer description; x (device) [M, K] in dtype; y (device) [M, N]
+ *   in dtype; eps > 0 is the RMSNorm epsilon; dbg (host struct, device
+ *   pointers) may be NULL. M = 0 is allowed and does nothing.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, CUDA. */
+mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_dtype dtype, int32_t M,
+                         void* y, float eps, void* ws, size_t ws_bytes, void* stream,
+                         const mmf_bitlinear_debug* dbg);
+
+/* ------------------------------------------------------------------------- */
+/* MLGRU scan                                                                 */
+/* ------------------------------------------------------------------------- */
+
+/* MLGRU gates and gated recurrence over T tokens for B sequences.
+ * [DC] "Core components: MLGRU and GLU" (token-by-token update of a hidden
+ * state through element-wise gates valued in [0,1]); [HL] "HGRN attention".
+ * With f~, c~, g~ the pre-activations of token t:
+ *   f = sigmoid(f~), c = SiLU(c~), g = sigmoid(g~)
+ *   h_t = f * h_{t-1} + (1 - f) * c,   o'_t = g * h_t
+ *   pre (device) [B, T, 3, d] in dtype: for each token the rows f~, c~, g~
+ *   h   (device) float [B, d]: h_0 on entry, h_T on return (in place)
+ *   o   (device) [B, T, d] in dtype: o'
+ * T = 0 leaves h unchanged. Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d % 8),
+ * MISALIGNED, CUDA. */
+mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
+                          float* h, void* o, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* MatMul-free GLU                                                            */
+/* ------------------------------------------------------------------------- */
+
+/* Scratch bytes mmf_glu needs for M tokens, hidden d, inner size I. */
+size_t mmf_glu_ws_size(int32_t M, int32_t d, int32_t I);
+
+/* MatMul-free GLU channel mixer. [DC] "Core components: MLGRU and GLU": two
+ * separate BitLinear layers, SiLU on one branch, element-wise product, then a
+ * third BitLinear.
+ *   p = SiLU(BitLinear_gate(x)) * BitLinear_up(x)   (stored in dtype, [M, I])
+ *   y = BitLinear_down(p) (+ residual)
+ * gate and up must share one RMSNorm gain (same pointer or both NULL) because x
+ * is normalised and quantised once for both.
+ *   x (device) [M, d]; residual (device) [M, d] or NULL; y (device) [M, d].
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (shapes disagree, gains differ),
+ * MISALIGNED, WORKSPACE, CUDA. */
+mmf_status mmf_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tlinear* down,
+                   const void* x, const void* residual, void* y, int32_t M, mmf_dtype dtype,
+                   float eps, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Blocks and recurrent state                                                 */
+/* ------------------------------------------------------------------------- */
+
+/* Weights of one MatMul-free block: MLGRU projections f, c, g, o (d x d) and
+ * GLU gate, up (I x d) and down (d x I). f, c and g share one gain, gate and up
+ * share one gain. */
+typedef struct mmf_block_weights {
+  mmf_tlinear f, c, g, o, gate, up, down;
+} mmf_block_weights;
+
+typedef struct mmf_block mmf_block;   /* opaque */
+typedef struct mmf_state mmf_state;   /* opaque */
+
+/* Validate a block's weights and build its launch descriptors. The device
+ * buffers named in `w` are NOT copied: they must stay valid and unchanged
+ * until mmf_block_destroy. The handle is host memory owned by the library.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, NOMEM, CUDA. */
+mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, int32_t I, mmf_block** out);
+void mmf_block_destroy(mmf_block* blk);
+
+/* Recurrent state h for L layers x B sequences x d channels, fp32, zeroed.
+ * The library allocates it with cudaMalloc on the current device and frees it
+ * in mmf_state_destroy. */
+mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_state** out);
+void mmf_state_destroy(mmf_state* st);
+/* Zero every layer's state (asynchronous on stream). */
+mmf_status mmf_state_reset(mmf_state* st, void* stream);
+/* Device address of layer `layer`'s state, float [B, d]; NULL if out of range. */
+float* mmf_state_layer(mmf_state* st, int32_t layer);
+/* Copy the whole state [L, B, d] fp32 to / from host memory; synchronises stream. */
+mmf_status mmf_state_get(const mmf_state* st, float* host_dst, void* stream);
+mmf_status mmf_state_set(mmf_state* st, const float* host_src, void* stream);
+
+/* Scratch bytes mmf_block_forward / mmf_stack_forward need for B x T tokens. */
+size_t mmf_block_ws_size(const mmf_block* blk, int32_t B, int32_t T);
+
+/* One MatMul-free block on x [B, T, d] -> y [B, T, d] (both device, dtype):
+ *   y1 = x + o_proj(MLGRU(x)),  y = y1 + GLU(y1)
+ * [HL] "HGRN attention" (the block input is normalised first, then f/c/g
+ * projections, recurrence and o-projection) and [DC] "Core components".
+ * The MLGRU continues from the state of `layer` in `st` and leaves h_T there,
+ * so T = 1 is one decode step and consecutive calls may split a prompt.
+ * x and y must not overlap. Errors: INVALID_ARG, UNSUPPORTED_SHAPE,
+ * MISALIGNED, WORKSPACE, CUDA. */
+mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf_state* st,
+                             const void* x, void* y, int32_t B, int32_t T, mmf_dtype dtype,
+                             float eps, void* ws, size_t ws_bytes, void* stream);
+
+/* L blocks in sequence (block l uses state layer l): y = block_{L-1}(...block_0(x)).
+ * blocks (host) array of L handles. x and y (device) [B, T, d] must not overlap;
+ * intermediate activations live in the workspace (mmf_block_ws_size of the
+ * largest block). Errors as mmf_block_forward. */
+mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t L, mmf_state* st,
+                             const void* x, void* y, int32_t B, int32_t T, mmf_dtype dtype,
+                             float eps, void* ws, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Kernel timing (tracing)                                                    */
+/* ------------------------------------------------------------------------- */
+
+/* When enabled, every kernel launch the library makes is bracketed by two CUDA
+ * events recorded on the launch's stream (process-wide switch, off by default;
+ * do not enable it while capturing a CUDA graph). Costs two event records per
+ * launch and nothing on the device. */
+mmf_status mmf_prof_enable(int32_t on);
+/* Wait for every recorded event pair and fold the durations into per-kernel
+ * totals. Returns the number of kernel kinds seen since the last reset, or -1
+ * on a CUDA error (see mmf_last_error). */
+int32_t mmf_prof_collect(void);
+/* Totals of kernel kind i (0 <= i < mmf_prof_collect()): its name (host buffer,
+ * truncated to name_len - 1 bytes), its number of launches and the summed
+ * device time in milliseconds. */
+mmf_status mmf_prof_get(int32_t i, char* name, size_t name_len, int64_t* launches, double* total_ms);
+/* Forget all totals and pending events. */
+void mmf_prof_reset(void);
+
+#ifdef __cplusplus
+}  /* extern "C" */
+#endif
+
+#endif  /* MMF_H_ */

@@ -1,0 +1,268 @@
+"""Thin torch-facing binding of libmmf.so: argument marshalling only.
+
+Every step of the computation runs in the library's CUDA kernels. Torch is
+used to hold device memory and to name the current CUDA stream. There is no
+CPU path: without the built library or without a CUDA tensor, calls fail.
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Sequence
+
+import torch
+
+from . import _lib as L
+
+_DT = {torch.float32: L.MMF_F32, torch.bfloat16: L.MMF_BF16}
+DEFAULT_EPS = 1e-6
+
+
+def _vp(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(device: torch.device) -> ctypes.c_void_p:
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _need_cuda(*ts: Optional[torch.Tensor]) -> None:
+    for t in ts:
+        if t is not None:
+            if not t.is_cuda:
+                raise ValueError("mmf needs CUDA tensors (there is no CPU path)")
+            if not t.is_contiguous():
+                raise ValueError("mmf needs contiguous tensors")
+
+
+def _dtype(t: torch.Tensor) -> int:
+    if t.dtype not in _DT:
+        raise ValueError(f"unsupported activation dtype {t.dtype}")
+    return _DT[t.dtype]
+
+
+def _workspace(nbytes: int, device, ws: Optional[torch.Tensor]) -> torch.Tensor:
+    if ws is not None:
+        if ws.numel() * ws.element_size() < nbytes:
+            raise ValueError(f"workspace too small: {ws.numel() * ws.element_size()} < {nbytes}")
+        return ws
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def version() -> str:
+    return L.load().mmf_version().decode()
+
+
+def check(stream: Optional[torch.cuda.Stream] = None) -> None:
+    """Synchronise and raise if a kernel recorded a device-side error."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    L.check(L.load().mmf_check(ctypes.c_void_p(s.cuda_stream)), "mmf_check")
+
+
+class TLinear:
+    """A ternary BitLinear held on the device: packed [N, K/16] (int32 storage of uint32), gamma [1]."""
+
+    def __init__(self, packed: torch.Tensor, gamma: torch.Tensor, N: int, K: int,
+                 gain: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None):
+        _need_cuda(packed, gamma, gain, bias)
+        self.packed, self.gamma, self.gain, self.bias = packed, gamma, gain, bias
+        self.N, self.K = int(N), int(K)
+
+    def c(self) -> L.TLinear:
+        return L.TLinear(self.packed.data_ptr(), self.gamma.data_ptr(),
+                         self.gain.data_ptr() if self.gain is not None else None,
+                         self.bias.data_ptr() if self.bias is not None else None, self.N, self.K)
+
+
+def quantize_weights(W: torch.Tensor, gain: Optional[torch.Tensor] = None,
+                     bias: Optional[torch.Tensor] = None) -> TLinear:
+    """Absmean-ternarise and pack a latent fp32 weight [N, K] on the device (mmf_quantize_weights)."""
+    _need_cuda(W)
+    if W.dtype != torch.float32 or W.dim() != 2:
+        raise ValueError("W must be a 2-D float32 CUDA tensor")
+    lib = L.load()
+    N, K = W.shape
+    packed = torch.empty((N, max(K // 16, 1)), dtype=torch.int32, device=W.device)
+    gamma = torch.empty(4, dtype=torch.float32, device=W.device)   # 16-byte slot, element 0 used
+    ws = _workspace(lib.mmf_quantize_weights_ws_size(N, K), W.device, None)
+    L.check(lib.mmf_quantize_weights(_vp(W), N, K, _vp(packed), _vp(gamma), _vp(ws), ws.numel(),
+                                     _stream(W.device)), "mmf_quantize_weights")
+    return TLinear(packed, gamma, N, K, gain, bias)
+
+
+def bitlinear(lin: TLinear, x: torch.Tensor, eps: float = DEFAULT_EPS, debug: bool = False,
+              ws: Optional[torch.Tensor] = None):
+    """y = BitLinear(x) for x [..., K]; with debug=True also returns (q, s, acc)."""
+    _need_cuda(x)
+    lib = L.load()
+    lead = x.shape[:-1]
+    M = int(x.numel() // x.shape[-1]) if x.shape[-1] else 0
+    y = torch.empty(*lead, lin.N, dtype=x.dtype, device=x.device)
+    w = _workspace(lib.mmf_bitlinear_ws_size(M, lin.K), x.device, ws)
+    dbg = None
+    if debug:
+        q = torch.empty(M, lin.K, dtype=torch.int8, device=x.device)
+        s = torch.empty(M, dtype=torch.float32, device=x.device)
+        acc = torch.empty(M, lin.N, dtype=torch.int32, device=x.device)
+        dbg = L.BitlinearDebug(q.data_ptr(), s.data_ptr(), acc.data_ptr())
+    cl = lin.c()
+    L.check(lib.mmf_bitlinear(ctypes.byref(cl), _vp(x), _dtype(x), M, _vp(y), eps, _vp(w),
+                              w.numel() * w.element_size(), _stream(x.device),
+                              ctypes.byref(dbg) if dbg is not None else None), "mmf_bitlinear")
+    if debug:
+        return y, q, s, acc
+    return y
+
+
+def mlgru_scan(pre: torch.Tensor, h: torch.Tensor) -> torch.Tensor:
+    """pre [B, T, 3, d] -> o' [B, T, d]; h [B, d] fp32 is updated in place to h_T."""
+    _need_cuda(pre, h)
+    if pre.dim() != 4 or pre.shape[2] != 3:
+        raise ValueError("pre must be [B, T, 3, d]")
+    B, T, _, d = pre.shape
+    if h.dtype != torch.float32 or tuple(h.shape) != (B, d):
+        raise ValueError("h must be float32 [B, d]")
+    o = torch.empty(B, T, d, dtype=pre.dtype, device=pre.device)
+    lib = L.load()
+    L.check(lib.mmf_mlgru_scan(_vp(pre), _dtype(pre), B, T, d, _vp(h), _vp(o), _stream(pre.device)),
+            "mmf_mlgru_scan")
+    return o
+
+
+def glu(gate: TLinear, up: TLinear, down: TLinear, x: torch.Tensor, residual: Optional[torch.Tensor] = None,
+        eps: float = DEFAULT_EPS, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """y = down(SiLU(gate(x)) * up(x)) (+ residual) for x [..., d]."""
+    _need_cuda(x, residual)
+    lib = L.load()
+    d = x.shape[-1]
+    M = int(x.numel() // d)
+    y = torch.empty_like(x)
+    w = _workspace(lib.mmf_glu_ws_size(M, d, gate.N), x.device, ws)
+    cg, cu, cd = gate.c(), up.c(), down.c()
+    L.check(lib.mmf_glu(ctypes.byref(cg), ctypes.byref(cu), ctypes.byref(cd), _vp(x), _vp(residual), _vp(y), M,
+                        _dtype(x), eps, _vp(w), w.numel() * w.element_size(), _stream(x.device)), "mmf_glu")
+    return y
+
+
+class Block:
+    """Handle of one MatMul-free block (mmf_block_create); keeps its weight tensors alive."""
+
+    NAMES = ("f", "c", "g", "o", "gate", "up", "down")
+
+    def __init__(self, lins: dict):
+        self.lins = dict(lins)
+        self.d = self.lins["f"].K
+        self.inner = self.lins["gate"].N
+        bw = L.BlockWeights(*[self.lins[n].c() for n in self.NAMES])
+        h = ctypes.c_void_p()
+        lib = L.load()
+        L.check(lib.mmf_block_create(ctypes.byref(bw), self.d, self.inner, ctypes.byref(h)), "mmf_block_create")
+        self.handle = h
+
+    def ws_size(self, B: int, T: int) -> int:
+        return int(L.load().mmf_block_ws_size(self.handle, B, T))
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            L.load().mmf_block_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+class State:
+    """Recurrent MLGRU state h [L, B, d] fp32 owned by the library (mmf_state_create)."""
+
+    def __init__(self, L_: int, B: int, d: int):
+        self.L, self.B, self.d = int(L_), int(B), int(d)
+        h = ctypes.c_void_p()
+        L.check(L.load().mmf_state_create(self.L, self.B, self.d, ctypes.byref(h)), "mmf_state_create")
+        self.handle = h
+
+    def reset(self):
+        L.check(L.load().mmf_state_reset(self.handle, _stream(torch.device("cuda"))), "mmf_state_reset")
+
+    def get(self) -> torch.Tensor:
+        out = torch.empty(self.L, self.B, self.d, dtype=torch.float32)
+        L.check(L.load().mmf_state_get(self.handle, ctypes.c_void_p(out.data_ptr()),
+                                       _stream(torch.device("cuda"))), "mmf_state_get")
+        return out
+
+    def set(self, h: torch.Tensor):
+        h = h.detach().to("cpu", torch.float32).contiguous()
+        if tuple(h.shape) != (self.L, self.B, self.d):
+            raise ValueError("state shape mismatch")
+        L.check(L.load().mmf_state_set(self.handle, ctypes.c_void_p(h.data_ptr()),
+                                       _stream(torch.device("cuda"))), "mmf_state_set")
+
+    def close(self):
+        if getattr(self, "handle", None) is not None and self.handle.value:
+            L.load().mmf_state_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def block_forward(block: Block, layer: int, state: State, x: torch.Tensor, eps: float = DEFAULT_EPS,
+                  ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """x [B, T, d] -> y [B, T, d] through one block, continuing state layer `layer`."""
+    _need_cuda(x)
+    B, T, d = x.shape
+    y = out if out is not None else torch.empty_like(x)
+    w = _workspace(block.ws_size(B, T), x.device, ws)
+    L.check(L.load().mmf_block_forward(block.handle, layer, state.handle, _vp(x), _vp(y), B, T, _dtype(x), eps,
+                                       _vp(w), w.numel() * w.element_size(), _stream(x.device)),
+            "mmf_block_forward")
+    return y
+
+
+def stack_ws_size(blocks: Sequence[Block], B: int, T: int) -> int:
+    return max(b.ws_size(B, T) for b in blocks)
+
+
+def stack_forward(blocks: Sequence[Block], state: State, x: torch.Tensor, eps: float = DEFAULT_EPS,
+                  ws: Optional[torch.Tensor] = None, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """x [B, T, d] through len(blocks) blocks (state layer l for block l)."""
+    _need_cuda(x)
+    B, T, d = x.shape
+    y = out if out is not None else torch.empty_like(x)
+    w = _workspace(stack_ws_size(blocks, B, T), x.device, ws)
+    arr = (ctypes.c_void_p * len(blocks))(*[b.handle.value for b in blocks])
+    L.check(L.load().mmf_stack_forward(arr, len(blocks), state.handle, _vp(x), _vp(y), B, T, _dtype(x), eps,
+                                       _vp(w), w.numel() * w.element_size(), _stream(x.device)),
+            "mmf_stack_forward")
+    return y
+
+
+# ---------------------------------------------------------------- launch timing
+
+def prof_enable(on: bool = True) -> None:
+    """Bracket every library kernel launch with CUDA events (mmf_prof_enable)."""
+    L.check(L.load().mmf_prof_enable(1 if on else 0), "mmf_prof_enable")
+
+
+def prof_reset() -> None:
+    L.load().mmf_prof_reset()
+
+
+def prof_collect() -> dict:
+    """{kernel name: (launches, total device ms)} since the last prof_reset()."""
+    lib = L.load()
+    n = lib.mmf_prof_collect()
+    if n < 0:
+        raise L.MMFError(5, "mmf_prof_collect", lib.mmf_last_error().decode())
+    out = {}
+    buf = ctypes.create_string_buffer(128)
+    for i in range(n):
+        launches = ctypes.c_int64()
+        ms = ctypes.c_double()
+        L.check(lib.mmf_prof_get(i, buf, 128, ctypes.byref(launches), ctypes.byref(ms)), "mmf_prof_get")
+        out[buf.value.decode()] = (int(launches.value), float(ms.value))
+    return out

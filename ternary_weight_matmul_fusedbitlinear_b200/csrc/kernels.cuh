@@ -1,0 +1,50 @@
+// Internal launchers of the mmf CUDA library. Not part of the C ABI.
+#pragma once
+
+#include <algorithm>
+
+#include "common.cuh"
+
+namespace mmf {
+
+constexpr int kQuantPartials = 592;   // CTAs of the absmean partial-sum pass (4 x 148 SMs)
+
+size_t quantize_weights_ws_bytes();
+cudaError_t launch_quantize_weights(const float* W, int N, int K, uint32_t* packed, float* gamma, void* ws,
+                                    cudaStream_t stream);
+
+cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
+                                 int8_t* q, float* scale, int32_t* qsum, cudaStream_t stream);
+
+// Epilogues of the ternary contraction.
+enum class Epi : int {
+  kStore = 0,     // y[m, seg*N + n] = acc*gamma_seg/s + bias (+ residual[m, n] when 1 segment)
+  kAcc = 1,       // int32 acc[m, n]
+  kScanStep = 2,  // 3 segments f,c,g: one MLGRU step, h[m, n] in place, o'[m, n]
+  kGlu = 3,       // 2 segments gate,up: p[m, n] = SiLU(u) * v
+};
+
+struct TGemmArgs {
+  const uint32_t* w[3];     // packed ternary weights per segment, [N, K/16]
+  const float* gamma[3];    // per-segment scale (device scalar)
+  const float* bias[3];     // per-segment bias [N] or null
+  int nseg;                 // 1..3
+  int N;                    // rows per segment
+  int K;
+  const int8_t* q;          // [M, K] activation codes
+  const float* s;           // [M] activation scales
+  const int32_t* qsum;      // [M] row sums of q
+  int M;
+  void* out;                // see Epi
+  int ldo;                  // leading dimension of out (elements)
+  const void* residual;     // [M, N] in the activation dtype, or null
+  float* h;                 // kScanStep: [M, N] fp32 state, updated in place
+};
+
+// mma.sync-based contraction (weights as the 16-row A operand, tokens as N=8 tiles).
+cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t stream);
+
+cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o,
+                              cudaStream_t stream);
+
+}  // namespace mmf

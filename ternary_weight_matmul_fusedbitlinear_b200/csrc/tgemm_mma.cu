@@ -1,0 +1,214 @@
+// Packed-ternary x int8 contraction on the warp-level tensor-core MMA
+// (mma.sync m16n8k32, u8 x s8 -> s32). Used for decode-sized token counts,
+// where the kernel streams the 2-bit weights from HBM once.
+//
+// "MatMul-free language models" (DataCamp blog), section "Replacing MatMul
+// with ternary operations": a product with a weight of -1, 0 or 1 is a
+// negation, a drop or a copy, so acc[m, n] = sum_k q[m,k] * w[n,k] is exact
+// integer add/subtract work. Here the stored code is w + 1 in {0,1,2}; the
+// kernel multiplies the stored code as an unsigned byte and subtracts the
+// per-token code sum afterwards: sum_k (w+1) q = acc + sum_k q.
+//
+// Work split: a CTA owns 16 output rows of each of its R weight segments and
+// 8*NT tokens; its 8 warps split K into 256-column segments round-robin. Per
+// 256-column segment a lane (group g, thread t) loads 16 bytes of packed codes
+// for rows g and g+8 (64 columns) and the 64 activation bytes [64t, 64t+64) of
+// its token; the column order inside the segment is permuted identically on
+// both operands, which the sum does not see. Partial sums meet in shared
+// memory through integer atomics (exact in any order), then the epilogue
+// rescales and applies the mode.
+#include "kernels.cuh"
+
+namespace mmf {
+
+namespace {
+
+constexpr int kThreads = 256;
+constexpr int kWarps = 8;
+constexpr uint32_t kLow2 = 0x03030303u;
+
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t u4get(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+// Load 4 consecutive 32-bit words starting at word index `w0` of a row with
+// `nw` words; words at or beyond nw read as 0. One 16-byte load only when the
+// rows are 16-byte aligned (nw % 4 == 0, so every row starts on a 16-byte
+// boundary of the 16-byte aligned matrix) and all 4 words are in the row.
+__device__ __forceinline__ uint4 load_words4(const uint32_t* row, int w0, int nw, bool row_ok) {
+  uint4 r = make_uint4(0u, 0u, 0u, 0u);
+  if (!row_ok) return r;
+  if ((nw & 3) == 0 && w0 + 4 <= nw) return __ldg(reinterpret_cast<const uint4*>(row + w0));
+  if (w0 + 0 < nw) r.x = __ldg(row + w0 + 0);
+  if (w0 + 1 < nw) r.y = __ldg(row + w0 + 1);
+  if (w0 + 2 < nw) r.z = __ldg(row + w0 + 2);
+  if (w0 + 3 < nw) r.w = __ldg(row + w0 + 3);
+  return r;
+}
+
+template <int NT, int R, Epi EPI, typename T>
+__global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
+  __shared__ int red[R][16][NT * 8];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int n0 = blockIdx.x * 16;
+  const int m0 = blockIdx.y * NT * 8;
+  const int K = a.K, N = a.N, M = a.M;
+  const int wpr = K / 16;            // packed words per row
+  const int nkseg = ceil_div(K, 256);
+
+  for (int i = threadIdx.x; i < R * 16 * NT * 8; i += kThreads) (&red[0][0][0])[i] = 0;
+
+  int acc[R][NT][4];
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < NT; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[r][j][e] = 0;
+
+  for (int seg = warp; seg < nkseg; seg += kWarps) {
+    const int w0 = seg * 16 + 4 * t;   // first packed word of this lane
+    uint4 wa[R], wb[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint32_t* W = a.w[r];
+      wa[r] = load_words4(W + (size_t)(n0 + g) * wpr, w0, wpr, n0 + g < N);
+      wb[r] = load_words4(W + (size_t)(n0 + g + 8) * wpr, w0, wpr, n0 + g + 8 < N);
+    }
+    uint4 act[NT][4];
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      const int m = m0 + 8 * j + g;
+      const int8_t* qrow = a.q + (size_t)m * K;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        // bytes [64t + 16u, +16) of this segment = packed word w0 + u's 16 columns
+        const bool ok = (m < M) && (w0 + u < wpr);
+        act[j][u] = ok ? __ldg(reinterpret_cast<const uint4*>(qrow + (size_t)(w0 + u) * 16))
+                       : make_uint4(0u, 0u, 0u, 0u);
+      }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int u = i >> 1, sub = (i & 1) * 2;
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint32_t wg = u4get(wa[r], u), wg8 = u4get(wb[r], u);
+        const uint32_t a0 = (wg >> (2 * sub)) & kLow2;
+        const uint32_t a2 = (wg >> (2 * sub + 2)) & kLow2;
+        const uint32_t a1 = (wg8 >> (2 * sub)) & kLow2;
+        const uint32_t a3 = (wg8 >> (2 * sub + 2)) & kLow2;
+#pragma unroll
+        for (int j = 0; j < NT; ++j) {
+          const uint32_t b0 = u4get(act[j][u], sub), b1 = u4get(act[j][u], sub + 1);
+          mma_u8s8(acc[r][j], a0, a1, a2, a3, b0, b1);
+        }
+      }
+    }
+  }
+  __syncthreads();   // red[] zeroed
+#pragma unroll
+  for (int r = 0; r < R; ++r)
+#pragma unroll
+    for (int j = 0; j < NT; ++j) {
+      atomicAdd(&red[r][g][8 * j + 2 * t], acc[r][j][0]);
+      atomicAdd(&red[r][g][8 * j + 2 * t + 1], acc[r][j][1]);
+      atomicAdd(&red[r][g + 8][8 * j + 2 * t], acc[r][j][2]);
+      atomicAdd(&red[r][g + 8][8 * j + 2 * t + 1], acc[r][j][3]);
+    }
+  __syncthreads();
+
+  // ---------------------------------------------------------------- epilogue
+  constexpr int kCols = NT * 8;
+  if constexpr (EPI == Epi::kStore || EPI == Epi::kAcc) {
+    for (int idx = threadIdx.x; idx < R * 16 * kCols; idx += kThreads) {
+      const int row = idx & 15, r = (idx >> 4) % R, mc = idx / (16 * R);
+      const int n = n0 + row, m = m0 + mc;
+      if (n >= N || m >= M) continue;
+      const int accv = red[r][row][mc] - a.qsum[m];
+      if constexpr (EPI == Epi::kAcc) {
+        static_cast<int32_t*>(a.out)[(size_t)m * a.ldo + r * N + n] = accv;
+      } else {
+        float v = __fdiv_rn(__fmul_rn((float)accv, *a.gamma[r]), a.s[m]);
+        if (a.bias[r] != nullptr) v += a.bias[r][n];
+        if (a.residual != nullptr) v += to_f32(static_cast<const T*>(a.residual)[(size_t)m * N + n]);
+        static_cast<T*>(a.out)[(size_t)m * a.ldo + r * N + n] = from_f32<T>(v);
+      }
+    }
+  } else if constexpr (EPI == Epi::kScanStep) {
+    for (int idx = threadIdx.x; idx < 16 * kCols; idx += kThreads) {
+      const int row = idx & 15, mc = idx >> 4;
+      const int n = n0 + row, m = m0 + mc;
+      if (n >= N || m >= M) continue;
+      float pre[3];
+#pragma unroll
+      for (int r = 0; r < 3; ++r) {
+        float v = __fdiv_rn(__fmul_rn((float)(red[r][row][mc] - a.qsum[m]), *a.gamma[r]), a.s[m]);
+        if (a.bias[r] != nullptr) v += a.bias[r][n];
+        pre[r] = round_to<T>(v);   // the pre-activations are a storage point
+      }
+      const float f = sigmoidf_(pre[0]), c = siluf_(pre[1]), gg = sigmoidf_(pre[2]);
+      float* hp = a.h + (size_t)m * N + n;
+      const float hn = f * (*hp) + (1.0f - f) * c;
+      *hp = hn;
+      static_cast<T*>(a.out)[(size_t)m * a.ldo + n] = from_f32<T>(gg * hn);
+    }
+  } else {  // kGlu
+    for (int idx = threadIdx.x; idx < 16 * kCols; idx += kThreads) {
+      const int row = idx & 15, mc = idx >> 4;
+      const int n = n0 + row, m = m0 + mc;
+      if (n >= N || m >= M) continue;
+      float uv[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        float v = __fdiv_rn(__fmul_rn((float)(red[r][row][mc] - a.qsum[m]), *a.gamma[r]), a.s[m]);
+        if (a.bias[r] != nullptr) v += a.bias[r][n];
+        uv[r] = v;
+      }
+      static_cast<T*>(a.out)[(size_t)m * a.ldo + n] = from_f32<T>(siluf_(uv[0]) * uv[1]);
+    }
+  }
+}
+
+template <int NT, typename T>
+cudaError_t launch_nt(const TGemmArgs& a, Epi epi, cudaStream_t stream) {
+  dim3 grid(ceil_div(a.N, 16), ceil_div(a.M, NT * 8));
+  switch (epi) {
+    case Epi::kStore:
+      if (a.nseg == 1) tgemm_mma_kernel<NT, 1, Epi::kStore, T><<<grid, kThreads, 0, stream>>>(a);
+      else if (a.nseg == 2) tgemm_mma_kernel<NT, 2, Epi::kStore, T><<<grid, kThreads, 0, stream>>>(a);
+      else tgemm_mma_kernel<NT, 3, Epi::kStore, T><<<grid, kThreads, 0, stream>>>(a);
+      break;
+    case Epi::kAcc: tgemm_mma_kernel<NT, 1, Epi::kAcc, T><<<grid, kThreads, 0, stream>>>(a); break;
+    case Epi::kScanStep: tgemm_mma_kernel<NT, 3, Epi::kScanStep, T><<<grid, kThreads, 0, stream>>>(a); break;
+    case Epi::kGlu: tgemm_mma_kernel<NT, 2, Epi::kGlu, T><<<grid, kThreads, 0, stream>>>(a); break;
+  }
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_t(const TGemmArgs& a, Epi epi, cudaStream_t stream) {
+  if (a.M <= 8) return launch_nt<1, T>(a, epi, stream);
+  if (a.M <= 16) return launch_nt<2, T>(a, epi, stream);
+  if (a.M <= 32) return launch_nt<4, T>(a, epi, stream);
+  return launch_nt<8, T>(a, epi, stream);
+}
+
+}  // namespace
+
+cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t stream) {
+  if (a.M == 0 || a.N == 0) return cudaSuccess;
+  return dt == MMF_BF16 ? launch_t<bf16>(a, epi, stream) : launch_t<float>(a, epi, stream);
+}
+
+}  // namespace mmf

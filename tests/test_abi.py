@@ -1,0 +1,96 @@
+"""The C-ABI library loads, exports every declared symbol and validates arguments (no GPU needed)."""
+import ctypes
+import subprocess
+
+import pytest
+
+from ternary_weight_matmul_fusedbitlinear_b200 import _lib as L
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from ternary_weight_matmul_fusedbitlinear_b200 import build
+    build.build()
+    return L.load()
+
+
+def test_every_header_function_is_exported(lib):
+    names = L.header_functions()
+    assert len(names) >= 20
+    out = subprocess.run(["nm", "-D", "--defined-only", L.LIB_PATH], capture_output=True, text=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    missing = [n for n in names if n not in exported]
+    assert not missing, missing
+    assert set(L.SIGNATURES) == set(names)
+
+
+def test_build_targets_sm100a_only():
+    from ternary_weight_matmul_fusedbitlinear_b200 import build
+    assert build.ARCH_FLAGS == ["-gencode", "arch=compute_100a,code=sm_100a"]
+    assert all("sm_" not in f or "100a" in f for f in build.NVCC_FLAGS)
+
+
+def test_version_and_error_message(lib):
+    assert lib.mmf_version().decode().startswith("mmf ")
+    st = lib.mmf_quantize_weights(None, 4, 16, None, None, None, 0, None)
+    assert st == 1
+    assert b"null" in lib.mmf_last_error()
+
+
+def _tl(N, K, packed=16, gamma=16):
+    return L.TLinear(packed, gamma, None, None, N, K)
+
+
+def test_bitlinear_validation_codes(lib):
+    x = ctypes.c_void_p(4096)
+    y = ctypes.c_void_p(8192)
+    ws = ctypes.c_void_p(1 << 20)
+    bad_k = _tl(8, 24)
+    assert lib.mmf_bitlinear(ctypes.byref(bad_k), x, 0, 4, y, 1e-6, ws, 1 << 20, None, None) == 2
+    assert b"multiple of 16" in lib.mmf_last_error()
+    mis = _tl(8, 32, packed=18)
+    assert lib.mmf_bitlinear(ctypes.byref(mis), x, 0, 4, y, 1e-6, ws, 1 << 20, None, None) == 3
+    ok = _tl(8, 32)
+    assert lib.mmf_bitlinear(ctypes.byref(ok), x, 0, 4, y, 1e-6, ws, 16, None, None) == 4      # workspace
+    assert lib.mmf_bitlinear(ctypes.byref(ok), x, 7, 4, y, 1e-6, ws, 1 << 20, None, None) == 1  # dtype
+    assert lib.mmf_bitlinear(ctypes.byref(ok), x, 0, -1, y, 1e-6, ws, 1 << 20, None, None) == 1
+    assert lib.mmf_bitlinear(ctypes.byref(ok), x, 0, 4, y, 0.0, ws, 1 << 20, None, None) == 1   # eps
+    # M = 0 is a no-op that touches nothing
+    assert lib.mmf_bitlinear(ctypes.byref(ok), None, 0, 0, None, 1e-6, None, 0, None, None) == 0
+
+
+def test_scan_and_glu_validation(lib):
+    p = ctypes.c_void_p(4096)
+    assert lib.mmf_mlgru_scan(p, 0, 2, 3, 12, p, p, None) == 2          # d % 8
+    assert lib.mmf_mlgru_scan(p, 0, -1, 3, 16, p, p, None) == 1
+    assert lib.mmf_mlgru_scan(None, 0, 0, 3, 16, None, None, None) == 0  # B = 0 no-op
+    gate, up, down = _tl(64, 32), _tl(64, 32), _tl(32, 64)
+    bad_up = _tl(48, 32)
+    assert lib.mmf_glu(ctypes.byref(gate), ctypes.byref(bad_up), ctypes.byref(down), p, None, p, 4, 0, 1e-6, p,
+                       1 << 20, None) == 2
+    up_gain = L.TLinear(16, 16, 32, None, 64, 32)
+    assert lib.mmf_glu(ctypes.byref(gate), ctypes.byref(up_gain), ctypes.byref(down), p, None, p, 4, 0, 1e-6, p,
+                       1 << 20, None) == 2
+    assert b"share one gain" in lib.mmf_last_error()
+
+
+def test_block_create_validation(lib):
+    d, I = 32, 64
+    sq = lambda: _tl(d, d)
+    w = L.BlockWeights(sq(), sq(), sq(), sq(), _tl(I, d), _tl(I, d), _tl(d, I))
+    h = ctypes.c_void_p()
+    assert lib.mmf_block_create(ctypes.byref(w), d, I, ctypes.byref(h)) == 0
+    assert h.value
+    assert lib.mmf_block_ws_size(h, 2, 8) > 0
+    lib.mmf_block_destroy(h)
+    w.c = L.TLinear(16, 16, 32, None, d, d)  # c has its own gain
+    assert lib.mmf_block_create(ctypes.byref(w), d, I, ctypes.byref(h)) == 2
+    w.c = _tl(d, d)
+    w.down = _tl(d, 48)
+    assert lib.mmf_block_create(ctypes.byref(w), d, I, ctypes.byref(h)) == 2
+
+
+def test_workspace_sizes_grow_with_size(lib):
+    assert lib.mmf_bitlinear_ws_size(16, 2048) < lib.mmf_bitlinear_ws_size(64, 2048)
+    assert lib.mmf_glu_ws_size(4, 1024, 2816) > 4 * 2816
+    assert lib.mmf_quantize_weights_ws_size(2048, 2048) >= 8

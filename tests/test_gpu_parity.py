@@ -1,0 +1,214 @@
+"""CUDA path vs the CPU oracle, element by element, through the C ABI.
+
+Bit-exact: ternary codes (given the GPU's gamma), int32 accumulators (given the
+GPU's activation codes). Activation codes: within 1 on <= 0.01% of elements.
+Floating outputs: normwise 2e-3, storage-type rounding flips allowed (tests/parity.py).
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+import synth
+from parity import (TORCH_DT, assert_close, assert_codes_close, make_block, make_layer, packed_to_np, to_np)
+
+pytestmark = pytest.mark.gpu
+
+mmf = pytest.importorskip("ternary_weight_matmul_fusedbitlinear_b200")
+
+
+# ------------------------------------------------------------------ weights
+
+@pytest.mark.parametrize("n,k", [(2048, 2048), (5632, 2048), (2048, 5632), (37, 48), (1, 16), (3, 4096)])
+def test_quantize_weights_bit_exact(n, k):
+    W = synth.latent_weight(100 + n + k, n, k)
+    lin = mmf.quantize_weights(W.cuda())
+    g_gpu = np.float32(lin.gamma[0].item())
+    g_ref, codes_ref = O.ternarize(W.numpy())
+    assert abs(float(g_gpu) - float(g_ref)) <= float(np.spacing(g_ref)), (g_gpu, g_ref)
+    _, codes_given = O.ternarize(W.numpy(), gamma=g_gpu)
+    codes_gpu = O.unpack_codes(packed_to_np(lin.packed), k)
+    np.testing.assert_array_equal(codes_gpu, codes_given)
+    if g_gpu == g_ref:
+        np.testing.assert_array_equal(codes_gpu, codes_ref)
+
+
+def test_quantize_weights_is_deterministic():
+    W = synth.latent_weight(5, 1024, 1024).cuda()
+    a = mmf.quantize_weights(W)
+    b = mmf.quantize_weights(W)
+    assert torch.equal(a.packed, b.packed) and torch.equal(a.gamma[:1], b.gamma[:1])
+
+
+# ------------------------------------------------------------------ BitLinear
+
+SWEEP = [(k, n, m) for (k, n) in synth.GEMV_SWEEP_SHAPES for m in synth.GEMV_SWEEP_TOKENS]
+RAGGED = [(48, 37, 3), (16, 1, 1), (272, 130, 9), (2048, 2048, 33), (1024, 3072, 130)]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("k,n,m", SWEEP + RAGGED)
+def test_bitlinear_parity(k, n, m, dtype):
+    W, lin, olin = make_layer(200 + k + n, n, k)
+    x = synth.activations(300 + m, m, k, TORCH_DT[dtype], outlier_p=synth.GEMV_OUTLIER_P,
+                          outlier_scale=synth.GEMV_OUTLIER_SCALE)
+    y, q, s, acc = mmf.bitlinear(lin, x.cuda(), debug=True)
+    torch.cuda.synchronize()
+    xn = to_np(x)
+    y_ref, parts = O.bitlinear(xn, olin, parts=True)
+    np.testing.assert_allclose(to_np(s), parts["s"], rtol=1e-6)
+    assert_codes_close(q.cpu().numpy(), parts["q"], "activation codes")
+    codes_gpu = O.unpack_codes(packed_to_np(lin.packed), k)
+    np.testing.assert_array_equal(acc.cpu().numpy().astype(np.int64),
+                                  O.ternary_accumulate(q.cpu().numpy(), codes_gpu))
+    assert_close(to_np(y), y_ref, dtype, "y")
+
+
+def test_bitlinear_empty_and_gain_bias():
+    k, n = 64, 40
+    W, lin, olin = make_layer(17, n, k)
+    y = mmf.bitlinear(lin, torch.empty(0, k, device="cuda"))
+    assert y.shape == (0, n)
+    gain = torch.linspace(-1.5, 2.0, k)
+    bias = torch.linspace(-0.3, 0.4, n)
+    lin2 = mmf.TLinear(lin.packed, lin.gamma, n, k, gain=gain.cuda(), bias=bias.cuda())
+    olin2 = O.TLinear(olin.codes, olin.gamma, gain.numpy(), bias.numpy().astype(np.float64))
+    x = synth.activations(18, 7, k)
+    y = mmf.bitlinear(lin2, x.cuda())
+    assert_close(to_np(y), O.bitlinear(x.numpy(), olin2), "f32", "y with gain and bias")
+
+
+def test_bitlinear_zero_rows():
+    k, n = 128, 64
+    _, lin, _ = make_layer(19, n, k)
+    x = torch.zeros(5, k, device="cuda")
+    x[2] = 1.0
+    y, q, s, acc = mmf.bitlinear(lin, x, debug=True)
+    assert torch.all(y[[0, 1, 3, 4]] == 0) and torch.all(q[0] == 0)
+    assert torch.all(q[2] == 127)
+
+
+# ------------------------------------------------------------------ MLGRU scan
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("b,t,d", [(2, 64, 256), (1, 3, 16), (3, 200, 264), (8, 1, 1024), (4, 517, 2048)])
+def test_scan_parity(b, t, d, dtype):
+    pre = synth.preacts(400 + t, b, t, d, TORCH_DT[dtype], scale=2.0)
+    h0 = synth.activations(401, b, d)
+    h = h0.cuda().clone()
+    o = mmf.mlgru_scan(pre.cuda(), h)
+    p = to_np(pre)
+    o_ref, h_ref = O.mlgru_scan(p[:, :, 0], p[:, :, 1], p[:, :, 2], h0.numpy().astype(np.float64))
+    assert_close(to_np(o), O.store(o_ref, dtype), dtype, "o'")
+    assert_close(to_np(h), h_ref, "f32", "h_T")
+
+
+def test_scan_closed_forms_on_gpu():
+    b, t, d = 2, 10, 32
+    pre = synth.preacts(402, b, t, d)
+    pre[:, :, 0] = -1e4   # f = 0 -> h = c
+    h = torch.full((b, d), 7.0, device="cuda")
+    o = mmf.mlgru_scan(pre.cuda(), h)
+    c = O.silu(pre[:, :, 1].numpy().astype(np.float64))
+    g = O.sigmoid(pre[:, :, 2].numpy().astype(np.float64))
+    assert_close(to_np(o), g * c, "f32", "f=0")
+    pre[:, :, 0] = 1e4    # f = 1 -> h = h0
+    h = torch.full((b, d), 7.0, device="cuda")
+    o = mmf.mlgru_scan(pre.cuda(), h)
+    assert torch.all(h == 7.0)
+    assert_close(to_np(o), g * 7.0, "f32", "f=1")
+
+
+def test_scan_chunked_equals_whole():
+    b, t, d = 2, 96, 64
+    pre = synth.preacts(403, b, t, d).cuda()
+    h1 = torch.zeros(b, d, device="cuda")
+    o1 = mmf.mlgru_scan(pre, h1)
+    h2 = torch.zeros(b, d, device="cuda")
+    oa = mmf.mlgru_scan(pre[:, :40].contiguous(), h2)
+    ob = mmf.mlgru_scan(pre[:, 40:].contiguous(), h2)
+    torch.testing.assert_close(torch.cat([oa, ob], 1), o1, rtol=1e-6, atol=1e-6)
+    torch.testing.assert_close(h2, h1, rtol=1e-6, atol=1e-6)
+
+
+# ------------------------------------------------------------------ GLU
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("m,d,inner", [(128, 256, 768), (4, 2048, 5632), (9, 64, 48)])
+def test_glu_parity(m, d, inner, dtype):
+    _, gate, og = make_layer(500, inner, d)
+    _, up, ou = make_layer(501, inner, d)
+    _, down, od = make_layer(502, d, inner)
+    x = synth.activations(503, m, d, TORCH_DT[dtype])
+    res = synth.activations(504, m, d, TORCH_DT[dtype])
+    y = mmf.glu(gate, up, down, x.cuda(), residual=res.cuda())
+    blk = O.Block(og, og, og, og, og, ou, od)
+    y_ref, parts = O.glu(to_np(x), blk, dtype, parts=True)
+    assert_close(to_np(y), to_np(res) + y_ref, dtype, "glu y")
+
+
+# ------------------------------------------------------------------ blocks
+
+def test_tiny_block_fp32_parity():
+    w = synth.TINY_BLOCK
+    blk, oblk = make_block(w.seed, w.d, w.inner)
+    x = synth.activations(w.seed + synth.ACT_SEED_OFFSET, w.batch * w.seq, w.d).reshape(w.batch, w.seq, w.d)
+    st = mmf.State(1, w.batch, w.d)
+    y = mmf.block_forward(blk, 0, st, x.cuda())
+    h = st.get()[0]
+    y_ref, h_ref = O.block_forward(x.numpy(), oblk, np.zeros((w.batch, w.d)), "f32")
+    assert_close(to_np(y), y_ref, "f32", "block y")
+    assert_close(h.numpy(), h_ref, "f32", "block h_T")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_block_decode_steps_parity(dtype):
+    d, inner, B, T = 256, 768, 4, 6
+    blk, oblk = make_block(7001, d, inner)
+    x = synth.activations(7002, B * T, d, TORCH_DT[dtype]).reshape(B, T, d)
+    st = mmf.State(1, B, d)
+    ys = [mmf.block_forward(blk, 0, st, x[:, t:t + 1].contiguous().cuda()) for t in range(T)]
+    y = torch.cat(ys, 1)
+    h = np.zeros((B, d))
+    yr = []
+    for t in range(T):
+        yt, h = O.block_forward(to_np(x[:, t:t + 1]), oblk, h, dtype)
+        yr.append(yt)
+    assert_close(to_np(y), np.concatenate(yr, 1), dtype, "decode y")
+    assert_close(st.get()[0].numpy(), h, "f32", "decode h")
+
+
+def test_block_prefill_then_decode_matches_oracle_bf16():
+    d, inner, B, T = 256, 768, 2, 40
+    blk, oblk = make_block(7003, d, inner)
+    x = synth.activations(7004, B * (T + 3), d, torch.bfloat16).reshape(B, T + 3, d)
+    st = mmf.State(1, B, d)
+    y0 = mmf.block_forward(blk, 0, st, x[:, :T].contiguous().cuda())
+    y1 = [mmf.block_forward(blk, 0, st, x[:, T + i:T + i + 1].contiguous().cuda()) for i in range(3)]
+    y = torch.cat([y0] + y1, 1)
+    y_ref, h_ref = O.block_forward(to_np(x[:, :T]), oblk, np.zeros((B, d)), "bf16")
+    ys = [y_ref]
+    h = h_ref
+    for i in range(3):
+        yt, h = O.block_forward(to_np(x[:, T + i:T + i + 1]), oblk, h, "bf16")
+        ys.append(yt)
+    assert_close(to_np(y), np.concatenate(ys, 1), "bf16", "prefill+decode y")
+    assert_close(st.get()[0].numpy(), h, "f32", "prefill+decode h")
+
+
+def test_stack_forward_matches_block_loop():
+    d, inner, B, T, L = 128, 256, 2, 24, 3
+    pairs = [make_block(7100, d, inner, layer=l) for l in range(L)]
+    blocks = [p[0] for p in pairs]
+    x = synth.activations(7101, B * T, d, torch.bfloat16).reshape(B, T, d).cuda()
+    st1 = mmf.State(L, B, d)
+    y1 = mmf.stack_forward(blocks, st1, x)
+    st2 = mmf.State(L, B, d)
+    z = x
+    for l in range(L):
+        z = mmf.block_forward(blocks[l], l, st2, z)
+    assert torch.equal(y1, z)
+    assert torch.equal(st1.get(), st2.get())
+    y_ref, h_ref = O.stack_forward(to_np(x.cpu()), [p[1] for p in pairs], np.zeros((L, B, d)), "bf16")
+    assert_close(to_np(y1), y_ref, "bf16", "stack y")
+    assert_close(st1.get().numpy(), h_ref, "f32", "stack h")
