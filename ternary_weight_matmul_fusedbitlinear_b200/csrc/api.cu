@@ -124,6 +124,32 @@ cudaError_t timed(const char* name, cudaStream_t s, F&& launch) {
   return e;
 }
 
+// Contraction dispatch: the tcgen05 kernel for prefill-sized token counts, the
+// mma.sync kernel for decode-sized ones and for shapes the tcgen05 kernel does
+// not take. MMF_GEMM_PATH=mma|tc|auto (default auto) pins one implementation;
+// both compute the same exact integer accumulators.
+constexpr int kTcMinTokens = 128;
+
+int gemm_path_pref() {
+  const char* e = getenv("MMF_GEMM_PATH");
+  if (e == nullptr) return 0;
+  if (strcmp(e, "mma") == 0) return 1;
+  if (strcmp(e, "tc") == 0) return 2;
+  return 0;
+}
+
+cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s) {
+  const int pref = gemm_path_pref();
+  const bool tc_ok = tgemm_tc_supported(a, epi);
+  const bool use_tc = tc_ok && (pref == 2 || (pref == 0 && a.M >= kTcMinTokens));
+  if (use_tc) {
+    int* st = nullptr;
+    if (device_status_ptr(&st) != MMF_OK) return cudaErrorUnknown;
+    return timed("tgemm_tc", s, [&] { return launch_tgemm_tc(a, epi, dt, st, s); });
+  }
+  return timed("tgemm_mma", s, [&] { return launch_tgemm_mma(a, epi, dt, s); });
+}
+
 mmf_status check_tlinear(const mmf_tlinear* l, const char* name) {
   if (l == nullptr) return fail(MMF_ERR_INVALID_ARG, "%s: null layer", name);
   if (l->packed == nullptr || l->gamma == nullptr) return fail(MMF_ERR_INVALID_ARG, "%s: null packed/gamma", name);
@@ -262,14 +288,14 @@ extern "C" mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_d
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, lin->K, lin->gain, eps, qa.q, qa.s, qa.qsum, s); }), "rmsnorm_quant");
   const mmf_tlinear* segs[1] = {lin};
   TGemmArgs a = gemm_args(segs, 1, qa.q, qa.s, qa.qsum, M, y, lin->N, nullptr, nullptr);
-  MMF_CUDA(timed("tgemm_mma", s, [&] { return launch_tgemm_mma(a, Epi::kStore, dtype, s); }), "tgemm");
+  MMF_CUDA(run_gemm(a, Epi::kStore, dtype, s), "tgemm");
   if (dbg) {
     if (dbg->q) MMF_CUDA(cudaMemcpyAsync(dbg->q, qa.q, (size_t)M * lin->K, cudaMemcpyDeviceToDevice, s), "dbg q");
     if (dbg->scale)
       MMF_CUDA(cudaMemcpyAsync(dbg->scale, qa.s, sizeof(float) * M, cudaMemcpyDeviceToDevice, s), "dbg scale");
     if (dbg->acc) {
       TGemmArgs d = gemm_args(segs, 1, qa.q, qa.s, qa.qsum, M, dbg->acc, lin->N, nullptr, nullptr);
-      MMF_CUDA(timed("tgemm_mma", s, [&] { return launch_tgemm_mma(d, Epi::kAcc, dtype, s); }), "tgemm acc");
+      MMF_CUDA(run_gemm(d, Epi::kAcc, dtype, s), "tgemm acc");
     }
   }
   return MMF_OK;
@@ -286,7 +312,11 @@ extern "C" mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B
   if (!pre || !h || !o) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan: null pointer");
   if (!aligned16(pre) || !aligned16(h) || !aligned16(o)) return fail(MMF_ERR_MISALIGNED, "mmf_mlgru_scan");
   cudaStream_t s = as_stream(stream);
-  MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(pre, dtype, B, T, d, h, o, s); }), "mlgru_scan");
+  int* status = nullptr;
+  mmf_status r = device_status_ptr(&status);
+  if (r != MMF_OK) return r;
+  MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(pre, dtype, B, T, d, h, o, status, s); }),
+           "mlgru_scan");
   return MMF_OK;
 }
 
@@ -319,11 +349,11 @@ mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tli
                    cudaStream_t s) {
   const mmf_tlinear* gu[2] = {gate, up};
   TGemmArgs a = gemm_args(gu, 2, qx.q, qx.s, qx.qsum, M, p, gate->N, nullptr, nullptr);
-  MMF_CUDA(timed("tgemm_mma", s, [&] { return launch_tgemm_mma(a, Epi::kGlu, dt, s); }), "glu gate/up");
+  MMF_CUDA(run_gemm(a, Epi::kGlu, dt, s), "glu gate/up");
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(p, dt, M, down->K, down->gain, eps, qp.q, qp.s, qp.qsum, s); }), "glu quant p");
   const mmf_tlinear* dn[1] = {down};
   TGemmArgs b = gemm_args(dn, 1, qp.q, qp.s, qp.qsum, M, y, down->N, residual, nullptr);
-  MMF_CUDA(timed("tgemm_mma", s, [&] { return launch_tgemm_mma(b, Epi::kStore, dt, s); }), "glu down");
+  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s), "glu down");
   return MMF_OK;
 }
 
@@ -488,16 +518,20 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   if (T == 1) {
     // decode: projections and one recurrence step in one launch; h updated in place
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, h);
-    MMF_CUDA(timed("tgemm_mma", s, [&] { return launch_tgemm_mma(a, Epi::kScanStep, dt, s); }), "block fcg+step");
+    MMF_CUDA(run_gemm(a, Epi::kScanStep, dt, s), "block fcg+step");
   } else {
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.pre, 3 * d, nullptr, nullptr);
-    MMF_CUDA(timed("tgemm_mma", s, [&] { return launch_tgemm_mma(a, Epi::kStore, dt, s); }), "block fcg");
-    MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, s); }), "block scan");
+    MMF_CUDA(run_gemm(a, Epi::kStore, dt, s), "block fcg");
+    int* status = nullptr;
+    mmf_status r = device_status_ptr(&status);
+    if (r != MMF_OK) return r;
+    MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, status, s); }),
+             "block scan");
   }
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.og, dt, M, d, W.o.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant o'");
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
-  MMF_CUDA(timed("tgemm_mma", s, [&] { return launch_tgemm_mma(b, Epi::kStore, dt, s); }), "block o-proj");
+  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s), "block o-proj");
   // channel mixer
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.y1, dt, M, d, W.gate.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant y1");
   return run_glu(&W.gate, &W.up, &W.down, w.qa, w.y1, y, M, dt, eps, w.p, w.qa, s);

@@ -1,6 +1,8 @@
 // Internal launchers of the mmf CUDA library. Not part of the C ABI.
 #pragma once
 
+#include <cuda.h>
+
 #include <algorithm>
 
 #include "common.cuh"
@@ -8,6 +10,12 @@
 namespace mmf {
 
 constexpr int kQuantPartials = 592;   // CTAs of the absmean partial-sum pass (4 x 148 SMs)
+
+// TMA tensor maps (host): a 2-D row-major [rows, cols] array of esize-byte elements.
+bool tma_available();
+bool make_tma_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
+                 uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
+int num_sms();
 
 size_t quantize_weights_ws_bytes();
 cudaError_t launch_quantize_weights(const float* W, int N, int K, uint32_t* packed, float* gamma, void* ws,
@@ -44,7 +52,12 @@ struct TGemmArgs {
 // mma.sync-based contraction (weights as the 16-row A operand, tokens as N=8 tiles).
 cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t stream);
 
-cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o,
+// tcgen05 (TMEM) contraction for prefill-sized token counts. Needs K % 64 == 0
+// and N % 128 == 0; `status` is the device status word for bounded-wait timeouts.
+bool tgemm_tc_supported(const TGemmArgs& a, Epi epi);
+cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
+
+cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, int* status,
                               cudaStream_t stream);
 
 }  // namespace mmf

@@ -1,0 +1,416 @@
+// Prefill ternary contraction on the 5th-generation tensor cores (tcgen05,
+// kind::i8, accumulators in tensor memory).
+//
+// "MatMul-free language models" (DataCamp blog), section "Replacing MatMul
+// with ternary operations": with weights in {-1,0,1} the contraction is exact
+// integer add/subtract work, so an int8 x int8 -> int32 tensor-core product of
+// the activation codes with the ternary codes gives the exact accumulators.
+// The stored weight code is w + 1 (unsigned byte 0..2); the kernel computes
+// sum_k q[m,k] (w[n,k] + 1) with an s8 x u8 MMA and the epilogue subtracts the
+// token's code sum: acc = raw - sum_k q[m,k].
+//
+// Tile: 128 tokens (M) x 256 output columns (N) x 128 k-bytes per stage.
+// Persistent CTAs (one per SM), warp-specialised:
+//   warp 0      TMA producer: int8 activation tile (128B-swizzled, the UMMA
+//               K-major SW128 layout) and the 2-bit packed weight tile
+//   warp 1      TMEM owner + single-thread MMA issuer (4 x K=32 per stage)
+//   warps 2..5  epilogue: tcgen05.ld of the int32 accumulators, rescale
+//               (+bias, +residual, SiLU*up), store
+//   warps 6..9  unpack: packed 2-bit codes -> int8 bytes in shared memory,
+//               written directly in the SW128 K-major layout the MMA reads
+// Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile overlap
+// the main loop of the next. Every mbarrier wait is bounded: on timeout the
+// kernel records an error in the status word, raises a CTA-wide abort flag,
+// and all roles leave their loops; nothing traps.
+#include "kernels.cuh"
+#include "tma.cuh"
+
+namespace mmf {
+
+namespace {
+
+constexpr int BM = 128, BN = 256, BK = 128, STAGES = 3;
+constexpr int A_BYTES = BM * BK;          // 16 KiB int8 activations
+constexpr int BP_BYTES = BN * BK / 4;     // 8 KiB packed codes (2 bit)
+constexpr int BU_BYTES = BN * BK;         // 32 KiB unpacked codes (int8)
+constexpr int HALF = BN / 2;              // rows per weight TMA box
+constexpr int kThreads = 320;             // 10 warps
+constexpr int kEpiWarp0 = 2, kUnpackWarp0 = 6;
+constexpr int kUnpackThreads = 128;
+constexpr uint32_t kTmemCols = 512;
+
+struct __align__(1024) SmemLayout {
+  uint8_t a[STAGES][A_BYTES];
+  uint8_t bu[STAGES][BU_BYTES];
+  uint32_t bp[STAGES][BP_BYTES / 4];
+  uint64_t full_tma[STAGES];
+  uint64_t full_bu[STAGES];
+  uint64_t empty[STAGES];
+  uint64_t tmem_full[2];
+  uint64_t tmem_empty[2];
+  uint64_t mma_drain;
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// UMMA shared-memory descriptor: K-major, 128-byte swizzle, 8-row groups 1024 B apart.
+__device__ __forceinline__ uint64_t umma_desc_sw128(uint32_t saddr) {
+  uint64_t d = 0;
+  d |= (uint64_t)((saddr & 0x3FFFFu) >> 4);   // start address
+  d |= (uint64_t)1 << 16;                       // leading byte offset (unused for swizzled K-major)
+  d |= (uint64_t)(1024 >> 4) << 32;             // stride byte offset: next 8-row group
+  d |= (uint64_t)1 << 46;                       // descriptor version (sm_100)
+  d |= (uint64_t)2 << 61;                       // layout: SWIZZLE_128B
+  return d;
+}
+
+// Instruction descriptor: kind::i8, D s32, A s8 (activations), B u8 (codes w+1),
+// both K-major, M = 128, N = 256.
+constexpr uint32_t kIdesc = (2u << 4)            // D format s32
+                            | (1u << 7)          // A format s8
+                            | (0u << 10)         // B format u8
+                            | ((uint32_t)(BN >> 3) << 17) | ((uint32_t)(BM >> 4) << 24);
+
+__device__ __forceinline__ void umma_i8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t accum) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n"
+      " tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(kIdesc), "r"(accum)
+      : "memory");
+}
+__device__ __forceinline__ void umma_commit(uint64_t* bar) {
+  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+      "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+  asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- tile geometry
+struct TcArgs {
+  TGemmArgs g;
+  int m_tiles, n_tiles;
+  int* status;
+};
+
+// Rows of weight segment `seg` starting at `row0` feed half `h` of tile `nt`.
+__device__ __forceinline__ void half_source(const TcArgs& p, Epi epi, int nt, int h, int& seg, int& row0) {
+  if (epi == Epi::kGlu) {
+    seg = h;
+    row0 = nt * HALF;
+  } else {
+    const int gcol = nt * BN + h * HALF;
+    const int total = p.g.nseg * p.g.N;
+    if (gcol >= total) {   // past the last segment: a fully out-of-bounds box reads zeros
+      seg = p.g.nseg - 1;
+      row0 = p.g.N;
+    } else {
+      seg = gcol / p.g.N;
+      row0 = gcol % p.g.N;
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void store32(T* dst, const float (&v)[32]);
+template <>
+__device__ __forceinline__ void store32<bf16>(bf16* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) store8(dst + 8 * q, v + 8 * q);
+}
+template <>
+__device__ __forceinline__ void store32<float>(float* dst, const float (&v)[32]) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) store8(dst + 8 * q, v + 8 * q);
+}
+
+template <Epi EPI, typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    tgemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
+                    const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_b2,
+                    const TcArgs p) {
+  extern __shared__ uint8_t smem_raw[];
+  SmemLayout& sm = *reinterpret_cast<SmemLayout*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  volatile int* abort_flag = &sm.abort_flag;
+  const int n_tiles_total = p.m_tiles * p.n_tiles;
+  const int nk = ceil_div(p.g.K, BK);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(&sm.full_tma[s], 1);
+      mbar_init(&sm.full_bu[s], kUnpackThreads);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&sm.tmem_full[a], 1);
+      mbar_init(&sm.tmem_empty[a], 128);
+    }
+    mbar_init(&sm.mma_drain, 1);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = sm.tmem_base;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const CUtensorMap* maps[3] = {&map_b0, &map_b1, &map_b2};
+      uint32_t it = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
+        const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+        int seg0, row0, seg1, row1;
+        half_source(p, EPI, nt, 0, seg0, row0);
+        half_source(p, EPI, nt, 1, seg1, row1);
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&sm.empty[s], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&sm.full_tma[s], A_BYTES + BP_BYTES);
+          tma_load_2d(sm.a[s], &map_a, kb * BK, mt * BM, &sm.full_tma[s]);
+          tma_load_2d(&sm.bp[s][0], maps[seg0], kb * (BK / 16), row0, &sm.full_tma[s]);
+          tma_load_2d(&sm.bp[s][HALF * (BK / 16)], maps[seg1], kb * (BK / 16), row1, &sm.full_tma[s]);
+        }
+      }
+      // let every copy this thread issued land before the CTA can exit
+      for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
+        mbar_wait(&sm.full_tma[j % STAGES], (j / STAGES) & 1, abort_flag, nullptr);
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      uint32_t it = 0, tl = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++tl) {
+        const int acc = tl & 1;
+        const uint32_t acc_ph = (tl >> 1) & 1;
+        if (!mbar_wait(&sm.tmem_empty[acc], acc_ph ^ 1, abort_flag, p.status)) break;
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * BN;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = it % STAGES;
+          const uint32_t ph = (it / STAGES) & 1;
+          if (!mbar_wait(&sm.full_bu[s], ph, abort_flag, p.status)) { ok = false; break; }
+          tc_fence_after();
+          const uint64_t adesc = umma_desc_sw128(smem_u32(sm.a[s]));
+          const uint64_t bdesc = umma_desc_sw128(smem_u32(sm.bu[s]));
+#pragma unroll
+          for (int j = 0; j < BK / 32; ++j)   // advance 32 bytes of K inside the swizzle atom
+            umma_i8(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), (kb | j) != 0);
+          umma_commit(&sm.empty[s]);
+        }
+        if (ok) umma_commit(&sm.tmem_full[acc]);
+      }
+      // every MMA this thread issued has finished before TMEM can be released
+      umma_commit(&sm.mma_drain);
+      mbar_wait(&sm.mma_drain, 0, abort_flag, nullptr);
+    }
+  } else if (warp >= kUnpackWarp0) {
+    // ------------------------------------------------------------ unpack 2-bit codes to int8
+    const int u = threadIdx.x - kUnpackWarp0 * 32;   // 0..127: rows u and u + 128
+    uint32_t it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        const int s = it % STAGES;
+        const uint32_t ph = (it / STAGES) & 1;
+        if (!mbar_wait(&sm.full_tma[s], ph, abort_flag, p.status)) { ok = false; break; }
+#pragma unroll
+        for (int rr = 0; rr < 2; ++rr) {
+          const int n = u + rr * HALF;
+          const uint4* src = reinterpret_cast<const uint4*>(&sm.bp[s][n * (BK / 16)]);
+          uint8_t* dst = sm.bu[s] + n * BK;
+#pragma unroll
+          for (int hq = 0; hq < 2; ++hq) {
+            const uint4 w4 = src[hq];
+            const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const int c = hq * 4 + e;     // 16-column chunk of this row
+              const uint32_t w = ws[e];
+              uint4 v;
+              v.x = w & 0x03030303u;
+              v.y = (w >> 2) & 0x03030303u;
+              v.z = (w >> 4) & 0x03030303u;
+              v.w = (w >> 6) & 0x03030303u;
+              *reinterpret_cast<uint4*>(dst + ((c ^ (n & 7)) << 4)) = v;
+            }
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(&sm.full_bu[s]);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ epilogue (warps 2..5)
+    const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int row_in_tile = quarter * 32 + lane;
+    uint32_t tl = 0;
+    for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++tl) {
+      const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
+      const int acc = tl & 1;
+      const uint32_t acc_ph = (tl >> 1) & 1;
+      const bool got = mbar_wait(&sm.tmem_full[acc], acc_ph, abort_flag, p.status);
+      __syncwarp();                               // tcgen05.ld below is warp-collective
+      if (!__all_sync(0xffffffffu, got)) break;
+      tc_fence_after();
+      const int m = mt * BM + row_in_tile;
+      const bool row_ok = m < p.g.M;
+      const float inv_s = row_ok ? 1.0f / p.g.s[m] : 0.0f;
+      const int qs = row_ok ? p.g.qsum[m] : 0;
+      const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
+      if constexpr (EPI == Epi::kGlu) {
+        const float sc_u = *p.g.gamma[0] * inv_s, sc_v = *p.g.gamma[1] * inv_s;
+        for (int c = 0; c < HALF / 32; ++c) {
+          uint32_t ru[32], rv[32];
+          tmem_ld32(tbase + 32 * c, ru);
+          tmem_ld32(tbase + HALF + 32 * c, rv);
+          const int n0 = nt * HALF + 32 * c;
+          if (row_ok) {
+            float out[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              float uu = (float)((int)ru[j] - qs) * sc_u;
+              float vv = (float)((int)rv[j] - qs) * sc_v;
+              if (p.g.bias[0] != nullptr) uu += p.g.bias[0][n0 + j];
+              if (p.g.bias[1] != nullptr) vv += p.g.bias[1][n0 + j];
+              out[j] = siluf_(uu) * vv;
+            }
+            store32<T>(static_cast<T*>(p.g.out) + (size_t)m * p.g.ldo + n0, out);
+          }
+        }
+      } else {
+        for (int h = 0; h < 2; ++h) {
+          int seg, row0;
+          half_source(p, EPI, nt, h, seg, row0);
+          if (nt * BN + h * HALF >= p.g.nseg * p.g.N) break;
+          const float sc = *p.g.gamma[seg] * inv_s;
+          const float* bias = p.g.bias[seg];
+          for (int c = 0; c < HALF / 32; ++c) {
+            uint32_t r[32];
+            tmem_ld32(tbase + h * HALF + 32 * c, r);
+            const int n0 = row0 + 32 * c;
+            if (!row_ok) continue;
+            if constexpr (EPI == Epi::kAcc) {
+              int32_t* dst = static_cast<int32_t*>(p.g.out) + (size_t)m * p.g.ldo + seg * p.g.N + n0;
+#pragma unroll
+              for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<int4*>(dst + j) =
+                    make_int4((int)r[j] - qs, (int)r[j + 1] - qs, (int)r[j + 2] - qs, (int)r[j + 3] - qs);
+            } else {
+              float out[32];
+#pragma unroll
+              for (int j = 0; j < 32; ++j) {
+                float v = (float)((int)r[j] - qs) * sc;
+                if (bias != nullptr) v += bias[n0 + j];
+                out[j] = v;
+              }
+              if (p.g.residual != nullptr) {
+                const T* res = static_cast<const T*>(p.g.residual) + (size_t)m * p.g.N + n0;
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                  float rv[8];
+                  load8(res + 8 * q, rv);
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) out[8 * q + j] += rv[j];
+                }
+              }
+              store32<T>(static_cast<T*>(p.g.out) + (size_t)m * p.g.ldo + seg * p.g.N + n0, out);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&sm.tmem_empty[acc]);
+    }
+  }
+
+  // ------------------------------------------------------------ teardown
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    __syncwarp();
+    tc_fence_after();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem_base), "r"(kTmemCols)
+                 : "memory");
+  }
+}
+
+// ---------------------------------------------------------------- host side
+template <Epi EPI, typename T>
+cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap (&mb)[3], const TcArgs& p, cudaStream_t stream) {
+  const size_t smem = sizeof(SmemLayout) + 1024;
+  auto kern = tgemm_tc_kernel<EPI, T>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int tiles = p.m_tiles * p.n_tiles;
+  const int grid = std::min(tiles, num_sms());
+  kern<<<grid, kThreads, smem, stream>>>(ma, mb[0], mb[1], mb[2], p);
+  return cudaGetLastError();
+}
+
+}  // namespace
+
+bool tgemm_tc_supported(const TGemmArgs& a, Epi epi) {
+  if (epi != Epi::kStore && epi != Epi::kAcc && epi != Epi::kGlu) return false;
+  if (a.K % 64 != 0 || a.N % HALF != 0) return false;   // 16-byte TMA row strides, whole 128-row halves
+  if (epi == Epi::kGlu && a.nseg != 2) return false;
+  if (a.residual != nullptr && a.nseg != 1) return false;
+  return tma_available();
+}
+
+cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream) {
+  if (a.M == 0) return cudaSuccess;
+  if (!tgemm_tc_supported(a, epi)) return cudaErrorNotSupported;
+  CUtensorMap ma, mb[3];
+  if (!make_tma_2d(&ma, a.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.K, (uint64_t)a.M, BK, BM,
+                CU_TENSOR_MAP_SWIZZLE_128B))
+    return cudaErrorInvalidValue;
+  for (int r = 0; r < 3; ++r) {
+    const int src = r < a.nseg ? r : 0;
+    if (!make_tma_2d(&mb[r], a.w[src], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(a.K / 16), (uint64_t)a.N, BK / 16,
+                  HALF, CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+  }
+  TcArgs p;
+  p.g = a;
+  p.status = status;
+  p.m_tiles = ceil_div(a.M, BM);
+  p.n_tiles = (epi == Epi::kGlu) ? ceil_div(a.N, HALF) : ceil_div(a.nseg * a.N, BN);
+  const bool b = dt == MMF_BF16;
+  switch (epi) {
+    case Epi::kStore:
+      return b ? launch_typed<Epi::kStore, bf16>(ma, mb, p, stream) : launch_typed<Epi::kStore, float>(ma, mb, p, stream);
+    case Epi::kAcc:
+      return b ? launch_typed<Epi::kAcc, bf16>(ma, mb, p, stream) : launch_typed<Epi::kAcc, float>(ma, mb, p, stream);
+    case Epi::kGlu:
+      return b ? launch_typed<Epi::kGlu, bf16>(ma, mb, p, stream) : launch_typed<Epi::kGlu, float>(ma, mb, p, stream);
+    default:
+      return cudaErrorNotSupported;
+  }
+}
+
+}  // namespace mmf

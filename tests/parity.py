@@ -7,8 +7,13 @@ import torch
 import oracle as O
 import synth
 
-# Floating outputs: normwise max relative error 2e-3 (bf16 I/O, fp32 accumulate).
+# Floating outputs: normwise max relative error 2e-3 (bf16 I/O, fp32 accumulate)
+# for every stage fed the oracle's own inputs (teacher forcing).
 TOL = 2e-3
+# Composite paths (a whole block, a stack, decode loops) are not teacher-forced:
+# one activation code that legitimately lands on the other side of a rounding tie
+# in an inner stage moves a few outputs by ~1/|acc|, so they gate at 1e-2.
+E2E_TOL = 1e-2
 # Elements next to a rounding boundary of the storage type may land one or two
 # units in the last place apart (fp32 vs fp64 evaluation before the rounding,
 # or an upstream stored value that flipped); at most this fraction of them.
