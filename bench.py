@@ -51,7 +51,9 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["mmf", "reference"], default="mmf")
-    ap.add_argument("--workload", choices=["stack370m"], default="stack370m")
+    ap.add_argument("--workload", choices=["stack370m", "bitlinear"], default="stack370m",
+                    help="stack370m: the 370M-shaped 24-block prefill (default); bitlinear: one prefill "
+                         "BitLinear of the 370M gate|up shape (16384 tokens, 1024 -> 5632)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) pass")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     return ap.parse_args(argv)
@@ -360,12 +362,69 @@ def run_mmf(args):
     return 0
 
 
+def run_bitlinear(args):
+    """One prefill BitLinear per step: 16384 tokens x (1024 -> 5632), bf16 (the 370M GLU gate|up shape)."""
+    world, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dist_init(world)
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    dev = torch.device("cuda", local)
+    M, K, N = 16384, 1024, 5632
+    peaks, peak_kind = load_peaks()
+    lin = mmf.quantize_weights(synth.latent_weight(synth.sub_seed(1002, 0, synth.PROJ_GATE), N, K, device=dev))
+    x = synth.activations(1002 + rank, M, K, torch.bfloat16, device=dev)
+    y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(mmf.api.L.load().mmf_bitlinear_ws_size(M, K), dtype=torch.uint8, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    for _ in range(args.warmup):
+        mmf.bitlinear(lin, x, ws=ws)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    for i in range(args.steps):
+        flush.zero_()
+        starts[i].record(stream)
+        y = mmf.bitlinear(lin, x, ws=ws)
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    mmf.prof_enable(False)
+    prof = mmf.prof_collect()
+    total_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(starts, ends)), world)
+    gemm = [k for k in prof if k.startswith("tgemm")]
+    gemm_ms = sum(prof[k][1] for k in gemm)
+    ops = 2.0 * M * N * K
+    achieved = ops * args.steps / (gemm_ms / 1e3) / 1e12
+    peak = peaks["bf16_tflops"] * INT8_OVER_BF16
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": world * M * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"bitlinear_prefill_m{M}_k{K}_n{N}_bf16", "l2": "flushed between timed steps"},
+            "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": ",".join(gemm),
+                         "peak_source": f"{peak_kind}: bf16 burst x {INT8_OVER_BF16}",
+                         "per_kernel_ms": {k: round(v[1] / args.steps, 4) for k, v in prof.items()}},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": int(sum(v[0] for v in prof.values())),
+            "clocks": clk}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
     if args.impl == "reference":
         return run_reference(args)
+    if args.workload == "bitlinear":
+        return run_bitlinear(args)
     return run_mmf(args)
 
 
