@@ -237,6 +237,35 @@ mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t L, mmf_stat
                              float eps, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
+/* FusedBitLinear without a workspace                                         */
+/* ------------------------------------------------------------------------- */
+
+/* Bytes of the fixed device array mmf_bitlinear_noalloc uses as scratch. */
+#define MMF_NOALLOC_SCRATCH_BYTES (2u * 1024u * 1024u)
+
+/* The same computation as mmf_bitlinear (y = BitLinear(x), x [M, K] -> y [M, N]),
+ * for callers that can neither allocate device memory nor pass a workspace:
+ * a custom-operator plug-in that is handed only its input and output buffers,
+ * or a process that reserved its whole device-memory budget up front. The
+ * paper has no counterpart to this call; it is a property of this library.
+ *
+ * Scratch (the int8 activation codes, scales and row sums) lives in one fixed
+ * array of MMF_NOALLOC_SCRATCH_BYTES that the library image places in device
+ * memory on every GPU that loads it and keeps until the process exits. The
+ * call never calls cudaMalloc, cudaFree or any allocating routine. Its size
+ * limit: round_up(M*K, 256) + 2 * round_up(4*M, 256) <= MMF_NOALLOC_SCRATCH_BYTES
+ * (for example M = 64 tokens of K = 16384, or M = 512 of K = 4096); larger calls
+ * return MMF_ERR_UNSUPPORTED_SHAPE with a message naming the limit.
+ * The first call on a device looks up the array's device address (a one-time
+ * set-up with that device current); make that first call before any stream
+ * capture. Every call shares the array and it keeps the last call's contents
+ * (each call overwrites everything it reads, so nothing needs clearing); calls
+ * that overlap on the GPU race on it and must be serialised by the caller.
+ * Arguments, layouts and the other errors are those of mmf_bitlinear. */
+mmf_status mmf_bitlinear_noalloc(const mmf_tlinear* lin, const void* x, mmf_dtype dtype, int32_t M,
+                                 void* y, float eps, void* stream);
+
+/* ------------------------------------------------------------------------- */
 /* Kernel timing (tracing)                                                    */
 /* ------------------------------------------------------------------------- */
 

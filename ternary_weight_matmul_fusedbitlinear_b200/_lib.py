@@ -60,6 +60,7 @@ SIGNATURES = {
                                          c_vp]),
     "mmf_stack_forward": (ctypes.c_int, [ctypes.POINTER(c_vp), c_i32, c_vp, c_vp, c_vp, c_i32, c_i32, ctypes.c_int,
                                          c_f, c_vp, c_sz, c_vp]),
+    "mmf_bitlinear_noalloc": (ctypes.c_int, [ctypes.POINTER(TLinear), c_vp, ctypes.c_int, c_i32, c_vp, c_f, c_vp]),
     "mmf_prof_enable": (ctypes.c_int, [c_i32]),
     "mmf_prof_collect": (c_i32, []),
     "mmf_prof_get": (ctypes.c_int, [c_i32, ctypes.c_char_p, c_sz, ctypes.POINTER(ctypes.c_int64),

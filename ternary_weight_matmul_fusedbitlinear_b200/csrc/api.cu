@@ -201,6 +201,8 @@ QAct carve_qact(Carver& c, int M, int K) {
 
 }  // namespace
 
+void mmf::set_last_error(const char* msg) { g_last_error = msg; }
+
 // ------------------------------------------------------------------ handles
 
 struct mmf_block {

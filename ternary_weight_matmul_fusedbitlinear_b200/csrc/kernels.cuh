@@ -17,6 +17,9 @@ bool make_tma_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int
                  uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 int num_sms();
 
+// Message returned by mmf_last_error() on this host thread.
+void set_last_error(const char* msg);
+
 size_t quantize_weights_ws_bytes();
 cudaError_t launch_quantize_weights(const float* W, int N, int K, uint32_t* packed, float* gamma, void* ws,
                                     cudaStream_t stream);
