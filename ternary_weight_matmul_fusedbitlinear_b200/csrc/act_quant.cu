@@ -105,11 +105,148 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_quant_kernel(const T* __rest
   }
 }
 
+// One warp per token row, the row held in registers as raw 16-byte vectors
+// (8 elements each): lane l owns vectors j*32 + l, j < VMAX, so every load and
+// every code store of the warp is one contiguous span. Same fp32 steps as the
+// CTA-per-row kernel; reductions are warp shuffles only.
+template <typename T>
+struct Vec16;
+template <>
+struct Vec16<bf16> {
+  using raw = uint4;   // 8 bf16
+  static constexpr int regs = 1;
+};
+template <>
+struct Vec16<float> {
+  using raw = uint4;   // 4 floats; two raws per 8 elements
+  static constexpr int regs = 2;
+};
+
+__device__ __forceinline__ void unpack8(const uint4 (&r)[1], float (&v)[8]) {
+  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r[0]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    float2 f = __bfloat1622float2(h[i]);
+    v[2 * i] = f.x;
+    v[2 * i + 1] = f.y;
+  }
+}
+__device__ __forceinline__ void unpack8(const uint4 (&r)[2], float (&v)[8]) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    v[4 * i + 0] = __uint_as_float(r[i].x);
+    v[4 * i + 1] = __uint_as_float(r[i].y);
+    v[4 * i + 2] = __uint_as_float(r[i].z);
+    v[4 * i + 3] = __uint_as_float(r[i].w);
+  }
+}
+
+template <typename T, int VMAX>
+__global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(const T* __restrict__ x, int M, int K,
+                                                                 const float* __restrict__ gain, float eps,
+                                                                 int8_t* __restrict__ q, float* __restrict__ scale,
+                                                                 int32_t* __restrict__ qsum) {
+  constexpr int R = Vec16<T>::regs;
+  const int lane = threadIdx.x & 31;
+  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  if (row >= M) return;
+  const int nvec = K / 8;
+  const T* xr = x + (size_t)row * K;
+  uint4 raw[VMAX][R];
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) {
+    const int vi = j * 32 + lane;
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+      raw[j][r] = vi < nvec ? __ldg(reinterpret_cast<const uint4*>(xr + (size_t)vi * 8) + r) : make_uint4(0, 0, 0, 0);
+  }
+  double ss = 0.0;
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) {
+    float v[8];
+    unpack8(raw[j], v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ss += (double)v[i] * (double)v[i];
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float ms = (float)(ss / (double)K);
+  const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
+
+  float amax = 0.0f;
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) {
+    const int vi = j * 32 + lane;
+    if (vi >= nvec) break;
+    float v[8];
+    unpack8(raw[j], v);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float h = __fmul_rn(v[i], rinv);
+      if (gain != nullptr) h = __fmul_rn(h, __ldg(gain + vi * 8 + i));
+      amax = fmaxf(amax, fabsf(h));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+
+  int isum = 0;
+  int8_t* qr = q + (size_t)row * K;
+#pragma unroll
+  for (int j = 0; j < VMAX; ++j) {
+    const int vi = j * 32 + lane;
+    if (vi >= nvec) break;
+    float v[8];
+    unpack8(raw[j], v);
+    uint32_t w[2] = {0u, 0u};
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float h = __fmul_rn(v[i], rinv);
+      if (gain != nullptr) h = __fmul_rn(h, __ldg(gain + vi * 8 + i));
+      int c = __float2int_rn(__fmul_rn(h, s));
+      c = max(-128, min(127, c));
+      isum += c;
+      w[i >> 2] |= (uint32_t)(c & 0xff) << (8 * (i & 3));
+    }
+    *reinterpret_cast<uint2*>(qr + (size_t)vi * 8) = make_uint2(w[0], w[1]);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+  if (lane == 0) {
+    scale[row] = s;
+    qsum[row] = isum;
+  }
+}
+
+template <typename T, int VMAX>
+void launch_warp(const void* x, int M, int K, const float* gain, float eps, int8_t* q, float* scale, int32_t* qsum,
+                 cudaStream_t stream) {
+  rmsnorm_quant_warp_kernel<T, VMAX><<<ceil_div(M, 8), 256, 0, stream>>>(static_cast<const T*>(x), M, K, gain, eps, q,
+                                                                          scale, qsum);
+}
+
 }  // namespace
 
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
                                  int8_t* q, float* scale, int32_t* qsum, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
+  // warp-per-row kernels while the row fits in registers (K / 256 vectors per lane)
+  const int vpl = ceil_div(K / 8, 32);
+  if (dt == MMF_BF16 && vpl <= 28) {
+    if (vpl <= 4) launch_warp<bf16, 4>(x, M, K, gain, eps, q, scale, qsum, stream);
+    else if (vpl <= 8) launch_warp<bf16, 8>(x, M, K, gain, eps, q, scale, qsum, stream);
+    else if (vpl <= 12) launch_warp<bf16, 12>(x, M, K, gain, eps, q, scale, qsum, stream);
+    else if (vpl <= 22) launch_warp<bf16, 22>(x, M, K, gain, eps, q, scale, qsum, stream);
+    else launch_warp<bf16, 28>(x, M, K, gain, eps, q, scale, qsum, stream);
+    return cudaGetLastError();
+  }
+  if (dt == MMF_F32 && vpl <= 12) {
+    if (vpl <= 4) launch_warp<float, 4>(x, M, K, gain, eps, q, scale, qsum, stream);
+    else if (vpl <= 8) launch_warp<float, 8>(x, M, K, gain, eps, q, scale, qsum, stream);
+    else launch_warp<float, 12>(x, M, K, gain, eps, q, scale, qsum, stream);
+    return cudaGetLastError();
+  }
   const size_t smem = sizeof(float) * (size_t)K;
   if (dt == MMF_BF16) {
     auto kern = rmsnorm_quant_kernel<bf16>;

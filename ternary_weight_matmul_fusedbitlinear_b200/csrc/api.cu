@@ -138,16 +138,19 @@ int gemm_path_pref() {
   return 0;
 }
 
-cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s) {
+// `what` names the projection for the launch-timing totals ("fcg", "o", ...).
+cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s, const char* what = "") {
   const int pref = gemm_path_pref();
   const bool tc_ok = tgemm_tc_supported(a, epi);
   const bool use_tc = tc_ok && (pref == 2 || (pref == 0 && a.M >= kTcMinTokens));
+  char name[48];
+  snprintf(name, sizeof(name), "%s%s%s", use_tc ? "tgemm_tc" : "tgemm_mma", what[0] ? ":" : "", what);
   if (use_tc) {
     int* st = nullptr;
     if (device_status_ptr(&st) != MMF_OK) return cudaErrorUnknown;
-    return timed("tgemm_tc", s, [&] { return launch_tgemm_tc(a, epi, dt, st, s); });
+    return timed(name, s, [&] { return launch_tgemm_tc(a, epi, dt, st, s); });
   }
-  return timed("tgemm_mma", s, [&] { return launch_tgemm_mma(a, epi, dt, s); });
+  return timed(name, s, [&] { return launch_tgemm_mma(a, epi, dt, s); });
 }
 
 mmf_status check_tlinear(const mmf_tlinear* l, const char* name) {
@@ -351,11 +354,11 @@ mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tli
                    cudaStream_t s) {
   const mmf_tlinear* gu[2] = {gate, up};
   TGemmArgs a = gemm_args(gu, 2, qx.q, qx.s, qx.qsum, M, p, gate->N, nullptr, nullptr);
-  MMF_CUDA(run_gemm(a, Epi::kGlu, dt, s), "glu gate/up");
+  MMF_CUDA(run_gemm(a, Epi::kGlu, dt, s, "gate_up"), "glu gate/up");
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(p, dt, M, down->K, down->gain, eps, qp.q, qp.s, qp.qsum, s); }), "glu quant p");
   const mmf_tlinear* dn[1] = {down};
   TGemmArgs b = gemm_args(dn, 1, qp.q, qp.s, qp.qsum, M, y, down->N, residual, nullptr);
-  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s), "glu down");
+  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s, "down"), "glu down");
   return MMF_OK;
 }
 
@@ -520,10 +523,10 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   if (T == 1) {
     // decode: projections and one recurrence step in one launch; h updated in place
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, h);
-    MMF_CUDA(run_gemm(a, Epi::kScanStep, dt, s), "block fcg+step");
+    MMF_CUDA(run_gemm(a, Epi::kScanStep, dt, s, "fcg_step"), "block fcg+step");
   } else {
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.pre, 3 * d, nullptr, nullptr);
-    MMF_CUDA(run_gemm(a, Epi::kStore, dt, s), "block fcg");
+    MMF_CUDA(run_gemm(a, Epi::kStore, dt, s, "fcg"), "block fcg");
     int* status = nullptr;
     mmf_status r = device_status_ptr(&status);
     if (r != MMF_OK) return r;
@@ -533,7 +536,7 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.og, dt, M, d, W.o.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant o'");
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
-  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s), "block o-proj");
+  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s, "o"), "block o-proj");
   // channel mixer
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.y1, dt, M, d, W.gate.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant y1");
   return run_glu(&W.gate, &W.up, &W.down, w.qa, w.y1, y, M, dt, eps, w.p, w.qa, s);

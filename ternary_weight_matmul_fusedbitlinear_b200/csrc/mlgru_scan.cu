@@ -19,6 +19,12 @@
 // one map, publishes it, folds the maps of warps 0..s-1 into the tile's carry
 // to get its starting state, then replays its 8 steps to produce o'. The carry
 // out of the last warp seeds the next tile.
+//
+// Gates: the three logistic functions of a step share one reciprocal. With
+// e_i = exp(-z_i) and D = (1+e_f)(1+e_c)(1+e_g), 1/(1+e_f) = (1+e_c)(1+e_g)/D
+// and so on; the arguments are clamped to [-20, 20] first so D stays finite
+// (sigmoid(20) rounds to 1 in fp32 and sigmoid(-20) = 2.1e-9 is below the
+// output tolerance), which takes 3 exponentials and 1 reciprocal per step.
 #include "kernels.cuh"
 #include "tma.cuh"
 
@@ -33,7 +39,18 @@ constexpr int LS = TC / SW;     // steps per warp per tile
 constexpr int STAGES = 3;
 constexpr int kThreads = SW * 32;
 
-__device__ __forceinline__ float sigmoid_fast(float z) { return __fdividef(1.0f, 1.0f + __expf(-z)); }
+// sigmoid of three arguments with one reciprocal (see the file comment)
+__device__ __forceinline__ void sigmoid3(float zf, float zc, float zg, float& sf, float& sc, float& sg) {
+  const float af = 1.0f + __expf(-fminf(fmaxf(zf, -20.0f), 20.0f));
+  const float ac = 1.0f + __expf(-fminf(fmaxf(zc, -20.0f), 20.0f));
+  const float ag = 1.0f + __expf(-fminf(fmaxf(zg, -20.0f), 20.0f));
+  const float fc = af * ac;
+  const float r = __fdividef(1.0f, fc * ag);
+  sg = r * fc;
+  const float rg = r * ag;
+  sf = rg * ac;
+  sc = rg * af;
+}
 
 template <typename T>
 struct ScanSmem {
@@ -86,12 +103,12 @@ __global__ void __launch_bounds__(kThreads) mlgru_scan_kernel(const __grid_const
     for (int j = 0; j < LS; ++j) {
       const int tl = warp * LS + j;
       if (t0 + j < T_) {
-        const float fv = sigmoid_fast(to_f32(sm.tile[s][0][tl][lane]));
         const float cz = to_f32(sm.tile[s][1][tl][lane]);
-        const float cv = cz * sigmoid_fast(cz);
-        gg[j] = sigmoid_fast(to_f32(sm.tile[s][2][tl][lane]));
+        float fv, sc, gv;
+        sigmoid3(to_f32(sm.tile[s][0][tl][lane]), cz, to_f32(sm.tile[s][2][tl][lane]), fv, sc, gv);
+        gg[j] = gv;
         f[j] = fv;
-        bb[j] = (1.0f - fv) * cv;
+        bb[j] = (1.0f - fv) * (cz * sc);
       } else {   // past the end: identity map
         f[j] = 1.0f;
         bb[j] = 0.0f;

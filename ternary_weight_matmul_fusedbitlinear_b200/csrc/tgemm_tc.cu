@@ -9,15 +9,16 @@
 // sum_k q[m,k] (w[n,k] + 1) with an s8 x u8 MMA and the epilogue subtracts the
 // token's code sum: acc = raw - sum_k q[m,k].
 //
-// Tile: 128 tokens (M) x 256 output columns (N) x 128 k-bytes per stage.
-// Persistent CTAs (one per SM), warp-specialised:
+// Tile: 128 tokens (M) x 256 output columns (N) x 128 k-bytes per K-step.
+// Persistent CTAs (one per SM, 320 threads), warp-specialised:
 //   warp 0      TMA producer: int8 activation tile (128B-swizzled, the UMMA
-//               K-major SW128 layout) and the 2-bit packed weight tile
-//   warp 1      TMEM owner + single-thread MMA issuer (4 x K=32 per stage)
+//               K-major SW128 layout) + 2-bit packed weight tile, 4-deep ring
+//   warp 1      TMEM owner + single-thread MMA issuer (4 x K=32 per K-step)
 //   warps 2..5  epilogue: tcgen05.ld of the int32 accumulators, rescale
-//               (+bias, +residual, SiLU*up), store
-//   warps 6..9  unpack: packed 2-bit codes -> int8 bytes in shared memory,
-//               written directly in the SW128 K-major layout the MMA reads
+//               (+bias, +residual, SiLU*up), swizzled staging in shared
+//               memory, TMA tensor store (coalesced, clipped at the M edge)
+//   warps 6..9  unpack: packed 2-bit codes -> int8 bytes written directly in
+//               the SW128 K-major layout the MMA reads, 2-deep ring
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile overlap
 // the main loop of the next. Every mbarrier wait is bounded: on timeout the
 // kernel records an error in the status word, raises a CTA-wide abort flag,
@@ -29,25 +30,37 @@ namespace mmf {
 
 namespace {
 
-constexpr int BM = 128, BN = 256, BK = 128, STAGES = 3;
+constexpr int BM = 128, BN = 256, BK = 128;
+constexpr int NB = 2;                     // unpacked-code ring depth
 constexpr int A_BYTES = BM * BK;          // 16 KiB int8 activations
 constexpr int BP_BYTES = BN * BK / 4;     // 8 KiB packed codes (2 bit)
 constexpr int BU_BYTES = BN * BK;         // 32 KiB unpacked codes (int8)
 constexpr int HALF = BN / 2;              // rows per weight TMA box
-constexpr int kThreads = 320;             // 10 warps
-constexpr int kEpiWarp0 = 2, kUnpackWarp0 = 6;
+constexpr int kEpiWarps = 8;              // two per TMEM lane quarter, splitting the columns
+constexpr int kEpiWarp0 = 2, kUnpackWarp0 = kEpiWarp0 + kEpiWarps;
 constexpr int kUnpackThreads = 128;
+constexpr int kThreads = (kUnpackWarp0 + kUnpackThreads / 32) * 32;   // 14 warps
+constexpr int kEpiChunk = 32;             // output columns per TMA store box (x 32 rows)
 constexpr uint32_t kTmemCols = 512;
 
+// Shared memory; OB = bytes of one output element (2: bf16, 4: fp32 / int32).
+// The TMA ring is 4 deep for 2-byte outputs and 3 deep for 4-byte outputs,
+// whose staging boxes are twice as large.
+template <int OB>
 struct __align__(1024) SmemLayout {
-  uint8_t a[STAGES][A_BYTES];
-  uint8_t bu[STAGES][BU_BYTES];
-  uint32_t bp[STAGES][BP_BYTES / 4];
-  uint64_t full_tma[STAGES];
-  uint64_t full_bu[STAGES];
-  uint64_t empty[STAGES];
+  static constexpr int NS = OB == 2 ? 4 : 3;
+  static constexpr int kStageBytes = 32 * kEpiChunk * OB;
+  uint8_t a[NS][A_BYTES];                          // 1024-aligned: SW128 atoms
+  uint8_t bu[NB][BU_BYTES];                        // 1024-aligned: SW128 atoms
+  uint8_t stage[kEpiWarps][2][kStageBytes];        // epilogue staging, double-buffered (1024-aligned)
+  uint32_t bp[NS][BP_BYTES / 4];
+  uint64_t tma_full[NS];
+  uint64_t tma_empty[NS];
+  uint64_t bu_full[NB];
+  uint64_t bu_empty[NB];
   uint64_t tmem_full[2];
   uint64_t tmem_empty[2];
+  uint64_t res_full[kEpiWarps];                    // residual box landed in a staging buffer
   uint64_t mma_drain;
   uint32_t tmem_base;
   int abort_flag;
@@ -98,6 +111,72 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+  asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                   reinterpret_cast<uint64_t>(map)),
+               "r"(x), "r"(y), "r"(smem_u32(src))
+               : "memory");
+  asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read_le1() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+
+// Stage one 32-row x 32-column box of the output in shared memory, in the
+// layout the output tensor map's swizzle expects (lane = row): 2-byte types use
+// 64-byte rows with the 64B swizzle (16-byte chunk c of row r at c ^ ((r>>1)&3)),
+// 4-byte types 128-byte rows with the 128B swizzle (chunk c at c ^ (r&7)).
+__device__ __forceinline__ void stage_row(uint8_t* buf, int r, const float (&v)[32], bf16*) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    uint4 u;
+    __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(v[8 * c + 2 * i], v[8 * c + 2 * i + 1]);
+    *reinterpret_cast<uint4*>(buf + r * 64 + ((c ^ ((r >> 1) & 3)) << 4)) = u;
+  }
+}
+__device__ __forceinline__ void stage_row(uint8_t* buf, int r, const float (&v)[32], float*) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<float4*>(buf + r * 128 + ((c ^ (r & 7)) << 4)) =
+        make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+}
+__device__ __forceinline__ void stage_row_i32(uint8_t* buf, int r, const uint32_t (&v)[32], int qs) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c)
+    *reinterpret_cast<int4*>(buf + r * 128 + ((c ^ (r & 7)) << 4)) =
+        make_int4((int)v[4 * c] - qs, (int)v[4 * c + 1] - qs, (int)v[4 * c + 2] - qs, (int)v[4 * c + 3] - qs);
+}
+
+// Add the residual box that TMA placed in `buf` (same swizzled layout as the
+// staged output) to this lane's row of outputs.
+__device__ __forceinline__ void add_staged_row(const uint8_t* buf, int r, float (&v)[32], bf16*) {
+#pragma unroll
+  for (int c = 0; c < 4; ++c) {
+    const uint4 u = *reinterpret_cast<const uint4*>(buf + r * 64 + ((c ^ ((r >> 1) & 3)) << 4));
+    const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&u);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float2 f = __bfloat1622float2(h[i]);
+      v[8 * c + 2 * i] += f.x;
+      v[8 * c + 2 * i + 1] += f.y;
+    }
+  }
+}
+__device__ __forceinline__ void add_staged_row(const uint8_t* buf, int r, float (&v)[32], float*) {
+#pragma unroll
+  for (int c = 0; c < 8; ++c) {
+    const float4 f = *reinterpret_cast<const float4*>(buf + r * 128 + ((c ^ (r & 7)) << 4));
+    v[4 * c] += f.x;
+    v[4 * c + 1] += f.y;
+    v[4 * c + 2] += f.z;
+    v[4 * c + 3] += f.w;
+  }
+}
+
+// SiLU with the hardware exponential and approximate reciprocal (a few ulp).
+__device__ __forceinline__ float silu_fast(float z) { return __fdividef(z, 1.0f + __expf(-z)); }
+
 // ---------------------------------------------------------------- tile geometry
 struct TcArgs {
   TGemmArgs g;
@@ -123,45 +202,41 @@ __device__ __forceinline__ void half_source(const TcArgs& p, Epi epi, int nt, in
   }
 }
 
-template <typename T>
-__device__ __forceinline__ void store32(T* dst, const float (&v)[32]);
-template <>
-__device__ __forceinline__ void store32<bf16>(bf16* dst, const float (&v)[32]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) store8(dst + 8 * q, v + 8 * q);
-}
-template <>
-__device__ __forceinline__ void store32<float>(float* dst, const float (&v)[32]) {
-#pragma unroll
-  for (int q = 0; q < 4; ++q) store8(dst + 8 * q, v + 8 * q);
-}
-
 template <Epi EPI, typename T>
 __global__ void __launch_bounds__(kThreads, 1)
     tgemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
                     const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_b2,
+                    const __grid_constant__ CUtensorMap map_out, const __grid_constant__ CUtensorMap map_res,
                     const TcArgs p) {
+  constexpr int OB = EPI == Epi::kAcc ? 4 : (int)sizeof(T);
+  using Smem = SmemLayout<OB>;
+  constexpr int NS = Smem::NS;
   extern __shared__ uint8_t smem_raw[];
-  SmemLayout& sm = *reinterpret_cast<SmemLayout*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort_flag = &sm.abort_flag;
   const int n_tiles_total = p.m_tiles * p.n_tiles;
   const int nk = ceil_div(p.g.K, BK);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < STAGES; ++s) {
-      mbar_init(&sm.full_tma[s], 1);
-      mbar_init(&sm.full_bu[s], kUnpackThreads);
-      mbar_init(&sm.empty[s], 1);
+    for (int s = 0; s < NS; ++s) {
+      mbar_init(&sm.tma_full[s], 1);
+      mbar_init(&sm.tma_empty[s], 1);
+    }
+    for (int u = 0; u < NB; ++u) {
+      mbar_init(&sm.bu_full[u], kUnpackThreads);
+      mbar_init(&sm.bu_empty[u], 1);
     }
     for (int a = 0; a < 2; ++a) {
       mbar_init(&sm.tmem_full[a], 1);
-      mbar_init(&sm.tmem_empty[a], 128);
+      mbar_init(&sm.tmem_empty[a], kEpiWarps * 32);
     }
+    for (int w = 0; w < kEpiWarps; ++w) mbar_init(&sm.res_full[w], 1);
     mbar_init(&sm.mma_drain, 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&map_a)) : "memory");
+    prefetch_tmap(&map_a);
+    prefetch_tmap(&map_out);
   }
   if (warp == 1) {
     asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(&sm.tmem_base)),
@@ -186,18 +261,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         half_source(p, EPI, nt, 0, seg0, row0);
         half_source(p, EPI, nt, 1, seg1, row1);
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&sm.empty[s], ph ^ 1, abort_flag, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sm.full_tma[s], A_BYTES + BP_BYTES);
-          tma_load_2d(sm.a[s], &map_a, kb * BK, mt * BM, &sm.full_tma[s]);
-          tma_load_2d(&sm.bp[s][0], maps[seg0], kb * (BK / 16), row0, &sm.full_tma[s]);
-          tma_load_2d(&sm.bp[s][HALF * (BK / 16)], maps[seg1], kb * (BK / 16), row1, &sm.full_tma[s]);
+          const int s = it % NS;
+          if (!mbar_wait(&sm.tma_empty[s], ((it / NS) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+          mbar_arrive_expect_tx(&sm.tma_full[s], A_BYTES + BP_BYTES);
+          tma_load_2d(sm.a[s], &map_a, kb * BK, mt * BM, &sm.tma_full[s]);
+          tma_load_2d(&sm.bp[s][0], maps[seg0], kb * (BK / 16), row0, &sm.tma_full[s]);
+          tma_load_2d(&sm.bp[s][HALF * (BK / 16)], maps[seg1], kb * (BK / 16), row1, &sm.tma_full[s]);
         }
       }
       // let every copy this thread issued land before the CTA can exit
-      for (uint32_t j = (it > STAGES ? it - STAGES : 0); j < it; ++j)
-        mbar_wait(&sm.full_tma[j % STAGES], (j / STAGES) & 1, abort_flag, nullptr);
+      for (uint32_t j = (it > NS ? it - NS : 0); j < it; ++j)
+        mbar_wait(&sm.tma_full[j % NS], (j / NS) & 1, abort_flag, nullptr);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -211,16 +285,20 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % STAGES;
-          const uint32_t ph = (it / STAGES) & 1;
-          if (!mbar_wait(&sm.full_bu[s], ph, abort_flag, p.status)) { ok = false; break; }
+          const int s = it % NS, u = it % NB;
+          if (!mbar_wait(&sm.bu_full[u], (it / NB) & 1, abort_flag, p.status) ||
+              !mbar_wait(&sm.tma_full[s], (it / NS) & 1, abort_flag, p.status)) {
+            ok = false;
+            break;
+          }
           tc_fence_after();
           const uint64_t adesc = umma_desc_sw128(smem_u32(sm.a[s]));
-          const uint64_t bdesc = umma_desc_sw128(smem_u32(sm.bu[s]));
+          const uint64_t bdesc = umma_desc_sw128(smem_u32(sm.bu[u]));
 #pragma unroll
           for (int j = 0; j < BK / 32; ++j)   // advance 32 bytes of K inside the swizzle atom
             umma_i8(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), (kb | j) != 0);
-          umma_commit(&sm.empty[s]);
+          umma_commit(&sm.tma_empty[s]);
+          umma_commit(&sm.bu_empty[u]);
         }
         if (ok) umma_commit(&sm.tmem_full[acc]);
       }
@@ -230,46 +308,70 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp >= kUnpackWarp0) {
     // ------------------------------------------------------------ unpack 2-bit codes to int8
-    const int u = threadIdx.x - kUnpackWarp0 * 32;   // 0..127: rows u and u + 128
+    // 512 (row, half-row) units per K-step; unit id = tid + 128 i reads the 16
+    // bytes at id * 16 of the packed tile (row id/2, columns 64 (id%2) ..+63),
+    // so each warp reads 512 contiguous bytes; writes land in distinct banks.
+    const int tid = threadIdx.x - kUnpackWarp0 * 32;
     uint32_t it = 0;
     bool ok = true;
     for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
       for (int kb = 0; kb < nk; ++kb, ++it) {
-        const int s = it % STAGES;
-        const uint32_t ph = (it / STAGES) & 1;
-        if (!mbar_wait(&sm.full_tma[s], ph, abort_flag, p.status)) { ok = false; break; }
+        const int s = it % NS, u = it % NB;
+        if (!mbar_wait(&sm.tma_full[s], (it / NS) & 1, abort_flag, p.status) ||
+            !mbar_wait(&sm.bu_empty[u], ((it / NB) & 1) ^ 1, abort_flag, p.status)) {
+          ok = false;
+          break;
+        }
+        const uint4* src = reinterpret_cast<const uint4*>(sm.bp[s]);
 #pragma unroll
-        for (int rr = 0; rr < 2; ++rr) {
-          const int n = u + rr * HALF;
-          const uint4* src = reinterpret_cast<const uint4*>(&sm.bp[s][n * (BK / 16)]);
-          uint8_t* dst = sm.bu[s] + n * BK;
+        for (int i = 0; i < 4; ++i) {
+          const int id = tid + kUnpackThreads * i;
+          const int n = id >> 1, h = id & 1;
+          const uint4 w4 = src[id];
+          const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
+          uint8_t* dst = sm.bu[u] + n * BK;
 #pragma unroll
-          for (int hq = 0; hq < 2; ++hq) {
-            const uint4 w4 = src[hq];
-            const uint32_t ws[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = hq * 4 + e;     // 16-column chunk of this row
-              const uint32_t w = ws[e];
-              uint4 v;
-              v.x = w & 0x03030303u;
-              v.y = (w >> 2) & 0x03030303u;
-              v.z = (w >> 4) & 0x03030303u;
-              v.w = (w >> 6) & 0x03030303u;
-              *reinterpret_cast<uint4*>(dst + ((c ^ (n & 7)) << 4)) = v;
-            }
+          for (int e = 0; e < 4; ++e) {
+            const int c = 4 * h + e;         // 16-column chunk of this row
+            const uint32_t w = ws[e];
+            uint4 v;
+            v.x = w & 0x03030303u;
+            v.y = (w >> 2) & 0x03030303u;
+            v.z = (w >> 4) & 0x03030303u;
+            v.w = (w >> 6) & 0x03030303u;
+            *reinterpret_cast<uint4*>(dst + ((c ^ (n & 7)) << 4)) = v;
           }
         }
         fence_proxy_async_smem();
-        mbar_arrive(&sm.full_bu[s]);
+        mbar_arrive(&sm.bu_full[u]);
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2..5)
+    // ------------------------------------------------------------ epilogue (8 warps)
+    const int ew = warp - kEpiWarp0;              // 0..7
     const int quarter = warp & 3;                 // TMEM lanes 32*quarter .. +31
+    const int group = ew >> 2;                    // which half of the columns this warp takes
     const int row_in_tile = quarter * 32 + lane;
+    uint8_t* stage0 = sm.stage[ew][0];
+    uint8_t* stage1 = sm.stage[ew][1];
+    int nst = 0;                                  // boxes stored by this warp so far
+    uint32_t nres = 0;                            // residual boxes loaded by this warp so far
     uint32_t tl = 0;
-    for (int tile = blockIdx.x; tile < n_tiles_total; tile += gridDim.x, ++tl) {
+    const bool has_res = EPI == Epi::kStore && p.g.residual != nullptr;
+    // Wait until the store that last used staging buffer (nst & 1) has read it.
+    auto claim = [&](uint8_t*& buf) {
+      if (lane == 0 && nst >= 2) bulk_wait_read_le1();
+      __syncwarp();
+      buf = (nst & 1) ? stage1 : stage0;
+    };
+    auto release = [&](int x, int y, uint8_t* buf) {
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) tma_store_2d(&map_out, buf, x, y);
+      ++nst;
+    };
+    bool alive = true;
+    for (int tile = blockIdx.x; tile < n_tiles_total && alive; tile += gridDim.x, ++tl) {
       const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
       const int acc = tl & 1;
       const uint32_t acc_ph = (tl >> 1) & 1;
@@ -278,48 +380,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
       const int m = mt * BM + row_in_tile;
+      const int y0 = mt * BM + quarter * 32;
       const bool row_ok = m < p.g.M;
       const float inv_s = row_ok ? 1.0f / p.g.s[m] : 0.0f;
       const int qs = row_ok ? p.g.qsum[m] : 0;
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
       if constexpr (EPI == Epi::kGlu) {
         const float sc_u = *p.g.gamma[0] * inv_s, sc_v = *p.g.gamma[1] * inv_s;
-        for (int c = 0; c < HALF / 32; ++c) {
+        for (int cc = 0; cc < 2; ++cc) {
+          const int c = group * 2 + cc;           // 32-column chunk of the gate / up halves
           uint32_t ru[32], rv[32];
           tmem_ld32(tbase + 32 * c, ru);
           tmem_ld32(tbase + HALF + 32 * c, rv);
           const int n0 = nt * HALF + 32 * c;
-          if (row_ok) {
-            float out[32];
+          float out[32];
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              float uu = (float)((int)ru[j] - qs) * sc_u;
-              float vv = (float)((int)rv[j] - qs) * sc_v;
-              if (p.g.bias[0] != nullptr) uu += p.g.bias[0][n0 + j];
-              if (p.g.bias[1] != nullptr) vv += p.g.bias[1][n0 + j];
-              out[j] = siluf_(uu) * vv;
-            }
-            store32<T>(static_cast<T*>(p.g.out) + (size_t)m * p.g.ldo + n0, out);
+          for (int j = 0; j < 32; ++j) {
+            float uu = (float)((int)ru[j] - qs) * sc_u;
+            float vv = (float)((int)rv[j] - qs) * sc_v;
+            if (p.g.bias[0] != nullptr) uu += p.g.bias[0][n0 + j];
+            if (p.g.bias[1] != nullptr) vv += p.g.bias[1][n0 + j];
+            out[j] = silu_fast(uu) * vv;
           }
+          uint8_t* buf;
+          claim(buf);
+          stage_row(buf, lane, out, (T*)nullptr);
+          release(n0, y0, buf);
         }
       } else {
-        for (int h = 0; h < 2; ++h) {
-          int seg, row0;
-          half_source(p, EPI, nt, h, seg, row0);
-          if (nt * BN + h * HALF >= p.g.nseg * p.g.N) break;
+        const int h = group;                      // 128-column half of the tile
+        int seg, row0;
+        half_source(p, EPI, nt, h, seg, row0);
+        if (nt * BN + h * HALF < p.g.nseg * p.g.N) {
           const float sc = *p.g.gamma[seg] * inv_s;
           const float* bias = p.g.bias[seg];
-          for (int c = 0; c < HALF / 32; ++c) {
+          for (int c = 0; c < HALF / kEpiChunk; ++c) {
+            const int n0 = row0 + 32 * c;
+            const int x0 = seg * p.g.N + n0;
+            uint8_t* buf;
+            claim(buf);
+            if (has_res && lane == 0) {           // residual box -> this staging buffer
+              mbar_arrive_expect_tx(&sm.res_full[ew], 32 * kEpiChunk * OB);
+              tma_load_2d(buf, &map_res, n0, y0, &sm.res_full[ew]);
+            }
             uint32_t r[32];
             tmem_ld32(tbase + h * HALF + 32 * c, r);
-            const int n0 = row0 + 32 * c;
-            if (!row_ok) continue;
             if constexpr (EPI == Epi::kAcc) {
-              int32_t* dst = static_cast<int32_t*>(p.g.out) + (size_t)m * p.g.ldo + seg * p.g.N + n0;
-#pragma unroll
-              for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<int4*>(dst + j) =
-                    make_int4((int)r[j] - qs, (int)r[j + 1] - qs, (int)r[j + 2] - qs, (int)r[j + 3] - qs);
+              stage_row_i32(buf, lane, r, qs);
             } else {
               float out[32];
 #pragma unroll
@@ -328,24 +435,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (bias != nullptr) v += bias[n0 + j];
                 out[j] = v;
               }
-              if (p.g.residual != nullptr) {
-                const T* res = static_cast<const T*>(p.g.residual) + (size_t)m * p.g.N + n0;
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                  float rv[8];
-                  load8(res + 8 * q, rv);
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) out[8 * q + j] += rv[j];
-                }
+              if (has_res) {
+                const bool ok = mbar_wait(&sm.res_full[ew], nres & 1, abort_flag, p.status);
+                ++nres;
+                if (!__all_sync(0xffffffffu, ok)) { alive = false; break; }
+                add_staged_row(buf, lane, out, (T*)nullptr);
+                __syncwarp();                     // every row read before any row is overwritten
               }
-              store32<T>(static_cast<T*>(p.g.out) + (size_t)m * p.g.ldo + seg * p.g.N + n0, out);
+              stage_row(buf, lane, out, (T*)nullptr);
             }
+            release(x0, y0, buf);
           }
         }
       }
       tc_fence_before();
       mbar_arrive(&sm.tmem_empty[acc]);
     }
+    if (lane == 0) bulk_wait_all();   // stores complete before the CTA exits
+    __syncwarp();
   }
 
   // ------------------------------------------------------------ teardown
@@ -362,13 +469,26 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------- host side
 template <Epi EPI, typename T>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap (&mb)[3], const TcArgs& p, cudaStream_t stream) {
-  const size_t smem = sizeof(SmemLayout) + 1024;
+  CUtensorMap mo;
+  const bool acc_out = EPI == Epi::kAcc;
+  const int esize = acc_out ? 4 : (int)sizeof(T);
+  const CUtensorMapDataType odt = acc_out ? CU_TENSOR_MAP_DATA_TYPE_INT32
+                                          : (sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16
+                                                            : CU_TENSOR_MAP_DATA_TYPE_FLOAT32);
+  const CUtensorMapSwizzle oswz = esize == 2 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B;
+  if (!make_tma_2d(&mo, p.g.out, odt, esize, (uint64_t)p.g.ldo, (uint64_t)p.g.M, kEpiChunk, 32, oswz))
+    return cudaErrorInvalidValue;
+  CUtensorMap mr = mo;   // unused unless there is a residual
+  if (EPI == Epi::kStore && p.g.residual != nullptr &&
+      !make_tma_2d(&mr, p.g.residual, odt, esize, (uint64_t)p.g.N, (uint64_t)p.g.M, kEpiChunk, 32, oswz))
+    return cudaErrorInvalidValue;
+  const size_t smem = sizeof(SmemLayout<(EPI == Epi::kAcc ? 4 : (int)sizeof(T))>) + 1024;
   auto kern = tgemm_tc_kernel<EPI, T>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = std::min(tiles, num_sms());
-  kern<<<grid, kThreads, smem, stream>>>(ma, mb[0], mb[1], mb[2], p);
+  kern<<<grid, kThreads, smem, stream>>>(ma, mb[0], mb[1], mb[2], mo, mr, p);
   return cudaGetLastError();
 }
 
