@@ -51,9 +51,15 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["mmf", "reference"], default="mmf")
-    ap.add_argument("--workload", choices=["stack370m", "bitlinear"], default="stack370m",
+    ap.add_argument("--workload", choices=["stack370m", "bitlinear", "scan", "gemv", "decode1p3b", "decode2p7b"],
+                    default="stack370m",
                     help="stack370m: the 370M-shaped 24-block prefill (default); bitlinear: one prefill "
-                         "BitLinear of the 370M gate|up shape (16384 tokens, 1024 -> 5632)")
+                         "BitLinear of the 370M gate|up shape (16384 tokens, 1024 -> 5632); scan: one MLGRU "
+                         "scan of the 370M layer shape (8 x 2048 tokens, d=1024); gemv: the decode BitLinear "
+                         "sweep (2048->2048, 2048->5632, 5632->2048 at 1/4/16 tokens) over a weight pool > L2; "
+                         "decode1p3b / decode2p7b: the 1.3B / 2.7B-shaped stacks, prompt prefill then decode "
+                         "steps (output fed back, state carried), each step one CUDA graph")
+    ap.add_argument("--batch", type=int, default=None, help="decode2p7b: concurrent sequences (1, 8 or 64)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) pass")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     return ap.parse_args(argv)
@@ -417,6 +423,187 @@ def run_bitlinear(args):
     return 0
 
 
+def run_scan(args):
+    """One MLGRU scan per step on the 370M layer shape; GB/s = 8 bytes per channel-step (bf16)."""
+    _, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    dev = torch.device("cuda", local)
+    w = synth.STACK_370M
+    B, T, d = w.batch, w.seq, w.d
+    peaks, peak_kind = load_peaks()
+    pre = synth.preacts(77, B, T, d, torch.bfloat16, scale=2.0, device=dev)
+    h = torch.zeros(B, d, device=dev)
+    flush = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        mmf.mlgru_scan(pre, h)
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    torch.cuda.synchronize()
+    for _ in range(args.steps):
+        flush.zero_()
+        mmf.mlgru_scan(pre, h)
+    torch.cuda.synchronize()
+    mmf.prof_enable(False)
+    prof = mmf.prof_collect()
+    ms = prof["mlgru_scan"][1] / prof["mlgru_scan"][0]
+    nbytes = 8.0 * B * T * d
+    gbs = nbytes / (ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic", "config": {"workload": f"mlgru_scan_b{B}_t{T}_d{d}_bf16",
+                                            "l2": "flushed between timed steps"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mlgru_scan",
+                         "peak_source": peak_kind},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": prof["mlgru_scan"][0]}), flush=True)
+    return 0
+
+
+def run_gemv(args):
+    """Decode BitLinear sweep: per shape and token count, calls cycle through a pool of distinct packed
+    matrices totalling more than 4x L2; GB/s = (N*K/4 + 4 + 2*M*K + 2*M*N) bytes per call / mean call time."""
+    _, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    dev = torch.device("cuda", local)
+    peaks, peak_kind = load_peaks()
+    rows = []
+    for (K, N) in synth.GEMV_SWEEP_SHAPES:
+        per = N * K // 4
+        pool_n = max(8, int(4 * L2_BYTES // per) + 1)
+        lins = [mmf.quantize_weights(synth.latent_weight(synth.GEMV_SWEEP_SEED * 4096 + i, N, K, device=dev))
+                for i in range(pool_n)]
+        for M in synth.GEMV_SWEEP_TOKENS:
+            x = synth.activations(synth.GEMV_SWEEP_SEED + M, M, K, torch.bfloat16, outlier_p=synth.GEMV_OUTLIER_P,
+                                  outlier_scale=synth.GEMV_OUTLIER_SCALE, device=dev)
+            ws = torch.empty(mmf.api.L.load().mmf_bitlinear_ws_size(M, K), dtype=torch.uint8, device=dev)
+            y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+            side = torch.cuda.Stream(dev)
+            side.wait_stream(torch.cuda.current_stream(dev))
+            with torch.cuda.stream(side):
+                for lin in lins[:max(args.warmup, 3)]:
+                    mmf.bitlinear(lin, x, ws=ws)
+            torch.cuda.current_stream(dev).wait_stream(side)
+            torch.cuda.synchronize()
+            # one graph replays the whole pool in order: launch cost leaves the host
+            calls = pool_n
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                for i in range(calls):
+                    mmf.bitlinear(lins[i], x, ws=ws)
+            graph.replay()
+            torch.cuda.synchronize()
+            reps = max(1, args.steps // 5)
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            e0.record()
+            for _ in range(reps):
+                graph.replay()
+            e1.record()
+            torch.cuda.synchronize()
+            del graph
+            calls = calls * reps
+            us = e0.elapsed_time(e1) * 1e3 / calls
+            nbytes = per + 4 + 2 * M * K + 2 * M * N
+            rows.append({"K": K, "N": N, "M": M, "us_per_call": round(us, 3),
+                         "GBps": round(nbytes / (us * 1e-6) / 1e9, 1),
+                         "frac": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
+                         "TOPS": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 3), "pool": pool_n})
+            del ws, y
+        del lins
+        torch.cuda.empty_cache()
+    best = max(r["GBps"] for r in rows)
+    mean = sum(r["GBps"] for r in rows) / len(rows)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": mean, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "bitlinear_decode_gemv_sweep", "l2": "weight pool > 4x L2, cycled"},
+            "roofline": {"bound": "hbm", "achieved": mean, "best": best, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": mean / peaks["hbm_gbs"], "traffic": None, "kernel": "rmsnorm_quant+tgemm_mma",
+                         "peak_source": peak_kind, "sweep": rows},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": None}), flush=True)
+    return 0
+
+
+def run_decode(args):
+    """Prompt prefill, then decode steps; each decode step (all layers, T=1) is one CUDA graph replay whose
+    output is copied back to its input. Reports decode tokens/s, and HBM GB/s of the packed-weight stream."""
+    _, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    dev = torch.device("cuda", local)
+    w = synth.STACK_1P3B if args.workload == "decode1p3b" else synth.STACK_2P7B
+    B = args.batch or w.batch
+    peaks, peak_kind = load_peaks()
+    blocks = build_stack(w, dev)
+    st = mmf.State(w.layers, B, w.d)
+    prompt = synth.activations(w.seed + synth.ACT_SEED_OFFSET, B * w.seq, w.d, torch.bfloat16,
+                               device=dev).reshape(B, w.seq, w.d)
+    ws_p = torch.empty(mmf.stack_ws_size(blocks, B, w.seq), dtype=torch.uint8, device=dev)
+    y_p = torch.empty_like(prompt)
+    # prompt prefill (timed separately)
+    mmf.stack_forward(blocks, st, prompt, ws=ws_p, out=y_p)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    st.reset()
+    e0.record()
+    mmf.stack_forward(blocks, st, prompt, ws=ws_p, out=y_p)
+    e1.record()
+    torch.cuda.synchronize()
+    prefill_ms = e0.elapsed_time(e1)
+    del ws_p
+    # decode: input = last prompt position's output
+    x = y_p[:, -1:, :].contiguous()
+    y = torch.empty_like(x)
+    ws = torch.empty(mmf.stack_ws_size(blocks, B, 1), dtype=torch.uint8, device=dev)
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):
+        for _ in range(3):
+            mmf.stack_forward(blocks, st, x, ws=ws, out=y)
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        mmf.stack_forward(blocks, st, x, ws=ws, out=y)
+        x.copy_(y)
+    steps = w.decode_steps
+    for _ in range(args.warmup):
+        graph.replay()
+    torch.cuda.synchronize()
+    clocks = ClockSampler(local)
+    clocks.start()
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    step_ms = e0.elapsed_time(e1) / steps
+    weights = w.layers * (4 * w.d * w.d + 3 * w.d * w.inner) / 4.0
+    state = 2.0 * w.layers * B * w.d * 4
+    gbs = (weights + state) / (step_ms / 1e3) / 1e9
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": B / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"{w.name}_b{B}", "batch": B, "layers": w.layers, "d": w.d, "inner": w.inner,
+                       "prompt": w.seq, "decode_steps": steps,
+                       "prefill_ms": prefill_ms, "prefill_tokens_per_s": B * w.seq / (prefill_ms / 1e3),
+                       "l2": "weight stream per step > L2"},
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "decode step (all kernels)",
+                         "bytes_per_step": weights + state, "peak_source": peak_kind},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": w.layers * 8, "clocks": clk}), flush=True)
+    return 0
+
+
 def main(argv=None):
     args = parse_args(argv)
     if args.warmup < 3:
@@ -425,6 +612,12 @@ def main(argv=None):
         return run_reference(args)
     if args.workload == "bitlinear":
         return run_bitlinear(args)
+    if args.workload == "scan":
+        return run_scan(args)
+    if args.workload == "gemv":
+        return run_gemv(args)
+    if args.workload in ("decode1p3b", "decode2p7b"):
+        return run_decode(args)
     return run_mmf(args)
 
 

@@ -141,18 +141,17 @@ __device__ __forceinline__ void unpack8(const uint4 (&r)[2], float (&v)[8]) {
   }
 }
 
+// Four int32 codes -> four saturated int8 bytes in memory order c0..c3.
+__device__ __forceinline__ uint32_t pack4_sat(int c0, int c1, int c2, int c3) {
+  uint32_t hi, w;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(c3), "r"(c2));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(w) : "r"(c1), "r"(c0), "r"(hi));
+  return w;
+}
+
 template <typename T, int VMAX>
-__global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(const T* __restrict__ x, int M, int K,
-                                                                 const float* __restrict__ gain, float eps,
-                                                                 int8_t* __restrict__ q, float* __restrict__ scale,
-                                                                 int32_t* __restrict__ qsum) {
+__device__ __forceinline__ void load_row(const T* __restrict__ xr, int nvec, int lane, uint4 (&raw)[VMAX][Vec16<T>::regs]) {
   constexpr int R = Vec16<T>::regs;
-  const int lane = threadIdx.x & 31;
-  const int row = blockIdx.x * 8 + (threadIdx.x >> 5);
-  if (row >= M) return;
-  const int nvec = K / 8;
-  const T* xr = x + (size_t)row * K;
-  uint4 raw[VMAX][R];
 #pragma unroll
   for (int j = 0; j < VMAX; ++j) {
     const int vi = j * 32 + lane;
@@ -160,70 +159,110 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(const T* __rest
     for (int r = 0; r < R; ++r)
       raw[j][r] = vi < nvec ? __ldg(reinterpret_cast<const uint4*>(xr + (size_t)vi * 8) + r) : make_uint4(0, 0, 0, 0);
   }
-  double ss = 0.0;
-#pragma unroll
-  for (int j = 0; j < VMAX; ++j) {
-    float v[8];
-    unpack8(raw[j], v);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) ss += (double)v[i] * (double)v[i];
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  const float ms = (float)(ss / (double)K);
-  const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
+}
 
-  float amax = 0.0f;
+// Persistent: each warp walks rows warp_id, warp_id + nwarps, ... and issues
+// the loads of its next row before reducing the current one, so the row's
+// HBM latency overlaps the previous row's arithmetic.
+template <typename T, int VMAX>
+__global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(const T* __restrict__ x, int M, int K,
+                                                                 const float* __restrict__ gain, float eps,
+                                                                 int8_t* __restrict__ q, float* __restrict__ scale,
+                                                                 int32_t* __restrict__ qsum) {
+  constexpr int R = Vec16<T>::regs;
+  constexpr bool kKeep = VMAX <= 8;   // keep x^ in registers between the max and the codes
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * 8;
+  int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+  pdl_trigger();
+  pdl_wait();
+  if (row >= M) return;
+  const int nvec = K / 8;
+  uint4 raw[VMAX][R], nxt[VMAX][R];
+  load_row<T, VMAX>(x + (size_t)row * K, nvec, lane, raw);
+  for (; row < M; row += nwarps) {
+    if (row + nwarps < M) load_row<T, VMAX>(x + (size_t)(row + nwarps) * K, nvec, lane, nxt);
+    double ss = 0.0;
 #pragma unroll
-  for (int j = 0; j < VMAX; ++j) {
-    const int vi = j * 32 + lane;
-    if (vi >= nvec) break;
-    float v[8];
-    unpack8(raw[j], v);
+    for (int j = 0; j < VMAX; ++j) {
+      float v[8];
+      unpack8(raw[j], v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float h = __fmul_rn(v[i], rinv);
-      if (gain != nullptr) h = __fmul_rn(h, __ldg(gain + vi * 8 + i));
-      amax = fmaxf(amax, fabsf(h));
+      for (int i = 0; i < 8; ++i) ss = fma((double)v[i], (double)v[i], ss);
     }
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-  const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    const float ms = (float)(ss / (double)K);
+    const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
 
-  int isum = 0;
-  int8_t* qr = q + (size_t)row * K;
+    float xh[kKeep ? VMAX : 1][8];
+    float amax = 0.0f;
 #pragma unroll
-  for (int j = 0; j < VMAX; ++j) {
-    const int vi = j * 32 + lane;
-    if (vi >= nvec) break;
-    float v[8];
-    unpack8(raw[j], v);
-    uint32_t w[2] = {0u, 0u};
+    for (int j = 0; j < VMAX; ++j) {
+      const int vi = j * 32 + lane;
+      float v[8];
+      unpack8(raw[j], v);
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float h = __fmul_rn(v[i], rinv);
-      if (gain != nullptr) h = __fmul_rn(h, __ldg(gain + vi * 8 + i));
-      int c = __float2int_rn(__fmul_rn(h, s));
-      c = max(-128, min(127, c));
-      isum += c;
-      w[i >> 2] |= (uint32_t)(c & 0xff) << (8 * (i & 3));
+      for (int i = 0; i < 8; ++i) {
+        float h = __fmul_rn(v[i], rinv);
+        if (gain != nullptr && vi < nvec) h = __fmul_rn(h, __ldg(gain + vi * 8 + i));
+        amax = fmaxf(amax, fabsf(h));
+        if constexpr (kKeep) xh[j][i] = h;
+      }
     }
-    *reinterpret_cast<uint2*>(qr + (size_t)vi * 8) = make_uint2(w[0], w[1]);
-  }
 #pragma unroll
-  for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
-  if (lane == 0) {
-    scale[row] = s;
-    qsum[row] = isum;
+    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+
+    int isum = 0;
+    int8_t* qr = q + (size_t)row * K;
+#pragma unroll
+    for (int j = 0; j < VMAX; ++j) {
+      const int vi = j * 32 + lane;
+      if (vi >= nvec) break;
+      float h[8];
+      if constexpr (kKeep) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) h[i] = xh[j][i];
+      } else {
+        float v[8];
+        unpack8(raw[j], v);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          h[i] = __fmul_rn(v[i], rinv);
+          if (gain != nullptr) h[i] = __fmul_rn(h[i], __ldg(gain + vi * 8 + i));
+        }
+      }
+      int c[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) c[i] = __float2int_rn(__fmul_rn(h[i], s));
+      const uint32_t w0 = pack4_sat(c[0], c[1], c[2], c[3]);
+      const uint32_t w1 = pack4_sat(c[4], c[5], c[6], c[7]);
+      isum = __dp4a((int)w0, 0x01010101, isum);
+      isum = __dp4a((int)w1, 0x01010101, isum);
+      *reinterpret_cast<uint2*>(qr + (size_t)vi * 8) = make_uint2(w0, w1);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+    if (lane == 0) {
+      scale[row] = s;
+      qsum[row] = isum;
+    }
+#pragma unroll
+    for (int j = 0; j < VMAX; ++j)
+#pragma unroll
+      for (int r = 0; r < R; ++r) raw[j][r] = nxt[j][r];
   }
 }
 
 template <typename T, int VMAX>
 void launch_warp(const void* x, int M, int K, const float* gain, float eps, int8_t* q, float* scale, int32_t* qsum,
                  cudaStream_t stream) {
-  rmsnorm_quant_warp_kernel<T, VMAX><<<ceil_div(M, 8), 256, 0, stream>>>(static_cast<const T*>(x), M, K, gain, eps, q,
-                                                                          scale, qsum);
+  auto kern = rmsnorm_quant_warp_kernel<T, VMAX>;
+  int per_sm = 1;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
+  const int grid = std::max(1, std::min(ceil_div(M, 8), num_sms() * std::max(per_sm, 1)));
+  launch_pdl(kern, dim3(grid), dim3(256), 0, stream, static_cast<const T*>(x), M, K, gain, eps, q, scale, qsum);
 }
 
 }  // namespace
@@ -231,20 +270,16 @@ void launch_warp(const void* x, int M, int K, const float* gain, float eps, int8
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
                                  int8_t* q, float* scale, int32_t* qsum, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
-  // warp-per-row kernels while the row fits in registers (K / 256 vectors per lane)
+  // warp-per-row kernels while two rows fit in registers (K / 256 vectors per lane)
   const int vpl = ceil_div(K / 8, 32);
-  if (dt == MMF_BF16 && vpl <= 28) {
+  if (dt == MMF_BF16 && vpl <= 12) {
     if (vpl <= 4) launch_warp<bf16, 4>(x, M, K, gain, eps, q, scale, qsum, stream);
     else if (vpl <= 8) launch_warp<bf16, 8>(x, M, K, gain, eps, q, scale, qsum, stream);
-    else if (vpl <= 12) launch_warp<bf16, 12>(x, M, K, gain, eps, q, scale, qsum, stream);
-    else if (vpl <= 22) launch_warp<bf16, 22>(x, M, K, gain, eps, q, scale, qsum, stream);
-    else launch_warp<bf16, 28>(x, M, K, gain, eps, q, scale, qsum, stream);
+    else launch_warp<bf16, 12>(x, M, K, gain, eps, q, scale, qsum, stream);
     return cudaGetLastError();
   }
-  if (dt == MMF_F32 && vpl <= 12) {
-    if (vpl <= 4) launch_warp<float, 4>(x, M, K, gain, eps, q, scale, qsum, stream);
-    else if (vpl <= 8) launch_warp<float, 8>(x, M, K, gain, eps, q, scale, qsum, stream);
-    else launch_warp<float, 12>(x, M, K, gain, eps, q, scale, qsum, stream);
+  if (dt == MMF_F32 && vpl <= 4) {
+    launch_warp<float, 4>(x, M, K, gain, eps, q, scale, qsum, stream);
     return cudaGetLastError();
   }
   const size_t smem = sizeof(float) * (size_t)K;

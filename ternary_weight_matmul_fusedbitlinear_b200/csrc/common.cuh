@@ -62,6 +62,15 @@ __device__ __forceinline__ void store8(float* p, const float v[8]) {
 __device__ __forceinline__ float sigmoidf_(float z) { return __frcp_rn(1.0f + __expf(-z)); }
 __device__ __forceinline__ float siluf_(float z) { return z * sigmoidf_(z); }
 
+// ---------------------------------------------------------------- programmatic dependent launch
+// A kernel launched with programmatic stream serialization may start before
+// its predecessor in the stream has finished. pdl_wait() blocks until every
+// predecessor grid has completed and its memory is visible: call it before the
+// first read of a predecessor's output and before the first global write.
+// pdl_trigger() lets the next kernel in the stream start launching.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ---------------------------------------------------------------- misc
 __host__ __device__ __forceinline__ int ceil_div(int a, int b) { return (a + b - 1) / b; }
 

@@ -4,6 +4,7 @@
 #include <cuda.h>
 
 #include <algorithm>
+#include <utility>
 
 #include "common.cuh"
 
@@ -16,6 +17,24 @@ bool tma_available();
 bool make_tma_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
                  uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 int num_sms();
+
+// Launch `kern` with programmatic stream serialization (the kernel must call
+// pdl_wait() before touching anything a predecessor wrote or reads).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
 
 // Message returned by mmf_last_error() on this host thread.
 void set_last_error(const char* msg);

@@ -9,6 +9,11 @@
 // kernel multiplies the stored code as an unsigned byte and subtracts the
 // per-token code sum afterwards: sum_k (w+1) q = acc + sum_k q.
 //
+// Launch: programmatic dependent launch. Before waiting on its predecessor a
+// CTA copies its whole weight slice (16 rows x K of each segment) into shared
+// memory with cp.async, so the weight stream overlaps the previous kernel; the
+// activations are read only after pdl_wait().
+//
 // Work split: a CTA owns 16 output rows of each of its R weight segments and
 // 8*NT tokens; its 8 warps split K into 256-column segments round-robin. Per
 // 256-column segment a lane (group g, thread t) loads 16 bytes of packed codes
@@ -55,9 +60,19 @@ __device__ __forceinline__ uint4 load_words4(const uint32_t* row, int w0, int nw
   return r;
 }
 
-template <int NT, int R, Epi EPI, typename T>
+__device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool valid) {
+  const uint32_t s = static_cast<uint32_t>(__cvta_generic_to_shared(smem));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(s), "l"(gmem), "r"(valid ? 16 : 0) : "memory");
+}
+
+// Shared-memory pitch of one weight row in 16-byte units: the row plus 64 bytes,
+// so the 8 rows a quarter-warp reads start in different banks.
+__host__ __device__ __forceinline__ int wsm_pitch4(int wpr) { return wpr / 4 + 4; }
+
+template <int NT, int R, Epi EPI, typename T, bool SMEMW>
 __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
   __shared__ int red[R][16][NT * 8];
+  extern __shared__ uint4 wsm[];     // SMEMW: [R][16][pitch4] weight slice
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int n0 = blockIdx.x * 16;
@@ -65,8 +80,25 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
   const int K = a.K, N = a.N, M = a.M;
   const int wpr = K / 16;            // packed words per row
   const int nkseg = ceil_div(K, 256);
+  const int wpr4 = wpr / 4, pitch4 = wsm_pitch4(wpr);
 
+  if constexpr (SMEMW) {             // weights do not depend on the predecessor
+    for (int idx = threadIdx.x; idx < R * 16 * wpr4; idx += kThreads) {
+      const int r = idx / (16 * wpr4), rem = idx - r * 16 * wpr4;
+      const int row = rem / wpr4, c4 = rem - row * wpr4;
+      const bool ok = n0 + row < N;
+      const uint32_t* src = ok ? a.w[r] + (size_t)(n0 + row) * wpr + c4 * 4 : a.w[r];
+      cp_async16(&wsm[(r * 16 + row) * pitch4 + c4], src, ok);
+    }
+    asm volatile("cp.async.commit_group;" ::: "memory");
+  }
+  pdl_trigger();
+  pdl_wait();
   for (int i = threadIdx.x; i < R * 16 * NT * 8; i += kThreads) (&red[0][0][0])[i] = 0;
+  if constexpr (SMEMW) {
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+  }
 
   int acc[R][NT][4];
 #pragma unroll
@@ -81,9 +113,15 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
     uint4 wa[R], wb[R];
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      const uint32_t* W = a.w[r];
-      wa[r] = load_words4(W + (size_t)(n0 + g) * wpr, w0, wpr, n0 + g < N);
-      wb[r] = load_words4(W + (size_t)(n0 + g + 8) * wpr, w0, wpr, n0 + g + 8 < N);
+      if constexpr (SMEMW) {
+        const bool in = w0 < wpr;    // wpr % 4 == 0: a 16-byte group is all in or all out
+        wa[r] = in ? wsm[(r * 16 + g) * pitch4 + (w0 >> 2)] : make_uint4(0u, 0u, 0u, 0u);
+        wb[r] = in ? wsm[(r * 16 + g + 8) * pitch4 + (w0 >> 2)] : make_uint4(0u, 0u, 0u, 0u);
+      } else {
+        const uint32_t* W = a.w[r];
+        wa[r] = load_words4(W + (size_t)(n0 + g) * wpr, w0, wpr, n0 + g < N);
+        wb[r] = load_words4(W + (size_t)(n0 + g + 8) * wpr, w0, wpr, n0 + g + 8 < N);
+      }
     }
     uint4 act[NT][4];
 #pragma unroll
@@ -180,20 +218,32 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
   }
 }
 
+template <int NT, int R, Epi EPI, typename T>
+cudaError_t launch_one(const TGemmArgs& a, cudaStream_t stream) {
+  dim3 grid(ceil_div(a.N, 16), ceil_div(a.M, NT * 8));
+  const int wpr = a.K / 16;
+  const size_t smem = (size_t)R * 16 * wsm_pitch4(wpr) * 16;
+  if (wpr % 4 == 0 && smem <= 100 * 1024) {
+    auto kern = tgemm_mma_kernel<NT, R, EPI, T, true>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(kern, grid, dim3(kThreads), smem, stream, a);
+  }
+  return launch_pdl(tgemm_mma_kernel<NT, R, EPI, T, false>, grid, dim3(kThreads), 0, stream, a);
+}
+
 template <int NT, typename T>
 cudaError_t launch_nt(const TGemmArgs& a, Epi epi, cudaStream_t stream) {
-  dim3 grid(ceil_div(a.N, 16), ceil_div(a.M, NT * 8));
   switch (epi) {
     case Epi::kStore:
-      if (a.nseg == 1) tgemm_mma_kernel<NT, 1, Epi::kStore, T><<<grid, kThreads, 0, stream>>>(a);
-      else if (a.nseg == 2) tgemm_mma_kernel<NT, 2, Epi::kStore, T><<<grid, kThreads, 0, stream>>>(a);
-      else tgemm_mma_kernel<NT, 3, Epi::kStore, T><<<grid, kThreads, 0, stream>>>(a);
-      break;
-    case Epi::kAcc: tgemm_mma_kernel<NT, 1, Epi::kAcc, T><<<grid, kThreads, 0, stream>>>(a); break;
-    case Epi::kScanStep: tgemm_mma_kernel<NT, 3, Epi::kScanStep, T><<<grid, kThreads, 0, stream>>>(a); break;
-    case Epi::kGlu: tgemm_mma_kernel<NT, 2, Epi::kGlu, T><<<grid, kThreads, 0, stream>>>(a); break;
+      if (a.nseg == 1) return launch_one<NT, 1, Epi::kStore, T>(a, stream);
+      if (a.nseg == 2) return launch_one<NT, 2, Epi::kStore, T>(a, stream);
+      return launch_one<NT, 3, Epi::kStore, T>(a, stream);
+    case Epi::kAcc: return launch_one<NT, 1, Epi::kAcc, T>(a, stream);
+    case Epi::kScanStep: return launch_one<NT, 3, Epi::kScanStep, T>(a, stream);
+    case Epi::kGlu: return launch_one<NT, 2, Epi::kGlu, T>(a, stream);
   }
-  return cudaGetLastError();
+  return cudaErrorInvalidValue;
 }
 
 template <typename T>
