@@ -83,11 +83,11 @@ def dist_env():
     return world, rank, local
 
 
-def dist_init(world):
+def dist_init(world, backend="nccl"):
     if world > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
 
 
 def barrier(world):
@@ -97,12 +97,19 @@ def barrier(world):
 
 
 def max_over_ranks(v: float, world: int) -> float:
+    """Max of a per-rank value over all ranks (the whole job is as slow as its slowest rank)."""
     if world == 1:
         return v
     import torch.distributed as dist
-    t = torch.tensor([v], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_total_ms: float) -> float:
+    """Units per second of the whole job: every rank's units over the slowest rank's time."""
+    return world * units_per_rank_step * steps / (max_total_ms / 1e3)
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -304,7 +311,7 @@ def run_mmf(args):
     total_ms = max_over_ranks(sum(step_ms), world)
     ms_per_step = total_ms / args.steps
     tokens_per_step = w.batch * w.seq
-    value = world * tokens_per_step * args.steps / (total_ms / 1e3)
+    value = whole_job_rate(world, tokens_per_step, args.steps, total_ms)
 
     # dominant kernel: the ternary contraction (tensor-bound)
     gemm_names = [k for k in prof if k.startswith("tgemm")]
@@ -341,7 +348,7 @@ def run_mmf(args):
         barrier(world)
         e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), world)
         nbytes = x_pin.numel() * x_pin.element_size()
-        e2e = {"value": world * tokens_per_step * args.steps / (e2e_ms / 1e3), "unit": "tokens/s",
+        e2e = {"value": whole_job_rate(world, tokens_per_step, args.steps, e2e_ms), "unit": "tokens/s",
                "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
 
     cpu = None
