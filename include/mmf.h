@@ -144,6 +144,9 @@ mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_dtype dtype,
 /* MLGRU scan                                                                 */
 /* ------------------------------------------------------------------------- */
 
+/* Scratch bytes mmf_mlgru_scan needs for B sequences of T tokens and d channels. */
+size_t mmf_mlgru_scan_ws_size(int32_t B, int32_t T, int32_t d);
+
 /* MLGRU gates and gated recurrence over T tokens for B sequences.
  * [DC] "Core components: MLGRU and GLU" (token-by-token update of a hidden
  * state through element-wise gates valued in [0,1]); [HL] "HGRN attention".
@@ -153,10 +156,14 @@ mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_dtype dtype,
  *   pre (device) [B, T, 3, d] in dtype: for each token the rows f~, c~, g~
  *   h   (device) float [B, d]: h_0 on entry, h_T on return (in place)
  *   o   (device) [B, T, d] in dtype: o'
+ *   ws  (device) scratch of mmf_mlgru_scan_ws_size(B, T, d) bytes.
+ * The sequence is split into chunks processed in parallel; a chunk takes its
+ * entering state from the previous chunk through a bounded wait (a timeout is
+ * reported by mmf_check as MMF_ERR_TIMEOUT).
  * T = 0 leaves h unchanged. Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d % 8),
- * MISALIGNED, CUDA. */
+ * MISALIGNED, WORKSPACE, CUDA. */
 mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
-                          float* h, void* o, void* stream);
+                          float* h, void* o, void* ws, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* MatMul-free GLU                                                            */

@@ -113,7 +113,7 @@ def bitlinear(lin: TLinear, x: torch.Tensor, eps: float = DEFAULT_EPS, debug: bo
     return y
 
 
-def mlgru_scan(pre: torch.Tensor, h: torch.Tensor) -> torch.Tensor:
+def mlgru_scan(pre: torch.Tensor, h: torch.Tensor, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """pre [B, T, 3, d] -> o' [B, T, d]; h [B, d] fp32 is updated in place to h_T."""
     _need_cuda(pre, h)
     if pre.dim() != 4 or pre.shape[2] != 3:
@@ -123,8 +123,9 @@ def mlgru_scan(pre: torch.Tensor, h: torch.Tensor) -> torch.Tensor:
         raise ValueError("h must be float32 [B, d]")
     o = torch.empty(B, T, d, dtype=pre.dtype, device=pre.device)
     lib = L.load()
-    L.check(lib.mmf_mlgru_scan(_vp(pre), _dtype(pre), B, T, d, _vp(h), _vp(o), _stream(pre.device)),
-            "mmf_mlgru_scan")
+    w = _workspace(lib.mmf_mlgru_scan_ws_size(B, T, d), pre.device, ws)
+    L.check(lib.mmf_mlgru_scan(_vp(pre), _dtype(pre), B, T, d, _vp(h), _vp(o), _vp(w), w.numel() * w.element_size(),
+                               _stream(pre.device)), "mmf_mlgru_scan")
     return o
 
 

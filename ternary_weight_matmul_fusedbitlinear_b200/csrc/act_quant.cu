@@ -141,14 +141,6 @@ __device__ __forceinline__ void unpack8(const uint4 (&r)[2], float (&v)[8]) {
   }
 }
 
-// Four int32 codes -> four saturated int8 bytes in memory order c0..c3.
-__device__ __forceinline__ uint32_t pack4_sat(int c0, int c1, int c2, int c3) {
-  uint32_t hi, w;
-  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(c3), "r"(c2));
-  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(w) : "r"(c1), "r"(c0), "r"(hi));
-  return w;
-}
-
 template <typename T, int VMAX>
 __device__ __forceinline__ void load_row(const T* __restrict__ xr, int nvec, int lane, uint4 (&raw)[VMAX][Vec16<T>::regs]) {
   constexpr int R = Vec16<T>::regs;

@@ -288,10 +288,10 @@ extern "C" mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_d
   if (ws_bytes < mmf_bitlinear_ws_size(M, lin->K))
     return fail(MMF_ERR_WORKSPACE, "mmf_bitlinear: ws_bytes=%zu < %zu", ws_bytes, mmf_bitlinear_ws_size(M, lin->K));
   cudaStream_t s = as_stream(stream);
+  const mmf_tlinear* segs[1] = {lin};
   Carver c(ws);
   QAct qa = carve_qact(c, M, lin->K);
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, lin->K, lin->gain, eps, qa.q, qa.s, qa.qsum, s); }), "rmsnorm_quant");
-  const mmf_tlinear* segs[1] = {lin};
   TGemmArgs a = gemm_args(segs, 1, qa.q, qa.s, qa.qsum, M, y, lin->N, nullptr, nullptr);
   MMF_CUDA(run_gemm(a, Epi::kStore, dtype, s), "tgemm");
   if (dbg) {
@@ -308,19 +308,27 @@ extern "C" mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_d
 
 // ------------------------------------------------------------------ MLGRU scan
 
+extern "C" size_t mmf_mlgru_scan_ws_size(int32_t B, int32_t T, int32_t d) {
+  if (B < 0 || T < 0 || d < 0) return 0;
+  return mlgru_scan_ws_bytes(B, T, d);
+}
+
 extern "C" mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d, float* h,
-                                     void* o, void* stream) {
+                                     void* o, void* ws, size_t ws_bytes, void* stream) {
   if (!dtype_ok(dtype)) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan: bad dtype");
   if (B < 0 || T < 0 || d < 1) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan: B=%d T=%d d=%d", B, T, d);
   if (d % 8 != 0) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_mlgru_scan: d=%d %% 8 != 0", d);
   if (B == 0 || T == 0) return MMF_OK;
-  if (!pre || !h || !o) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan: null pointer");
-  if (!aligned16(pre) || !aligned16(h) || !aligned16(o)) return fail(MMF_ERR_MISALIGNED, "mmf_mlgru_scan");
+  if (!pre || !h || !o || !ws) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan: null pointer");
+  if (!aligned16(pre) || !aligned16(h) || !aligned16(o) || !aligned16(ws))
+    return fail(MMF_ERR_MISALIGNED, "mmf_mlgru_scan");
+  if (ws_bytes < mlgru_scan_ws_bytes(B, T, d))
+    return fail(MMF_ERR_WORKSPACE, "mmf_mlgru_scan: ws_bytes=%zu < %zu", ws_bytes, mlgru_scan_ws_bytes(B, T, d));
   cudaStream_t s = as_stream(stream);
   int* status = nullptr;
   mmf_status r = device_status_ptr(&status);
   if (r != MMF_OK) return r;
-  MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(pre, dtype, B, T, d, h, o, status, s); }),
+  MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(pre, dtype, B, T, d, h, o, ws, status, s); }),
            "mlgru_scan");
   return MMF_OK;
 }
@@ -495,10 +503,12 @@ struct BlockWs {
   void* p;     // [M, I] GLU product
   void* ping;  // [M, d] stack intermediates
   void* pong;
+  void* scan;  // scan scratch
   size_t bytes;
 };
 
-BlockWs carve_block(void* base, int M, int d, int I, mmf_dtype dt) {
+BlockWs carve_block(void* base, int B, int T, int d, int I, mmf_dtype dt) {
+  const int M = B * T;
   Carver c(base);
   BlockWs w;
   const size_t e = elem_bytes(dt);
@@ -509,6 +519,7 @@ BlockWs carve_block(void* base, int M, int d, int I, mmf_dtype dt) {
   w.p = c.take<char>((size_t)M * I * e);
   w.ping = c.take<char>((size_t)M * d * e);
   w.pong = c.take<char>((size_t)M * d * e);
+  w.scan = c.take<char>(mlgru_scan_ws_bytes(B, T, d));
   w.bytes = c.off + 256;
   return w;
 }
@@ -530,7 +541,7 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
     int* status = nullptr;
     mmf_status r = device_status_ptr(&status);
     if (r != MMF_OK) return r;
-    MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, status, s); }),
+    MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, w.scan, status, s); }),
              "block scan");
   }
   MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.og, dt, M, d, W.o.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant o'");
@@ -565,7 +576,7 @@ mmf_status check_forward_args(const mmf_block* blk, mmf_state* st, const void* x
 
 extern "C" size_t mmf_block_ws_size(const mmf_block* blk, int32_t B, int32_t T) {
   if (!blk || B < 0 || T < 0) return 0;
-  return carve_block(nullptr, B * T, blk->d, blk->I, MMF_F32).bytes;
+  return carve_block(nullptr, B, T, blk->d, blk->I, MMF_F32).bytes;
 }
 
 extern "C" mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf_state* st, const void* x, void* y,
@@ -575,7 +586,7 @@ extern "C" mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf
   if (r != MMF_OK) return r;
   if (layer < 0 || layer >= st->L) return fail(MMF_ERR_INVALID_ARG, "mmf_block_forward: layer %d of %d", layer, st->L);
   if (T == 0) return MMF_OK;
-  BlockWs w = carve_block(ws, B * T, blk->d, blk->I, dtype);
+  BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype);
   if (ws_bytes < mmf_block_ws_size(blk, B, T))
     return fail(MMF_ERR_WORKSPACE, "mmf_block_forward: ws_bytes=%zu < %zu", ws_bytes, mmf_block_ws_size(blk, B, T));
   return block_forward_impl(blk, mmf_state_layer(st, layer), x, y, B, T, dtype, eps, w, as_stream(stream));
@@ -599,7 +610,7 @@ extern "C" mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t 
   cudaStream_t s = as_stream(stream);
   const void* cur = x;
   for (int l = 0; l < L; ++l) {
-    BlockWs w = carve_block(ws, B * T, blocks[l]->d, blocks[l]->I, dtype);
+    BlockWs w = carve_block(ws, B, T, blocks[l]->d, blocks[l]->I, dtype);
     void* dst = (l == L - 1) ? y : ((l % 2 == 0) ? w.ping : w.pong);
     mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), cur, dst, B, T, dtype, eps, w, s);
     if (r != MMF_OK) return r;

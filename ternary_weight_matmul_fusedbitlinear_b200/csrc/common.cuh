@@ -56,6 +56,14 @@ __device__ __forceinline__ void store8(float* p, const float v[8]) {
   *reinterpret_cast<float4*>(p + 4) = make_float4(v[4], v[5], v[6], v[7]);
 }
 
+// Four int32 codes -> four saturated int8 bytes in memory order c0..c3.
+__device__ __forceinline__ uint32_t pack4_sat(int c0, int c1, int c2, int c3) {
+  uint32_t hi, w;
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, 0;" : "=r"(hi) : "r"(c3), "r"(c2));
+  asm("cvt.pack.sat.s8.s32.b32 %0, %1, %2, %3;" : "=r"(w) : "r"(c1), "r"(c0), "r"(hi));
+  return w;
+}
+
 // ---------------------------------------------------------------- gates
 // sigmoid(z) = 1 / (1 + e^-z); e^-z overflows to +inf for very negative z and
 // the reciprocal then gives exactly 0, which is the limit.

@@ -71,6 +71,8 @@ struct TGemmArgs {
   float* h;                 // kScanStep: [M, N] fp32 state, updated in place
 };
 
+
+
 // mma.sync-based contraction (weights as the 16-row A operand, tokens as N=8 tiles).
 cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t stream);
 
@@ -79,7 +81,10 @@ cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStre
 bool tgemm_tc_supported(const TGemmArgs& a, Epi epi);
 cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
 
-cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, int* status,
-                              cudaStream_t stream);
+// Chunk-parallel MLGRU scan; `ws` holds mlgru_scan_ws_bytes(B, T, d) bytes of
+// per-launch scratch (ticket counter, chunk flags, chunk carries).
+size_t mlgru_scan_ws_bytes(int B, int T, int d);
+cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, void* ws,
+                              int* status, cudaStream_t stream);
 
 }  // namespace mmf

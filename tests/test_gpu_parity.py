@@ -64,6 +64,20 @@ def test_bitlinear_parity(k, n, m, dtype):
     assert_close(to_np(y), y_ref, dtype, "y")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("k,n,m", SWEEP + [(48, 37, 3), (272, 130, 9), (6912, 2560, 16), (1024, 64, 11)])
+def test_bitlinear_gain_parity_no_debug(k, n, m, dtype):
+    # decode-sized calls without debug outputs, with a non-trivial RMSNorm gain
+    W, lin, olin = make_layer(600 + k + n, n, k)
+    gain = torch.linspace(0.5, 1.5, k)
+    lin = mmf.TLinear(lin.packed, lin.gamma, n, k, gain=gain.cuda())
+    olin = O.TLinear(olin.codes, olin.gamma, gain.numpy())
+    x = synth.activations(601 + m, m, k, TORCH_DT[dtype], outlier_p=synth.GEMV_OUTLIER_P,
+                          outlier_scale=synth.GEMV_OUTLIER_SCALE)
+    y = mmf.bitlinear(lin, x.cuda())
+    assert_close(to_np(y), O.bitlinear(to_np(x), olin), dtype, "y (gain)")
+
+
 def test_bitlinear_empty_and_gain_bias():
     k, n = 64, 40
     W, lin, olin = make_layer(17, n, k)
