@@ -329,27 +329,55 @@ def run_mmf(args):
                 "per_kernel_ms": {k: round(v[1] / args.steps, 4) for k, v in prof.items()}}
 
     # ------------------------------------------------------------ end to end through the public API
+    # Every step's input is copied from pinned host memory and its output copied
+    # back, all inside the timed region; the copies run on their own streams so
+    # step i+1's upload and step i-1's download overlap step i's kernels
+    # (double-buffered device input/output).
     e2e = None
     if not args.no_e2e:
-        x_pin = x_host.pin_memory()
-        y_pin = torch.empty_like(x_pin).pin_memory()
-        e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
-        e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+        x_pin = [x_host.pin_memory(), x_host.clone().pin_memory()]
+        y_pin = [torch.empty_like(x_host).pin_memory() for _ in range(2)]
+        x_d = [x, torch.empty_like(x)]
+        y_d = [y, torch.empty_like(y)]
+        h2d, d2h = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        up = [torch.cuda.Event() for _ in range(args.steps)]
+        done = [torch.cuda.Event() for _ in range(args.steps)]
+        down = [torch.cuda.Event() for _ in range(args.steps)]
+        t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         barrier(world)
         torch.cuda.synchronize()
+        t0.record(stream)
+        h2d.wait_stream(stream)
+        d2h.wait_stream(stream)
+        with torch.cuda.stream(h2d):
+            x_d[0].copy_(x_pin[0], non_blocking=True)
+            up[0].record(h2d)
         for i in range(args.steps):
-            flush.zero_()
-            e_s[i].record(stream)
-            x.copy_(x_pin, non_blocking=True)
-            step(x, y)
-            y_pin.copy_(y, non_blocking=True)
-            e_e[i].record(stream)
+            b = i % 2
+            if i + 1 < args.steps:
+                with torch.cuda.stream(h2d):
+                    if i >= 1:
+                        h2d.wait_event(done[i - 1])        # step i-1 has finished reading x_d[(i+1)%2]
+                    x_d[(i + 1) % 2].copy_(x_pin[(i + 1) % 2], non_blocking=True)
+                    up[i + 1].record(h2d)
+            stream.wait_event(up[i])
+            if i >= 2:
+                stream.wait_event(down[i - 2])            # y_d[b] has been copied out
+            step(x_d[b], y_d[b])
+            done[i].record(stream)
+            with torch.cuda.stream(d2h):
+                d2h.wait_event(done[i])
+                y_pin[b].copy_(y_d[b], non_blocking=True)
+                down[i].record(d2h)
+        stream.wait_event(down[args.steps - 1])
+        t1.record(stream)
         torch.cuda.synchronize()
         barrier(world)
-        e2e_ms = max_over_ranks(sum(s.elapsed_time(e) for s, e in zip(e_s, e_e)), world)
-        nbytes = x_pin.numel() * x_pin.element_size()
+        e2e_ms = max_over_ranks(t0.elapsed_time(t1), world)
+        nbytes = x_host.numel() * x_host.element_size()
         e2e = {"value": whole_job_rate(world, tokens_per_step, args.steps, e2e_ms), "unit": "tokens/s",
-               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes}
+               "h2d_bytes_per_step": nbytes, "d2h_bytes_per_step": nbytes,
+               "note": "copies on side streams overlap neighbouring steps; all inside the timed region"}
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -124,10 +124,13 @@ cudaError_t timed(const char* name, cudaStream_t s, F&& launch) {
   return e;
 }
 
-// Contraction dispatch: the tcgen05 kernel for prefill-sized token counts, the
-// mma.sync kernel for decode-sized ones and for shapes the tcgen05 kernel does
-// not take. MMF_GEMM_PATH=mma|tc|auto (default auto) pins one implementation;
-// both compute the same exact integer accumulators.
+// Contraction dispatch: the single-SM tcgen05 kernel from 128 tokens, the
+// mma.sync kernel for decode-sized token counts and for shapes the tcgen05
+// kernels do not take. The SM-pair tcgen05 kernel (M >= 256) is selected only
+// on request: it is correct but measured slower than the single-SM kernel on
+// the 370M shapes. MMF_GEMM_PATH=mma|tc|tc1|tc2|auto (default auto; tc and tc1
+// both mean the single-SM kernel) pins one implementation; all compute the
+// same exact integer accumulators.
 constexpr int kTcMinTokens = 128;
 
 int gemm_path_pref() {
@@ -135,6 +138,8 @@ int gemm_path_pref() {
   if (e == nullptr) return 0;
   if (strcmp(e, "mma") == 0) return 1;
   if (strcmp(e, "tc") == 0) return 2;
+  if (strcmp(e, "tc1") == 0) return 3;
+  if (strcmp(e, "tc2") == 0) return 4;
   return 0;
 }
 
@@ -142,12 +147,16 @@ int gemm_path_pref() {
 cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s, const char* what = "") {
   const int pref = gemm_path_pref();
   const bool tc_ok = tgemm_tc_supported(a, epi);
-  const bool use_tc = tc_ok && (pref == 2 || (pref == 0 && a.M >= kTcMinTokens));
+  const bool tc2_ok = tgemm_tc2_supported(a, epi);
+  bool use_tc = tc_ok && (pref >= 2 || (pref == 0 && a.M >= kTcMinTokens));
+  const bool use_tc2 = use_tc && tc2_ok && pref == 4;
   char name[48];
-  snprintf(name, sizeof(name), "%s%s%s", use_tc ? "tgemm_tc" : "tgemm_mma", what[0] ? ":" : "", what);
+  snprintf(name, sizeof(name), "%s%s%s", use_tc2 ? "tgemm_tc2" : (use_tc ? "tgemm_tc" : "tgemm_mma"),
+           what[0] ? ":" : "", what);
   if (use_tc) {
     int* st = nullptr;
     if (device_status_ptr(&st) != MMF_OK) return cudaErrorUnknown;
+    if (use_tc2) return timed(name, s, [&] { return launch_tgemm_tc2(a, epi, dt, st, s); });
     return timed(name, s, [&] { return launch_tgemm_tc(a, epi, dt, st, s); });
   }
   return timed(name, s, [&] { return launch_tgemm_mma(a, epi, dt, s); });

@@ -81,6 +81,10 @@ cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStre
 bool tgemm_tc_supported(const TGemmArgs& a, Epi epi);
 cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
 
+// The same contraction on SM pairs (tcgen05 cta_group::2, 256-token tiles); needs M >= 256.
+bool tgemm_tc2_supported(const TGemmArgs& a, Epi epi);
+cudaError_t launch_tgemm_tc2(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
+
 // Chunk-parallel MLGRU scan; `ws` holds mlgru_scan_ws_bytes(B, T, d) bytes of
 // per-launch scratch (ticket counter, chunk flags, chunk carries).
 size_t mlgru_scan_ws_bytes(int B, int T, int d);

@@ -16,7 +16,7 @@ pytestmark = pytest.mark.gpu
 mmf = pytest.importorskip("ternary_weight_matmul_fusedbitlinear_b200")
 
 
-@pytest.fixture(params=["tc", "mma"])
+@pytest.fixture(params=["tc", "tc2", "mma"])
 def path(request, monkeypatch):
     monkeypatch.setenv("MMF_GEMM_PATH", request.param)
     return request.param
