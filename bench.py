@@ -115,7 +115,7 @@ def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_total
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms during the timed region."""
+    """nvidia-smi clocks and throttle reasons sampled every 50 ms during the timed region."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
@@ -132,7 +132,7 @@ class ClockSampler:
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except OSError:
             self.proc = None
 
@@ -620,6 +620,14 @@ def run_decode(args):
     torch.cuda.synchronize()
     clk = clocks.stop()
     step_ms = e0.elapsed_time(e1) / steps
+    # per-kernel device time of a decode step (eager launches, outside the timed region)
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    for _ in range(5):
+        mmf.stack_forward(blocks, st, x, ws=ws, out=y)
+    torch.cuda.synchronize()
+    mmf.prof_enable(False)
+    per_kernel = {k: round(v[1] / 5, 4) for k, v in mmf.prof_collect().items()}
     weights = w.layers * (4 * w.d * w.d + 3 * w.d * w.inner) / 4.0
     state = 2.0 * w.layers * B * w.d * 4
     gbs = (weights + state) / (step_ms / 1e3) / 1e9
@@ -634,7 +642,8 @@ def run_decode(args):
                        "l2": "weight stream per step > L2"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "decode step (all kernels)",
-                         "bytes_per_step": weights + state, "peak_source": peak_kind},
+                         "bytes_per_step": weights + state, "peak_source": peak_kind,
+                         "per_kernel_ms_eager_step": per_kernel},
             "cpu_baseline": None, "e2e": None, "gpu_launches": w.layers * 8, "clocks": clk}), flush=True)
     return 0
 

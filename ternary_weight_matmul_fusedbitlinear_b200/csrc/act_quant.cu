@@ -141,6 +141,50 @@ __device__ __forceinline__ void unpack8(const uint4 (&r)[2], float (&v)[8]) {
   }
 }
 
+// fp32 bit pattern -> the same value as an fp64, built with integer operations
+// (the conversion instruction issues at a fraction of the ALU rate). Exact for
+// every normal value. Zero and subnormals come out as magnitudes below 2^-126
+// instead; their squares stay below 2^-252 and can move a row's sum only when
+// every element of the row is that small, and then the fp32 mean square
+// underflows to 0 either way.
+__device__ __forceinline__ double f32bits_to_f64(uint32_t u) {
+  const uint32_t a = u & 0x7fffffffu;          // the sign does not matter for a square
+  return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
+}
+
+// Sum of squares of the 8 elements of one raw vector, accumulated in fp64.
+__device__ __forceinline__ void sumsq8(const uint4 (&r)[1], double& ss) {
+  const uint32_t w[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const double a = f32bits_to_f64(w[i] << 16), b = f32bits_to_f64(w[i] & 0xffff0000u);
+    ss = fma(a, a, ss);
+    ss = fma(b, b, ss);
+  }
+}
+__device__ __forceinline__ void sumsq8(const uint4 (&r)[2], double& ss) {
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t w[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const double a = f32bits_to_f64(w[k]);
+      ss = fma(a, a, ss);
+    }
+  }
+}
+
+// rint(t) for |t| < 2^22 by adding 1.5 * 2^23: the sum's unit in the last
+// place is 1, so the fp32 add rounds t half-to-even to an integer, and the
+// sum's bit pattern is 0x4B400000 + rint(t) with rint(t) in two's complement
+// in the low bits. Returns that bit pattern; its low byte is the int8 code.
+__device__ __forceinline__ uint32_t rint_bits(float t) { return __float_as_uint(__fadd_rn(t, 12582912.0f)); }
+
+// Low bytes of four rint_bits() patterns -> one word, bytes in order a, b, c, d.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
 template <typename T, int VMAX>
 __device__ __forceinline__ void load_row(const T* __restrict__ xr, int nvec, int lane, uint4 (&raw)[VMAX][Vec16<T>::regs]) {
   constexpr int R = Vec16<T>::regs;
@@ -176,12 +220,7 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(const T* __rest
     if (row + nwarps < M) load_row<T, VMAX>(x + (size_t)(row + nwarps) * K, nvec, lane, nxt);
     double ss = 0.0;
 #pragma unroll
-    for (int j = 0; j < VMAX; ++j) {
-      float v[8];
-      unpack8(raw[j], v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) ss = fma((double)v[i], (double)v[i], ss);
-    }
+    for (int j = 0; j < VMAX; ++j) sumsq8(raw[j], ss);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float ms = (float)(ss / (double)K);
@@ -225,11 +264,13 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(const T* __rest
           if (gain != nullptr) h[i] = __fmul_rn(h[i], __ldg(gain + vi * 8 + i));
         }
       }
-      int c[8];
+      // |x^ * s| <= 127 (to within rounding) by the choice of s, so the codes
+      // need no clamp and never reach -128
+      uint32_t c[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) c[i] = __float2int_rn(__fmul_rn(h[i], s));
-      const uint32_t w0 = pack4_sat(c[0], c[1], c[2], c[3]);
-      const uint32_t w1 = pack4_sat(c[4], c[5], c[6], c[7]);
+      for (int i = 0; i < 8; ++i) c[i] = rint_bits(__fmul_rn(h[i], s));
+      const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
+      const uint32_t w1 = pack_low_bytes(c[4], c[5], c[6], c[7]);
       isum = __dp4a((int)w0, 0x01010101, isum);
       isum = __dp4a((int)w1, 0x01010101, isum);
       *reinterpret_cast<uint2*>(qr + (size_t)vi * 8) = make_uint2(w0, w1);
