@@ -13,6 +13,7 @@
 // depend on how the kernel is laid out; only the fp64 sum's order could, and
 // it is fixed here (per-thread strided order, xor-shuffle tree, warps in order).
 #include "kernels.cuh"
+#include "tma.cuh"
 
 namespace mmf {
 
@@ -105,73 +106,25 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_quant_kernel(const T* __rest
   }
 }
 
-// One warp per token row, the row held in registers as raw 16-byte vectors
-// (8 elements each): lane l owns vectors j*32 + l, j < VMAX, so every load and
-// every code store of the warp is one contiguous span. Same fp32 steps as the
-// CTA-per-row kernel; reductions are warp shuffles only.
-template <typename T>
-struct Vec16;
-template <>
-struct Vec16<bf16> {
-  using raw = uint4;   // 8 bf16
-  static constexpr int regs = 1;
-};
-template <>
-struct Vec16<float> {
-  using raw = uint4;   // 4 floats; two raws per 8 elements
-  static constexpr int regs = 2;
-};
+// ---------------------------------------------------------------- staged warp-per-row kernel
+// One warp per token row. Each warp keeps a ring of `slots` row buffers in
+// shared memory and fills them with 1-D bulk copies (cp.async.bulk, one per
+// row), so the next rows stream in while the current one is reduced; the row
+// itself is read from shared memory in 16-byte vectors (lane l takes vectors
+// l, l+32, ...), twice or three times, never from HBM again.
+// Pass 1 sums the squares in fp64 and takes the largest |x|. Without a gain
+// vector that already fixes the scale: rounding is monotone, so
+// fl(max|x| * rinv) = max fl(|x| * rinv) = max|x^|. With a gain vector a
+// second pass takes max|(x * rinv) * gain|. The last pass writes the codes.
 
-__device__ __forceinline__ void unpack8(const uint4 (&r)[1], float (&v)[8]) {
-  const __nv_bfloat162* h = reinterpret_cast<const __nv_bfloat162*>(&r[0]);
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    float2 f = __bfloat1622float2(h[i]);
-    v[2 * i] = f.x;
-    v[2 * i + 1] = f.y;
-  }
-}
-__device__ __forceinline__ void unpack8(const uint4 (&r)[2], float (&v)[8]) {
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    v[4 * i + 0] = __uint_as_float(r[i].x);
-    v[4 * i + 1] = __uint_as_float(r[i].y);
-    v[4 * i + 2] = __uint_as_float(r[i].z);
-    v[4 * i + 3] = __uint_as_float(r[i].w);
-  }
-}
-
-// fp32 bit pattern -> the same value as an fp64, built with integer operations
-// (the conversion instruction issues at a fraction of the ALU rate). Exact for
-// every normal value. Zero and subnormals come out as magnitudes below 2^-126
-// instead; their squares stay below 2^-252 and can move a row's sum only when
-// every element of the row is that small, and then the fp32 mean square
-// underflows to 0 either way.
-__device__ __forceinline__ double f32bits_to_f64(uint32_t u) {
-  const uint32_t a = u & 0x7fffffffu;          // the sign does not matter for a square
+// fp32 bit pattern (sign cleared) -> the same value as an fp64, built with
+// integer operations (the conversion instruction issues at a fraction of the
+// ALU rate). Exact for every normal value. Zero and subnormals come out as
+// magnitudes below 2^-126 instead; their squares stay below 2^-252 and can
+// move a row's sum only when every element of the row is that small, and then
+// the fp32 mean square underflows to 0 either way.
+__device__ __forceinline__ double magbits_to_f64(uint32_t a) {
   return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
-}
-
-// Sum of squares of the 8 elements of one raw vector, accumulated in fp64.
-__device__ __forceinline__ void sumsq8(const uint4 (&r)[1], double& ss) {
-  const uint32_t w[4] = {r[0].x, r[0].y, r[0].z, r[0].w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const double a = f32bits_to_f64(w[i] << 16), b = f32bits_to_f64(w[i] & 0xffff0000u);
-    ss = fma(a, a, ss);
-    ss = fma(b, b, ss);
-  }
-}
-__device__ __forceinline__ void sumsq8(const uint4 (&r)[2], double& ss) {
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint32_t w[4] = {r[i].x, r[i].y, r[i].z, r[i].w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-      const double a = f32bits_to_f64(w[k]);
-      ss = fma(a, a, ss);
-    }
-  }
 }
 
 // rint(t) for |t| < 2^22 by adding 1.5 * 2^23: the sum's unit in the last
@@ -185,136 +138,225 @@ __device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint3
   return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
 }
 
-template <typename T, int VMAX>
-__device__ __forceinline__ void load_row(const T* __restrict__ xr, int nvec, int lane, uint4 (&raw)[VMAX][Vec16<T>::regs]) {
-  constexpr int R = Vec16<T>::regs;
-#pragma unroll
-  for (int j = 0; j < VMAX; ++j) {
-    const int vi = j * 32 + lane;
-#pragma unroll
-    for (int r = 0; r < R; ++r)
-      raw[j][r] = vi < nvec ? __ldg(reinterpret_cast<const uint4*>(xr + (size_t)vi * 8) + r) : make_uint4(0, 0, 0, 0);
+// Per element type: E elements per 16-byte vector, their fp32 magnitude bits
+// and values.
+template <typename T>
+struct Vec;
+template <>
+struct Vec<bf16> {
+  static constexpr int E = 8;
+  __device__ __forceinline__ static uint32_t mag(const uint4& r, int i) {
+    const uint32_t w = (&r.x)[i >> 1];
+    return (i & 1) ? (w & 0x7fff0000u) : ((w << 16) & 0x7fffffffu);
   }
+  __device__ __forceinline__ static float val(const uint4& r, int i) {
+    const uint32_t w = (&r.x)[i >> 1];
+    return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+  __device__ __forceinline__ static void store_codes(int8_t* p, const uint32_t (&c)[8], int& isum) {
+    const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
+    const uint32_t w1 = pack_low_bytes(c[4], c[5], c[6], c[7]);
+    isum = __dp4a((int)w0, 0x01010101, isum);
+    isum = __dp4a((int)w1, 0x01010101, isum);
+    *reinterpret_cast<uint2*>(p) = make_uint2(w0, w1);
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int E = 4;
+  __device__ __forceinline__ static uint32_t mag(const uint4& r, int i) { return (&r.x)[i] & 0x7fffffffu; }
+  __device__ __forceinline__ static float val(const uint4& r, int i) { return __uint_as_float((&r.x)[i]); }
+  __device__ __forceinline__ static void store_codes(int8_t* p, const uint32_t (&c)[4], int& isum) {
+    const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
+    isum = __dp4a((int)w0, 0x01010101, isum);
+    *reinterpret_cast<uint32_t*>(p) = w0;
+  }
+};
+
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
 }
 
-// Persistent: each warp walks rows warp_id, warp_id + nwarps, ... and issues
-// the loads of its next row before reducing the current one, so the row's
-// HBM latency overlaps the previous row's arithmetic.
-template <typename T, int VMAX>
-__global__ void __launch_bounds__(256) rmsnorm_quant_warp_kernel(const T* __restrict__ x, int M, int K,
-                                                                 const float* __restrict__ gain, float eps,
-                                                                 int8_t* __restrict__ q, float* __restrict__ scale,
-                                                                 int32_t* __restrict__ qsum) {
-  constexpr int R = Vec16<T>::regs;
-  constexpr bool kKeep = VMAX <= 8;   // keep x^ in registers between the max and the codes
-  const int lane = threadIdx.x & 31;
-  const int nwarps = gridDim.x * 8;
-  int row = blockIdx.x * 8 + (threadIdx.x >> 5);
+// Bounded wait on a row buffer (all lanes); false after the time limit, with
+// status code 1 recorded when a status word is given.
+__device__ __forceinline__ bool slot_wait(uint64_t* bar, uint32_t parity, int* status) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (clock64() - t0 > kWaitCycles) {
+      if (status && (threadIdx.x & 31) == 0) atomicExch(status, 1);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <typename T, bool GAIN>
+__global__ void __launch_bounds__(256) rmsnorm_quant_staged_kernel(const T* __restrict__ x, int M, int K,
+                                                                   const float* __restrict__ gain, float eps,
+                                                                   int8_t* __restrict__ q, float* __restrict__ scale,
+                                                                   int32_t* __restrict__ qsum, int slots,
+                                                                   int stride, int* status) {
+  using V = Vec<T>;
+  constexpr int E = V::E;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int warps = blockDim.x >> 5;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* ring = base + (size_t)warp * slots * stride;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(base + (size_t)warps * slots * stride) + warp * slots;
+  const int nwarps = gridDim.x * warps;
+  const int row0 = blockIdx.x * warps + warp;
+  const uint32_t row_bytes = (uint32_t)K * sizeof(T);
+  const int nvec = (int)(row_bytes / 16);
+
+  if (lane == 0) {
+    for (int s = 0; s < slots; ++s) mbar_init(&bars[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncwarp();
   pdl_trigger();
-  pdl_wait();
-  if (row >= M) return;
-  const int nvec = K / 8;
-  uint4 raw[VMAX][R], nxt[VMAX][R];
-  load_row<T, VMAX>(x + (size_t)row * K, nvec, lane, raw);
-  for (; row < M; row += nwarps) {
-    if (row + nwarps < M) load_row<T, VMAX>(x + (size_t)(row + nwarps) * K, nvec, lane, nxt);
+  pdl_wait();   // x is the previous kernel's output
+  if (lane == 0) {
+    for (int s = 0; s < slots; ++s) {
+      const int r = row0 + s * nwarps;
+      if (r >= M) break;
+      mbar_arrive_expect_tx(&bars[s], row_bytes);
+      bulk_load(ring + (size_t)s * stride, x + (size_t)r * K, row_bytes, &bars[s]);
+    }
+  }
+
+  int k = 0;
+  for (int row = row0; row < M; row += nwarps, ++k) {
+    const int s = k % slots;
+    if (!slot_wait(&bars[s], (uint32_t)(k / slots) & 1u, status)) {
+      // give up on this warp's rows; let the copies in flight land (bounded)
+      if (lane == 0)
+        for (int i = 1; i < slots; ++i) {
+          const int si = (k + i) % slots;
+          if (row + i * nwarps < M) slot_wait(&bars[si], (uint32_t)((k + i) / slots) & 1u, nullptr);
+        }
+      return;
+    }
+    const uint4* v = reinterpret_cast<const uint4*>(ring + (size_t)s * stride);
+
+    // pass 1: sum of squares (fp64) and max |x|
     double ss = 0.0;
+    uint32_t am = 0;
+#pragma unroll 4
+    for (int vi = lane; vi < nvec; vi += 32) {
+      const uint4 r = v[vi];
 #pragma unroll
-    for (int j = 0; j < VMAX; ++j) sumsq8(raw[j], ss);
+      for (int i = 0; i < E; ++i) {
+        const uint32_t a = V::mag(r, i);
+        am = max(am, a);
+        const double xd = magbits_to_f64(a);
+        ss = fma(xd, xd, ss);
+      }
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     const float ms = (float)(ss / (double)K);
     const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
 
-    float xh[kKeep ? VMAX : 1][8];
-    float amax = 0.0f;
+    float amax;
+    if constexpr (GAIN) {   // pass 2: max |(x * rinv) * gain|
+      uint32_t hm = 0;
+#pragma unroll 4
+      for (int vi = lane; vi < nvec; vi += 32) {
+        const uint4 r = v[vi];
 #pragma unroll
-    for (int j = 0; j < VMAX; ++j) {
-      const int vi = j * 32 + lane;
-      float v[8];
-      unpack8(raw[j], v);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        float h = __fmul_rn(v[i], rinv);
-        if (gain != nullptr && vi < nvec) h = __fmul_rn(h, __ldg(gain + vi * 8 + i));
-        amax = fmaxf(amax, fabsf(h));
-        if constexpr (kKeep) xh[j][i] = h;
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-    const float s = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
-
-    int isum = 0;
-    int8_t* qr = q + (size_t)row * K;
-#pragma unroll
-    for (int j = 0; j < VMAX; ++j) {
-      const int vi = j * 32 + lane;
-      if (vi >= nvec) break;
-      float h[8];
-      if constexpr (kKeep) {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) h[i] = xh[j][i];
-      } else {
-        float v[8];
-        unpack8(raw[j], v);
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          h[i] = __fmul_rn(v[i], rinv);
-          if (gain != nullptr) h[i] = __fmul_rn(h[i], __ldg(gain + vi * 8 + i));
+        for (int i = 0; i < E; ++i) {
+          const float hv = __fmul_rn(__fmul_rn(V::val(r, i), rinv), __ldg(gain + vi * E + i));
+          hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
         }
       }
-      // |x^ * s| <= 127 (to within rounding) by the choice of s, so the codes
-      // need no clamp and never reach -128
-      uint32_t c[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) c[i] = rint_bits(__fmul_rn(h[i], s));
-      const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
-      const uint32_t w1 = pack_low_bytes(c[4], c[5], c[6], c[7]);
-      isum = __dp4a((int)w0, 0x01010101, isum);
-      isum = __dp4a((int)w1, 0x01010101, isum);
-      *reinterpret_cast<uint2*>(qr + (size_t)vi * 8) = make_uint2(w0, w1);
+      amax = __uint_as_float(__reduce_max_sync(0xffffffffu, hm));
+    } else {
+      amax = __fmul_rn(__uint_as_float(__reduce_max_sync(0xffffffffu, am)), rinv);
     }
+    const float sc = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+
+    // last pass: codes (|x^ * s| <= 127 up to rounding, so no clamp is needed
+    // and -128 never occurs) and their sum
+    int isum = 0;
+    int8_t* qr = q + (size_t)row * K;
+#pragma unroll 4
+    for (int vi = lane; vi < nvec; vi += 32) {
+      const uint4 r = v[vi];
+      uint32_t c[E];
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+      for (int i = 0; i < E; ++i) {
+        float hv = __fmul_rn(V::val(r, i), rinv);
+        if constexpr (GAIN) hv = __fmul_rn(hv, __ldg(gain + vi * E + i));
+        c[i] = rint_bits(__fmul_rn(hv, sc));
+      }
+      V::store_codes(qr + (size_t)vi * E, c, isum);
+    }
+    isum = __reduce_add_sync(0xffffffffu, isum);
     if (lane == 0) {
-      scale[row] = s;
+      scale[row] = sc;
       qsum[row] = isum;
     }
-#pragma unroll
-    for (int j = 0; j < VMAX; ++j)
-#pragma unroll
-      for (int r = 0; r < R; ++r) raw[j][r] = nxt[j][r];
+
+    // refill this buffer with the row `slots` rows ahead
+    __syncwarp();
+    if (lane == 0) {
+      const int nr = row + slots * nwarps;
+      if (nr < M) {
+        fence_proxy_async_smem();
+        mbar_arrive_expect_tx(&bars[s], row_bytes);
+        bulk_load(ring + (size_t)s * stride, x + (size_t)nr * K, row_bytes, &bars[s]);
+      }
+    }
   }
 }
 
-template <typename T, int VMAX>
-void launch_warp(const void* x, int M, int K, const float* gain, float eps, int8_t* q, float* scale, int32_t* qsum,
-                 cudaStream_t stream) {
-  auto kern = rmsnorm_quant_warp_kernel<T, VMAX>;
+// Geometry of the staged kernel for one row length; false when a row does not fit.
+struct StagedGeom {
+  int warps, slots, stride;
+  size_t smem;
+};
+bool staged_geometry(int K, int esize, StagedGeom& g) {
+  g.stride = (K * esize + 127) / 128 * 128;
+  constexpr int kBudget = 200 * 1024;   // shared memory per CTA
+  g.warps = 2 * 8 * g.stride <= kBudget ? 8 : 4;
+  if (2 * g.warps * g.stride > kBudget) return false;
+  g.slots = std::max(2, std::min(4, (96 * 1024) / (g.warps * g.stride)));
+  g.smem = (size_t)g.warps * g.slots * g.stride + sizeof(uint64_t) * g.warps * g.slots + 128;
+  return true;
+}
+
+template <typename T, bool GAIN>
+cudaError_t launch_staged(const StagedGeom& g, const void* x, int M, int K, const float* gain, float eps, int8_t* q,
+                          float* scale, int32_t* qsum, int* status, cudaStream_t stream) {
+  auto kern = rmsnorm_quant_staged_kernel<T, GAIN>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
+  if (e != cudaSuccess) return e;
   int per_sm = 1;
-  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, 256, 0);
-  const int grid = std::max(1, std::min(ceil_div(M, 8), num_sms() * std::max(per_sm, 1)));
-  launch_pdl(kern, dim3(grid), dim3(256), 0, stream, static_cast<const T*>(x), M, K, gain, eps, q, scale, qsum);
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.warps * 32, g.smem);
+  const int grid = std::max(1, std::min(ceil_div(M, g.warps), num_sms() * std::max(per_sm, 1)));
+  return launch_pdl(kern, dim3(grid), dim3(g.warps * 32), g.smem, stream, static_cast<const T*>(x), M, K, gain, eps,
+                    q, scale, qsum, g.slots, g.stride, status);
 }
 
 }  // namespace
 
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
-                                 int8_t* q, float* scale, int32_t* qsum, cudaStream_t stream) {
+                                 int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream) {
   if (M == 0) return cudaSuccess;
-  // warp-per-row kernels while two rows fit in registers (K / 256 vectors per lane)
-  const int vpl = ceil_div(K / 8, 32);
-  if (dt == MMF_BF16 && vpl <= 12) {
-    if (vpl <= 4) launch_warp<bf16, 4>(x, M, K, gain, eps, q, scale, qsum, stream);
-    else if (vpl <= 8) launch_warp<bf16, 8>(x, M, K, gain, eps, q, scale, qsum, stream);
-    else launch_warp<bf16, 12>(x, M, K, gain, eps, q, scale, qsum, stream);
-    return cudaGetLastError();
+  StagedGeom g;
+  if (staged_geometry(K, dt == MMF_BF16 ? 2 : 4, g)) {
+    if (dt == MMF_BF16)
+      return gain ? launch_staged<bf16, true>(g, x, M, K, gain, eps, q, scale, qsum, status, stream)
+                  : launch_staged<bf16, false>(g, x, M, K, gain, eps, q, scale, qsum, status, stream);
+    return gain ? launch_staged<float, true>(g, x, M, K, gain, eps, q, scale, qsum, status, stream)
+                : launch_staged<float, false>(g, x, M, K, gain, eps, q, scale, qsum, status, stream);
   }
-  if (dt == MMF_F32 && vpl <= 4) {
-    launch_warp<float, 4>(x, M, K, gain, eps, q, scale, qsum, stream);
-    return cudaGetLastError();
-  }
+  // rows too long for the staged ring: one CTA per row
   const size_t smem = sizeof(float) * (size_t)K;
   if (dt == MMF_BF16) {
     auto kern = rmsnorm_quant_kernel<bf16>;

@@ -162,6 +162,12 @@ cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s, 
   return timed(name, s, [&] { return launch_tgemm_mma(a, epi, dt, s); });
 }
 
+// Device status word for kernels with bounded waits, or null when it cannot be had.
+int* status_word() {
+  int* st = nullptr;
+  return device_status_ptr(&st) == MMF_OK ? st : nullptr;
+}
+
 mmf_status check_tlinear(const mmf_tlinear* l, const char* name) {
   if (l == nullptr) return fail(MMF_ERR_INVALID_ARG, "%s: null layer", name);
   if (l->packed == nullptr || l->gamma == nullptr) return fail(MMF_ERR_INVALID_ARG, "%s: null packed/gamma", name);
@@ -300,7 +306,7 @@ extern "C" mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_d
   const mmf_tlinear* segs[1] = {lin};
   Carver c(ws);
   QAct qa = carve_qact(c, M, lin->K);
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, lin->K, lin->gain, eps, qa.q, qa.s, qa.qsum, s); }), "rmsnorm_quant");
+  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, lin->K, lin->gain, eps, qa.q, qa.s, qa.qsum, status_word(), s); }), "rmsnorm_quant");
   TGemmArgs a = gemm_args(segs, 1, qa.q, qa.s, qa.qsum, M, y, lin->N, nullptr, nullptr);
   MMF_CUDA(run_gemm(a, Epi::kStore, dtype, s), "tgemm");
   if (dbg) {
@@ -337,7 +343,11 @@ extern "C" mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B
   int* status = nullptr;
   mmf_status r = device_status_ptr(&status);
   if (r != MMF_OK) return r;
-  MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(pre, dtype, B, T, d, h, o, ws, status, s); }),
+  MMF_CUDA(timed("mlgru_scan", s,
+                 [&] {
+                   cudaError_t e = reset_mlgru_scan_ws(ws, B, T, d, s);
+                   return e != cudaSuccess ? e : launch_mlgru_scan(pre, dtype, B, T, d, h, o, ws, status, s);
+                 }),
            "mlgru_scan");
   return MMF_OK;
 }
@@ -372,7 +382,7 @@ mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tli
   const mmf_tlinear* gu[2] = {gate, up};
   TGemmArgs a = gemm_args(gu, 2, qx.q, qx.s, qx.qsum, M, p, gate->N, nullptr, nullptr);
   MMF_CUDA(run_gemm(a, Epi::kGlu, dt, s, "gate_up"), "glu gate/up");
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(p, dt, M, down->K, down->gain, eps, qp.q, qp.s, qp.qsum, s); }), "glu quant p");
+  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(p, dt, M, down->K, down->gain, eps, qp.q, qp.s, qp.qsum, status_word(), s); }), "glu quant p");
   const mmf_tlinear* dn[1] = {down};
   TGemmArgs b = gemm_args(dn, 1, qp.q, qp.s, qp.qsum, M, y, down->N, residual, nullptr);
   MMF_CUDA(run_gemm(b, Epi::kStore, dt, s, "down"), "glu down");
@@ -407,7 +417,7 @@ extern "C" mmf_status mmf_glu(const mmf_tlinear* gate, const mmf_tlinear* up, co
   Carver c(ws);
   QAct qa = carve_qact(c, M, std::max(d, I));
   void* p = c.take<char>((size_t)M * I * elem_bytes(dtype));
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, d, gate->gain, eps, qa.q, qa.s, qa.qsum, s); }), "glu quant x");
+  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, d, gate->gain, eps, qa.q, qa.s, qa.qsum, status_word(), s); }), "glu quant x");
   return run_glu(gate, up, down, qa, residual, y, M, dtype, eps, p, qa, s);
 }
 
@@ -538,8 +548,11 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   const int M = B * T, d = blk->d;
   const mmf_block_weights& W = blk->w;
   const mmf_tlinear* fcg[3] = {&W.f, &W.c, &W.g};
+  // prefill: the scan's scratch is reset here, so that fcg projection -> scan
+  // are back-to-back kernels (the scan starts as a programmatic dependent)
+  if (T > 1) MMF_CUDA(timed("mlgru_scan_reset", s, [&] { return reset_mlgru_scan_ws(w.scan, B, T, d, s); }), "block scan reset");
   // token mixer: quantise x once for f, c, g (shared gain)
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dt, M, d, W.f.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant x");
+  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dt, M, d, W.f.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(), s); }), "block quant x");
   if (T == 1) {
     // decode: projections and one recurrence step in one launch; h updated in place
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, h);
@@ -553,12 +566,12 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
     MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, w.scan, status, s); }),
              "block scan");
   }
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.og, dt, M, d, W.o.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant o'");
+  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.og, dt, M, d, W.o.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(), s); }), "block quant o'");
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
   MMF_CUDA(run_gemm(b, Epi::kStore, dt, s, "o"), "block o-proj");
   // channel mixer
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.y1, dt, M, d, W.gate.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s); }), "block quant y1");
+  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.y1, dt, M, d, W.gate.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(), s); }), "block quant y1");
   return run_glu(&W.gate, &W.up, &W.down, w.qa, w.y1, y, M, dt, eps, w.p, w.qa, s);
 }
 

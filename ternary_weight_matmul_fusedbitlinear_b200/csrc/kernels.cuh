@@ -43,8 +43,9 @@ size_t quantize_weights_ws_bytes();
 cudaError_t launch_quantize_weights(const float* W, int N, int K, uint32_t* packed, float* gamma, void* ws,
                                     cudaStream_t stream);
 
+// `status` (nullable) is the device status word for bounded-wait timeouts.
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
-                                 int8_t* q, float* scale, int32_t* qsum, cudaStream_t stream);
+                                 int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream);
 
 // Epilogues of the ternary contraction.
 enum class Epi : int {
@@ -86,8 +87,12 @@ bool tgemm_tc2_supported(const TGemmArgs& a, Epi epi);
 cudaError_t launch_tgemm_tc2(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
 
 // Chunk-parallel MLGRU scan; `ws` holds mlgru_scan_ws_bytes(B, T, d) bytes of
-// per-launch scratch (ticket counter, chunk flags, chunk carries).
+// scratch, which reset_mlgru_scan_ws() must prepare (stream-ordered) before
+// every launch; launch_mlgru_scan() itself enqueues only the kernel (launched
+// as a programmatic dependent of the kernel before it). `status` is the device
+// status word for bounded-wait timeouts.
 size_t mlgru_scan_ws_bytes(int B, int T, int d);
+cudaError_t reset_mlgru_scan_ws(void* ws, int B, int T, int d, cudaStream_t stream);
 cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, void* ws,
                               int* status, cudaStream_t stream);
 

@@ -65,8 +65,9 @@ struct ScanSmem {
   int abort_flag;
 };
 
-// Per-launch scratch: ticket counter, then per item three fields of 32 lane
-// words (float2 each): aggregate multiplier, aggregate offset, leaving state.
+// Per-launch scratch, filled with all-ones bytes before the launch: ticket
+// counter (starts at -1), then per item three fields of 32 lane words (float2
+// each): aggregate multiplier, aggregate offset, leaving state.
 struct ScanWs {
   int* ticket;
   float2* rec;
@@ -162,11 +163,13 @@ __global__ void __launch_bounds__(kThreads, sizeof(T) == 2 ? 2 : 1)
     }
   };
 
+  pdl_trigger();
+  pdl_wait();   // the pre-activations are the previous kernel's output
   if (threadIdx.x == 0) {
     for (int s = 0; s < NST; ++s) mbar_init(&sm.full[s], 1);
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    for (int s = 0; s < NST; ++s) issue(s, atomicAdd(ws.ticket, 1));
+    for (int s = 0; s < NST; ++s) issue(s, atomicAdd(ws.ticket, 1) + 1);
   }
   __syncthreads();
 
@@ -192,7 +195,7 @@ __global__ void __launch_bounds__(kThreads, sizeof(T) == 2 ? 2 : 1)
     const int item = sm.tk[s];
     if (item >= items) break;   // tickets rise, so every later stage is out of range too
     int next_ticket = 0;
-    if (threadIdx.x == 0) next_ticket = atomicAdd(ws.ticket, 1);   // used at the end of the item
+    if (threadIdx.x == 0) next_ticket = atomicAdd(ws.ticket, 1) + 1;   // used at the end of the item
 
     const int j = item / per_chunk, rem = item - j * per_chunk;
     const int b = rem / n_cb, cb = rem - b * n_cb;
@@ -296,6 +299,11 @@ __global__ void __launch_bounds__(kThreads, sizeof(T) == 2 ? 2 : 1)
   }
 }
 
+size_t ws_used_bytes(int B, int T_, int d) {
+  const size_t items = (size_t)ceil_div(T_, TC) * B * ceil_div(d, CC);
+  return 256 + sizeof(float) * items * kWsPerItem;
+}
+
 template <typename T>
 cudaError_t launch_typed(const void* pre, int B, int T_, int d, float* h, void* o, void* ws, int* status,
                          cudaStream_t stream) {
@@ -311,26 +319,27 @@ cudaError_t launch_typed(const void* pre, int B, int T_, int d, float* h, void* 
   ScanWs w;
   w.ticket = reinterpret_cast<int*>(base);
   w.rec = reinterpret_cast<float2*>(base + 256);
-  cudaError_t e = cudaMemsetAsync(base, 0, sizeof(int), stream);
-  if (e == cudaSuccess) e = cudaMemsetAsync(w.rec, 0xff, sizeof(float) * kWsPerItem * (size_t)items, stream);
-  if (e != cudaSuccess) return e;
   const size_t smem = sizeof(ScanSmem<T>) + 128;
   auto kern = mlgru_scan_kernel<T>;
-  e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   int per_sm = 1;
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
   const int grid = std::max(1, std::min(items, num_sms() * std::max(per_sm, 1)));
-  kern<<<grid, kThreads, smem, stream>>>(map, B, T_, d, n_cb, nchunk, h, static_cast<T*>(o), w, status);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, map, B, T_, d, n_cb, nchunk, h,
+                    static_cast<T*>(o), w, status);
 }
 
 }  // namespace
 
 size_t mlgru_scan_ws_bytes(int B, int T, int d) {
   if (B <= 0 || T <= 0 || d <= 0) return 256;
-  const size_t items = (size_t)ceil_div(T, TC) * B * ceil_div(d, CC);
-  return 256 + sizeof(float) * items * kWsPerItem;
+  return ws_used_bytes(B, T, d);
+}
+
+cudaError_t reset_mlgru_scan_ws(void* ws, int B, int T, int d, cudaStream_t stream) {
+  if (B <= 0 || T <= 0 || d <= 0) return cudaSuccess;
+  return cudaMemsetAsync(ws, 0xff, ws_used_bytes(B, T, d), stream);
 }
 
 cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, void* ws,

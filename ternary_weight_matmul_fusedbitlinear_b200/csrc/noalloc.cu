@@ -102,7 +102,9 @@ extern "C" mmf_status mmf_bitlinear_noalloc(const mmf_tlinear* lin, const void* 
   int32_t* qsum = reinterpret_cast<int32_t*>(cur);
 
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  e = launch_rmsnorm_quant(x, dtype, M, lin->K, lin->gain, eps, q, s, qsum, st);
+  // no status word here (obtaining it may allocate): a timed-out wait in the
+  // quantiser leaves its rows unwritten without a recorded code
+  e = launch_rmsnorm_quant(x, dtype, M, lin->K, lin->gain, eps, q, s, qsum, nullptr, st);
   if (e == cudaSuccess) {
     TGemmArgs a{};
     for (int i = 0; i < 3; ++i) {

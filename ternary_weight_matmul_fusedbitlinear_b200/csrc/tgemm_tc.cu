@@ -139,6 +139,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = sm.tmem_base;
+  // programmatic dependent launch: the set-up above overlaps the predecessor's
+  // tail; its outputs (codes, scales, residual) are read only after this
+  pdl_trigger();
+  pdl_wait();
 
   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
@@ -379,8 +383,7 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap (&mb)[3], cons
   if (e != cudaSuccess) return e;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = std::min(tiles, num_sms());
-  kern<<<grid, kThreads, smem, stream>>>(ma, mb[0], mb[1], mb[2], mo, mr, p);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kThreads), smem, stream, ma, mb[0], mb[1], mb[2], mo, mr, p);
 }
 
 }  // namespace
