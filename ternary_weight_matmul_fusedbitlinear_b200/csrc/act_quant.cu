@@ -14,6 +14,7 @@
 // it is fixed here (per-thread strided order, xor-shuffle tree, warps in order).
 #include "kernels.cuh"
 #include "tma.cuh"
+#include "quant_row.cuh"
 
 namespace mmf {
 
@@ -110,68 +111,7 @@ __global__ void __launch_bounds__(kThreads) rmsnorm_quant_kernel(const T* __rest
 // One warp per token row. Each warp keeps a ring of `slots` row buffers in
 // shared memory and fills them with 1-D bulk copies (cp.async.bulk, one per
 // row), so the next rows stream in while the current one is reduced; the row
-// itself is read from shared memory in 16-byte vectors (lane l takes vectors
-// l, l+32, ...), twice or three times, never from HBM again.
-// Pass 1 sums the squares in fp64 and takes the largest |x|. Without a gain
-// vector that already fixes the scale: rounding is monotone, so
-// fl(max|x| * rinv) = max fl(|x| * rinv) = max|x^|. With a gain vector a
-// second pass takes max|(x * rinv) * gain|. The last pass writes the codes.
-
-// fp32 bit pattern (sign cleared) -> the same value as an fp64, built with
-// integer operations (the conversion instruction issues at a fraction of the
-// ALU rate). Exact for every normal value. Zero and subnormals come out as
-// magnitudes below 2^-126 instead; their squares stay below 2^-252 and can
-// move a row's sum only when every element of the row is that small, and then
-// the fp32 mean square underflows to 0 either way.
-__device__ __forceinline__ double magbits_to_f64(uint32_t a) {
-  return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
-}
-
-// rint(t) for |t| < 2^22 by adding 1.5 * 2^23: the sum's unit in the last
-// place is 1, so the fp32 add rounds t half-to-even to an integer, and the
-// sum's bit pattern is 0x4B400000 + rint(t) with rint(t) in two's complement
-// in the low bits. Returns that bit pattern; its low byte is the int8 code.
-__device__ __forceinline__ uint32_t rint_bits(float t) { return __float_as_uint(__fadd_rn(t, 12582912.0f)); }
-
-// Low bytes of four rint_bits() patterns -> one word, bytes in order a, b, c, d.
-__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
-  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
-}
-
-// Per element type: E elements per 16-byte vector, their fp32 magnitude bits
-// and values.
-template <typename T>
-struct Vec;
-template <>
-struct Vec<bf16> {
-  static constexpr int E = 8;
-  __device__ __forceinline__ static uint32_t mag(const uint4& r, int i) {
-    const uint32_t w = (&r.x)[i >> 1];
-    return (i & 1) ? (w & 0x7fff0000u) : ((w << 16) & 0x7fffffffu);
-  }
-  __device__ __forceinline__ static float val(const uint4& r, int i) {
-    const uint32_t w = (&r.x)[i >> 1];
-    return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
-  }
-  __device__ __forceinline__ static void store_codes(int8_t* p, const uint32_t (&c)[8], int& isum) {
-    const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
-    const uint32_t w1 = pack_low_bytes(c[4], c[5], c[6], c[7]);
-    isum = __dp4a((int)w0, 0x01010101, isum);
-    isum = __dp4a((int)w1, 0x01010101, isum);
-    *reinterpret_cast<uint2*>(p) = make_uint2(w0, w1);
-  }
-};
-template <>
-struct Vec<float> {
-  static constexpr int E = 4;
-  __device__ __forceinline__ static uint32_t mag(const uint4& r, int i) { return (&r.x)[i] & 0x7fffffffu; }
-  __device__ __forceinline__ static float val(const uint4& r, int i) { return __uint_as_float((&r.x)[i]); }
-  __device__ __forceinline__ static void store_codes(int8_t* p, const uint32_t (&c)[4], int& isum) {
-    const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
-    isum = __dp4a((int)w0, 0x01010101, isum);
-    *reinterpret_cast<uint32_t*>(p) = w0;
-  }
-};
+// itself is read from shared memory by quant_row(), never from HBM again.
 
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -200,8 +140,6 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_staged_kernel(const T* __re
                                                                    int8_t* __restrict__ q, float* __restrict__ scale,
                                                                    int32_t* __restrict__ qsum, int slots,
                                                                    int stride, int* status) {
-  using V = Vec<T>;
-  constexpr int E = V::E;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warps = blockDim.x >> 5;
@@ -242,64 +180,10 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_staged_kernel(const T* __re
       return;
     }
     const uint4* v = reinterpret_cast<const uint4*>(ring + (size_t)s * stride);
-
-    // pass 1: sum of squares (fp64) and max |x|
-    double ss = 0.0;
-    uint32_t am = 0;
-#pragma unroll 4
-    for (int vi = lane; vi < nvec; vi += 32) {
-      const uint4 r = v[vi];
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const uint32_t a = V::mag(r, i);
-        am = max(am, a);
-        const double xd = magbits_to_f64(a);
-        ss = fma(xd, xd, ss);
-      }
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-    const float ms = (float)(ss / (double)K);
-    const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
-
-    float amax;
-    if constexpr (GAIN) {   // pass 2: max |(x * rinv) * gain|
-      uint32_t hm = 0;
-#pragma unroll 4
-      for (int vi = lane; vi < nvec; vi += 32) {
-        const uint4 r = v[vi];
-#pragma unroll
-        for (int i = 0; i < E; ++i) {
-          const float hv = __fmul_rn(__fmul_rn(V::val(r, i), rinv), __ldg(gain + vi * E + i));
-          hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
-        }
-      }
-      amax = __uint_as_float(__reduce_max_sync(0xffffffffu, hm));
-    } else {
-      amax = __fmul_rn(__uint_as_float(__reduce_max_sync(0xffffffffu, am)), rinv);
-    }
-    const float sc = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
-
-    // last pass: codes (|x^ * s| <= 127 up to rounding, so no clamp is needed
-    // and -128 never occurs) and their sum
-    int isum = 0;
-    int8_t* qr = q + (size_t)row * K;
-#pragma unroll 4
-    for (int vi = lane; vi < nvec; vi += 32) {
-      const uint4 r = v[vi];
-      uint32_t c[E];
-#pragma unroll
-      for (int i = 0; i < E; ++i) {
-        float hv = __fmul_rn(V::val(r, i), rinv);
-        if constexpr (GAIN) hv = __fmul_rn(hv, __ldg(gain + vi * E + i));
-        c[i] = rint_bits(__fmul_rn(hv, sc));
-      }
-      V::store_codes(qr + (size_t)vi * E, c, isum);
-    }
-    isum = __reduce_add_sync(0xffffffffu, isum);
+    const RowCode rc = quant_row<T, GAIN, false>(v, nvec, K, gain, eps, q + (size_t)row * K, lane);
     if (lane == 0) {
-      scale[row] = sc;
-      qsum[row] = isum;
+      scale[row] = rc.scale;
+      qsum[row] = rc.qsum;
     }
 
     // refill this buffer with the row `slots` rows ahead

@@ -143,12 +143,28 @@ int gemm_path_pref() {
   return 0;
 }
 
+bool gemm_uses_tc(const TGemmArgs& a, Epi epi) {
+  const int pref = gemm_path_pref();
+  return tgemm_tc_supported(a, epi) && (pref >= 2 || (pref == 0 && a.M >= kTcMinTokens));
+}
+
+// Whether the decode contraction quantises its own token rows (both ways give
+// the same codes). Every CTA then repeats the row work, which on one B200 beat
+// the standalone quantiser plus one kernel boundary only for single-token
+// calls (1.3B decode at 4 tokens: 0.69 ms per step fused, 0.59 ms split).
+// MMF_DECODE_FUSED_QUANT=1 fuses whenever the shapes allow, =0 never.
+bool decode_fused_quant_wanted(int M) {
+  const char* e = getenv("MMF_DECODE_FUSED_QUANT");
+  if (e != nullptr && strcmp(e, "1") == 0) return true;
+  if (e != nullptr && strcmp(e, "0") == 0) return false;
+  return M == 1;
+}
+
 // `what` names the projection for the launch-timing totals ("fcg", "o", ...).
 cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s, const char* what = "") {
   const int pref = gemm_path_pref();
-  const bool tc_ok = tgemm_tc_supported(a, epi);
   const bool tc2_ok = tgemm_tc2_supported(a, epi);
-  bool use_tc = tc_ok && (pref >= 2 || (pref == 0 && a.M >= kTcMinTokens));
+  bool use_tc = gemm_uses_tc(a, epi);
   const bool use_tc2 = use_tc && tc2_ok && pref == 4;
   char name[48];
   snprintf(name, sizeof(name), "%s%s%s", use_tc2 ? "tgemm_tc2" : (use_tc ? "tgemm_tc" : "tgemm_mma"),
@@ -166,6 +182,38 @@ cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s, 
 int* status_word() {
   int* st = nullptr;
   return device_status_ptr(&st) == MMF_OK ? st : nullptr;
+}
+
+// Quantised activations of M tokens of length K.
+struct QAct {
+  int8_t* q;
+  float* s;
+  int32_t* qsum;
+};
+
+// RMSNorm + int8 quantisation of x (a.M tokens of length a.K, RMSNorm gain
+// `gain`), then the contraction `a` (whose q/s/qsum point at qa). Single-token
+// calls on the mma.sync kernel quantise inside the contraction (one launch);
+// the codes also land in qa when `want_codes`. Otherwise the quantiser fills qa
+// and the contraction reads it.
+mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& qa, TGemmArgs a, Epi epi,
+                      mmf_dtype dt, cudaStream_t s, const char* what, bool want_codes) {
+  if (!gemm_uses_tc(a, epi) && decode_fused_quant_wanted(a.M) &&
+      tgemm_mma_fused_quant_supported(a.M, a.K, elem_bytes(dt))) {
+    a.x = x;
+    a.gain = gain;
+    a.eps = eps;
+    a.q_out = want_codes ? qa.q : nullptr;
+    a.s_out = want_codes ? qa.s : nullptr;
+    a.qsum_out = want_codes ? qa.qsum : nullptr;
+    MMF_CUDA(run_gemm(a, epi, dt, s, what), "fused quant + contraction");
+    return MMF_OK;
+  }
+  MMF_CUDA(timed("rmsnorm_quant", s,
+                 [&] { return launch_rmsnorm_quant(x, dt, a.M, a.K, gain, eps, qa.q, qa.s, qa.qsum, status_word(), s); }),
+           "rmsnorm_quant");
+  MMF_CUDA(run_gemm(a, epi, dt, s, what), "contraction");
+  return MMF_OK;
 }
 
 mmf_status check_tlinear(const mmf_tlinear* l, const char* name) {
@@ -202,12 +250,6 @@ TGemmArgs gemm_args(const mmf_tlinear* const* segs, int nseg, const int8_t* q, c
   return a;
 }
 
-// Quantised activations of M tokens of length K.
-struct QAct {
-  int8_t* q;
-  float* s;
-  int32_t* qsum;
-};
 
 QAct carve_qact(Carver& c, int M, int K) {
   QAct a;
@@ -306,9 +348,9 @@ extern "C" mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_d
   const mmf_tlinear* segs[1] = {lin};
   Carver c(ws);
   QAct qa = carve_qact(c, M, lin->K);
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, lin->K, lin->gain, eps, qa.q, qa.s, qa.qsum, status_word(), s); }), "rmsnorm_quant");
   TGemmArgs a = gemm_args(segs, 1, qa.q, qa.s, qa.qsum, M, y, lin->N, nullptr, nullptr);
-  MMF_CUDA(run_gemm(a, Epi::kStore, dtype, s), "tgemm");
+  mmf_status r = quant_gemm(x, lin->gain, eps, qa, a, Epi::kStore, dtype, s, "", dbg != nullptr);
+  if (r != MMF_OK) return r;
   if (dbg) {
     if (dbg->q) MMF_CUDA(cudaMemcpyAsync(dbg->q, qa.q, (size_t)M * lin->K, cudaMemcpyDeviceToDevice, s), "dbg q");
     if (dbg->scale)
@@ -375,18 +417,18 @@ mmf_status check_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_t
   return MMF_OK;
 }
 
-// p = SiLU(gate(x)) * up(x); y = down(p) + residual. x already quantised in qx.
-mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tlinear* down, const QAct& qx,
-                   const void* residual, void* y, int M, mmf_dtype dt, float eps, void* p, const QAct& qp,
+// p = SiLU(gate(x)) * up(x); y = down(p) + residual. x is quantised with the
+// gate's RMSNorm gain (gate and up share it), p with the down projection's.
+mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tlinear* down, const void* x,
+                   const void* residual, void* y, int M, mmf_dtype dt, float eps, void* p, const QAct& qa,
                    cudaStream_t s) {
   const mmf_tlinear* gu[2] = {gate, up};
-  TGemmArgs a = gemm_args(gu, 2, qx.q, qx.s, qx.qsum, M, p, gate->N, nullptr, nullptr);
-  MMF_CUDA(run_gemm(a, Epi::kGlu, dt, s, "gate_up"), "glu gate/up");
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(p, dt, M, down->K, down->gain, eps, qp.q, qp.s, qp.qsum, status_word(), s); }), "glu quant p");
+  TGemmArgs a = gemm_args(gu, 2, qa.q, qa.s, qa.qsum, M, p, gate->N, nullptr, nullptr);
+  mmf_status r = quant_gemm(x, gate->gain, eps, qa, a, Epi::kGlu, dt, s, "gate_up", false);
+  if (r != MMF_OK) return r;
   const mmf_tlinear* dn[1] = {down};
-  TGemmArgs b = gemm_args(dn, 1, qp.q, qp.s, qp.qsum, M, y, down->N, residual, nullptr);
-  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s, "down"), "glu down");
-  return MMF_OK;
+  TGemmArgs b = gemm_args(dn, 1, qa.q, qa.s, qa.qsum, M, y, down->N, residual, nullptr);
+  return quant_gemm(p, down->gain, eps, qa, b, Epi::kStore, dt, s, "down", false);
 }
 
 }  // namespace
@@ -417,8 +459,7 @@ extern "C" mmf_status mmf_glu(const mmf_tlinear* gate, const mmf_tlinear* up, co
   Carver c(ws);
   QAct qa = carve_qact(c, M, std::max(d, I));
   void* p = c.take<char>((size_t)M * I * elem_bytes(dtype));
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dtype, M, d, gate->gain, eps, qa.q, qa.s, qa.qsum, status_word(), s); }), "glu quant x");
-  return run_glu(gate, up, down, qa, residual, y, M, dtype, eps, p, qa, s);
+  return run_glu(gate, up, down, x, residual, y, M, dtype, eps, p, qa, s);
 }
 
 // ------------------------------------------------------------------ blocks and state
@@ -551,28 +592,28 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   // prefill: the scan's scratch is reset here, so that fcg projection -> scan
   // are back-to-back kernels (the scan starts as a programmatic dependent)
   if (T > 1) MMF_CUDA(timed("mlgru_scan_reset", s, [&] { return reset_mlgru_scan_ws(w.scan, B, T, d, s); }), "block scan reset");
-  // token mixer: quantise x once for f, c, g (shared gain)
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(x, dt, M, d, W.f.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(), s); }), "block quant x");
+  // token mixer: x quantised once for f, c, g (shared gain)
   if (T == 1) {
     // decode: projections and one recurrence step in one launch; h updated in place
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, h);
-    MMF_CUDA(run_gemm(a, Epi::kScanStep, dt, s, "fcg_step"), "block fcg+step");
+    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kScanStep, dt, s, "fcg_step", false);
+    if (r != MMF_OK) return r;
   } else {
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.pre, 3 * d, nullptr, nullptr);
-    MMF_CUDA(run_gemm(a, Epi::kStore, dt, s, "fcg"), "block fcg");
+    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", false);
+    if (r != MMF_OK) return r;
     int* status = nullptr;
-    mmf_status r = device_status_ptr(&status);
+    r = device_status_ptr(&status);
     if (r != MMF_OK) return r;
     MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, w.scan, status, s); }),
              "block scan");
   }
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.og, dt, M, d, W.o.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(), s); }), "block quant o'");
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
-  MMF_CUDA(run_gemm(b, Epi::kStore, dt, s, "o"), "block o-proj");
+  mmf_status r = quant_gemm(w.og, W.o.gain, eps, w.qa, b, Epi::kStore, dt, s, "o", false);
+  if (r != MMF_OK) return r;
   // channel mixer
-  MMF_CUDA(timed("rmsnorm_quant", s, [&] { return launch_rmsnorm_quant(w.y1, dt, M, d, W.gate.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(), s); }), "block quant y1");
-  return run_glu(&W.gate, &W.up, &W.down, w.qa, w.y1, y, M, dt, eps, w.p, w.qa, s);
+  return run_glu(&W.gate, &W.up, &W.down, w.y1, w.y1, y, M, dt, eps, w.p, w.qa, s);
 }
 
 mmf_status check_forward_args(const mmf_block* blk, mmf_state* st, const void* x, void* y, int B, int T,

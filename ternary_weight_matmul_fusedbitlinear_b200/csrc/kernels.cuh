@@ -70,12 +70,26 @@ struct TGemmArgs {
   int ldo;                  // leading dimension of out (elements)
   const void* residual;     // [M, N] in the activation dtype, or null
   float* h;                 // kScanStep: [M, N] fp32 state, updated in place
+  // Decode contraction only: when x is set, the kernel quantises the token
+  // rows x [M, K] (activation dtype, RMSNorm gain `gain` or null, `eps`)
+  // itself and q/s/qsum above are not read; q_out/s_out/qsum_out (nullable)
+  // then receive the codes, scales and sums.
+  const void* x;
+  const float* gain;
+  float eps;
+  int8_t* q_out;
+  float* s_out;
+  int32_t* qsum_out;
 };
 
 
 
 // mma.sync-based contraction (weights as the 16-row A operand, tokens as N=8 tiles).
 cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t stream);
+// Whether launch_tgemm_mma can quantise the token rows itself (TGemmArgs::x):
+// up to 16 tokens whose rows (esize bytes per element) and codes fit the
+// kernel's shared memory.
+bool tgemm_mma_fused_quant_supported(int M, int K, int esize);
 
 // tcgen05 (TMEM) contraction for prefill-sized token counts. Needs K % 64 == 0
 // and N % 128 == 0; `status` is the device status word for bounded-wait timeouts.

@@ -1,0 +1,156 @@
+// One token row of the fused RMSNorm + absmax int8 quantisation, computed by
+// one warp (sm_100a). Shared by the standalone quantiser and by the decode
+// contraction, which quantises its few token rows itself.
+//
+// "MatMul-free language models" (DataCamp blog), overview figure panel
+// "RMS Norm", and the hysenlabs review, section "FusedBitLinear": RMSNorm on
+// the input, then per-token absmax quantisation to int8. Per row x[0..K):
+//   ms  = (float)(sum x^2 in fp64 / K)
+//   rinv = 1 / sqrt(ms + eps)                        (IEEE fp32)
+//   x^  = (x * rinv) * gain                          (IEEE fp32 products)
+//   s   = 127 / max(max|x^|, 1e-5)
+//   q   = rint(x^ * s) (|x^ s| <= 127 up to rounding, so no clamp is needed
+//         and -128 never occurs),  qsum = sum q      (int32)
+// Every fp32 step is a correctly rounded single operation, so the codes do not
+// depend on the kernel's layout; the fp64 sum's order is fixed (lane l sums
+// vectors l, l+32, ... in order, then an xor-shuffle tree).
+// Pass 1 sums the squares and takes max|x|. Without a gain vector that already
+// fixes the scale: rounding is monotone, so fl(max|x| * rinv) =
+// max fl(|x| * rinv) = max|x^|. With a gain vector a second pass takes
+// max|(x * rinv) * gain|. The last pass writes the codes.
+#pragma once
+
+#include "common.cuh"
+
+namespace mmf {
+
+// fp32 bit pattern (sign cleared) -> the same value as an fp64, built with
+// integer operations (the conversion instruction issues at a fraction of the
+// ALU rate). Exact for every normal value. Zero and subnormals come out as
+// magnitudes below 2^-126 instead; their squares stay below 2^-252 and can
+// move a row's sum only when every element of the row is that small, and then
+// the fp32 mean square underflows to 0 either way.
+__device__ __forceinline__ double magbits_to_f64(uint32_t a) {
+  return __hiloint2double((int)((a >> 3) + 0x38000000u), (int)(a << 29));
+}
+
+// rint(t) for |t| < 2^22 by adding 1.5 * 2^23: the sum's unit in the last
+// place is 1, so the fp32 add rounds t half-to-even to an integer, and the
+// sum's bit pattern is 0x4B400000 + rint(t) with rint(t) in two's complement
+// in the low bits. Returns that bit pattern; its low byte is the int8 code.
+__device__ __forceinline__ uint32_t rint_bits(float t) { return __float_as_uint(__fadd_rn(t, 12582912.0f)); }
+
+// Low bytes of four rint_bits() patterns -> one word, bytes in order a, b, c, d.
+__device__ __forceinline__ uint32_t pack_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return __byte_perm(__byte_perm(a, b, 0x0040), __byte_perm(c, d, 0x0040), 0x5410);
+}
+
+// Per element type: E elements per 16-byte vector, their fp32 magnitude bits
+// and values.
+template <typename T>
+struct Vec;
+template <>
+struct Vec<bf16> {
+  static constexpr int E = 8;
+  __device__ __forceinline__ static uint32_t mag(const uint4& r, int i) {
+    const uint32_t w = (&r.x)[i >> 1];
+    return (i & 1) ? (w & 0x7fff0000u) : ((w << 16) & 0x7fffffffu);
+  }
+  __device__ __forceinline__ static float val(const uint4& r, int i) {
+    const uint32_t w = (&r.x)[i >> 1];
+    return __uint_as_float((i & 1) ? (w & 0xffff0000u) : (w << 16));
+  }
+  __device__ __forceinline__ static void store_codes(int8_t* p, const uint32_t (&c)[8], int& isum) {
+    const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
+    const uint32_t w1 = pack_low_bytes(c[4], c[5], c[6], c[7]);
+    isum = __dp4a((int)w0, 0x01010101, isum);
+    isum = __dp4a((int)w1, 0x01010101, isum);
+    *reinterpret_cast<uint2*>(p) = make_uint2(w0, w1);
+  }
+};
+template <>
+struct Vec<float> {
+  static constexpr int E = 4;
+  __device__ __forceinline__ static uint32_t mag(const uint4& r, int i) { return (&r.x)[i] & 0x7fffffffu; }
+  __device__ __forceinline__ static float val(const uint4& r, int i) { return __uint_as_float((&r.x)[i]); }
+  __device__ __forceinline__ static void store_codes(int8_t* p, const uint32_t (&c)[4], int& isum) {
+    const uint32_t w0 = pack_low_bytes(c[0], c[1], c[2], c[3]);
+    isum = __dp4a((int)w0, 0x01010101, isum);
+    *reinterpret_cast<uint32_t*>(p) = w0;
+  }
+};
+
+struct RowCode {
+  float scale;
+  int qsum;
+};
+
+// Warp-collective: all 32 lanes call it with the same row. `v` points at the
+// row as nvec 16-byte vectors (K elements), in global memory when GLOBAL
+// (read through the read-only path) or in shared memory; codes go to qr
+// (16-byte aligned, global or shared). Returns the scale and the code sum on
+// every lane.
+template <typename T, bool GAIN, bool GLOBAL>
+__device__ __forceinline__ RowCode quant_row(const uint4* v, int nvec, int K, const float* __restrict__ gain,
+                                             float eps, int8_t* qr, int lane) {
+  using V = Vec<T>;
+  constexpr int E = V::E;
+  auto ld = [&](int vi) -> uint4 {
+    if constexpr (GLOBAL) return __ldg(v + vi);
+    else return v[vi];
+  };
+  // pass 1: sum of squares (fp64) and max |x|
+  double ss = 0.0;
+  uint32_t am = 0;
+#pragma unroll 4
+  for (int vi = lane; vi < nvec; vi += 32) {
+    const uint4 r = ld(vi);
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const uint32_t a = V::mag(r, i);
+      am = max(am, a);
+      const double xd = magbits_to_f64(a);
+      ss = fma(xd, xd, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  const float ms = (float)(ss / (double)K);
+  const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
+
+  float amax;
+  if constexpr (GAIN) {   // pass 2: max |(x * rinv) * gain|
+    uint32_t hm = 0;
+#pragma unroll 4
+    for (int vi = lane; vi < nvec; vi += 32) {
+      const uint4 r = ld(vi);
+#pragma unroll
+      for (int i = 0; i < E; ++i) {
+        const float hv = __fmul_rn(__fmul_rn(V::val(r, i), rinv), __ldg(gain + vi * E + i));
+        hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
+      }
+    }
+    amax = __uint_as_float(__reduce_max_sync(0xffffffffu, hm));
+  } else {
+    amax = __fmul_rn(__uint_as_float(__reduce_max_sync(0xffffffffu, am)), rinv);
+  }
+  const float sc = __fdiv_rn(127.0f, fmaxf(amax, 1e-5f));
+
+  // last pass: codes and their sum
+  int isum = 0;
+#pragma unroll 4
+  for (int vi = lane; vi < nvec; vi += 32) {
+    const uint4 r = ld(vi);
+    uint32_t c[E];
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      float hv = __fmul_rn(V::val(r, i), rinv);
+      if constexpr (GAIN) hv = __fmul_rn(hv, __ldg(gain + vi * E + i));
+      c[i] = rint_bits(__fmul_rn(hv, sc));
+    }
+    V::store_codes(qr + (size_t)vi * E, c, isum);
+  }
+  return RowCode{sc, __reduce_add_sync(0xffffffffu, isum)};
+}
+
+}  // namespace mmf

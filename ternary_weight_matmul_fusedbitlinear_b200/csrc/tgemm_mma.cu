@@ -14,6 +14,13 @@
 // memory with cp.async, so the weight stream overlaps the previous kernel; the
 // activations are read only after pdl_wait().
 //
+// Fused quantisation (FQ): for decode-sized token counts every CTA can take the
+// raw activations instead of int8 codes and quantise its (at most 16) token
+// rows itself, one warp per row, with the same row routine and the same fp32
+// steps as the standalone quantiser, so the codes are identical; one kernel per
+// projection instead of two. The rows are first copied whole into shared
+// memory (all copies in flight at once), so their latency is paid once.
+//
 // Work split: a CTA owns 16 output rows of each of its R weight segments and
 // 8*NT tokens; its 8 warps split K into 256-column segments round-robin. Per
 // 256-column segment a lane (group g, thread t) loads 16 bytes of packed codes
@@ -23,6 +30,7 @@
 // memory through integer atomics (exact in any order), then the epilogue
 // rescales and applies the mode.
 #include "kernels.cuh"
+#include "quant_row.cuh"
 
 namespace mmf {
 
@@ -69,10 +77,17 @@ __device__ __forceinline__ void cp_async16(void* smem, const void* gmem, bool va
 // so the 8 rows a quarter-warp reads start in different banks.
 __host__ __device__ __forceinline__ int wsm_pitch4(int wpr) { return wpr / 4 + 4; }
 
-template <int NT, int R, Epi EPI, typename T, bool SMEMW>
+// Shared-memory row pitch (bytes) of the fused-quantisation codes: 16 bytes
+// more than a row, which spreads the 8 rows of a fragment load over the banks.
+__host__ __device__ __forceinline__ int fq_pitch(int K) { return K + 16; }
+
+template <int NT, int R, Epi EPI, typename T, bool SMEMW, bool FQ>
 __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
   __shared__ int red[R][16][NT * 8];
-  extern __shared__ uint4 wsm[];     // SMEMW: [R][16][pitch4] weight slice
+  __shared__ float s_sm[FQ ? NT * 8 : 1];
+  __shared__ int qsum_sm[FQ ? NT * 8 : 1];
+  extern __shared__ uint4 wsm[];     // SMEMW: [R][16][pitch4] weight slice; FQ: then [NT*8][fq_pitch] codes,
+                                     // then the token rows [rows][K] in the activation dtype
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int n0 = blockIdx.x * 16;
@@ -95,10 +110,40 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
   pdl_trigger();
   pdl_wait();
   for (int i = threadIdx.x; i < R * 16 * NT * 8; i += kThreads) (&red[0][0][0])[i] = 0;
-  if constexpr (SMEMW) {
+  int8_t* qs = reinterpret_cast<int8_t*>(wsm + (SMEMW ? R * 16 * pitch4 : 0));
+  const int qpitch = fq_pitch(K);
+  if constexpr (FQ) {   // quantise this CTA's token rows, one warp per row
+    const int nvec = (int)(K * sizeof(T) / 16);
+    const int rows = min(NT * 8, M - m0);
+    uint4* xs = reinterpret_cast<uint4*>(qs + (size_t)NT * 8 * qpitch);
+    const uint4* xg = reinterpret_cast<const uint4*>(static_cast<const T*>(a.x) + (size_t)m0 * K);
+    for (int i = threadIdx.x; i < rows * nvec; i += kThreads) cp_async16(xs + i, xg + i, true);
+    asm volatile("cp.async.commit_group;" ::: "memory");
     asm volatile("cp.async.wait_all;" ::: "memory");
     __syncthreads();
+    for (int mc = warp; mc < rows; mc += kWarps) {
+      const int m = m0 + mc;
+      const uint4* xr = xs + (size_t)mc * nvec;
+      int8_t* qr = qs + (size_t)mc * qpitch;
+      const RowCode rc = a.gain != nullptr ? quant_row<T, true, false>(xr, nvec, K, a.gain, a.eps, qr, lane)
+                                           : quant_row<T, false, false>(xr, nvec, K, nullptr, a.eps, qr, lane);
+      if (lane == 0) {
+        s_sm[mc] = rc.scale;
+        qsum_sm[mc] = rc.qsum;
+      }
+      if (blockIdx.x == 0 && a.q_out != nullptr) {   // one CTA also hands the codes out
+        __syncwarp();
+        for (int i = lane; i < K / 16; i += 32)
+          *reinterpret_cast<uint4*>(a.q_out + (size_t)m * K + i * 16) = *reinterpret_cast<const uint4*>(qr + i * 16);
+        if (lane == 0) {
+          if (a.s_out) a.s_out[m] = rc.scale;
+          if (a.qsum_out) a.qsum_out[m] = rc.qsum;
+        }
+      }
+    }
   }
+  if constexpr (SMEMW) asm volatile("cp.async.wait_all;" ::: "memory");
+  if constexpr (SMEMW || FQ) __syncthreads();
 
   int acc[R][NT][4];
 #pragma unroll
@@ -127,13 +172,17 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
 #pragma unroll
     for (int j = 0; j < NT; ++j) {
       const int m = m0 + 8 * j + g;
-      const int8_t* qrow = a.q + (size_t)m * K;
+      const int8_t* qrow = FQ ? nullptr : a.q + (size_t)m * K;
 #pragma unroll
       for (int u = 0; u < 4; ++u) {
         // bytes [64t + 16u, +16) of this segment = packed word w0 + u's 16 columns
         const bool ok = (m < M) && (w0 + u < wpr);
-        act[j][u] = ok ? __ldg(reinterpret_cast<const uint4*>(qrow + (size_t)(w0 + u) * 16))
-                       : make_uint4(0u, 0u, 0u, 0u);
+        if constexpr (FQ)
+          act[j][u] = ok ? *reinterpret_cast<const uint4*>(qs + (size_t)(8 * j + g) * qpitch + (w0 + u) * 16)
+                         : make_uint4(0u, 0u, 0u, 0u);
+        else
+          act[j][u] = ok ? __ldg(reinterpret_cast<const uint4*>(qrow + (size_t)(w0 + u) * 16))
+                         : make_uint4(0u, 0u, 0u, 0u);
       }
     }
 #pragma unroll
@@ -168,16 +217,18 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
 
   // ---------------------------------------------------------------- epilogue
   constexpr int kCols = NT * 8;
+  auto row_scale = [&](int mc) { return FQ ? s_sm[mc] : a.s[m0 + mc]; };
+  auto row_qsum = [&](int mc) { return FQ ? qsum_sm[mc] : a.qsum[m0 + mc]; };
   if constexpr (EPI == Epi::kStore || EPI == Epi::kAcc) {
     for (int idx = threadIdx.x; idx < R * 16 * kCols; idx += kThreads) {
       const int row = idx & 15, r = (idx >> 4) % R, mc = idx / (16 * R);
       const int n = n0 + row, m = m0 + mc;
       if (n >= N || m >= M) continue;
-      const int accv = red[r][row][mc] - a.qsum[m];
+      const int accv = red[r][row][mc] - row_qsum(mc);
       if constexpr (EPI == Epi::kAcc) {
         static_cast<int32_t*>(a.out)[(size_t)m * a.ldo + r * N + n] = accv;
       } else {
-        float v = __fdiv_rn(__fmul_rn((float)accv, *a.gamma[r]), a.s[m]);
+        float v = __fdiv_rn(__fmul_rn((float)accv, *a.gamma[r]), row_scale(mc));
         if (a.bias[r] != nullptr) v += a.bias[r][n];
         if (a.residual != nullptr) v += to_f32(static_cast<const T*>(a.residual)[(size_t)m * N + n]);
         static_cast<T*>(a.out)[(size_t)m * a.ldo + r * N + n] = from_f32<T>(v);
@@ -191,7 +242,7 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
       float pre[3];
 #pragma unroll
       for (int r = 0; r < 3; ++r) {
-        float v = __fdiv_rn(__fmul_rn((float)(red[r][row][mc] - a.qsum[m]), *a.gamma[r]), a.s[m]);
+        float v = __fdiv_rn(__fmul_rn((float)(red[r][row][mc] - row_qsum(mc)), *a.gamma[r]), row_scale(mc));
         if (a.bias[r] != nullptr) v += a.bias[r][n];
         pre[r] = round_to<T>(v);   // the pre-activations are a storage point
       }
@@ -209,7 +260,7 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
       float uv[2];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
-        float v = __fdiv_rn(__fmul_rn((float)(red[r][row][mc] - a.qsum[m]), *a.gamma[r]), a.s[m]);
+        float v = __fdiv_rn(__fmul_rn((float)(red[r][row][mc] - row_qsum(mc)), *a.gamma[r]), row_scale(mc));
         if (a.bias[r] != nullptr) v += a.bias[r][n];
         uv[r] = v;
       }
@@ -218,18 +269,33 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
   }
 }
 
+constexpr size_t kFqBytes = 128 * 1024;   // fused-quantisation limit: codes + staged token rows
+
+template <int NT, int R, Epi EPI, typename T, bool SMEMW, bool FQ>
+cudaError_t launch_variant(const TGemmArgs& a, dim3 grid, size_t smem, cudaStream_t stream) {
+  auto kern = tgemm_mma_kernel<NT, R, EPI, T, SMEMW, FQ>;
+  if (smem > 48 * 1024) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(kern, grid, dim3(kThreads), smem, stream, a);
+}
+
 template <int NT, int R, Epi EPI, typename T>
 cudaError_t launch_one(const TGemmArgs& a, cudaStream_t stream) {
   dim3 grid(ceil_div(a.N, 16), ceil_div(a.M, NT * 8));
   const int wpr = a.K / 16;
-  const size_t smem = (size_t)R * 16 * wsm_pitch4(wpr) * 16;
-  if (wpr % 4 == 0 && smem <= 100 * 1024) {
-    auto kern = tgemm_mma_kernel<NT, R, EPI, T, true>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
-    if (e != cudaSuccess) return e;
-    return launch_pdl(kern, grid, dim3(kThreads), smem, stream, a);
-  }
-  return launch_pdl(tgemm_mma_kernel<NT, R, EPI, T, false>, grid, dim3(kThreads), 0, stream, a);
+  const size_t wbytes = (size_t)R * 16 * wsm_pitch4(wpr) * 16;
+  const bool fq = a.x != nullptr;
+  const size_t qbytes = fq ? (size_t)NT * 8 * fq_pitch(a.K) + (size_t)std::min(a.M, NT * 8) * a.K * sizeof(T) : 0;
+  if (fq && (NT > 2 || qbytes > kFqBytes)) return cudaErrorInvalidValue;
+  // the weight slice goes to shared memory when it fits next to the codes
+  const bool smemw = wpr % 4 == 0 && wbytes <= 100 * 1024 && wbytes + qbytes <= 200 * 1024;
+  const size_t smem = (smemw ? wbytes : 0) + qbytes;
+  if (smemw) return fq ? launch_variant<NT, R, EPI, T, true, true>(a, grid, smem, stream)
+                       : launch_variant<NT, R, EPI, T, true, false>(a, grid, smem, stream);
+  return fq ? launch_variant<NT, R, EPI, T, false, true>(a, grid, smem, stream)
+            : launch_variant<NT, R, EPI, T, false, false>(a, grid, smem, stream);
 }
 
 template <int NT, typename T>
@@ -255,6 +321,11 @@ cudaError_t launch_t(const TGemmArgs& a, Epi epi, cudaStream_t stream) {
 }
 
 }  // namespace
+
+bool tgemm_mma_fused_quant_supported(int M, int K, int esize) {
+  const int nt = M <= 8 ? 1 : 2;
+  return M >= 1 && M <= 16 && (size_t)nt * 8 * fq_pitch(K) + (size_t)M * K * esize <= kFqBytes;
+}
 
 cudaError_t launch_tgemm_mma(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t stream) {
   if (a.M == 0 || a.N == 0) return cudaSuccess;

@@ -193,6 +193,35 @@ def test_block_decode_steps_parity(dtype):
     assert_close(st.get()[0].numpy(), h, "f32", "decode h", tol=E2E_TOL)
 
 
+@pytest.mark.parametrize("k,n,m", [(2048, 2048, 1), (2048, 5632, 4), (5632, 2048, 16), (272, 130, 9)])
+def test_decode_fused_quant_matches_standalone_quantiser(k, n, m, monkeypatch):
+    # the decode contraction quantises its token rows itself with the same row
+    # routine as the standalone quantiser: codes, scales and outputs are identical
+    _, lin, _ = make_layer(900 + k + n, n, k)
+    x = synth.activations(901 + m, m, k, torch.bfloat16, outlier_p=synth.GEMV_OUTLIER_P,
+                          outlier_scale=synth.GEMV_OUTLIER_SCALE).cuda()
+    monkeypatch.setenv("MMF_DECODE_FUSED_QUANT", "1")
+    fused = mmf.bitlinear(lin, x, debug=True)
+    monkeypatch.setenv("MMF_DECODE_FUSED_QUANT", "0")
+    split = mmf.bitlinear(lin, x, debug=True)
+    for a, b, what in zip(fused, split, ("y", "q", "s", "acc")):
+        assert torch.equal(a, b), what
+
+
+def test_block_decode_fused_quant_matches_standalone_quantiser(monkeypatch):
+    d, inner, B = 256, 768, 4
+    blk, _ = make_block(7011, d, inner)
+    x = synth.activations(7012, B, d, torch.bfloat16).reshape(B, 1, d).cuda()
+    h0 = synth.activations(7013, B, d) * 0.5
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MMF_DECODE_FUSED_QUANT", flag)
+        st = mmf.State(1, B, d)
+        st.set(h0.reshape(1, B, d))
+        outs.append((mmf.block_forward(blk, 0, st, x), st.get()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
 def test_block_prefill_then_decode_matches_oracle_bf16():
     d, inner, B, T = 256, 768, 2, 40
     blk, oblk = make_block(7003, d, inner)
