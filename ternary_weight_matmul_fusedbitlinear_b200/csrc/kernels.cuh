@@ -100,6 +100,18 @@ cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* stat
 bool tgemm_tc2_supported(const TGemmArgs& a, Epi epi);
 cudaError_t launch_tgemm_tc2(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
 
+// Prefill token mixer in one kernel: the f|c|g contraction (a.nseg == 3, rows
+// of the three matrices for the same channels) with the MLGRU gates and
+// recurrence in its epilogue; writes o' [M, d] (a.out, activation dtype) and
+// updates the state h [B, d]. Needs T % 128 == 0 and d % 64 == 0. `ws` holds
+// tgemm_tc_mlgru_ws_bytes(B, T, d) bytes that reset_tgemm_tc_mlgru_ws() must
+// prepare (stream-ordered) before every launch.
+bool tgemm_tc_mlgru_supported(const TGemmArgs& a, int T, int d);
+size_t tgemm_tc_mlgru_ws_bytes(int B, int T, int d);
+cudaError_t reset_tgemm_tc_mlgru_ws(void* ws, int B, int T, int d, cudaStream_t stream);
+cudaError_t launch_tgemm_tc_mlgru(const TGemmArgs& a, mmf_dtype dt, int T, int d, float* h, void* ws, int* status,
+                                  cudaStream_t stream);
+
 // Chunk-parallel MLGRU scan; `ws` holds mlgru_scan_ws_bytes(B, T, d) bytes of
 // scratch, which reset_mlgru_scan_ws() must prepare (stream-ordered) before
 // every launch; launch_mlgru_scan() itself enqueues only the kernel (launched

@@ -222,6 +222,45 @@ def test_block_decode_fused_quant_matches_standalone_quantiser(monkeypatch):
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_block_prefill_fused_mixer_parity(dtype, monkeypatch):
+    # T % 128 == 0 and MMF_FUSED_MLGRU=1: the token mixer runs as one kernel
+    # (contraction + MLGRU epilogue); checked against the oracle and against
+    # the default path (contraction, pre-activations, scan)
+    d, inner, B, T = 256, 768, 2, 256
+    blk, oblk = make_block(7021, d, inner)
+    x = synth.activations(7022, B * T, d, TORCH_DT[dtype]).reshape(B, T, d)
+    h0 = synth.activations(7023, B, d) * 0.5
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MMF_FUSED_MLGRU", flag)
+        st = mmf.State(1, B, d)
+        st.set(h0.reshape(1, B, d))
+        outs.append((mmf.block_forward(blk, 0, st, x.cuda()), st.get()))
+    mmf.check()
+    y_ref, h_ref = O.block_forward(to_np(x), oblk, h0.numpy().astype(np.float64), dtype)
+    assert_close(to_np(outs[0][0]), y_ref, dtype, "fused block y", tol=E2E_TOL)
+    assert_close(outs[0][1][0].numpy(), h_ref, "f32", "fused block h_T", tol=E2E_TOL)
+    torch.testing.assert_close(outs[0][1], outs[1][1], rtol=1e-4, atol=1e-5)
+    # the two paths round the scan in a different order, so an o' code can land
+    # on the other side of a tie: composite tolerance, as for any whole block
+    assert_close(to_np(outs[0][0]), to_np(outs[1][0]), dtype, "fused vs unfused y", tol=E2E_TOL)
+
+
+def test_block_prefill_fused_mixer_chunked_equals_whole(monkeypatch):
+    monkeypatch.setenv("MMF_FUSED_MLGRU", "1")
+    d, inner, B, T = 256, 768, 2, 256
+    blk, _ = make_block(7031, d, inner)
+    x = synth.activations(7032, B * T, d, torch.bfloat16).reshape(B, T, d).cuda()
+    st1 = mmf.State(1, B, d)
+    y1 = mmf.block_forward(blk, 0, st1, x)
+    st2 = mmf.State(1, B, d)
+    ya = mmf.block_forward(blk, 0, st2, x[:, :128].contiguous())
+    yb = mmf.block_forward(blk, 0, st2, x[:, 128:].contiguous())
+    torch.testing.assert_close(st2.get(), st1.get(), rtol=1e-5, atol=1e-6)
+    assert_close(to_np(torch.cat([ya, yb], 1)), to_np(y1), "bf16", "chunked vs whole")
+
+
 def test_block_prefill_then_decode_matches_oracle_bf16():
     d, inner, B, T = 256, 768, 2, 40
     blk, oblk = make_block(7003, d, inner)
