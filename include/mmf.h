@@ -203,6 +203,14 @@ typedef struct mmf_state mmf_state;   /* opaque */
 /* Validate a block's weights and build its launch descriptors. The device
  * buffers named in `w` are NOT copied: they must stay valid and unchanged
  * until mmf_block_destroy. The handle is host memory owned by the library.
+ * For the prefill contraction the library also keeps the seven matrices' codes
+ * one byte per weight (the stored value w + 1; 4x the packed size, e.g. 303 MB
+ * for a 24-block d=1024 / I=2816 stack): it allocates them with cudaMalloc on
+ * the current device, fills them with one kernel on the legacy default stream,
+ * waits for it, and frees them in mmf_block_destroy. The environment variable
+ * MMF_PREFILL_UNPACKED=0 turns the copy off, and when the memory cannot be
+ * allocated the block goes without it (the contraction then expands the packed
+ * codes in shared memory; same results).
  * Errors: INVALID_ARG, UNSUPPORTED_SHAPE, MISALIGNED, NOMEM, CUDA. */
 mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, int32_t I, mmf_block** out);
 void mmf_block_destroy(mmf_block* blk);

@@ -226,6 +226,13 @@ mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& q
   return MMF_OK;
 }
 
+// Blocks keep one-byte copies of their codes for the prefill contraction
+// (4x the packed weight memory) unless MMF_PREFILL_UNPACKED=0.
+bool prefill_unpacked_enabled() {
+  const char* e = getenv("MMF_PREFILL_UNPACKED");
+  return e == nullptr || strcmp(e, "0") != 0;
+}
+
 mmf_status check_tlinear(const mmf_tlinear* l, const char* name) {
   if (l == nullptr) return fail(MMF_ERR_INVALID_ARG, "%s: null layer", name);
   if (l->packed == nullptr || l->gamma == nullptr) return fail(MMF_ERR_INVALID_ARG, "%s: null packed/gamma", name);
@@ -275,9 +282,12 @@ void mmf::set_last_error(const char* msg) { g_last_error = msg; }
 
 // ------------------------------------------------------------------ handles
 
+// wu: one-byte copies of the seven matrices' codes (f, c, g, o, gate, up,
+// down), made at creation for the prefill contraction; all null when disabled.
 struct mmf_block {
   mmf_block_weights w;
   int d, I;
+  uint8_t* wu[7];
 };
 
 struct mmf_state {
@@ -431,13 +441,18 @@ mmf_status check_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_t
 // gate's RMSNorm gain (gate and up share it), p with the down projection's.
 mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tlinear* down, const void* x,
                    const void* residual, void* y, int M, mmf_dtype dt, float eps, void* p, const QAct& qa,
-                   cudaStream_t s) {
+                   cudaStream_t s, const uint8_t* const* wu = nullptr /* gate, up, down one-byte codes */) {
   const mmf_tlinear* gu[2] = {gate, up};
   TGemmArgs a = gemm_args(gu, 2, qa.q, qa.s, qa.qsum, M, p, gate->N, nullptr, nullptr);
+  if (wu) {
+    a.wu[0] = wu[0];
+    a.wu[1] = wu[1];
+  }
   mmf_status r = quant_gemm(x, gate->gain, eps, qa, a, Epi::kGlu, dt, s, "gate_up", false);
   if (r != MMF_OK) return r;
   const mmf_tlinear* dn[1] = {down};
   TGemmArgs b = gemm_args(dn, 1, qa.q, qa.s, qa.qsum, M, y, down->N, residual, nullptr);
+  if (wu) b.wu[0] = wu[2];
   return quant_gemm(p, down->gain, eps, qa, b, Epi::kStore, dt, s, "down", false);
 }
 
@@ -496,11 +511,49 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
   b->w = *w;
   b->d = d;
   b->I = I;
+  for (int i = 0; i < 7; ++i) b->wu[i] = nullptr;
+  if (prefill_unpacked_enabled()) {
+    // the copy only speeds prefill up: without device memory for it the block
+    // keeps using the packed codes
+    const mmf_tlinear* all[7] = {&w->f, &w->c, &w->g, &w->o, &w->gate, &w->up, &w->down};
+    bool have = true;
+    for (int i = 0; i < 7 && have; ++i) {
+      if (cudaMalloc(&b->wu[i], (size_t)all[i]->N * all[i]->K) != cudaSuccess) {
+        b->wu[i] = nullptr;
+        have = false;
+      }
+    }
+    if (!have) {
+      (void)cudaGetLastError();   // clear the allocation error
+      for (int i = 0; i < 7; ++i) {
+        cudaFree(b->wu[i]);
+        b->wu[i] = nullptr;
+      }
+    }
+    for (int i = 0; i < 7 && have; ++i) {
+      cudaError_t e = launch_unpack_codes(all[i]->packed, all[i]->N, all[i]->K, b->wu[i], 0);
+      if (e != cudaSuccess) {
+        mmf_block_destroy(b);
+        return cuda_fail(e, "mmf_block_create: unpack codes");
+      }
+    }
+    if (have) {
+      cudaError_t e = cudaStreamSynchronize(0);
+      if (e != cudaSuccess) {
+        mmf_block_destroy(b);
+        return cuda_fail(e, "mmf_block_create: synchronise");
+      }
+    }
+  }
   *out = b;
   return MMF_OK;
 }
 
-extern "C" void mmf_block_destroy(mmf_block* blk) { delete blk; }
+extern "C" void mmf_block_destroy(mmf_block* blk) {
+  if (!blk) return;
+  for (int i = 0; i < 7; ++i) cudaFree(blk->wu[i]);
+  delete blk;
+}
 
 extern "C" mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_state** out) {
   if (!out) return fail(MMF_ERR_INVALID_ARG, "mmf_state_create: null out");
@@ -600,6 +653,7 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   const mmf_block_weights& W = blk->w;
   const mmf_tlinear* fcg[3] = {&W.f, &W.c, &W.g};
   TGemmArgs tm = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, nullptr);
+  for (int i = 0; i < 3; ++i) tm.wu[i] = blk->wu[i];
   const bool fused_mixer = T > 1 && fused_mlgru_enabled() && gemm_uses_tc(tm, Epi::kStore) &&
                            tgemm_tc_mlgru_supported(tm, T, d);
   // prefill: the scan's scratch is reset here, so that the kernels that read
@@ -625,6 +679,7 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
     if (r != MMF_OK) return r;
   } else {
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.pre, 3 * d, nullptr, nullptr);
+    for (int i = 0; i < 3; ++i) a.wu[i] = blk->wu[i];
     mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", false);
     if (r != MMF_OK) return r;
     int* status = nullptr;
@@ -635,10 +690,11 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   }
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
+  b.wu[0] = blk->wu[3];
   mmf_status r = quant_gemm(w.og, W.o.gain, eps, w.qa, b, Epi::kStore, dt, s, "o", false);
   if (r != MMF_OK) return r;
   // channel mixer
-  return run_glu(&W.gate, &W.up, &W.down, w.y1, w.y1, y, M, dt, eps, w.p, w.qa, s);
+  return run_glu(&W.gate, &W.up, &W.down, w.y1, w.y1, y, M, dt, eps, w.p, w.qa, s, blk->wu + 4);
 }
 
 mmf_status check_forward_args(const mmf_block* blk, mmf_state* st, const void* x, void* y, int B, int T,

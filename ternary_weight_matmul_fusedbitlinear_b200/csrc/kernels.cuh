@@ -40,6 +40,9 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
 void set_last_error(const char* msg);
 
 size_t quantize_weights_ws_bytes();
+// Packed codes [N, K/16] -> one byte per weight [N, K] holding the stored code
+// w + 1 (K % 16 == 0; `out` 16-byte aligned).
+cudaError_t launch_unpack_codes(const uint32_t* packed, int N, int K, uint8_t* out, cudaStream_t stream);
 cudaError_t launch_quantize_weights(const float* W, int N, int K, uint32_t* packed, float* gamma, void* ws,
                                     cudaStream_t stream);
 
@@ -57,6 +60,8 @@ enum class Epi : int {
 
 struct TGemmArgs {
   const uint32_t* w[3];     // packed ternary weights per segment, [N, K/16]
+  const uint8_t* wu[3];     // optional: the same codes one byte per weight, [N, K] (tcgen05 path reads
+                            // them with TMA instead of unpacking the packed words); null = not available
   const float* gamma[3];    // per-segment scale (device scalar)
   const float* bias[3];     // per-segment bias [N] or null
   int nseg;                 // 1..3

@@ -81,7 +81,25 @@ __global__ void __launch_bounds__(kThreads) ternarize_pack_kernel(const float* _
   }
 }
 
+// One thread per packed word: the 16 stored codes (w + 1) of columns
+// 16j .. 16j+15 as 16 bytes, in column order.
+__global__ void __launch_bounds__(kThreads) unpack_codes_kernel(const uint32_t* __restrict__ packed, size_t nwords,
+                                                                uint4* __restrict__ out) {
+  for (size_t w = (size_t)blockIdx.x * kThreads + threadIdx.x; w < nwords; w += (size_t)gridDim.x * kThreads) {
+    const uint32_t v = packed[w];
+    out[w] = make_uint4(v & 0x03030303u, (v >> 2) & 0x03030303u, (v >> 4) & 0x03030303u, (v >> 6) & 0x03030303u);
+  }
+}
+
 }  // namespace
+
+cudaError_t launch_unpack_codes(const uint32_t* packed, int N, int K, uint8_t* out, cudaStream_t stream) {
+  const size_t nwords = (size_t)N * (K / 16);
+  if (nwords == 0) return cudaSuccess;
+  const int blocks = (int)std::min<size_t>((nwords + kThreads - 1) / kThreads, (size_t)148 * 16);
+  unpack_codes_kernel<<<blocks, kThreads, 0, stream>>>(packed, nwords, reinterpret_cast<uint4*>(out));
+  return cudaGetLastError();
+}
 
 size_t quantize_weights_ws_bytes() { return sizeof(double) * kQuantPartials; }
 

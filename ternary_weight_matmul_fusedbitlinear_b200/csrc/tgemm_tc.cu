@@ -20,7 +20,12 @@
 //   warps 6..9  unpack: packed 2-bit codes -> int8 bytes written directly in
 //               the SW128 K-major layout the MMA reads, 2-deep ring
 // Two TMEM accumulators (2 x 256 columns) let the epilogue of one tile overlap
-// the main loop of the next. Every mbarrier wait is bounded: on timeout the
+// the main loop of the next.
+// Variant UNP: when the codes are also held one byte per weight in HBM (a
+// block keeps such a copy for prefill), the producer TMA-loads the weight tile
+// straight into the SW128 layout next to the activation tile (3-stage ring of
+// 16 + 32 KiB) and the unpack warps stay idle; unpacking 32 KiB per k-step
+// through shared memory was the largest cost of the main loop. Every mbarrier wait is bounded: on timeout the
 // kernel records an error in the status word, raises a CTA-wide abort flag,
 // and all roles leave their loops; nothing traps.
 #include "kernels.cuh"
@@ -45,15 +50,18 @@ constexpr uint32_t kTmemCols = 512;
 
 // Shared memory; OB = bytes of one output element (2: bf16, 4: fp32 / int32).
 // The TMA ring is 4 deep for 2-byte outputs and 3 deep for 4-byte outputs,
-// whose staging boxes are twice as large.
-template <int OB>
+// whose staging boxes are twice as large; 3 deep (with a weight tile per
+// stage) for UNP.
+template <int OB, bool UNP>
 struct __align__(1024) SmemLayout {
-  static constexpr int NS = OB == 2 ? 4 : 3;
+  static constexpr int NS = UNP ? 3 : (OB == 2 ? 4 : 3);
+  static constexpr int NBU = UNP ? NS : NB;        // int8 weight tiles: per TMA stage (UNP) or unpack ring
+  static constexpr int NBP = UNP ? 1 : NS;         // packed weight tiles (unused with UNP)
   static constexpr int kStageBytes = 32 * kEpiChunk * OB;
   uint8_t a[NS][A_BYTES];                          // 1024-aligned: SW128 atoms
-  uint8_t bu[NB][BU_BYTES];                        // 1024-aligned: SW128 atoms
+  uint8_t bu[NBU][BU_BYTES];                       // 1024-aligned: SW128 atoms
   uint8_t stage[kEpiWarps][2][kStageBytes];        // epilogue staging, double-buffered (1024-aligned)
-  uint32_t bp[NS][BP_BYTES / 4];
+  uint32_t bp[NBP][BP_BYTES / 4];
   uint64_t tma_full[NS];
   uint64_t tma_empty[NS];
   uint64_t bu_full[NB];
@@ -93,14 +101,14 @@ __device__ __forceinline__ void half_source(const TcArgs& p, Epi epi, int nt, in
   }
 }
 
-template <Epi EPI, typename T>
+template <Epi EPI, typename T, bool UNP>
 __global__ void __launch_bounds__(kThreads, 1)
     tgemm_tc_kernel(const __grid_constant__ CUtensorMap map_a, const __grid_constant__ CUtensorMap map_b0,
                     const __grid_constant__ CUtensorMap map_b1, const __grid_constant__ CUtensorMap map_b2,
                     const __grid_constant__ CUtensorMap map_out, const __grid_constant__ CUtensorMap map_res,
                     const TcArgs p) {
   constexpr int OB = EPI == Epi::kAcc ? 4 : (int)sizeof(T);
-  using Smem = SmemLayout<OB>;
+  using Smem = SmemLayout<OB, UNP>;
   constexpr int NS = Smem::NS;
   extern __shared__ uint8_t smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -158,10 +166,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % NS;
           if (!mbar_wait(&sm.tma_empty[s], ((it / NS) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
-          mbar_arrive_expect_tx(&sm.tma_full[s], A_BYTES + BP_BYTES);
-          tma_load_2d(sm.a[s], &map_a, kb * BK, mt * BM, &sm.tma_full[s]);
-          tma_load_2d(&sm.bp[s][0], maps[seg0], kb * (BK / 16), row0, &sm.tma_full[s]);
-          tma_load_2d(&sm.bp[s][HALF * (BK / 16)], maps[seg1], kb * (BK / 16), row1, &sm.tma_full[s]);
+          if constexpr (UNP) {   // int8 weight rows straight into the SW128 tile of this stage
+            mbar_arrive_expect_tx(&sm.tma_full[s], A_BYTES + BU_BYTES);
+            tma_load_2d(sm.a[s], &map_a, kb * BK, mt * BM, &sm.tma_full[s]);
+            tma_load_2d(sm.bu[s], maps[seg0], kb * BK, row0, &sm.tma_full[s]);
+            tma_load_2d(sm.bu[s] + HALF * BK, maps[seg1], kb * BK, row1, &sm.tma_full[s]);
+          } else {
+            mbar_arrive_expect_tx(&sm.tma_full[s], A_BYTES + BP_BYTES);
+            tma_load_2d(sm.a[s], &map_a, kb * BK, mt * BM, &sm.tma_full[s]);
+            tma_load_2d(&sm.bp[s][0], maps[seg0], kb * (BK / 16), row0, &sm.tma_full[s]);
+            tma_load_2d(&sm.bp[s][HALF * (BK / 16)], maps[seg1], kb * (BK / 16), row1, &sm.tma_full[s]);
+          }
         }
       }
       // let every copy this thread issued land before the CTA can exit
@@ -180,8 +195,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
-          const int s = it % NS, u = it % NB;
-          if (!mbar_wait(&sm.bu_full[u], (it / NB) & 1, abort_flag, p.status) ||
+          const int s = it % NS, u = UNP ? s : (int)(it % NB);
+          if ((!UNP && !mbar_wait(&sm.bu_full[u], (it / NB) & 1, abort_flag, p.status)) ||
               !mbar_wait(&sm.tma_full[s], (it / NS) & 1, abort_flag, p.status)) {
             ok = false;
             break;
@@ -193,7 +208,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < BK / 32; ++j)   // advance 32 bytes of K inside the swizzle atom
             umma_i8(d_tmem, adesc + (uint64_t)(2 * j), bdesc + (uint64_t)(2 * j), kIdesc, (kb | j) != 0);
           umma_commit(&sm.tma_empty[s]);
-          umma_commit(&sm.bu_empty[u]);
+          if constexpr (!UNP) umma_commit(&sm.bu_empty[u]);
         }
         if (ok) umma_commit(&sm.tmem_full[acc]);
       }
@@ -202,7 +217,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_wait(&sm.mma_drain, 0, abort_flag, nullptr);
     }
   } else if (warp >= kUnpackWarp0) {
-    // ------------------------------------------------------------ unpack 2-bit codes to int8
+    // ------------------------------------------------------------ unpack 2-bit codes to int8 (idle with UNP)
+    if constexpr (!UNP) {
     // 512 (row, half-row) units per K-step; unit id = tid + 128 i reads the 16
     // bytes at id * 16 of the packed tile (row id/2, columns 64 (id%2) ..+63),
     // so each warp reads 512 contiguous bytes; writes land in distinct banks.
@@ -240,6 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         fence_proxy_async_smem();
         mbar_arrive(&sm.bu_full[u]);
       }
+    }
     }
   } else {
     // ------------------------------------------------------------ epilogue (8 warps)
@@ -362,7 +379,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ---------------------------------------------------------------- host side
-template <Epi EPI, typename T>
+template <Epi EPI, typename T, bool UNP>
 cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap (&mb)[3], const TcArgs& p, cudaStream_t stream) {
   CUtensorMap mo;
   const bool acc_out = EPI == Epi::kAcc;
@@ -377,8 +394,8 @@ cudaError_t launch_typed(const CUtensorMap& ma, const CUtensorMap (&mb)[3], cons
   if (EPI == Epi::kStore && p.g.residual != nullptr &&
       !make_tma_2d(&mr, p.g.residual, odt, esize, (uint64_t)p.g.N, (uint64_t)p.g.M, kEpiChunk, 32, oswz))
     return cudaErrorInvalidValue;
-  const size_t smem = sizeof(SmemLayout<(EPI == Epi::kAcc ? 4 : (int)sizeof(T))>) + 1024;
-  auto kern = tgemm_tc_kernel<EPI, T>;
+  const size_t smem = sizeof(SmemLayout<(EPI == Epi::kAcc ? 4 : (int)sizeof(T)), UNP>) + 1024;
+  auto kern = tgemm_tc_kernel<EPI, T, UNP>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const int tiles = p.m_tiles * p.n_tiles;
@@ -403,11 +420,15 @@ cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* stat
   if (!make_tma_2d(&ma, a.q, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.K, (uint64_t)a.M, BK, BM,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return cudaErrorInvalidValue;
+  bool unp = true;   // every segment has its one-byte copy
+  for (int r = 0; r < a.nseg; ++r) unp = unp && a.wu[r] != nullptr;
   for (int r = 0; r < 3; ++r) {
     const int src = r < a.nseg ? r : 0;
-    if (!make_tma_2d(&mb[r], a.w[src], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(a.K / 16), (uint64_t)a.N, BK / 16,
-                  HALF, CU_TENSOR_MAP_SWIZZLE_NONE))
-      return cudaErrorInvalidValue;
+    const bool ok = unp ? make_tma_2d(&mb[r], a.wu[src], CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, (uint64_t)a.K, (uint64_t)a.N,
+                                      BK, HALF, CU_TENSOR_MAP_SWIZZLE_128B)
+                        : make_tma_2d(&mb[r], a.w[src], CU_TENSOR_MAP_DATA_TYPE_UINT32, 4, (uint64_t)(a.K / 16),
+                                      (uint64_t)a.N, BK / 16, HALF, CU_TENSOR_MAP_SWIZZLE_NONE);
+    if (!ok) return cudaErrorInvalidValue;
   }
   TcArgs p;
   p.g = a;
@@ -415,16 +436,16 @@ cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* stat
   p.m_tiles = ceil_div(a.M, BM);
   p.n_tiles = (epi == Epi::kGlu) ? ceil_div(a.N, HALF) : ceil_div(a.nseg * a.N, BN);
   const bool b = dt == MMF_BF16;
+#define MMF_TC_LAUNCH(E)                                                                                      \
+  (unp ? (b ? launch_typed<E, bf16, true>(ma, mb, p, stream) : launch_typed<E, float, true>(ma, mb, p, stream)) \
+       : (b ? launch_typed<E, bf16, false>(ma, mb, p, stream) : launch_typed<E, float, false>(ma, mb, p, stream)))
   switch (epi) {
-    case Epi::kStore:
-      return b ? launch_typed<Epi::kStore, bf16>(ma, mb, p, stream) : launch_typed<Epi::kStore, float>(ma, mb, p, stream);
-    case Epi::kAcc:
-      return b ? launch_typed<Epi::kAcc, bf16>(ma, mb, p, stream) : launch_typed<Epi::kAcc, float>(ma, mb, p, stream);
-    case Epi::kGlu:
-      return b ? launch_typed<Epi::kGlu, bf16>(ma, mb, p, stream) : launch_typed<Epi::kGlu, float>(ma, mb, p, stream);
-    default:
-      return cudaErrorNotSupported;
+    case Epi::kStore: return MMF_TC_LAUNCH(Epi::kStore);
+    case Epi::kAcc: return MMF_TC_LAUNCH(Epi::kAcc);
+    case Epi::kGlu: return MMF_TC_LAUNCH(Epi::kGlu);
+    default: return cudaErrorNotSupported;
   }
+#undef MMF_TC_LAUNCH
 }
 
 }  // namespace mmf

@@ -261,6 +261,22 @@ def test_block_prefill_fused_mixer_chunked_equals_whole(monkeypatch):
     assert_close(to_np(torch.cat([ya, yb], 1)), to_np(y1), "bf16", "chunked vs whole")
 
 
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_block_prefill_unpacked_copy_is_bit_identical(dtype, monkeypatch):
+    # a block keeps one-byte copies of its codes for the prefill contraction
+    # (TMA-loaded instead of expanded in shared memory): identical results
+    d, inner, B, T = 256, 768, 2, 192
+    x = synth.activations(7042, B * T, d, TORCH_DT[dtype]).reshape(B, T, d).cuda()
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MMF_PREFILL_UNPACKED", flag)
+        blk, _ = make_block(7041, d, inner)
+        st = mmf.State(1, B, d)
+        outs.append((mmf.block_forward(blk, 0, st, x), st.get()))
+    mmf.check()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
 def test_block_prefill_then_decode_matches_oracle_bf16():
     d, inner, B, T = 256, 768, 2, 40
     blk, oblk = make_block(7003, d, inner)
