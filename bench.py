@@ -22,6 +22,7 @@ workload on this host's cores (the baseline arm; rank 0 only).
 from __future__ import annotations
 
 import argparse
+import dataclasses
 import json
 import os
 import statistics
@@ -60,6 +61,10 @@ def parse_args(argv=None):
                          "decode1p3b / decode2p7b: the 1.3B / 2.7B-shaped stacks, prompt prefill then decode "
                          "steps (output fed back, state carried), each step one CUDA graph")
     ap.add_argument("--batch", type=int, default=None, help="decode2p7b: concurrent sequences (1, 8 or 64)")
+    ap.add_argument("--packed-only", action="store_true",
+                    help="bitlinear: contract from the 2-bit codes only (no one-byte copy of the codes)")
+    ap.add_argument("--layers", type=int, default=None,
+                    help="stack370m: number of blocks (default 24; fewer for short profiler captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) pass")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     return ap.parse_args(argv)
@@ -170,8 +175,13 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
-def stack_workload():
-    return synth.STACK_370M
+def stack_workload(layers=None):
+    """The 370M-shaped stack; `layers` overrides the block count (a one-block run has the same
+    kernel shapes, for short profiler captures), and the workload name then says so."""
+    w = synth.STACK_370M
+    if layers is not None and layers != w.layers:
+        w = dataclasses.replace(w, layers=layers, name=f"{w.name}_layers{layers}")
+    return w
 
 
 def gemm_ops_per_step(w) -> float:
@@ -266,7 +276,7 @@ def run_mmf(args):
     import ternary_weight_matmul_fusedbitlinear_b200 as mmf
     mmf.load()
     dev = torch.device("cuda", local)
-    w = stack_workload()
+    w = stack_workload(args.layers)
     peaks, peak_kind = load_peaks()
 
     blocks = build_stack(w, dev)
@@ -413,6 +423,8 @@ def run_bitlinear(args):
     M, K, N = 16384, 1024, 5632
     peaks, peak_kind = load_peaks()
     lin = mmf.quantize_weights(synth.latent_weight(synth.sub_seed(1002, 0, synth.PROJ_GATE), N, K, device=dev))
+    if not args.packed_only:   # one byte per weight as well: the prefill contraction loads it directly
+        lin = mmf.unpack_codes(lin)
     x = synth.activations(1002 + rank, M, K, torch.bfloat16, device=dev)
     y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
     ws = torch.empty(mmf.api.L.load().mmf_bitlinear_ws_size(M, K), dtype=torch.uint8, device=dev)
@@ -448,7 +460,8 @@ def run_bitlinear(args):
             "metric": METRIC, "value": world * M * args.steps / (total_ms / 1e3), "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": f"bitlinear_prefill_m{M}_k{K}_n{N}_bf16", "l2": "flushed between timed steps"},
+            "config": {"workload": f"bitlinear_prefill_m{M}_k{K}_n{N}_bf16", "l2": "flushed between timed steps",
+                       "weight_codes": "2-bit packed only" if args.packed_only else "2-bit packed + one byte per weight"},
             "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                          "frac": achieved / peak, "traffic": None, "kernel": ",".join(gemm),
                          "peak_source": f"{peak_kind}: bf16 burst x {INT8_OVER_BF16}",

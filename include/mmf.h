@@ -82,6 +82,10 @@ mmf_status mmf_check(void* stream);
  *   gamma  (device) one float: the absmean weight scale of the whole matrix.
  *   gain   (device) float [K] RMSNorm gain, or NULL for all ones.
  *   bias   (device) float [N], or NULL for all zeros.
+ *   codes  (device) uint8 [N, K], or NULL: the same stored values one byte per
+ *          weight (mmf_unpack_codes builds it). When given, prefill-sized
+ *          contractions load it directly instead of expanding `packed` in
+ *          shared memory (same results; 4x the memory). It must match `packed`.
  * The struct itself is read during the call only. */
 typedef struct mmf_tlinear {
   const uint32_t* packed;
@@ -90,6 +94,7 @@ typedef struct mmf_tlinear {
   const float* bias;
   int32_t N;
   int32_t K;
+  const uint8_t* codes;
 } mmf_tlinear;
 
 /* Scratch bytes mmf_quantize_weights needs for an N x K matrix. */
@@ -109,6 +114,15 @@ size_t mmf_quantize_weights_ws_size(int32_t N, int32_t K);
  *         MISALIGNED, WORKSPACE. */
 mmf_status mmf_quantize_weights(const float* W, int32_t N, int32_t K, uint32_t* packed,
                                 float* gamma, void* ws, size_t ws_bytes, void* stream);
+
+/* One byte per weight from the packed codes: codes[n, k] = the stored value
+ * w + 1 of column k of row n (format as in mmf_tlinear), for the optional
+ * mmf_tlinear.codes. Asynchronous on stream.
+ *   packed (device) uint32 [N, K/16], read only
+ *   codes  (device) uint8 [N, K], output, 16-byte aligned
+ * Errors: INVALID_ARG (null, N or K < 1), UNSUPPORTED_SHAPE (K % 16 != 0),
+ *         MISALIGNED, CUDA. */
+mmf_status mmf_unpack_codes(const uint32_t* packed, int32_t N, int32_t K, uint8_t* codes, void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* FusedBitLinear                                                             */
@@ -203,11 +217,12 @@ typedef struct mmf_state mmf_state;   /* opaque */
 /* Validate a block's weights and build its launch descriptors. The device
  * buffers named in `w` are NOT copied: they must stay valid and unchanged
  * until mmf_block_destroy. The handle is host memory owned by the library.
- * For the prefill contraction the library also keeps the seven matrices' codes
- * one byte per weight (the stored value w + 1; 4x the packed size, e.g. 303 MB
- * for a 24-block d=1024 / I=2816 stack): it allocates them with cudaMalloc on
- * the current device, fills them with one kernel on the legacy default stream,
- * waits for it, and frees them in mmf_block_destroy. The environment variable
+ * For the prefill contraction the block uses each matrix's codes one byte per
+ * weight: the caller's mmf_tlinear.codes when given, otherwise a copy the
+ * library makes (4x the packed size, e.g. 303 MB for a 24-block d=1024 /
+ * I=2816 stack): it allocates them with cudaMalloc on the current device,
+ * fills them with one kernel on the legacy default stream, waits for it, and
+ * frees them in mmf_block_destroy. The environment variable
  * MMF_PREFILL_UNPACKED=0 turns the copy off, and when the memory cannot be
  * allocated the block goes without it (the contraction then expands the packed
  * codes in shared memory; same results).

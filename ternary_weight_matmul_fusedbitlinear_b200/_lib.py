@@ -22,7 +22,8 @@ c_f = ctypes.c_float
 
 
 class TLinear(ctypes.Structure):
-    _fields_ = [("packed", c_vp), ("gamma", c_vp), ("gain", c_vp), ("bias", c_vp), ("N", c_i32), ("K", c_i32)]
+    _fields_ = [("packed", c_vp), ("gamma", c_vp), ("gain", c_vp), ("bias", c_vp), ("N", c_i32), ("K", c_i32),
+                ("codes", c_vp)]
 
 
 class BitlinearDebug(ctypes.Structure):
@@ -40,6 +41,7 @@ SIGNATURES = {
     "mmf_check": (ctypes.c_int, [c_vp]),
     "mmf_quantize_weights_ws_size": (c_sz, [c_i32, c_i32]),
     "mmf_quantize_weights": (ctypes.c_int, [c_vp, c_i32, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "mmf_unpack_codes": (ctypes.c_int, [c_vp, c_i32, c_i32, c_vp, c_vp]),
     "mmf_bitlinear_ws_size": (c_sz, [c_i32, c_i32]),
     "mmf_bitlinear": (ctypes.c_int, [ctypes.POINTER(TLinear), c_vp, ctypes.c_int, c_i32, c_vp, c_f, c_vp, c_sz,
                                      c_vp, ctypes.POINTER(BitlinearDebug)]),

@@ -59,18 +59,31 @@ def check(stream: Optional[torch.cuda.Stream] = None) -> None:
 
 
 class TLinear:
-    """A ternary BitLinear held on the device: packed [N, K/16] (int32 storage of uint32), gamma [1]."""
+    """A ternary BitLinear held on the device: packed [N, K/16] (int32 storage of uint32), gamma [1],
+    optionally codes [N, K] uint8 (the same codes one byte per weight, see unpack_codes)."""
 
     def __init__(self, packed: torch.Tensor, gamma: torch.Tensor, N: int, K: int,
-                 gain: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None):
-        _need_cuda(packed, gamma, gain, bias)
-        self.packed, self.gamma, self.gain, self.bias = packed, gamma, gain, bias
+                 gain: Optional[torch.Tensor] = None, bias: Optional[torch.Tensor] = None,
+                 codes: Optional[torch.Tensor] = None):
+        _need_cuda(packed, gamma, gain, bias, codes)
+        self.packed, self.gamma, self.gain, self.bias, self.codes = packed, gamma, gain, bias, codes
         self.N, self.K = int(N), int(K)
 
     def c(self) -> L.TLinear:
         return L.TLinear(self.packed.data_ptr(), self.gamma.data_ptr(),
                          self.gain.data_ptr() if self.gain is not None else None,
-                         self.bias.data_ptr() if self.bias is not None else None, self.N, self.K)
+                         self.bias.data_ptr() if self.bias is not None else None, self.N, self.K,
+                         self.codes.data_ptr() if self.codes is not None else None)
+
+
+def unpack_codes(lin: TLinear) -> TLinear:
+    """The same layer with its codes also held one byte per weight (mmf_unpack_codes), which the
+    prefill contraction loads directly instead of expanding the packed words."""
+    lib = L.load()
+    codes = torch.empty((lin.N, lin.K), dtype=torch.uint8, device=lin.packed.device)
+    L.check(lib.mmf_unpack_codes(_vp(lin.packed), lin.N, lin.K, _vp(codes), _stream(lin.packed.device)),
+            "mmf_unpack_codes")
+    return TLinear(lin.packed, lin.gamma, lin.N, lin.K, lin.gain, lin.bias, codes)
 
 
 def quantize_weights(W: torch.Tensor, gain: Optional[torch.Tensor] = None,

@@ -239,8 +239,8 @@ mmf_status check_tlinear(const mmf_tlinear* l, const char* name) {
   if (l->N < 1 || l->K < 1) return fail(MMF_ERR_INVALID_ARG, "%s: N=%d K=%d must be >= 1", name, l->N, l->K);
   if (l->K % 16 != 0) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "%s: K=%d is not a multiple of 16", name, l->K);
   if (!aligned16(l->packed)) return fail(MMF_ERR_MISALIGNED, "%s: packed not 16-byte aligned", name);
-  if ((l->gain && !aligned16(l->gain)) || (l->bias && !aligned16(l->bias)))
-    return fail(MMF_ERR_MISALIGNED, "%s: gain/bias not 16-byte aligned", name);
+  if ((l->gain && !aligned16(l->gain)) || (l->bias && !aligned16(l->bias)) || (l->codes && !aligned16(l->codes)))
+    return fail(MMF_ERR_MISALIGNED, "%s: gain/bias/codes not 16-byte aligned", name);
   return MMF_OK;
 }
 
@@ -250,6 +250,7 @@ TGemmArgs gemm_args(const mmf_tlinear* const* segs, int nseg, const int8_t* q, c
   for (int i = 0; i < 3; ++i) {
     const mmf_tlinear* l = segs[i < nseg ? i : 0];
     a.w[i] = l->packed;
+    a.wu[i] = l->codes;
     a.gamma[i] = l->gamma;
     a.bias[i] = l->bias;
   }
@@ -282,12 +283,14 @@ void mmf::set_last_error(const char* msg) { g_last_error = msg; }
 
 // ------------------------------------------------------------------ handles
 
-// wu: one-byte copies of the seven matrices' codes (f, c, g, o, gate, up,
-// down), made at creation for the prefill contraction; all null when disabled.
+// wu: one-byte codes of the seven matrices (f, c, g, o, gate, up, down) for
+// the prefill contraction: the caller's mmf_tlinear.codes, or copies made at
+// creation (owned[i]); all null when disabled.
 struct mmf_block {
   mmf_block_weights w;
   int d, I;
-  uint8_t* wu[7];
+  const uint8_t* wu[7];
+  uint8_t* owned[7];
 };
 
 struct mmf_state {
@@ -347,6 +350,15 @@ extern "C" size_t mmf_bitlinear_ws_size(int32_t M, int32_t K) {
   Carver c(nullptr);
   carve_qact(c, M, K);
   return c.off + 256;
+}
+
+extern "C" mmf_status mmf_unpack_codes(const uint32_t* packed, int32_t N, int32_t K, uint8_t* codes, void* stream) {
+  if (!packed || !codes) return fail(MMF_ERR_INVALID_ARG, "mmf_unpack_codes: null pointer");
+  if (N < 1 || K < 1) return fail(MMF_ERR_INVALID_ARG, "mmf_unpack_codes: N=%d K=%d", N, K);
+  if (K % 16 != 0) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_unpack_codes: K=%d %% 16 != 0", K);
+  if (!aligned16(packed) || !aligned16(codes)) return fail(MMF_ERR_MISALIGNED, "mmf_unpack_codes");
+  MMF_CUDA(launch_unpack_codes(packed, N, K, codes, as_stream(stream)), "mmf_unpack_codes");
+  return MMF_OK;
 }
 
 extern "C" mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_dtype dtype, int32_t M, void* y,
@@ -447,7 +459,7 @@ mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tli
   if (wu) {
     a.wu[0] = wu[0];
     a.wu[1] = wu[1];
-  }
+  }   // otherwise the layers' own codes (if any), set by gemm_args
   mmf_status r = quant_gemm(x, gate->gain, eps, qa, a, Epi::kGlu, dt, s, "gate_up", false);
   if (r != MMF_OK) return r;
   const mmf_tlinear* dn[1] = {down};
@@ -511,33 +523,42 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
   b->w = *w;
   b->d = d;
   b->I = I;
-  for (int i = 0; i < 7; ++i) b->wu[i] = nullptr;
+  const mmf_tlinear* all[7] = {&w->f, &w->c, &w->g, &w->o, &w->gate, &w->up, &w->down};
+  for (int i = 0; i < 7; ++i) {
+    b->wu[i] = all[i]->codes;
+    b->owned[i] = nullptr;
+  }
   if (prefill_unpacked_enabled()) {
-    // the copy only speeds prefill up: without device memory for it the block
-    // keeps using the packed codes
-    const mmf_tlinear* all[7] = {&w->f, &w->c, &w->g, &w->o, &w->gate, &w->up, &w->down};
+    // copies for the matrices the caller gave no codes for; they only speed
+    // prefill up, so without device memory for them the block keeps using the
+    // packed codes
     bool have = true;
     for (int i = 0; i < 7 && have; ++i) {
-      if (cudaMalloc(&b->wu[i], (size_t)all[i]->N * all[i]->K) != cudaSuccess) {
-        b->wu[i] = nullptr;
+      if (b->wu[i] != nullptr) continue;
+      if (cudaMalloc(&b->owned[i], (size_t)all[i]->N * all[i]->K) != cudaSuccess) {
+        b->owned[i] = nullptr;
         have = false;
       }
     }
     if (!have) {
       (void)cudaGetLastError();   // clear the allocation error
       for (int i = 0; i < 7; ++i) {
-        cudaFree(b->wu[i]);
-        b->wu[i] = nullptr;
+        cudaFree(b->owned[i]);
+        b->owned[i] = nullptr;
       }
     }
+    bool launched = false;
     for (int i = 0; i < 7 && have; ++i) {
-      cudaError_t e = launch_unpack_codes(all[i]->packed, all[i]->N, all[i]->K, b->wu[i], 0);
+      if (b->owned[i] == nullptr) continue;
+      cudaError_t e = launch_unpack_codes(all[i]->packed, all[i]->N, all[i]->K, b->owned[i], 0);
       if (e != cudaSuccess) {
         mmf_block_destroy(b);
         return cuda_fail(e, "mmf_block_create: unpack codes");
       }
+      b->wu[i] = b->owned[i];
+      launched = true;
     }
-    if (have) {
+    if (launched) {
       cudaError_t e = cudaStreamSynchronize(0);
       if (e != cudaSuccess) {
         mmf_block_destroy(b);
@@ -551,7 +572,7 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
 
 extern "C" void mmf_block_destroy(mmf_block* blk) {
   if (!blk) return;
-  for (int i = 0; i < 7; ++i) cudaFree(blk->wu[i]);
+  for (int i = 0; i < 7; ++i) cudaFree(blk->owned[i]);
   delete blk;
 }
 

@@ -277,6 +277,28 @@ def test_block_prefill_unpacked_copy_is_bit_identical(dtype, monkeypatch):
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
+@pytest.mark.parametrize("m", [128, 300])
+def test_bitlinear_and_glu_with_byte_codes_bit_identical(m):
+    # mmf_tlinear.codes (mmf_unpack_codes) lets the prefill contraction load the
+    # codes directly: identical outputs and debug values to the packed path
+    k, n = 1024, 768
+    _, lin, _ = make_layer(911, n, k)
+    lin_u = mmf.unpack_codes(lin)
+    codes_ref = O.unpack_codes(packed_to_np(lin.packed), k) + 1
+    np.testing.assert_array_equal(lin_u.codes.cpu().numpy().astype(np.int64), codes_ref)
+    x = synth.activations(912, m, k, torch.bfloat16).cuda()
+    for a, b, what in zip(mmf.bitlinear(lin, x, debug=True), mmf.bitlinear(lin_u, x, debug=True),
+                          ("y", "q", "s", "acc")):
+        assert torch.equal(a, b), what
+    _, gate, _ = make_layer(913, 768, k)
+    _, up, _ = make_layer(914, 768, k)
+    _, down, _ = make_layer(915, k, 768)
+    res = synth.activations(916, m, k, torch.bfloat16).cuda()
+    y1 = mmf.glu(gate, up, down, x, residual=res)
+    y2 = mmf.glu(mmf.unpack_codes(gate), mmf.unpack_codes(up), mmf.unpack_codes(down), x, residual=res)
+    assert torch.equal(y1, y2)
+
+
 def test_block_prefill_then_decode_matches_oracle_bf16():
     d, inner, B, T = 256, 768, 2, 40
     blk, oblk = make_block(7003, d, inner)
