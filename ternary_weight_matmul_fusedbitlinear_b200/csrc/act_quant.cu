@@ -244,11 +244,13 @@ cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, cons
   const size_t smem = sizeof(float) * (size_t)K;
   if (dt == MMF_BF16) {
     auto kern = rmsnorm_quant_kernel<bf16>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     kern<<<M, kThreads, smem, stream>>>(static_cast<const bf16*>(x), K, gain, eps, q, scale, qsum);
   } else {
     auto kern = rmsnorm_quant_kernel<float>;
-    if (smem > 48 * 1024) cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
     kern<<<M, kThreads, smem, stream>>>(static_cast<const float*>(x), K, gain, eps, q, scale, qsum);
   }
   return cudaGetLastError();

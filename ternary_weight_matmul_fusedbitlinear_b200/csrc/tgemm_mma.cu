@@ -274,7 +274,7 @@ constexpr size_t kFqBytes = 128 * 1024;   // fused-quantisation limit: codes + s
 template <int NT, int R, Epi EPI, typename T, bool SMEMW, bool FQ>
 cudaError_t launch_variant(const TGemmArgs& a, dim3 grid, size_t smem, cudaStream_t stream) {
   auto kern = tgemm_mma_kernel<NT, R, EPI, T, SMEMW, FQ>;
-  if (smem > 48 * 1024) {
+  if (smem > 0) {   // the default limit covers static + dynamic together, so opt in whenever there is any
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
   }

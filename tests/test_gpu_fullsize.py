@@ -68,7 +68,8 @@ def test_370m_block_full_batch_sampled_sequence():
     assert_close(st.get()[0, b:b + 1].numpy(), h_ref, "f32", "block h_T (sequence 5)", tol=E2E_TOL)
 
 
-@pytest.mark.parametrize("wl,batch", [(synth.STACK_1P3B, 4), (synth.STACK_2P7B, 64)])
+@pytest.mark.parametrize("wl,batch", [(synth.STACK_1P3B, 4), (synth.STACK_2P7B, 1), (synth.STACK_2P7B, 8),
+                                      (synth.STACK_2P7B, 64)])
 def test_decode_step_full_width(wl, batch):
     d, I = wl.d, wl.inner
     blk, oblk = make_block(wl.seed, d, I, layer=0)
