@@ -175,6 +175,14 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
+# DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture summarised in
+# profiles/tgemm_tc_stack370m_block.md: mean over the four contraction launches of one 370M block with
+# one-byte weight codes. Valid while that kernel is unchanged; None elsewhere.
+STACK370M_CONTRACTION_TRAFFIC = 69.35e6
+# Same for the scan at the 370M layer shape (profiles/mlgru_scan_b8_t2048_d1024.md): 100.9 + 10.3 MB.
+SCAN370M_TRAFFIC = 111.16e6
+
+
 def stack_workload(layers=None):
     """The 370M-shaped stack; `layers` overrides the block count (a one-block run has the same
     kernel shapes, for short profiler captures), and the workload name then says so."""
@@ -331,8 +339,10 @@ def run_mmf(args):
     achieved = ops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
     peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_OVER_BF16
     launches = sum(v[0] for v in prof.values())
+    byte_codes = os.environ.get("MMF_PREFILL_UNPACKED", "1") != "0"
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": None,
+                "frac": achieved / peak, "traffic": STACK370M_CONTRACTION_TRAFFIC if byte_codes else None,
+                "traffic_note": "DRAM bytes per contraction launch, mean of one block's four (ncu)",
                 "kernel": ",".join(gemm_names), "launches": gemm_launches,
                 "share_of_step": gemm_ms / sum(step_ms) if step_ms else None,
                 "peak_source": f"{peak_kind}: bf16 sustained x {INT8_OVER_BF16} (int8 dense : bf16 dense nominal)",
@@ -504,7 +514,7 @@ def run_scan(args):
             "data": "synthetic", "config": {"workload": f"mlgru_scan_b{B}_t{T}_d{d}_bf16",
                                             "l2": "flushed between timed steps"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mlgru_scan",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": SCAN370M_TRAFFIC, "kernel": "mlgru_scan",
                          "peak_source": peak_kind},
             "cpu_baseline": None, "e2e": None, "gpu_launches": prof["mlgru_scan"][0]}), flush=True)
     return 0
