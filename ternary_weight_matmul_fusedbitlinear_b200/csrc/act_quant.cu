@@ -139,7 +139,8 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_staged_kernel(const T* __re
                                                                    const float* __restrict__ gain, float eps,
                                                                    int8_t* __restrict__ q, float* __restrict__ scale,
                                                                    int32_t* __restrict__ qsum, int slots,
-                                                                   int stride, int* status) {
+                                                                   int stride, int* status, uint4* fill,
+                                                                   size_t fill16) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warps = blockDim.x >> 5;
@@ -158,6 +159,9 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_staged_kernel(const T* __re
   __syncwarp();
   pdl_trigger();
   pdl_wait();   // x is the previous kernel's output
+  // side work for a later kernel: fill `fill16` 16-byte units with all-ones bytes
+  for (size_t i = (size_t)blockIdx.x * blockDim.x + threadIdx.x; i < fill16; i += (size_t)gridDim.x * blockDim.x)
+    fill[i] = make_uint4(~0u, ~0u, ~0u, ~0u);
   if (lane == 0) {
     for (int s = 0; s < slots; ++s) {
       const int r = row0 + s * nwarps;
@@ -216,7 +220,7 @@ bool staged_geometry(int K, int esize, StagedGeom& g) {
 
 template <typename T, bool GAIN>
 cudaError_t launch_staged(const StagedGeom& g, const void* x, int M, int K, const float* gain, float eps, int8_t* q,
-                          float* scale, int32_t* qsum, int* status, cudaStream_t stream) {
+                          float* scale, int32_t* qsum, int* status, void* fill, size_t fill_bytes, cudaStream_t stream) {
   auto kern = rmsnorm_quant_staged_kernel<T, GAIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
   if (e != cudaSuccess) return e;
@@ -224,21 +228,26 @@ cudaError_t launch_staged(const StagedGeom& g, const void* x, int M, int K, cons
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.warps * 32, g.smem);
   const int grid = std::max(1, std::min(ceil_div(M, g.warps), num_sms() * std::max(per_sm, 1)));
   return launch_pdl(kern, dim3(grid), dim3(g.warps * 32), g.smem, stream, static_cast<const T*>(x), M, K, gain, eps,
-                    q, scale, qsum, g.slots, g.stride, status);
+                    q, scale, qsum, g.slots, g.stride, status, static_cast<uint4*>(fill), fill_bytes / 16);
 }
 
 }  // namespace
 
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
-                                 int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream) {
-  if (M == 0) return cudaSuccess;
+                                 int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream, void* fill,
+                                 size_t fill_bytes) {
+  if (M == 0) return fill_bytes ? cudaMemsetAsync(fill, 0xff, fill_bytes, stream) : cudaSuccess;
   StagedGeom g;
-  if (staged_geometry(K, dt == MMF_BF16 ? 2 : 4, g)) {
+  if (staged_geometry(K, dt == MMF_BF16 ? 2 : 4, g) && fill_bytes % 16 == 0) {
     if (dt == MMF_BF16)
-      return gain ? launch_staged<bf16, true>(g, x, M, K, gain, eps, q, scale, qsum, status, stream)
-                  : launch_staged<bf16, false>(g, x, M, K, gain, eps, q, scale, qsum, status, stream);
-    return gain ? launch_staged<float, true>(g, x, M, K, gain, eps, q, scale, qsum, status, stream)
-                : launch_staged<float, false>(g, x, M, K, gain, eps, q, scale, qsum, status, stream);
+      return gain ? launch_staged<bf16, true>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream)
+                  : launch_staged<bf16, false>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream);
+    return gain ? launch_staged<float, true>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream)
+                : launch_staged<float, false>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream);
+  }
+  if (fill_bytes) {
+    const cudaError_t e = cudaMemsetAsync(fill, 0xff, fill_bytes, stream);
+    if (e != cudaSuccess) return e;
   }
   // rows too long for the staged ring: one CTA per row
   const size_t smem = sizeof(float) * (size_t)K;

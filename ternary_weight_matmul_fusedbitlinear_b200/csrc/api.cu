@@ -207,9 +207,11 @@ struct QAct {
 // the codes also land in qa when `want_codes`. Otherwise the quantiser fills qa
 // and the contraction reads it.
 mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& qa, TGemmArgs a, Epi epi,
-                      mmf_dtype dt, cudaStream_t s, const char* what, bool want_codes) {
+                      mmf_dtype dt, cudaStream_t s, const char* what, bool want_codes, void* fill = nullptr,
+                      size_t fill_bytes = 0) {
   if (!gemm_uses_tc(a, epi) && decode_fused_quant_wanted(a.M) &&
       tgemm_mma_fused_quant_supported(a.M, a.K, elem_bytes(dt))) {
+    if (fill_bytes) MMF_CUDA(cudaMemsetAsync(fill, 0xff, fill_bytes, s), "scratch fill");
     a.x = x;
     a.gain = gain;
     a.eps = eps;
@@ -220,7 +222,10 @@ mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& q
     return MMF_OK;
   }
   MMF_CUDA(timed("rmsnorm_quant", s,
-                 [&] { return launch_rmsnorm_quant(x, dt, a.M, a.K, gain, eps, qa.q, qa.s, qa.qsum, status_word(), s); }),
+                 [&] {
+                   return launch_rmsnorm_quant(x, dt, a.M, a.K, gain, eps, qa.q, qa.s, qa.qsum, status_word(), s,
+                                               fill, fill_bytes);
+                 }),
            "rmsnorm_quant");
   MMF_CUDA(run_gemm(a, epi, dt, s, what), "contraction");
   return MMF_OK;
@@ -677,16 +682,16 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   for (int i = 0; i < 3; ++i) tm.wu[i] = blk->wu[i];
   const bool fused_mixer = T > 1 && fused_mlgru_enabled() && gemm_uses_tc(tm, Epi::kStore) &&
                            tgemm_tc_mlgru_supported(tm, T, d);
-  // prefill: the scan's scratch is reset here, so that the kernels that read
-  // it follow their predecessors back to back (programmatic dependent launch)
-  if (fused_mixer)
-    MMF_CUDA(timed("mlgru_scratch_reset", s, [&] { return reset_tgemm_tc_mlgru_ws(w.scan, B, T, d, s); }), "block mixer reset");
-  else if (T > 1)
-    MMF_CUDA(timed("mlgru_scratch_reset", s, [&] { return reset_mlgru_scan_ws(w.scan, B, T, d, s); }), "block scan reset");
+  // prefill: the scan's scratch (all-ones before the scan) is filled by the
+  // quantiser of x as side work, so no memset sits between the kernels
+  const size_t scan_fill = fused_mixer ? tgemm_tc_mlgru_ws_bytes(B, T, d) : (T > 1 ? mlgru_scan_ws_bytes(B, T, d) : 0);
   // token mixer: x quantised once for f, c, g (shared gain)
   if (fused_mixer) {
     MMF_CUDA(timed("rmsnorm_quant", s,
-                   [&] { return launch_rmsnorm_quant(x, dt, M, d, W.f.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(), s); }),
+                   [&] {
+                     return launch_rmsnorm_quant(x, dt, M, d, W.f.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(),
+                                                 s, w.scan, scan_fill);
+                   }),
              "block quant x");
     int* status = nullptr;
     mmf_status r = device_status_ptr(&status);
@@ -701,7 +706,7 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   } else {
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.pre, 3 * d, nullptr, nullptr);
     for (int i = 0; i < 3; ++i) a.wu[i] = blk->wu[i];
-    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", false);
+    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", false, w.scan, scan_fill);
     if (r != MMF_OK) return r;
     int* status = nullptr;
     r = device_status_ptr(&status);

@@ -47,8 +47,11 @@ cudaError_t launch_quantize_weights(const float* W, int N, int K, uint32_t* pack
                                     cudaStream_t stream);
 
 // `status` (nullable) is the device status word for bounded-wait timeouts.
+// Optionally, as side work for a later kernel, it sets `fill_bytes` bytes at
+// `fill` (16-byte aligned) to 0xff, stream-ordered like a memset.
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
-                                 int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream);
+                                 int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream,
+                                 void* fill = nullptr, size_t fill_bytes = 0);
 
 // Epilogues of the ternary contraction.
 enum class Epi : int {
