@@ -120,18 +120,49 @@ def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_total
 # ----------------------------------------------------------------------------- clocks
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 50 ms during the timed region."""
+    """SM clock and clock-event (throttle) reasons sampled during the timed region: read-only NVML queries
+    every 10 ms from a thread, or nvidia-smi every 50 ms when NVML is not importable."""
 
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    REASON_BITS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+                   "hw_thermal_slowdown": 0x40}
 
     def __init__(self, gpu_index: int):
         self.idx = gpu_index
         self.proc = None
         self.path = None
+        self.thread = None
+        self.rows = []
+
+    def _nvml_handle(self, nvml):
+        try:   # match the CUDA device by UUID: NVML indices ignore CUDA_VISIBLE_DEVICES
+            uuid = str(torch.cuda.get_device_properties(self.idx).uuid)
+            return nvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+        except Exception:
+            return nvml.nvmlDeviceGetHandleByIndex(self.idx)
 
     def start(self):
+        try:
+            import threading
+            import pynvml as nvml
+            nvml.nvmlInit()
+            h = self._nvml_handle(nvml)
+            reasons_fn = getattr(nvml, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+                nvml.nvmlDeviceGetCurrentClocksThrottleReasons
+            mx = nvml.nvmlDeviceGetMaxClockInfo(h, nvml.NVML_CLOCK_SM)
+            self.stop_flag = threading.Event()
+
+            def run():
+                while not self.stop_flag.is_set():
+                    self.rows.append((nvml.nvmlDeviceGetClockInfo(h, nvml.NVML_CLOCK_SM), mx, reasons_fn(h)))
+                    self.stop_flag.wait(0.01)
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            return
+        except Exception:
+            self.thread = None
         fd, self.path = tempfile.mkstemp(suffix=".csv")
         os.close(fd)
         try:
@@ -141,7 +172,22 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    @staticmethod
+    def _summary(sm, mx, reasons, n, source):
+        loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(loaded) if loaded else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": n, "source": source}
+
     def stop(self) -> dict:
+        if self.thread is not None:
+            self.stop_flag.set()
+            self.thread.join(timeout=5)
+            rows = self.rows
+            if not rows:
+                return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+            reasons = sorted({k for _, _, r in rows for k, bit in self.REASON_BITS.items() if r & bit})
+            return self._summary([float(r[0]) for r in rows], [float(r[1]) for r in rows], reasons, len(rows),
+                                 "nvml, 10 ms")
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
@@ -168,9 +214,7 @@ class ClockSampler:
         mx = [num(r[2]) for r in rows if num(r[2]) is not None]
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        loaded = [v for v in sm if mx and v > 0.5 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(loaded) if loaded else None,
-                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons, "samples": len(rows)}
+        return self._summary(sm, mx, reasons, len(rows), "nvidia-smi, 50 ms")
 
 
 # ----------------------------------------------------------------------------- workload
