@@ -140,7 +140,7 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_staged_kernel(const T* __re
                                                                    int8_t* __restrict__ q, float* __restrict__ scale,
                                                                    int32_t* __restrict__ qsum, int slots,
                                                                    int stride, int* status, uint4* fill,
-                                                                   size_t fill16, RowStats stats) {
+                                                                   size_t fill16) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* base = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   const int warps = blockDim.x >> 5;
@@ -184,10 +184,7 @@ __global__ void __launch_bounds__(256) rmsnorm_quant_staged_kernel(const T* __re
       return;
     }
     const uint4* v = reinterpret_cast<const uint4*>(ring + (size_t)s * stride);
-    const RowCode rc =
-        quant_row<T, GAIN, false>(v, nvec, K, gain, eps, q + (size_t)row * K, lane,
-                                  stats.ss ? stats.ss + (size_t)row * stats.parts : nullptr,
-                                  stats.am ? stats.am + (size_t)row * stats.parts : nullptr, stats.parts);
+    const RowCode rc = quant_row<T, GAIN, false>(v, nvec, K, gain, eps, q + (size_t)row * K, lane);
     if (lane == 0) {
       scale[row] = rc.scale;
       qsum[row] = rc.qsum;
@@ -223,8 +220,7 @@ bool staged_geometry(int K, int esize, StagedGeom& g) {
 
 template <typename T, bool GAIN>
 cudaError_t launch_staged(const StagedGeom& g, const void* x, int M, int K, const float* gain, float eps, int8_t* q,
-                          float* scale, int32_t* qsum, int* status, void* fill, size_t fill_bytes,
-                          const RowStats& stats, cudaStream_t stream) {
+                          float* scale, int32_t* qsum, int* status, void* fill, size_t fill_bytes, cudaStream_t stream) {
   auto kern = rmsnorm_quant_staged_kernel<T, GAIN>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
   if (e != cudaSuccess) return e;
@@ -232,23 +228,22 @@ cudaError_t launch_staged(const StagedGeom& g, const void* x, int M, int K, cons
   cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, g.warps * 32, g.smem);
   const int grid = std::max(1, std::min(ceil_div(M, g.warps), num_sms() * std::max(per_sm, 1)));
   return launch_pdl(kern, dim3(grid), dim3(g.warps * 32), g.smem, stream, static_cast<const T*>(x), M, K, gain, eps,
-                    q, scale, qsum, g.slots, g.stride, status, static_cast<uint4*>(fill), fill_bytes / 16, stats);
+                    q, scale, qsum, g.slots, g.stride, status, static_cast<uint4*>(fill), fill_bytes / 16);
 }
 
 }  // namespace
 
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
                                  int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream, void* fill,
-                                 size_t fill_bytes, const RowStats* stats) {
+                                 size_t fill_bytes) {
   if (M == 0) return fill_bytes ? cudaMemsetAsync(fill, 0xff, fill_bytes, stream) : cudaSuccess;
   StagedGeom g;
-  const RowStats st = stats ? *stats : RowStats{nullptr, nullptr, 0};
   if (staged_geometry(K, dt == MMF_BF16 ? 2 : 4, g) && fill_bytes % 16 == 0) {
     if (dt == MMF_BF16)
-      return gain ? launch_staged<bf16, true>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, st, stream)
-                  : launch_staged<bf16, false>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, st, stream);
-    return gain ? launch_staged<float, true>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, st, stream)
-                : launch_staged<float, false>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, st, stream);
+      return gain ? launch_staged<bf16, true>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream)
+                  : launch_staged<bf16, false>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream);
+    return gain ? launch_staged<float, true>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream)
+                : launch_staged<float, false>(g, x, M, K, gain, eps, q, scale, qsum, status, fill, fill_bytes, stream);
   }
   if (fill_bytes) {
     const cudaError_t e = cudaMemsetAsync(fill, 0xff, fill_bytes, stream);

@@ -153,13 +153,6 @@ bool fused_mlgru_enabled() {
   return e != nullptr && strcmp(e, "1") == 0;
 }
 
-// Prefill contractions hand the next quantiser per-row statistics of what
-// they store (it then skips its first pass) unless MMF_ROW_STATS=0.
-bool row_stats_enabled() {
-  const char* e = getenv("MMF_ROW_STATS");
-  return e == nullptr || strcmp(e, "0") != 0;
-}
-
 bool gemm_uses_tc(const TGemmArgs& a, Epi epi) {
   const int pref = gemm_path_pref();
   return tgemm_tc_supported(a, epi) && (pref >= 2 || (pref == 0 && a.M >= kTcMinTokens));
@@ -215,7 +208,7 @@ struct QAct {
 // and the contraction reads it.
 mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& qa, TGemmArgs a, Epi epi,
                       mmf_dtype dt, cudaStream_t s, const char* what, bool want_codes, void* fill = nullptr,
-                      size_t fill_bytes = 0, const RowStats* in_stats = nullptr) {
+                      size_t fill_bytes = 0) {
   if (!gemm_uses_tc(a, epi) && decode_fused_quant_wanted(a.M) &&
       tgemm_mma_fused_quant_supported(a.M, a.K, elem_bytes(dt))) {
     if (fill_bytes) MMF_CUDA(cudaMemsetAsync(fill, 0xff, fill_bytes, s), "scratch fill");
@@ -231,7 +224,7 @@ mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& q
   MMF_CUDA(timed("rmsnorm_quant", s,
                  [&] {
                    return launch_rmsnorm_quant(x, dt, a.M, a.K, gain, eps, qa.q, qa.s, qa.qsum, status_word(), s,
-                                               fill, fill_bytes, in_stats);
+                                               fill, fill_bytes);
                  }),
            "rmsnorm_quant");
   MMF_CUDA(run_gemm(a, epi, dt, s, what), "contraction");
@@ -463,43 +456,21 @@ mmf_status check_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_t
 
 // p = SiLU(gate(x)) * up(x); y = down(p) + residual. x is quantised with the
 // gate's RMSNorm gain (gate and up share it), p with the down projection's.
-// Row statistics buffers of one activation tensor [M rows x parts].
-struct StatsBuf {
-  double* ss;
-  uint32_t* am;
-  int parts;
-};
-
-// Ask the contraction `a` for statistics of its output rows in `out` (when the
-// tensor-core path runs it and statistics are on); returns whether it will.
-bool request_stats(TGemmArgs& a, Epi epi, const StatsBuf* out) {
-  if (out == nullptr || out->ss == nullptr || !row_stats_enabled() || !gemm_uses_tc(a, epi)) return false;
-  a.ss_out = out->ss;
-  a.am_out = out->am;
-  a.stats_parts = out->parts;
-  return true;
-}
-
 mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tlinear* down, const void* x,
                    const void* residual, void* y, int M, mmf_dtype dt, float eps, void* p, const QAct& qa,
-                   cudaStream_t s, const uint8_t* const* wu = nullptr /* gate, up, down one-byte codes */,
-                   const RowStats* x_stats = nullptr, const StatsBuf* p_stats = nullptr,
-                   const StatsBuf* y_stats = nullptr) {
+                   cudaStream_t s, const uint8_t* const* wu = nullptr /* gate, up, down one-byte codes */) {
   const mmf_tlinear* gu[2] = {gate, up};
   TGemmArgs a = gemm_args(gu, 2, qa.q, qa.s, qa.qsum, M, p, gate->N, nullptr, nullptr);
   if (wu) {
     a.wu[0] = wu[0];
     a.wu[1] = wu[1];
   }   // otherwise the layers' own codes (if any), set by gemm_args
-  const bool p_has = request_stats(a, Epi::kGlu, p_stats);
-  mmf_status r = quant_gemm(x, gate->gain, eps, qa, a, Epi::kGlu, dt, s, "gate_up", false, nullptr, 0, x_stats);
+  mmf_status r = quant_gemm(x, gate->gain, eps, qa, a, Epi::kGlu, dt, s, "gate_up", false);
   if (r != MMF_OK) return r;
   const mmf_tlinear* dn[1] = {down};
   TGemmArgs b = gemm_args(dn, 1, qa.q, qa.s, qa.qsum, M, y, down->N, residual, nullptr);
   if (wu) b.wu[0] = wu[2];
-  request_stats(b, Epi::kStore, y_stats);
-  const RowStats ps{p_has ? p_stats->ss : nullptr, p_has ? p_stats->am : nullptr, p_has ? p_stats->parts : 0};
-  return quant_gemm(p, down->gain, eps, qa, b, Epi::kStore, dt, s, "down", false, nullptr, 0, p_has ? &ps : nullptr);
+  return quant_gemm(p, down->gain, eps, qa, b, Epi::kStore, dt, s, "down", false);
 }
 
 }  // namespace
@@ -682,7 +653,6 @@ struct BlockWs {
   void* ping;  // [M, d] stack intermediates
   void* pong;
   void* scan;  // scan scratch
-  StatsBuf st_y1, st_p, st_ping, st_pong;   // row statistics of y1, p and the stack intermediates
   size_t bytes;
 };
 
@@ -699,27 +669,12 @@ BlockWs carve_block(void* base, int B, int T, int d, int I, mmf_dtype dt) {
   w.ping = c.take<char>((size_t)M * d * e);
   w.pong = c.take<char>((size_t)M * d * e);
   w.scan = c.take<char>(std::max(mlgru_scan_ws_bytes(B, T, d), tgemm_tc_mlgru_ws_bytes(B, T, d)));
-  auto stats = [&](int cols, int cp) {   // partial statistics for `cols` columns in groups of cp
-    StatsBuf b{nullptr, nullptr, cols / cp};
-    if (cols % cp != 0 || T < 2) return StatsBuf{nullptr, nullptr, 0};
-    b.ss = c.take<double>((size_t)M * b.parts);
-    b.am = c.take<uint32_t>((size_t)M * b.parts);
-    return b;
-  };
-  w.st_y1 = stats(d, 128);
-  w.st_p = stats(I, 64);
-  w.st_ping = stats(d, 128);
-  w.st_pong = stats(d, 128);
   w.bytes = c.off + 256;
   return w;
 }
 
-// x_stats: row statistics of x written by the previous block's down
-// projection (or null); y_stats: where this block's down projection writes
-// those of y (or null).
 mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, void* y, int B, int T, mmf_dtype dt,
-                              float eps, const BlockWs& w, cudaStream_t s, const RowStats* x_stats = nullptr,
-                              const StatsBuf* y_stats = nullptr) {
+                              float eps, const BlockWs& w, cudaStream_t s) {
   const int M = B * T, d = blk->d;
   const mmf_block_weights& W = blk->w;
   const mmf_tlinear* fcg[3] = {&W.f, &W.c, &W.g};
@@ -751,7 +706,7 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   } else {
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.pre, 3 * d, nullptr, nullptr);
     for (int i = 0; i < 3; ++i) a.wu[i] = blk->wu[i];
-    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", false, w.scan, scan_fill, x_stats);
+    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", false, w.scan, scan_fill);
     if (r != MMF_OK) return r;
     int* status = nullptr;
     r = device_status_ptr(&status);
@@ -762,13 +717,10 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
   b.wu[0] = blk->wu[3];
-  const bool y1_has = request_stats(b, Epi::kStore, &w.st_y1);
   mmf_status r = quant_gemm(w.og, W.o.gain, eps, w.qa, b, Epi::kStore, dt, s, "o", false);
   if (r != MMF_OK) return r;
   // channel mixer
-  const RowStats y1s{w.st_y1.ss, w.st_y1.am, w.st_y1.parts};
-  return run_glu(&W.gate, &W.up, &W.down, w.y1, w.y1, y, M, dt, eps, w.p, w.qa, s, blk->wu + 4,
-                 y1_has ? &y1s : nullptr, &w.st_p, y_stats);
+  return run_glu(&W.gate, &W.up, &W.down, w.y1, w.y1, y, M, dt, eps, w.p, w.qa, s, blk->wu + 4);
 }
 
 mmf_status check_forward_args(const mmf_block* blk, mmf_state* st, const void* x, void* y, int B, int T,
@@ -827,21 +779,12 @@ extern "C" mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t 
   if (ws_bytes < need) return fail(MMF_ERR_WORKSPACE, "mmf_stack_forward: ws_bytes=%zu < %zu", ws_bytes, need);
   cudaStream_t s = as_stream(stream);
   const void* cur = x;
-  RowStats cur_stats{nullptr, nullptr, 0};   // statistics of `cur` when its producer wrote them
   for (int l = 0; l < L; ++l) {
     BlockWs w = carve_block(ws, B, T, blocks[l]->d, blocks[l]->I, dtype);
-    const bool last = l == L - 1;
-    void* dst = last ? y : ((l % 2 == 0) ? w.ping : w.pong);
-    const StatsBuf* dst_stats = last ? nullptr : ((l % 2 == 0) ? &w.st_ping : &w.st_pong);
-    // the down projection writes them only on the tensor-core path (prefill), checked like the block does
-    const mmf_tlinear* dn[1] = {&blocks[l]->w.down};
-    TGemmArgs probe = gemm_args(dn, 1, nullptr, nullptr, nullptr, B * T, dst, blocks[l]->d, nullptr, nullptr);
-    const bool writes = dst_stats && dst_stats->ss && row_stats_enabled() && gemm_uses_tc(probe, Epi::kStore);
-    mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), cur, dst, B, T, dtype, eps, w, s,
-                                      cur_stats.ss ? &cur_stats : nullptr, writes ? dst_stats : nullptr);
+    void* dst = (l == L - 1) ? y : ((l % 2 == 0) ? w.ping : w.pong);
+    mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), cur, dst, B, T, dtype, eps, w, s);
     if (r != MMF_OK) return r;
     cur = dst;
-    cur_stats = writes ? RowStats{dst_stats->ss, dst_stats->am, dst_stats->parts} : RowStats{nullptr, nullptr, 0};
   }
   return MMF_OK;
 }

@@ -36,14 +36,6 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
-// Per-row partial statistics of an activation tensor, as written by the
-// contraction epilogue (TGemmArgs::ss_out / am_out).
-struct RowStats {
-  const double* ss;
-  const uint32_t* am;
-  int parts;
-};
-
 // Message returned by mmf_last_error() on this host thread.
 void set_last_error(const char* msg);
 
@@ -56,12 +48,10 @@ cudaError_t launch_quantize_weights(const float* W, int N, int K, uint32_t* pack
 
 // `status` (nullable) is the device status word for bounded-wait timeouts.
 // Optionally, as side work for a later kernel, it sets `fill_bytes` bytes at
-// `fill` (16-byte aligned) to 0xff, stream-ordered like a memset. With `stats`
-// (row partials written by the producer of x) the sum of squares and max|x|
-// are combined from them instead of a pass over the row.
+// `fill` (16-byte aligned) to 0xff, stream-ordered like a memset.
 cudaError_t launch_rmsnorm_quant(const void* x, mmf_dtype dt, int M, int K, const float* gain, float eps,
                                  int8_t* q, float* scale, int32_t* qsum, int* status, cudaStream_t stream,
-                                 void* fill = nullptr, size_t fill_bytes = 0, const RowStats* stats = nullptr);
+                                 void* fill = nullptr, size_t fill_bytes = 0);
 
 // Epilogues of the ternary contraction.
 enum class Epi : int {
@@ -98,17 +88,7 @@ struct TGemmArgs {
   int8_t* q_out;
   float* s_out;
   int32_t* qsum_out;
-  // tcgen05 path, kStore (one segment) and kGlu: when ss_out is set the
-  // epilogue also writes per-row partial statistics of the values it stores
-  // (rounded to the output type): for output columns [cp*i, cp*i + cp) of row
-  // m, ss_out[m * stats_parts + i] = sum of squares (fp64, columns in order)
-  // and am_out[...] = largest |value| as fp32 bits; cp = 128 (kStore) or 64
-  // (kGlu), stats_parts = output columns / cp.
-  double* ss_out;
-  uint32_t* am_out;
-  int stats_parts;
 };
-
 
 
 

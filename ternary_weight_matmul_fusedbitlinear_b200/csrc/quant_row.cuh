@@ -89,13 +89,10 @@ struct RowCode {
 // row as nvec 16-byte vectors (K elements), in global memory when GLOBAL
 // (read through the read-only path) or in shared memory; codes go to qr
 // (16-byte aligned, global or shared). Returns the scale and the code sum on
-// every lane. With `pss` (and `pam`, `nparts`): the row's sum of squares and
-// max|x| come from partials written by the row's producer instead of pass 1
-// (partial i by lane i % 32 in order, then the same xor tree).
+// every lane.
 template <typename T, bool GAIN, bool GLOBAL>
 __device__ __forceinline__ RowCode quant_row(const uint4* v, int nvec, int K, const float* __restrict__ gain,
-                                             float eps, int8_t* qr, int lane, const double* pss = nullptr,
-                                             const uint32_t* pam = nullptr, int nparts = 0) {
+                                             float eps, int8_t* qr, int lane) {
   using V = Vec<T>;
   constexpr int E = V::E;
   auto ld = [&](int vi) -> uint4 {
@@ -105,22 +102,15 @@ __device__ __forceinline__ RowCode quant_row(const uint4* v, int nvec, int K, co
   // pass 1: sum of squares (fp64) and max |x|
   double ss = 0.0;
   uint32_t am = 0;
-  if (pss != nullptr) {
-    for (int i = lane; i < nparts; i += 32) {
-      ss += __ldg(pss + i);
-      am = max(am, __ldg(pam + i));
-    }
-  } else {
 #pragma unroll 4
-    for (int vi = lane; vi < nvec; vi += 32) {
-      const uint4 r = ld(vi);
+  for (int vi = lane; vi < nvec; vi += 32) {
+    const uint4 r = ld(vi);
 #pragma unroll
-      for (int i = 0; i < E; ++i) {
-        const uint32_t a = V::mag(r, i);
-        am = max(am, a);
-        const double xd = magbits_to_f64(a);
-        ss = fma(xd, xd, ss);
-      }
+    for (int i = 0; i < E; ++i) {
+      const uint32_t a = V::mag(r, i);
+      am = max(am, a);
+      const double xd = magbits_to_f64(a);
+      ss = fma(xd, xd, ss);
     }
   }
 #pragma unroll

@@ -76,19 +76,6 @@ struct __align__(1024) SmemLayout {
 
 constexpr uint32_t kIdesc = umma_idesc_i8(BM, BN);
 
-// Row statistics of 32 output values as stored (rounded to T): sum of squares
-// in fp64 (in column order) and the largest |value| as fp32 bits.
-template <typename T>
-__device__ __forceinline__ void row_stats_add(const float (&v)[32], double& ss, uint32_t& am) {
-#pragma unroll
-  for (int j = 0; j < 32; ++j) {
-    const float r = round_to<T>(v[j]);
-    am = max(am, __float_as_uint(r) & 0x7fffffffu);
-    const double d = (double)r;
-    ss = fma(d, d, ss);
-  }
-}
-
 // ---------------------------------------------------------------- tile geometry
 struct TcArgs {
   TGemmArgs g;
@@ -312,8 +299,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tbase = tmem_base + ((uint32_t)(quarter * 32) << 16) + acc * BN;
       if constexpr (EPI == Epi::kGlu) {
         const float sc_u = *p.g.gamma[0] * inv_s, sc_v = *p.g.gamma[1] * inv_s;
-        double ss = 0.0;                          // row statistics of this warp's 64 output columns
-        uint32_t am = 0;
         for (int cc = 0; cc < 2; ++cc) {
           const int c = group * 2 + cc;           // 32-column chunk of the gate / up halves
           uint32_t ru[32], rv[32];
@@ -329,16 +314,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.g.bias[1] != nullptr) vv += p.g.bias[1][n0 + j];
             out[j] = silu_fast(uu) * vv;
           }
-          if (p.g.ss_out != nullptr) row_stats_add<T>(out, ss, am);
           uint8_t* buf;
           claim(buf);
           stage_row(buf, lane, out, (T*)nullptr);
           release(n0, y0, buf);
-        }
-        if (p.g.ss_out != nullptr && row_ok) {    // output columns [64 (2 nt + group), +64)
-          const size_t idx = (size_t)m * p.g.stats_parts + 2 * nt + group;
-          p.g.ss_out[idx] = ss;
-          p.g.am_out[idx] = am;
         }
       } else {
         const int h = group;                      // 128-column half of the tile
@@ -347,8 +326,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (nt * BN + h * HALF < p.g.nseg * p.g.N) {
           const float sc = *p.g.gamma[seg] * inv_s;
           const float* bias = p.g.bias[seg];
-          double ss = 0.0;                        // row statistics of this warp's 128 output columns
-          uint32_t am = 0;
           for (int c = 0; c < HALF / kEpiChunk; ++c) {
             const int n0 = row0 + 32 * c;
             const int x0 = seg * p.g.N + n0;
@@ -377,15 +354,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 add_staged_row(buf, lane, out, (T*)nullptr);
                 __syncwarp();                     // every row read before any row is overwritten
               }
-              if (p.g.ss_out != nullptr) row_stats_add<T>(out, ss, am);
               stage_row(buf, lane, out, (T*)nullptr);
             }
             release(x0, y0, buf);
-          }
-          if (EPI == Epi::kStore && p.g.ss_out != nullptr && alive && row_ok) {   // columns [128 i, +128)
-            const size_t idx = (size_t)m * p.g.stats_parts + (seg * p.g.N + row0) / HALF;
-            p.g.ss_out[idx] = ss;
-            p.g.am_out[idx] = am;
           }
         }
       }

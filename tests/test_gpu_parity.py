@@ -299,27 +299,6 @@ def test_bitlinear_and_glu_with_byte_codes_bit_identical(m):
     assert torch.equal(y1, y2)
 
 
-def test_stack_prefill_row_statistics_match_full_quantiser(monkeypatch):
-    # prefill contractions hand the next quantiser per-row partial sums of
-    # squares and max|x|; only the fp64 summation order differs from the
-    # quantiser's own pass, so nearly every output is identical and the rest
-    # stays within the composite tolerance
-    d, inner, B, T, L = 256, 768, 2, 128, 3
-    pairs = [make_block(7051 + 17 * l, d, inner, layer=l) for l in range(L)]
-    blocks = [p[0] for p in pairs]
-    x = synth.activations(7052, B * T, d, torch.bfloat16).reshape(B, T, d).cuda()
-    outs = []
-    for flag in ("1", "0"):
-        monkeypatch.setenv("MMF_ROW_STATS", flag)
-        st = mmf.State(L, B, d)
-        outs.append((mmf.stack_forward(blocks, st, x), st.get()))
-    mmf.check()
-    a, b = to_np(outs[0][0]), to_np(outs[1][0])
-    assert np.mean(a == b) > 0.99
-    assert_close(a, b, "bf16", "stack y with row statistics", tol=E2E_TOL)
-    torch.testing.assert_close(outs[0][1], outs[1][1], rtol=1e-2, atol=1e-3)
-
-
 def test_block_prefill_then_decode_matches_oracle_bf16():
     d, inner, B, T = 256, 768, 2, 40
     blk, oblk = make_block(7003, d, inner)
