@@ -222,7 +222,7 @@ class ClockSampler:
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture summarised in
 # profiles/tgemm_tc_stack370m_block.md: mean over the four contraction launches of one 370M block with
 # one-byte weight codes. Valid while that kernel is unchanged; None elsewhere.
-STACK370M_CONTRACTION_TRAFFIC = 69.35e6
+STACK370M_CONTRACTION_TRAFFIC = None   # kernel changed since the last capture (4-stage ring); recapture pending
 # Same for the scan at the 370M layer shape (profiles/mlgru_scan_b8_t2048_d1024.md): 100.9 + 10.3 MB.
 SCAN370M_TRAFFIC = 111.16e6
 

@@ -50,18 +50,18 @@ constexpr uint32_t kTmemCols = 512;
 
 // Shared memory; OB = bytes of one output element (2: bf16, 4: fp32 / int32).
 // The TMA ring is 4 deep for 2-byte outputs and 3 deep for 4-byte outputs,
-// whose staging boxes are twice as large; 3 deep (with a weight tile per
-// stage) for UNP.
+// whose staging boxes are twice as large; with UNP (a weight tile per stage)
+// also 4 deep for 2-byte outputs (225 KB of the 227 KB) and 3 for 4-byte ones.
 template <int OB, bool UNP>
 struct __align__(1024) SmemLayout {
-  static constexpr int NS = UNP ? 3 : (OB == 2 ? 4 : 3);
+  static constexpr int NS = UNP ? (OB == 2 ? 4 : 3) : (OB == 2 ? 4 : 3);
   static constexpr int NBU = UNP ? NS : NB;        // int8 weight tiles: per TMA stage (UNP) or unpack ring
   static constexpr int NBP = UNP ? 1 : NS;         // packed weight tiles (unused with UNP)
   static constexpr int kStageBytes = 32 * kEpiChunk * OB;
   uint8_t a[NS][A_BYTES];                          // 1024-aligned: SW128 atoms
   uint8_t bu[NBU][BU_BYTES];                       // 1024-aligned: SW128 atoms
   uint8_t stage[kEpiWarps][2][kStageBytes];        // epilogue staging, double-buffered (1024-aligned)
-  uint32_t bp[NBP][BP_BYTES / 4];
+  uint32_t bp[NBP][UNP ? 4 : BP_BYTES / 4];
   uint64_t tma_full[NS];
   uint64_t tma_empty[NS];
   uint64_t bu_full[NB];
