@@ -119,6 +119,12 @@ def whole_job_rate(world: int, units_per_rank_step: float, steps: int, max_total
 
 # ----------------------------------------------------------------------------- clocks
 
+def wait_event(ev) -> None:
+    """Wait for a CUDA event by polling with short sleeps, so the clock-sampling thread keeps running."""
+    while not ev.query():
+        time.sleep(0.0005)
+
+
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons sampled during the timed region: read-only NVML queries
     every 10 ms from a thread, or nvidia-smi every 50 ms when NVML is not importable."""
@@ -222,7 +228,7 @@ class ClockSampler:
 # DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture summarised in
 # profiles/tgemm_tc_stack370m_block.md: mean over the four contraction launches of one 370M block with
 # one-byte weight codes. Valid while that kernel is unchanged; None elsewhere.
-STACK370M_CONTRACTION_TRAFFIC = None   # kernel changed since the last capture (4-stage ring); recapture pending
+STACK370M_CONTRACTION_TRAFFIC = 69.38e6
 # Same for the scan at the 370M layer shape (profiles/mlgru_scan_b8_t2048_d1024.md): 100.9 + 10.3 MB.
 SCAN370M_TRAFFIC = 111.16e6
 
@@ -364,6 +370,7 @@ def run_mmf(args):
             starts[i].record(stream)
             step(x, y)
             ends[i].record(stream)
+        wait_event(ends[-1])
         torch.cuda.synchronize()
         barrier(world)
         mmf.prof_enable(False)
@@ -507,6 +514,7 @@ def run_bitlinear(args):
             starts[i].record(stream)
             mmf.bitlinear(lin, x, ws=ws)
             ends[i].record(stream)
+        wait_event(ends[-1])
         torch.cuda.synchronize()
         mmf.prof_enable(False)
         return sum(s.elapsed_time(e) for s, e in zip(starts, ends)), (mmf.prof_collect() if profile else {})
