@@ -333,3 +333,15 @@ def test_stack_forward_matches_block_loop():
     y_ref, h_ref = O.stack_forward(to_np(x.cpu()), [p[1] for p in pairs], np.zeros((L, B, d)), "bf16")
     assert_close(to_np(y1), y_ref, "bf16", "stack y", tol=E2E_TOL)
     assert_close(st1.get().numpy(), h_ref, "f32", "stack h", tol=E2E_TOL)
+
+
+def test_graft_entry_smoke():
+    # the packaged smoke check: a 2 x 64-token prefill (tensor-core contraction)
+    # and one decode step of a d=256 block against the oracle
+    import importlib.util
+    import pathlib
+    path = pathlib.Path(__file__).resolve().parents[1] / "__graft_entry__.py"
+    spec = importlib.util.spec_from_file_location("graft_entry", path)
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    mod.smoke()
