@@ -715,7 +715,9 @@ def run_decode(args):
         mmf.stack_forward(blocks, st, x, ws=ws, out=y)
     torch.cuda.synchronize()
     mmf.prof_enable(False)
-    per_kernel = {k: round(v[1] / 5, 4) for k, v in mmf.prof_collect().items()}
+    prof = mmf.prof_collect()
+    per_kernel = {k: round(v[1] / 5, 4) for k, v in prof.items()}
+    launches_per_step = sum(v[0] for v in prof.values()) // 5
     weights = w.layers * (4 * w.d * w.d + 3 * w.d * w.inner) / 4.0
     state = 2.0 * w.layers * B * w.d * 4
     gbs = (weights + state) / (step_ms / 1e3) / 1e9
@@ -732,7 +734,8 @@ def run_decode(args):
                          "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "decode step (all kernels)",
                          "bytes_per_step": weights + state, "peak_source": peak_kind,
                          "per_kernel_ms_eager_step": per_kernel},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": w.layers * 8, "clocks": clk}), flush=True)
+            "cpu_baseline": None, "e2e": None, "gpu_launches": launches_per_step * steps, "clocks": clk}),
+              flush=True)
     return 0
 
 

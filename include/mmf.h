@@ -232,10 +232,16 @@ void mmf_block_destroy(mmf_block* blk);
 
 /* Recurrent state h for L layers x B sequences x d channels, fp32, zeroed.
  * The library allocates it with cudaMalloc on the current device and frees it
- * in mmf_state_destroy. */
+ * in mmf_state_destroy. It also holds the two barrier words of the opt-in
+ * one-launch decode step (environment variable MMF_DECODE_BLOCK_KERNEL=1:
+ * T == 1, B <= 8, d and I multiples of 64), which must be zero between
+ * launches; calls that share a state are stream-ordered anyway, since h is
+ * updated in place. */
 mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_state** out);
 void mmf_state_destroy(mmf_state* st);
-/* Zero every layer's state (asynchronous on stream). */
+/* Zero every layer's state and the barrier words (asynchronous on stream);
+ * also the way to recover after mmf_check reported a barrier wait that gave
+ * up (code 4). */
 mmf_status mmf_state_reset(mmf_state* st, void* stream);
 /* Device address of layer `layer`'s state, float [B, d]; NULL if out of range. */
 float* mmf_state_layer(mmf_state* st, int32_t layer);

@@ -298,8 +298,12 @@ struct mmf_block {
   uint8_t* owned[7];
 };
 
+// bar: 256 bytes holding the counter and generation words of the one-launch
+// decode step's grid barrier, zero between launches; calls sharing a state are stream-ordered
+// anyway (h is updated in place), so one pair serves every layer.
 struct mmf_state {
   float* h;
+  unsigned* bar;
   int L, B, d;
 };
 
@@ -593,9 +597,17 @@ extern "C" mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_stat
     delete st;
     return fail(MMF_ERR_NOMEM, "mmf_state_create: cudaMalloc(%zu): %s", bytes, cudaGetErrorString(e));
   }
-  e = cudaMemset(st->h, 0, bytes);
+  e = cudaMalloc(&st->bar, 256);
   if (e != cudaSuccess) {
     cudaFree(st->h);
+    delete st;
+    return fail(MMF_ERR_NOMEM, "mmf_state_create: cudaMalloc(256): %s", cudaGetErrorString(e));
+  }
+  e = cudaMemset(st->h, 0, bytes);
+  if (e == cudaSuccess) e = cudaMemset(st->bar, 0, 256);
+  if (e != cudaSuccess) {
+    cudaFree(st->h);
+    cudaFree(st->bar);
     delete st;
     return cuda_fail(e, "mmf_state_create: cudaMemset");
   }
@@ -609,6 +621,7 @@ extern "C" mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_stat
 extern "C" void mmf_state_destroy(mmf_state* st) {
   if (!st) return;
   cudaFree(st->h);
+  cudaFree(st->bar);
   delete st;
 }
 
@@ -616,6 +629,7 @@ extern "C" mmf_status mmf_state_reset(mmf_state* st, void* stream) {
   if (!st) return fail(MMF_ERR_INVALID_ARG, "mmf_state_reset: null state");
   MMF_CUDA(cudaMemsetAsync(st->h, 0, sizeof(float) * (size_t)st->L * st->B * st->d, as_stream(stream)),
            "mmf_state_reset");
+  MMF_CUDA(cudaMemsetAsync(st->bar, 0, 256, as_stream(stream)), "mmf_state_reset: barrier words");
   return MMF_OK;
 }
 
@@ -673,11 +687,64 @@ BlockWs carve_block(void* base, int B, int T, int d, int I, mmf_dtype dt) {
   return w;
 }
 
-mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, void* y, int B, int T, mmf_dtype dt,
-                              float eps, const BlockWs& w, cudaStream_t s) {
+// With MMF_DECODE_BLOCK_KERNEL=1 a decode step of up to 8 tokens runs as one
+// launch per block (four stages, grid barriers between them) instead of four
+// contractions; both compute the same values. Off by default: on one B200 a
+// 2.7B-shaped block step took 41.5 us that way against 29.1 us for the
+// separate kernels (each stage's row quantisation, contraction and epilogue
+// stay serial, and a grid barrier costs about as much as a kernel boundary
+// with programmatic dependent launch).
+bool decode_block_enabled() {
+  const char* e = getenv("MMF_DECODE_BLOCK_KERNEL");
+  return e != nullptr && strcmp(e, "1") == 0;
+}
+
+DecodeStage decode_stage(const mmf_tlinear* const* segs, int nseg) {
+  DecodeStage st{};
+  for (int i = 0; i < 3; ++i) {
+    const mmf_tlinear* l = segs[i < nseg ? i : 0];
+    st.w[i] = l->packed;
+    st.gamma[i] = l->gamma;
+    st.bias[i] = l->bias;
+  }
+  st.gain = segs[0]->gain;
+  st.nseg = nseg;
+  st.N = segs[0]->N;
+  st.K = segs[0]->K;
+  return st;
+}
+
+mmf_status block_forward_impl(const mmf_block* blk, float* h, unsigned* bar, const void* x, void* y, int B, int T,
+                              mmf_dtype dt, float eps, const BlockWs& w, cudaStream_t s) {
   const int M = B * T, d = blk->d;
   const mmf_block_weights& W = blk->w;
   const mmf_tlinear* fcg[3] = {&W.f, &W.c, &W.g};
+  if (T == 1 && decode_block_enabled()) {
+    const mmf_tlinear* o1[1] = {&W.o};
+    const mmf_tlinear* gu[2] = {&W.gate, &W.up};
+    const mmf_tlinear* dn[1] = {&W.down};
+    DecodeBlockArgs a{};
+    a.st[0] = decode_stage(fcg, 3);
+    a.st[1] = decode_stage(o1, 1);
+    a.st[2] = decode_stage(gu, 2);
+    a.st[3] = decode_stage(dn, 1);
+    a.x = x;
+    a.og = w.og;
+    a.y1 = w.y1;
+    a.p = w.p;
+    a.y = y;
+    a.h = h;
+    a.M = M;
+    a.d = d;
+    a.I = blk->I;
+    a.eps = eps;
+    a.bar = bar;
+    a.status = status_word();
+    if (a.status != nullptr && decode_block_supported(a, dt)) {
+      MMF_CUDA(timed("decode_block", s, [&] { return launch_decode_block(a, dt, s); }), "decode block");
+      return MMF_OK;
+    }
+  }
   TGemmArgs tm = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, nullptr);
   for (int i = 0; i < 3; ++i) tm.wu[i] = blk->wu[i];
   const bool fused_mixer = T > 1 && fused_mlgru_enabled() && gemm_uses_tc(tm, Epi::kStore) &&
@@ -759,7 +826,7 @@ extern "C" mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf
   BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype);
   if (ws_bytes < mmf_block_ws_size(blk, B, T))
     return fail(MMF_ERR_WORKSPACE, "mmf_block_forward: ws_bytes=%zu < %zu", ws_bytes, mmf_block_ws_size(blk, B, T));
-  return block_forward_impl(blk, mmf_state_layer(st, layer), x, y, B, T, dtype, eps, w, as_stream(stream));
+  return block_forward_impl(blk, mmf_state_layer(st, layer), st->bar, x, y, B, T, dtype, eps, w, as_stream(stream));
 }
 
 extern "C" mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t L, mmf_state* st, const void* x,
@@ -782,7 +849,7 @@ extern "C" mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t 
   for (int l = 0; l < L; ++l) {
     BlockWs w = carve_block(ws, B, T, blocks[l]->d, blocks[l]->I, dtype);
     void* dst = (l == L - 1) ? y : ((l % 2 == 0) ? w.ping : w.pong);
-    mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), cur, dst, B, T, dtype, eps, w, s);
+    mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), st->bar, cur, dst, B, T, dtype, eps, w, s);
     if (r != MMF_OK) return r;
     cur = dst;
   }

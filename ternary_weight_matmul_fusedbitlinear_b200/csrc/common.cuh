@@ -70,6 +70,20 @@ __device__ __forceinline__ uint32_t pack4_sat(int c0, int c1, int c2, int c3) {
 __device__ __forceinline__ float sigmoidf_(float z) { return __frcp_rn(1.0f + __expf(-z)); }
 __device__ __forceinline__ float siluf_(float z) { return z * sigmoidf_(z); }
 
+// ---------------------------------------------------------------- decode epilogue steps
+// Written once so that every decode kernel rounds them the same way.
+// Rescale of an int32 accumulator: acc * gamma / s, each a correctly rounded fp32 operation.
+__device__ __forceinline__ float rescale_acc(int acc, float gamma, float s) {
+  return __fdiv_rn(__fmul_rn((float)acc, gamma), s);
+}
+// One MLGRU step of one channel from its f, c, g pre-activations: h becomes
+// f h + (1 - f) c (f = sigmoid, c = SiLU); returns the gated output g h.
+__device__ __forceinline__ float mlgru_step(float pf, float pc, float pg, float& h) {
+  const float f = sigmoidf_(pf), c = siluf_(pc), g = sigmoidf_(pg);
+  h = __fmaf_rn(f, h, __fmul_rn(1.0f - f, c));
+  return g * h;
+}
+
 // ---------------------------------------------------------------- programmatic dependent launch
 // A kernel launched with programmatic stream serialization may start before
 // its predecessor in the stream has finished. pdl_wait() blocks until every

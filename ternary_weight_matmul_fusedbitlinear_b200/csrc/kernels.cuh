@@ -120,6 +120,38 @@ cudaError_t reset_tgemm_tc_mlgru_ws(void* ws, int B, int T, int d, cudaStream_t 
 cudaError_t launch_tgemm_tc_mlgru(const TGemmArgs& a, mmf_dtype dt, int T, int d, float* h, void* ws, int* status,
                                   cudaStream_t stream);
 
+// One decode step (T = 1, M <= 8 tokens) of a whole block in one cooperative
+// launch (grid = one CTA per SM): stage 0 quantises x with st[0].gain and runs
+// f|c|g (3 segments, N = d) with the MLGRU step (h in place, o' -> og); stage 1
+// quantises og and runs o (+ x) -> y1; stage 2 quantises y1 and runs gate|up
+// (2 segments, N = I) with SiLU(gate) * up -> p; stage 3 quantises p and runs
+// down (+ y1) -> y. `bar` holds 256 bytes (words 0 and 32 used) that are zero
+// between launches.
+constexpr int kDecodeMaxTiles = 4;   // 16-row weight tiles per CTA and stage
+struct DecodeStage {
+  const uint32_t* w[3];     // packed codes per segment, [N, K/16]
+  const float* gamma[3];    // per-segment scale (device scalar)
+  const float* bias[3];     // per-segment bias [N] or null
+  const float* gain;        // RMSNorm gain [K] of the stage's input, or null
+  int nseg, N, K;
+};
+struct DecodeBlockArgs {
+  DecodeStage st[4];        // f|c|g, o, gate|up, down
+  const void* x;            // [M, d] block input (activation dtype)
+  void* og;                 // [M, d] o'
+  void* y1;                 // [M, d] token-mixer output
+  void* p;                  // [M, I] GLU product
+  void* y;                  // [M, d] block output
+  float* h;                 // [M, d] recurrent state
+  int M, d, I;
+  float eps;
+  unsigned* bar;            // grid-barrier words (counter, generation)
+  int* status;              // device status word (code 4: a barrier wait gave up)
+  int slot_bytes;           // set by the launcher
+};
+bool decode_block_supported(const DecodeBlockArgs& a, mmf_dtype dt);
+cudaError_t launch_decode_block(DecodeBlockArgs a, mmf_dtype dt, cudaStream_t stream);
+
 // Chunk-parallel MLGRU scan; `ws` holds mlgru_scan_ws_bytes(B, T, d) bytes of
 // scratch, which reset_mlgru_scan_ws() must prepare (stream-ordered) before
 // every launch; launch_mlgru_scan() itself enqueues only the kernel (launched

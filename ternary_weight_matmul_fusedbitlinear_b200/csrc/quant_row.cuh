@@ -88,9 +88,12 @@ struct RowCode {
 // Warp-collective: all 32 lanes call it with the same row. `v` points at the
 // row as nvec 16-byte vectors (K elements), in global memory when GLOBAL
 // (read through the read-only path) or in shared memory; codes go to qr
-// (16-byte aligned, global or shared). Returns the scale and the code sum on
-// every lane.
-template <typename T, bool GAIN, bool GLOBAL>
+// (16-byte aligned, global or shared). With INPLACE, qr is the row itself: the
+// codes of vector vi overwrite bytes [E vi, E vi + E), which hold vectors read
+// in the same or an earlier step of the last pass, and a compiler barrier
+// keeps each step's accesses in program order. Returns the scale and the code
+// sum on every lane.
+template <typename T, bool GAIN, bool GLOBAL, bool INPLACE = false>
 __device__ __forceinline__ RowCode quant_row(const uint4* v, int nvec, int K, const float* __restrict__ gain,
                                              float eps, int8_t* qr, int lane) {
   using V = Vec<T>;
@@ -149,6 +152,7 @@ __device__ __forceinline__ RowCode quant_row(const uint4* v, int nvec, int K, co
       c[i] = rint_bits(__fmul_rn(hv, sc));
     }
     V::store_codes(qr + (size_t)vi * E, c, isum);
+    if constexpr (INPLACE) asm volatile("" ::: "memory");
   }
   return RowCode{sc, __reduce_add_sync(0xffffffffu, isum)};
 }

@@ -209,6 +209,7 @@ def test_decode_fused_quant_matches_standalone_quantiser(k, n, m, monkeypatch):
 
 
 def test_block_decode_fused_quant_matches_standalone_quantiser(monkeypatch):
+    monkeypatch.setenv("MMF_DECODE_BLOCK_KERNEL", "0")   # the separate kernels
     d, inner, B = 256, 768, 4
     blk, _ = make_block(7011, d, inner)
     x = synth.activations(7012, B, d, torch.bfloat16).reshape(B, 1, d).cuda()
@@ -219,6 +220,81 @@ def test_block_decode_fused_quant_matches_standalone_quantiser(monkeypatch):
         st = mmf.State(1, B, d)
         st.set(h0.reshape(1, B, d))
         outs.append((mmf.block_forward(blk, 0, st, x), st.get()))
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B", [1, 3, 8])
+def test_block_decode_one_launch_matches_separate_kernels(dtype, B, monkeypatch):
+    # a decode step of up to 8 tokens runs as one launch (four stages, grid
+    # barriers between them) with the same codes and fp32 steps as the
+    # separate kernels: identical outputs and state, step after step; and both
+    # against the oracle. d = 320 and I = 2432 give some CTAs two tiles of the
+    # gate|up stage and leave others idle.
+    d, inner, T = 320, 2432, 3
+    blk, oblk = make_block(7051 + B, d, inner)
+    x = synth.activations(7052 + B, B * T, d, TORCH_DT[dtype]).reshape(B, T, d)
+    h0 = synth.activations(7053 + B, B, d) * 0.5
+    runs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MMF_DECODE_BLOCK_KERNEL", flag)
+        st = mmf.State(1, B, d)
+        st.set(h0.reshape(1, B, d))
+        ys = [mmf.block_forward(blk, 0, st, x[:, t:t + 1].contiguous().cuda()) for t in range(T)]
+        mmf.check()
+        runs.append((torch.cat(ys, 1), st.get()))
+    assert torch.equal(runs[0][0], runs[1][0]) and torch.equal(runs[0][1], runs[1][1])
+    h = h0.numpy().astype(np.float64)
+    yr = []
+    for t in range(T):
+        yt, h = O.block_forward(to_np(x[:, t:t + 1]), oblk, h, dtype)
+        yr.append(yt)
+    assert_close(to_np(runs[0][0]), np.concatenate(yr, 1), dtype, "one-launch decode y", tol=E2E_TOL)
+    assert_close(runs[0][1][0].numpy(), h, "f32", "one-launch decode h", tol=E2E_TOL)
+
+
+def test_block_decode_one_launch_with_gains_and_biases(monkeypatch):
+    # RMSNorm gains (f|c|g share one, gate|up share one) and biases on every
+    # projection: the one-launch step and the separate kernels agree exactly
+    d, inner, B = 256, 768, 5
+    shapes = {"f": (d, d), "c": (d, d), "g": (d, d), "o": (d, d), "gate": (inner, d), "up": (inner, d),
+              "down": (d, inner)}
+    gain_of = {"f": 0, "c": 0, "g": 0, "o": 1, "gate": 2, "up": 2, "down": 3}
+    gains = [(1.0 + 0.2 * synth.activations(7071 + i, 1, d if i < 3 else inner)[0]).cuda() for i in range(4)]
+    lins = {}
+    for i, name in enumerate(synth.PROJ_NAMES):
+        W = synth.latent_weight(synth.sub_seed(7072, 0, i), *shapes[name])
+        bias = (0.05 * synth.activations(7073 + i, 1, shapes[name][0])[0]).cuda()
+        lins[name] = mmf.quantize_weights(W.cuda(), gain=gains[gain_of[name]], bias=bias)
+    blk = mmf.Block(lins)
+    x = synth.activations(7074, B, d, torch.bfloat16).reshape(B, 1, d).cuda()
+    h0 = synth.activations(7075, B, d) * 0.5
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MMF_DECODE_BLOCK_KERNEL", flag)
+        st = mmf.State(1, B, d)
+        st.set(h0.reshape(1, B, d))
+        y = mmf.block_forward(blk, 0, st, x)
+        mmf.check()
+        outs.append((y, st.get()))
+    assert torch.isfinite(outs[0][0].float()).all()
+    assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
+
+
+def test_stack_decode_one_launch_per_block_matches_separate_kernels(monkeypatch):
+    # several layers in a row share the state's barrier words
+    d, inner, B, L = 256, 768, 2, 3
+    blocks = [make_block(7061 + l, d, inner)[0] for l in range(L)]
+    x = synth.activations(7062, B, d, torch.bfloat16).reshape(B, 1, d).cuda()
+    outs = []
+    for flag in ("1", "0"):
+        monkeypatch.setenv("MMF_DECODE_BLOCK_KERNEL", flag)
+        st = mmf.State(L, B, d)
+        y = x
+        for _ in range(4):
+            y = mmf.stack_forward(blocks, st, y)
+        mmf.check()
+        outs.append((y, st.get()))
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
