@@ -245,6 +245,11 @@ void mmf_state_destroy(mmf_state* st);
 mmf_status mmf_state_reset(mmf_state* st, void* stream);
 /* Device address of layer `layer`'s state, float [B, d]; NULL if out of range. */
 float* mmf_state_layer(mmf_state* st, int32_t layer);
+/* Device address of the state's 256 bytes of barrier words (counter at byte
+ * 0, generation at byte 128, uint32 each), for diagnostics and tests; NULL for
+ * a null state. Nonzero words between launches make the one-launch decode
+ * step's barriers give up after their bounded wait (status code 4). */
+uint32_t* mmf_state_barrier(mmf_state* st);
 /* Copy the whole state [L, B, d] fp32 to / from host memory; synchronises stream. */
 mmf_status mmf_state_get(const mmf_state* st, float* host_dst, void* stream);
 mmf_status mmf_state_set(mmf_state* st, const float* host_src, void* stream);

@@ -56,6 +56,7 @@ SIGNATURES = {
     "mmf_state_destroy": (None, [c_vp]),
     "mmf_state_reset": (ctypes.c_int, [c_vp, c_vp]),
     "mmf_state_layer": (c_vp, [c_vp, c_i32]),
+    "mmf_state_barrier": (c_vp, [c_vp]),
     "mmf_state_get": (ctypes.c_int, [c_vp, c_vp, c_vp]),
     "mmf_state_set": (ctypes.c_int, [c_vp, c_vp, c_vp]),
     "mmf_block_ws_size": (c_sz, [c_vp, c_i32, c_i32]),

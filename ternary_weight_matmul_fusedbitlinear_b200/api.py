@@ -199,6 +199,15 @@ class State:
     def reset(self):
         L.check(L.load().mmf_state_reset(self.handle, _stream(torch.device("cuda"))), "mmf_state_reset")
 
+    def barrier_words(self) -> torch.Tensor:
+        """uint32 view [64] of the state's barrier words (mmf_state_barrier): counter at [0], generation at [32]."""
+        ptr = L.load().mmf_state_barrier(self.handle)
+
+        class _Words:
+            __cuda_array_interface__ = {"shape": (64,), "typestr": "<u4", "data": (ptr, False), "version": 2}
+
+        return torch.as_tensor(_Words(), device="cuda")
+
     def get(self) -> torch.Tensor:
         out = torch.empty(self.L, self.B, self.d, dtype=torch.float32)
         L.check(L.load().mmf_state_get(self.handle, ctypes.c_void_p(out.data_ptr()),

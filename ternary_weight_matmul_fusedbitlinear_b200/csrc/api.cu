@@ -633,6 +633,8 @@ extern "C" mmf_status mmf_state_reset(mmf_state* st, void* stream) {
   return MMF_OK;
 }
 
+extern "C" uint32_t* mmf_state_barrier(mmf_state* st) { return st ? st->bar : nullptr; }
+
 extern "C" float* mmf_state_layer(mmf_state* st, int32_t layer) {
   if (!st || layer < 0 || layer >= st->L) return nullptr;
   return st->h + (size_t)layer * st->B * st->d;

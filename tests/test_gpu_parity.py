@@ -281,6 +281,34 @@ def test_block_decode_one_launch_with_gains_and_biases(monkeypatch):
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
+def test_decode_block_barrier_gives_up_and_reports(monkeypatch):
+    # failure detection without a fault: barrier words left nonzero make every
+    # CTA's barrier wait run out (bounded, ~2 s); the kernel returns, mmf_check
+    # reports the timeout (code 4), and after a state reset the next step runs
+    # normally and matches the separate kernels
+    monkeypatch.setenv("MMF_DECODE_BLOCK_KERNEL", "1")
+    d, inner, B = 256, 768, 2
+    blk, _ = make_block(7081, d, inner)
+    x = synth.activations(7082, B, d, torch.bfloat16).reshape(B, 1, d).cuda()
+    st = mmf.State(1, B, d)
+    words = st.barrier_words()
+    words[0] = 1 << 30            # the counter never reaches "last arrival"
+    torch.cuda.synchronize()
+    mmf.block_forward(blk, 0, st, x)
+    with pytest.raises(mmf.MMFError) as err:
+        mmf.check()
+    assert err.value.status == 6 and "code 4" in str(err.value)
+    st.reset()
+    torch.cuda.synchronize()
+    assert int(words[0]) == 0 and int(words[32]) == 0
+    y1 = mmf.block_forward(blk, 0, st, x)
+    mmf.check()
+    monkeypatch.setenv("MMF_DECODE_BLOCK_KERNEL", "0")
+    st2 = mmf.State(1, B, d)
+    y2 = mmf.block_forward(blk, 0, st2, x)
+    assert torch.equal(y1, y2) and torch.equal(st.get(), st2.get())
+
+
 def test_stack_decode_one_launch_per_block_matches_separate_kernels(monkeypatch):
     # several layers in a row share the state's barrier words
     d, inner, B, L = 256, 768, 2, 3
