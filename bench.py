@@ -61,6 +61,8 @@ def parse_args(argv=None):
                          "decode1p3b / decode2p7b: the 1.3B / 2.7B-shaped stacks, prompt prefill then decode "
                          "steps (output fed back, state carried), each step one CUDA graph")
     ap.add_argument("--batch", type=int, default=None, help="decode2p7b: concurrent sequences (1, 8 or 64)")
+    ap.add_argument("--decode-steps", type=int, default=None,
+                    help="decode1p3b/decode2p7b: timed decode steps (default: the workload's own count)")
     ap.add_argument("--packed-only", action="store_true",
                     help="bitlinear: contract from the 2-bit codes only (no one-byte copy of the codes)")
     ap.add_argument("--layers", type=int, default=None,
@@ -695,7 +697,7 @@ def run_decode(args):
     with torch.cuda.graph(graph):
         mmf.stack_forward(blocks, st, x, ws=ws, out=y)
         x.copy_(y)
-    steps = w.decode_steps
+    steps = args.decode_steps or w.decode_steps
     for _ in range(args.warmup):
         graph.replay()
     torch.cuda.synchronize()
