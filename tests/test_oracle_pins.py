@@ -398,6 +398,88 @@ def test_glu_identity_weights_closed_form():
     assert np.max(np.abs(swapped - parts["p"])) > 0.1 * np.max(np.abs(parts["p"]))
 
 
+def _scaled_eye(d, alpha):
+    # latent alpha*d*I: gamma = |alpha|, codes sign(alpha)*I, so the BitLinear is alpha * q/s
+    lin = O.make_tlinear(np.eye(d, dtype=np.float32) * np.float32(alpha * d))
+    np.testing.assert_array_equal(lin.codes, np.sign(alpha) * np.eye(d, dtype=np.int8))
+    return lin
+
+
+def _dq(lin, x):
+    # identity-weight BitLinear: sign * gamma * q / s of RMSNorm(x) (pinned stage functions)
+    x2 = np.asarray(x).reshape(-1, x.shape[-1])
+    q, s = O.absmax_quantize(O.rmsnorm(x2))
+    sign = float(lin.codes[0, 0])
+    return (sign * float(lin.gamma) * q / s[:, None].astype(np.float64)).reshape(x.shape)
+
+
+def _unrolled_scan(f, c, g, h0):
+    # h_t = (prod_{r<=t} f_r) h0 + sum_{s<=t} (prod_{s<r<=t} f_r) (1 - f_s) c_s ; o'_t = g_t h_t
+    T = f.shape[1]
+    o = np.empty_like(f)
+    for t in range(T):
+        h = np.prod(f[:, :t + 1], axis=1) * h0
+        for s_ in range(t + 1):
+            h = h + np.prod(f[:, s_ + 1:t + 1], axis=1) * (1 - f[:, s_]) * c[:, s_]
+        o[:, t] = g[:, t] * h
+    return o, h
+
+
+ALPHAS = {"f": 0.7, "c": -1.3, "g": 2.1, "o": 0.45, "gate": 1.6, "up": -0.8, "down": 0.35}
+
+
+def _eye_block(d):
+    return O.Block(**{name: _scaled_eye(d, a) for name, a in ALPHAS.items()})
+
+
+def test_mlgru_identity_weights_closed_form():
+    # f, c, g, o = alpha_* I with distinct alphas: the projections reduce to
+    # alpha * q/s, the scan to its unrolled sum; any swap of the three gate
+    # projections, SiLU/sigmoid mix-up, missing (1 - f) or o-projection of h
+    # instead of o' changes the result
+    d, B, T = 32, 2, 6
+    blk = _eye_block(d)
+    x = O.round_f32(synth.activations(61, B * T, d).numpy().reshape(B, T, d))
+    h0 = synth.activations(62, B, d).numpy().astype(np.float64)
+    o, hT, parts = O.mlgru(x, blk, h0, "f32", parts=True)
+    pf, pc, pg = (O.round_f32(_dq(getattr(blk, n), x)) for n in ("f", "c", "g"))
+    np.testing.assert_array_equal(parts["pf"], pf)
+    np.testing.assert_array_equal(parts["pc"], pc)
+    np.testing.assert_array_equal(parts["pg"], pg)
+    og, h = _unrolled_scan(O.sigmoid(pf), O.silu(pc), O.sigmoid(pg), h0)
+    np.testing.assert_allclose(parts["o_gate"], O.round_f32(og), rtol=2e-7, atol=1e-12)
+    np.testing.assert_allclose(hT, O.round_f32(h), rtol=2e-7)
+    np.testing.assert_allclose(o, _dq(blk.o, parts["o_gate"]), rtol=1e-12)
+    # f and g swapped would give a different o'
+    og_swapped, _ = _unrolled_scan(O.sigmoid(pg), O.silu(pc), O.sigmoid(pf), h0)
+    assert np.max(np.abs(og_swapped - og)) > 0.05 * np.max(np.abs(og))
+
+
+def test_block_identity_weights_closed_form():
+    # all seven projections alpha_* I: y1 = x + alpha_o q/s(o'), y = y1 + alpha_d q/s(p),
+    # p = SiLU(alpha_gate q/s(y1)) * alpha_up q/s(y1): pins the residual wiring and which
+    # tensor each mixer reads
+    d, B, T = 32, 2, 5
+    blk = _eye_block(d)
+    x = O.round_f32(synth.activations(63, B * T, d).numpy().reshape(B, T, d))
+    h0 = synth.activations(64, B, d).numpy().astype(np.float64)
+    y, hT, parts = O.block_forward(x, blk, h0, "f32", parts=True)
+    pf, pc, pg = (O.round_f32(_dq(getattr(blk, n), x)) for n in ("f", "c", "g"))
+    og, h = _unrolled_scan(O.sigmoid(pf), O.silu(pc), O.sigmoid(pg), h0)
+    og = O.round_f32(og)
+    np.testing.assert_allclose(parts["o_gate"], og, rtol=2e-7, atol=1e-12)
+    y1 = O.round_f32(x + _dq(blk.o, parts["o_gate"]))
+    np.testing.assert_array_equal(parts["y1"], y1)
+    u, v = _dq(blk.gate, y1), _dq(blk.up, y1)
+    p = O.round_f32(O.silu(u) * v)
+    np.testing.assert_array_equal(parts["p"], p)
+    np.testing.assert_array_equal(y, O.round_f32(y1 + _dq(blk.down, p)))
+    np.testing.assert_allclose(hT, O.round_f32(h), rtol=2e-7)
+    # a block that skipped the first residual (GLU of x) would differ
+    p_x = O.round_f32(O.silu(_dq(blk.gate, x)) * _dq(blk.up, x))
+    assert np.max(np.abs(O.round_f32(x + _dq(blk.down, p_x)) - y)) > 1e-3
+
+
 def test_block_zero_weights_is_identity():
     d, inner, B, T = 32, 48, 2, 6
     blk = _block(43, d, inner)
