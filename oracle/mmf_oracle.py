@@ -29,8 +29,10 @@ both sides can agree bit for bit:
 
 Pins: every function below is checked in tests/test_oracle_pins.py against
 closed forms, hand-built cases, brute force or library routines. The
-composition ``block_forward`` / ``stack_forward`` is pinned only through its
-stages plus the zero-weight identity and the prefill == decode invariant.
+compositions ``mlgru``, ``block_forward`` and ``stack_forward`` are pinned
+through special cases only: scaled-identity weights, where every BitLinear
+reduces to alpha * q / s and the scan to its unrolled sum; zero weights; the
+prefill == decode invariant. The pages print no worked example for them.
 """
 from __future__ import annotations
 
