@@ -269,8 +269,8 @@ def build_stack(w, device):
 
 # ----------------------------------------------------------------------------- oracle timing
 
-def oracle_sample(w, tokens: int):
-    """Time the CPU oracle on one block over `tokens` tokens of one sequence; returns (seconds, threads)."""
+def oracle_sample(w, tokens: int, nseq: int = 1):
+    """Time the CPU oracle on one block over `tokens` tokens of `nseq` sequences; returns (seconds, threads)."""
     import numpy as np
     from threadpoolctl import threadpool_info
 
@@ -280,21 +280,22 @@ def oracle_sample(w, tokens: int):
     lat = {n: synth.latent_weight(synth.sub_seed(w.seed, 0, i), *shapes[n]).numpy()
            for i, n in enumerate(synth.PROJ_NAMES)}
     blk = O.make_block(lat)
-    x = synth.activations(w.seed + synth.ACT_SEED_OFFSET, tokens, w.d, torch.bfloat16)
-    x = x.float().numpy().astype(np.float64).reshape(1, tokens, w.d)
+    x = synth.activations(w.seed + synth.ACT_SEED_OFFSET, nseq * tokens, w.d, torch.bfloat16)
+    x = x.float().numpy().astype(np.float64).reshape(nseq, tokens, w.d)
     t0 = time.perf_counter()
-    O.block_forward(x, blk, np.zeros((1, w.d)), w.dtype)
+    O.block_forward(x, blk, np.zeros((nseq, w.d)), w.dtype)
     dt = time.perf_counter() - t0
     threads = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
     return dt, threads
 
 
 def cpu_baseline_entry(w, tokens: int):
-    dt, threads = oracle_sample(w, tokens)
-    tps = tokens / (dt * w.layers)
+    # one block over the whole batch (several seconds of CPU work), extrapolated to the stack
+    dt, threads = oracle_sample(w, tokens, w.batch)
+    tps = w.batch * tokens / (dt * w.layers)
     return {"value": tps, "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"1 of {w.layers} blocks on {tokens} tokens of 1 of {w.batch} sequences "
-                      f"({dt:.2f} s), extrapolated x{w.layers} blocks",
+            "sample": f"1 of {w.layers} blocks on {w.batch} x {tokens} tokens (the whole batch, "
+                      f"{dt:.2f} s), extrapolated x{w.layers} blocks",
             "host_cores_available": len(os.sched_getaffinity(0))}
 
 
