@@ -92,6 +92,12 @@ def test_block_create_validation(lib):
     assert lib.mmf_block_create(ctypes.byref(w), d, I, ctypes.byref(h)) == 2
 
 
+def test_state_accessors_on_null_handle(lib):
+    assert lib.mmf_state_layer(None, 0) is None
+    assert lib.mmf_state_barrier(None) is None
+    assert lib.mmf_state_reset(None, None) == 1
+
+
 def test_workspace_sizes_grow_with_size(lib):
     assert lib.mmf_bitlinear_ws_size(16, 2048) < lib.mmf_bitlinear_ws_size(64, 2048)
     assert lib.mmf_glu_ws_size(4, 1024, 2816) > 4 * 2816
