@@ -263,6 +263,10 @@ size_t mmf_block_ws_size(const mmf_block* blk, int32_t B, int32_t T);
  * projections, recurrence and o-projection) and [DC] "Core components".
  * The MLGRU continues from the state of `layer` in `st` and leaves h_T there,
  * so T = 1 is one decode step and consecutive calls may split a prompt.
+ * A decode step (T = 1) runs four contractions (f|c|g with the recurrence
+ * step in its epilogue, o, gate|up, down). With MMF_DECODE_BLOCK_KERNEL=1 and
+ * B <= 8, d and I multiples of 64, it runs as one cooperative launch instead,
+ * with the same results; that launch uses the state's barrier words.
  * x and y must not overlap. Errors: INVALID_ARG, UNSUPPORTED_SHAPE,
  * MISALIGNED, WORKSPACE, CUDA. */
 mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf_state* st,
