@@ -432,22 +432,25 @@ def _eye_block(d):
     return O.Block(**{name: _scaled_eye(d, a) for name, a in ALPHAS.items()})
 
 
-def test_mlgru_identity_weights_closed_form():
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_mlgru_identity_weights_closed_form(dtype):
     # f, c, g, o = alpha_* I with distinct alphas: the projections reduce to
     # alpha * q/s, the scan to its unrolled sum; any swap of the three gate
     # projections, SiLU/sigmoid mix-up, missing (1 - f) or o-projection of h
-    # instead of o' changes the result
+    # instead of o' changes the result. Storage points in the run dtype.
     d, B, T = 32, 2, 6
     blk = _eye_block(d)
-    x = O.round_f32(synth.activations(61, B * T, d).numpy().reshape(B, T, d))
+    x = O.store(synth.activations(61, B * T, d).numpy().reshape(B, T, d), dtype)
     h0 = synth.activations(62, B, d).numpy().astype(np.float64)
-    o, hT, parts = O.mlgru(x, blk, h0, "f32", parts=True)
-    pf, pc, pg = (O.round_f32(_dq(getattr(blk, n), x)) for n in ("f", "c", "g"))
+    o, hT, parts = O.mlgru(x, blk, h0, dtype, parts=True)
+    pf, pc, pg = (O.store(_dq(getattr(blk, n), x), dtype) for n in ("f", "c", "g"))
     np.testing.assert_array_equal(parts["pf"], pf)
     np.testing.assert_array_equal(parts["pc"], pc)
     np.testing.assert_array_equal(parts["pg"], pg)
     og, h = _unrolled_scan(O.sigmoid(pf), O.silu(pc), O.sigmoid(pg), h0)
-    np.testing.assert_allclose(parts["o_gate"], O.round_f32(og), rtol=2e-7, atol=1e-12)
+    # o' is stored: agreement up to one storage ulp where the two sums round apart
+    ulp = 2.0 ** -7 if dtype == "bf16" else 2.0 ** -23
+    np.testing.assert_allclose(parts["o_gate"], O.store(og, dtype), rtol=ulp, atol=1e-12)
     np.testing.assert_allclose(hT, O.round_f32(h), rtol=2e-7)
     np.testing.assert_allclose(o, _dq(blk.o, parts["o_gate"]), rtol=1e-12)
     # f and g swapped would give a different o'
