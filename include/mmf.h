@@ -299,7 +299,7 @@ mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t L, mmf_stat
  * memory on every GPU that loads it and keeps until the process exits. The
  * call never calls cudaMalloc, cudaFree or any allocating routine. Its size
  * limit: round_up(M*K, 256) + 2 * round_up(4*M, 256) <= MMF_NOALLOC_SCRATCH_BYTES
- * (for example M = 64 tokens of K = 16384, or M = 512 of K = 4096); larger calls
+ * (for example M = 64 tokens of K = 16384, or at most M = 511 of K = 4096); larger calls
  * return MMF_ERR_UNSUPPORTED_SHAPE with a message naming the limit.
  * The first call on a device looks up the array's device address (a one-time
  * set-up with that device current); make that first call before any stream

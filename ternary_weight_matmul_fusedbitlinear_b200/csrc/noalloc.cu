@@ -66,6 +66,9 @@ extern "C" mmf_status mmf_bitlinear_noalloc(const mmf_tlinear* lin, const void* 
   if (x == nullptr || y == nullptr) return noalloc_fail(MMF_ERR_INVALID_ARG, "mmf_bitlinear_noalloc: null x/y");
   if (((uintptr_t)x | (uintptr_t)y | (uintptr_t)lin->packed) & 15u)
     return noalloc_fail(MMF_ERR_MISALIGNED, "mmf_bitlinear_noalloc: pointer not 16-byte aligned");
+  // the same layer checks as mmf_bitlinear: optional vectors must be 16-byte aligned too
+  if (((uintptr_t)lin->gain | (uintptr_t)lin->bias | (uintptr_t)lin->codes) & 15u)
+    return noalloc_fail(MMF_ERR_MISALIGNED, "mmf_bitlinear_noalloc: gain/bias/codes not 16-byte aligned");
   if (need_bytes(M, lin->K) > kNoallocBytes) {
     snprintf(msg, sizeof(msg),
              "mmf_bitlinear_noalloc: M=%d x K=%d needs %zu bytes of scratch, more than the fixed %zu-byte "

@@ -61,3 +61,33 @@ def test_noalloc_rejects_sizes_beyond_its_array():
                                    ctypes.c_void_p(y.data_ptr()), 1e-6, None)
     assert st == 2
     assert b"scratch" in lib.mmf_last_error()
+
+
+def test_noalloc_size_limit_boundary():
+    # K = 4096: M = 511 tokens fill the array exactly (511*4096 bytes of codes
+    # plus two 2048-byte slots for scales and row sums); M = 512 is one too many
+    k, n = 4096, 128
+    lin = mmf.quantize_weights(synth.latent_weight(1401, n, k).cuda())
+    lib = L.load()
+    cl = lin.c()
+    for m, want in ((511, 0), (512, 2)):
+        x = synth.activations(1402 + m, m, k, torch.bfloat16).cuda()
+        y = torch.empty(m, n, dtype=torch.bfloat16, device="cuda")
+        st = lib.mmf_bitlinear_noalloc(ctypes.byref(cl), ctypes.c_void_p(x.data_ptr()), L.MMF_BF16, m,
+                                       ctypes.c_void_p(y.data_ptr()), 1e-6,
+                                       ctypes.c_void_p(torch.cuda.current_stream().cuda_stream))
+        assert st == want, (m, st, lib.mmf_last_error())
+        if want == 0:
+            assert_close(to_np(y), to_np(mmf.bitlinear(lin, x)), "bf16", f"M={m}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_noalloc_with_gain_and_bias_matches_bitlinear(dtype):
+    k, n, m = 1024, 768, 8
+    W = synth.latent_weight(1410, n, k).cuda()
+    gain = (1.0 + 0.3 * synth.activations(1411, 1, k)[0]).cuda()
+    bias = (0.1 * synth.activations(1412, 1, n)[0]).cuda()
+    lin = mmf.quantize_weights(W, gain=gain, bias=bias)
+    for call in range(2):
+        x = synth.activations(1413 + call, m, k, TORCH_DT[dtype]).cuda()
+        assert_close(to_np(_noalloc(lin, x, dtype)), to_np(mmf.bitlinear(lin, x)), dtype, f"call {call + 1}")
