@@ -146,11 +146,26 @@ def unpack_codes(packed, K: int) -> np.ndarray:
 
 @dataclasses.dataclass
 class TLinear:
-    """A ternary BitLinear: codes [N,K] int8, per-matrix gamma, optional gain [K] / bias [N]."""
+    """A ternary BitLinear: codes [N,K] int8, per-matrix gamma, optional gain [K] / bias [N].
+
+    With ``cache`` set, the codes are also kept as the -1.0/0.0/+1.0 matrix that
+    ternary_accumulate multiplies (4 bytes per weight more memory, no
+    conversion per call); the results are the same either way.
+    """
     codes: np.ndarray
     gamma: np.float32
     gain: Optional[np.ndarray] = None
     bias: Optional[np.ndarray] = None
+    cache: bool = False
+    _dense: Optional[np.ndarray] = dataclasses.field(default=None, repr=False, compare=False)
+
+    def weights(self) -> np.ndarray:
+        """What ternary_accumulate takes: the cached dense codes, or the int8 codes."""
+        if not self.cache:
+            return self.codes
+        if self._dense is None:
+            self._dense = ternary_weights_dense(self.codes)
+        return self._dense
 
     @property
     def N(self) -> int:
@@ -161,11 +176,11 @@ class TLinear:
         return self.codes.shape[1]
 
 
-def make_tlinear(W_latent, gain=None, bias=None) -> TLinear:
+def make_tlinear(W_latent, gain=None, bias=None, cache: bool = False) -> TLinear:
     gamma, codes = ternarize(W_latent)
     g = None if gain is None else np.asarray(gain, dtype=np.float32)
     b = None if bias is None else np.asarray(bias, dtype=np.float64)
-    return TLinear(codes, gamma, g, b)
+    return TLinear(codes, gamma, g, b, cache)
 
 
 # ---------------------------------------------------------------------------
@@ -207,19 +222,32 @@ def absmax_quantize(xhat):
     return q, s
 
 
+# Largest K for which every partial sum of q[k] * w[k] (|q| <= 128, w in {-1,0,1})
+# is an integer below 2^24, i.e. exactly representable in fp32.
+F32_EXACT_K = (1 << 24) // 128
+
+
+def ternary_weights_dense(codes) -> np.ndarray:
+    """The ternary codes as a matrix of -1.0 / 0.0 / +1.0, in fp32 when K <= F32_EXACT_K, else fp64."""
+    c = np.asarray(codes)
+    return c.astype(np.float32 if c.shape[-1] <= F32_EXACT_K else np.float64)
+
+
 def ternary_accumulate(q, codes) -> np.ndarray:
-    """acc[m, n] = sum over k of q[m,k] * w[n,k] with w in {-1,0,1}, done as add/subtract.
+    """acc[m, n] = sum over k of q[m,k] * w[n,k] with w in {-1,0,1}, exact.
 
     [DC] "Replacing MatMul with ternary operations": multiplying by -1 negates,
-    by 0 drops, by 1 keeps. So acc = (sum of q where w = +1) - (sum of q where
-    w = -1). The two masked sums use an fp64 matrix product as a library step;
-    every partial sum is an integer below 2^53, so the result is exact.
+    by 0 drops, by 1 keeps, so every term is -q, 0 or +q and acc is an integer
+    sum. It is evaluated as one library matrix product of q with the codes
+    written as -1.0 / 0.0 / +1.0: every partial sum, in whatever order the
+    library adds, is an integer of magnitude at most 128 * K, which fp32 holds
+    exactly for K <= F32_EXACT_K (fp64 beyond), so the result is exact.
+    ``codes`` may be int8 codes or the output of ternary_weights_dense.
     """
-    q64 = np.asarray(q, dtype=np.float64)
     c = np.asarray(codes)
-    plus = (c == 1).astype(np.float64)
-    minus = (c == -1).astype(np.float64)
-    acc = q64 @ plus.T - q64 @ minus.T
+    w = c if c.dtype.kind == "f" else ternary_weights_dense(c)
+    qf = np.asarray(q).astype(w.dtype)
+    acc = qf @ w.T
     return np.rint(acc).astype(np.int64)
 
 
@@ -245,7 +273,7 @@ def bitlinear(x, lin: TLinear, eps: float = EPS_NORM, parts: bool = False):
     x2 = x.reshape(-1, x.shape[-1])
     xhat = rmsnorm(x2, lin.gain, eps)
     q, s = absmax_quantize(xhat)
-    acc = ternary_accumulate(q, lin.codes)
+    acc = ternary_accumulate(q, lin.weights())
     y = rescale(acc, lin.gamma, s, lin.bias)
     y = y.reshape(*lead, lin.N)
     if parts:
@@ -318,9 +346,9 @@ class Block:
         return self.gate.N
 
 
-def make_block(latents: dict) -> Block:
+def make_block(latents: dict, cache: bool = False) -> Block:
     """latents: dict of name -> fp32 latent [N, K] for f, c, g, o, gate, up, down."""
-    return Block(**{k: make_tlinear(latents[k]) for k in ("f", "c", "g", "o", "gate", "up", "down")})
+    return Block(**{k: make_tlinear(latents[k], cache=cache) for k in ("f", "c", "g", "o", "gate", "up", "down")})
 
 
 def mlgru_preacts(x, blk: Block, dtype: str, eps: float = EPS_NORM):

@@ -239,6 +239,29 @@ def test_accumulate_extremes_and_library_matmul():
     assert acc[0, 0] == 127 * K and acc[0, 1] == -127 * K
 
 
+def test_accumulate_exact_at_the_fp32_bound():
+    # K = F32_EXACT_K: the extreme rows sum to +-128 * K = +-2^24 and must stay exact;
+    # one past the bound switches to fp64 and stays exact too
+    for K in (O.F32_EXACT_K, O.F32_EXACT_K + 16):
+        q = np.full((2, K), 127, dtype=np.int8)
+        q[1, ::2] = -128
+        codes = np.ones((3, K), dtype=np.int8)
+        codes[1] = -1
+        codes[2, 1::2] = 0
+        acc = O.ternary_accumulate(q, codes)
+        ref = torch.tensor(q, dtype=torch.int64) @ torch.tensor(codes, dtype=torch.int64).T
+        np.testing.assert_array_equal(acc, ref.numpy())
+        assert O.ternary_weights_dense(codes).dtype == (np.float32 if K <= O.F32_EXACT_K else np.float64)
+
+
+def test_accumulate_cached_dense_weights_same_result():
+    lin = O.make_tlinear(synth.latent_weight(7, 40, 64).numpy(), cache=True)
+    x = synth.activations(8, 5, 64).numpy()
+    plain = O.TLinear(lin.codes, lin.gamma)
+    np.testing.assert_array_equal(O.bitlinear(x, lin), O.bitlinear(x, plain))
+    assert lin.weights().dtype == np.float32 and plain.weights().dtype == np.int8
+
+
 def test_accumulate_via_packed_words():
     rng = np.random.default_rng(6)
     codes = rng.integers(-1, 2, size=(33, 96)).astype(np.int8)
@@ -516,10 +539,12 @@ def test_block_prefill_equals_decode_steps(dtype):
 
 
 def test_stack_composes_blocks():
+    # distinct non-zero initial states per layer, so a stack that handed one
+    # layer's state to another would not compose the same way
     d, inner, B, T = 16, 32, 1, 4
     blocks = [_block(50 + l, d, inner) for l in range(3)]
     x = O.round_f32(synth.activations(53, B * T, d).numpy().reshape(B, T, d))
-    h0s = np.zeros((3, B, d))
+    h0s = O.round_f32(synth.activations(54, 3 * B, d).numpy().reshape(3, B, d) * np.array([1.0, -2.0, 0.5])[:, None, None])
     y, hs = O.stack_forward(x, blocks, h0s, "f32")
     z = x
     for l in range(3):
