@@ -69,6 +69,8 @@ def parse_args(argv=None):
                     help="stack370m: number of blocks (default 24; fewer for short profiler captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) pass")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--no-sub", action="store_true",
+                    help="stack370m: skip the decode-step and GEMV-sweep sub-measurements")
     return ap.parse_args(argv)
 
 
@@ -79,6 +81,18 @@ def load_peaks():
             d = json.load(f)
         return d, "measured"
     return dict(FALLBACK_PEAKS), "fallback"
+
+
+def int8_peak(peaks, peak_kind, clk):
+    """Dense int8 tensor peak for a contraction timed in this run: 2 x the bf16 burst figure, or 2 x the
+    sustained one when the sampled clocks show power capping or SM clocks well below their maximum."""
+    burst = peaks["bf16_tflops"] * INT8_OVER_BF16
+    sustained = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_OVER_BF16
+    sm, mx = (clk or {}).get("sm_mhz"), (clk or {}).get("sm_max_mhz")
+    capped = "sw_power_cap" in (clk or {}).get("reasons", []) or bool(sm and mx and sm < 0.9 * mx)
+    kind = "sustained" if capped else "burst"
+    return (sustained if capped else burst), burst, sustained, \
+        f"{peak_kind}: bf16 {kind} x {INT8_OVER_BF16} (int8 dense : bf16 dense nominal)"
 
 
 # ----------------------------------------------------------------------------- distributed plumbing
@@ -227,12 +241,11 @@ class ClockSampler:
 
 # ----------------------------------------------------------------------------- workload
 
-# DRAM bytes (read + write) per launch of the dominant kernel, from the ncu capture summarised in
-# profiles/tgemm_tc_stack370m_block.md: mean over the four contraction launches of one 370M block with
-# one-byte weight codes. Valid while that kernel is unchanged; None elsewhere.
+# DRAM bytes (read + write) per launch of the dominant kernel, measured by an ncu capture of the same
+# kernel (mean over the four contraction launches of one 370M block, one-byte weight codes). Reported as
+# the `traffic` of the headline line with the capture named in `traffic_source`; None elsewhere.
 STACK370M_CONTRACTION_TRAFFIC = 69.38e6
-# Same for the scan at the 370M layer shape (profiles/mlgru_scan_b8_t2048_d1024.md): 100.9 + 10.3 MB.
-SCAN370M_TRAFFIC = 111.16e6
+STACK370M_TRAFFIC_SOURCE = "ncu capture, tgemm_tc at the four 370M block shapes (dram__bytes read + write)"
 
 
 def stack_workload(layers=None):
@@ -398,17 +411,34 @@ def run_mmf(args):
     gemm_launches = sum(prof[k][0] for k in gemm_names)
     ops = gemm_ops_per_step(w) * args.steps
     achieved = ops / (gemm_ms / 1e3) / 1e12 if gemm_ms > 0 else 0.0
-    peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]) * INT8_OVER_BF16
+    peak, peak_burst, peak_sus, peak_src = int8_peak(peaks, peak_kind, clk)
     launches = sum(v[0] for v in prof.values())
     byte_codes = os.environ.get("MMF_PREFILL_UNPACKED", "1") != "0"
     roofline = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                "frac": achieved / peak, "traffic": STACK370M_CONTRACTION_TRAFFIC if byte_codes else None,
-                "traffic_note": "DRAM bytes per contraction launch, mean of one block's four (ncu)",
+                "frac": achieved / peak, "frac_of_sustained": achieved / peak_sus, "peak_sustained": peak_sus,
+                "traffic": STACK370M_CONTRACTION_TRAFFIC if byte_codes else None,
+                "traffic_note": "DRAM bytes per contraction launch, mean of one block's four",
+                "traffic_source": STACK370M_TRAFFIC_SOURCE,
                 "kernel": ",".join(gemm_names), "launches": gemm_launches,
                 "share_of_step": gemm_ms / sum(prof_step_ms) if prof_step_ms else None,
                 "kernel_times": "CUDA events around each kernel in a second pass of the same steps",
-                "peak_source": f"{peak_kind}: bf16 sustained x {INT8_OVER_BF16} (int8 dense : bf16 dense nominal)",
+                "peak_source": peak_src,
                 "per_kernel_ms": {k: round(v[1] / args.steps, 4) for k, v in prof.items()}}
+    # the other kernels of the step against HBM, from the same per-kernel times
+    M = w.batch * w.seq
+    hbm = peaks["hbm_gbs"]
+    others = {}
+    if "mlgru_scan" in prof:
+        scan_ms = prof["mlgru_scan"][1] / prof["mlgru_scan"][0]
+        gbs = 8.0 * M * w.d / (scan_ms / 1e3) / 1e9   # 6 B read + 2 B written per channel-step (bf16)
+        others["mlgru_scan"] = {"us_per_layer": round(scan_ms * 1e3, 2), "GBps": round(gbs, 1),
+                                "frac": round(gbs / hbm, 4), "bytes_per_layer": 8.0 * M * w.d}
+    if "rmsnorm_quant" in prof:
+        q_ms = prof["rmsnorm_quant"][1] / args.steps
+        qbytes = 3.0 * M * (3 * w.d + w.inner) * w.layers   # 2 B read + 1 B written per element (bf16)
+        gbs = qbytes / (q_ms / 1e3) / 1e9
+        others["rmsnorm_quant"] = {"ms_per_step": round(q_ms, 4), "GBps": round(gbs, 1), "frac": round(gbs / hbm, 4),
+                                   "bytes_per_step": qbytes}
 
     # ------------------------------------------------------------ end to end through the public API
     # Every step's input is copied from pinned host memory and its output copied
@@ -465,6 +495,20 @@ def run_mmf(args):
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         cpu = cpu_baseline_entry(w, 2048)
 
+    # the metric's other clauses, each its own timed measurement after the headline: the decode
+    # BitLinear GEMV sweep and a 2.7B-shaped decode step (HBM-bound), on every rank like the headline
+    sub = None
+    if not args.no_sub:
+        del blocks, ws, flush
+        torch.cuda.empty_cache()
+        sub = {"kernels_in_step": others}
+        w27 = synth.STACK_2P7B
+        d27 = measure_decode(mmf, w27, 1, 128, 3, dev, peaks, prompt=False)
+        sub["decode_2p7b_b1"] = {k: d27[k] for k in ("ms_per_step", "tokens_per_s", "GBps", "frac", "bytes_per_step",
+                                                      "launches_per_step", "decode_steps", "clocks")}
+        torch.cuda.empty_cache()
+        sub["gemv_sweep"] = measure_gemv(mmf, dev, 2, 3, peaks)
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
@@ -475,7 +519,7 @@ def run_mmf(args):
                        "parallelism": f"replicas x{world} (independent sequences)",
                        "l2": "flushed between timed steps (252 MB write outside the step events)"},
             "roofline": roofline, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": int(launches), "clocks": clk,
+            "gpu_launches": int(launches), "clocks": clk, "sub": sub,
         }
         print(json.dumps(line), flush=True)
     barrier(world)
@@ -582,20 +626,16 @@ def run_scan(args):
             "data": "synthetic", "config": {"workload": f"mlgru_scan_b{B}_t{T}_d{d}_bf16",
                                             "l2": "flushed between timed steps"},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": SCAN370M_TRAFFIC, "kernel": "mlgru_scan",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mlgru_scan (with its scratch reset)",
                          "peak_source": peak_kind},
             "cpu_baseline": None, "e2e": None, "gpu_launches": prof["mlgru_scan"][0]}), flush=True)
     return 0
 
 
-def run_gemv(args):
+def measure_gemv(mmf, dev, reps: int, warmup: int, peaks) -> dict:
     """Decode BitLinear sweep: per shape and token count, calls cycle through a pool of distinct packed
-    matrices totalling more than 4x L2; GB/s = (N*K/4 + 4 + 2*M*K + 2*M*N) bytes per call / mean call time."""
-    _, rank, local = dist_env()
-    torch.cuda.set_device(local)
-    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
-    dev = torch.device("cuda", local)
-    peaks, peak_kind = load_peaks()
+    matrices totalling more than 4x L2, replayed as one CUDA graph; GB/s = (N*K/4 + 4 + 2*M*K + 2*M*N)
+    bytes per call / mean call time. The calls form a dependent chain on one stream."""
     rows = []
     for (K, N) in synth.GEMV_SWEEP_SHAPES:
         per = N * K // 4
@@ -606,23 +646,19 @@ def run_gemv(args):
             x = synth.activations(synth.GEMV_SWEEP_SEED + M, M, K, torch.bfloat16, outlier_p=synth.GEMV_OUTLIER_P,
                                   outlier_scale=synth.GEMV_OUTLIER_SCALE, device=dev)
             ws = torch.empty(mmf.api.L.load().mmf_bitlinear_ws_size(M, K), dtype=torch.uint8, device=dev)
-            y = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
             side = torch.cuda.Stream(dev)
             side.wait_stream(torch.cuda.current_stream(dev))
             with torch.cuda.stream(side):
-                for lin in lins[:max(args.warmup, 3)]:
+                for lin in lins[:max(warmup, 3)]:
                     mmf.bitlinear(lin, x, ws=ws)
             torch.cuda.current_stream(dev).wait_stream(side)
             torch.cuda.synchronize()
-            # one graph replays the whole pool in order: launch cost leaves the host
-            calls = pool_n
-            graph = torch.cuda.CUDAGraph()
+            graph = torch.cuda.CUDAGraph()   # the whole pool in order: launch cost leaves the host
             with torch.cuda.graph(graph):
-                for i in range(calls):
+                for i in range(pool_n):
                     mmf.bitlinear(lins[i], x, ws=ws)
             graph.replay()
             torch.cuda.synchronize()
-            reps = max(1, args.steps // 5)
             e0 = torch.cuda.Event(enable_timing=True)
             e1 = torch.cuda.Event(enable_timing=True)
             e0.record()
@@ -631,85 +667,103 @@ def run_gemv(args):
             e1.record()
             torch.cuda.synchronize()
             del graph
-            calls = calls * reps
-            us = e0.elapsed_time(e1) * 1e3 / calls
+            us = e0.elapsed_time(e1) * 1e3 / (pool_n * reps)
             nbytes = per + 4 + 2 * M * K + 2 * M * N
             rows.append({"K": K, "N": N, "M": M, "us_per_call": round(us, 3),
                          "GBps": round(nbytes / (us * 1e-6) / 1e9, 1),
                          "frac": round(nbytes / (us * 1e-6) / 1e9 / peaks["hbm_gbs"], 4),
                          "TOPS": round(2.0 * M * N * K / (us * 1e-6) / 1e12, 3), "pool": pool_n})
-            del ws, y
+            del ws
         del lins
         torch.cuda.empty_cache()
-    best = max(r["GBps"] for r in rows)
     mean = sum(r["GBps"] for r in rows) / len(rows)
-    if rank == 0:
-        print(json.dumps({
-            "metric": METRIC, "value": mean, "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": "bitlinear_decode_gemv_sweep", "l2": "weight pool > 4x L2, cycled"},
-            "roofline": {"bound": "hbm", "achieved": mean, "best": best, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": mean / peaks["hbm_gbs"], "traffic": None, "kernel": "rmsnorm_quant+tgemm_mma",
-                         "peak_source": peak_kind, "sweep": rows},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": None}), flush=True)
-    return 0
+    return {"mean_GBps": round(mean, 1), "best_GBps": max(r["GBps"] for r in rows),
+            "frac_mean": round(mean / peaks["hbm_gbs"], 4), "shapes": rows,
+            "note": "dependent chain of single calls (each waits for the previous one's output)"}
 
 
-def run_decode(args):
-    """Prompt prefill, then decode steps; each decode step (all layers, T=1) is one CUDA graph replay whose
-    output is copied back to its input. Reports decode tokens/s, and HBM GB/s of the packed-weight stream."""
+def run_gemv(args):
     _, rank, local = dist_env()
     torch.cuda.set_device(local)
     import ternary_weight_matmul_fusedbitlinear_b200 as mmf
     dev = torch.device("cuda", local)
-    w = synth.STACK_1P3B if args.workload == "decode1p3b" else synth.STACK_2P7B
-    B = args.batch or w.batch
     peaks, peak_kind = load_peaks()
-    blocks = build_stack(w, dev)
+    g = measure_gemv(mmf, dev, max(1, args.steps // 5), args.warmup, peaks)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": g["mean_GBps"], "unit": "GB/s", "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": None, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": "bitlinear_decode_gemv_sweep", "l2": "weight pool > 4x L2, cycled"},
+            "roofline": {"bound": "hbm", "achieved": g["mean_GBps"], "best": g["best_GBps"], "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": g["frac_mean"], "traffic": None, "kernel": "rmsnorm_quant+tgemm_mma",
+                         "peak_source": peak_kind, "sweep": g["shapes"]},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": None}), flush=True)
+    return 0
+
+
+def decode_bytes_per_step(w, B) -> float:
+    """Algorithmic bytes of one decode step: the packed weights (0.25 B/weight) + the state read and written."""
+    weights = w.layers * (4 * w.d * w.d + 3 * w.d * w.inner) / 4.0
+    return weights + 2.0 * w.layers * B * w.d * 4
+
+
+def measure_decode(mmf, w, B: int, steps: int, warmup: int, dev, peaks, prompt: bool = True, blocks=None) -> dict:
+    """Optional prompt prefill, then `steps` decode steps; each decode step (all layers, T=1) is one CUDA
+    graph replay whose output is copied back to its input. Returns the timings and the HBM GB/s of the
+    step's algorithmic bytes (packed weights + state)."""
+    blocks = blocks if blocks is not None else build_stack(w, dev)
     st = mmf.State(w.layers, B, w.d)
-    prompt = synth.activations(w.seed + synth.ACT_SEED_OFFSET, B * w.seq, w.d, torch.bfloat16,
+    out = {"batch": B, "layers": w.layers, "d": w.d, "inner": w.inner}
+    if prompt:
+        xp = synth.activations(w.seed + synth.ACT_SEED_OFFSET, B * w.seq, w.d, torch.bfloat16,
                                device=dev).reshape(B, w.seq, w.d)
-    ws_p = torch.empty(mmf.stack_ws_size(blocks, B, w.seq), dtype=torch.uint8, device=dev)
-    y_p = torch.empty_like(prompt)
-    # prompt prefill (timed separately)
-    mmf.stack_forward(blocks, st, prompt, ws=ws_p, out=y_p)
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    st.reset()
-    e0.record()
-    mmf.stack_forward(blocks, st, prompt, ws=ws_p, out=y_p)
-    e1.record()
-    torch.cuda.synchronize()
-    prefill_ms = e0.elapsed_time(e1)
-    del ws_p
-    # decode: input = last prompt position's output
-    x = y_p[:, -1:, :].contiguous()
+        ws_p = torch.empty(mmf.stack_ws_size(blocks, B, w.seq), dtype=torch.uint8, device=dev)
+        y_p = torch.empty_like(xp)
+        mmf.stack_forward(blocks, st, xp, ws=ws_p, out=y_p)   # warm-up
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        st.reset()
+        e0.record()
+        mmf.stack_forward(blocks, st, xp, ws=ws_p, out=y_p)
+        e1.record()
+        torch.cuda.synchronize()
+        out["prompt"] = w.seq
+        out["prefill_ms"] = e0.elapsed_time(e1)
+        out["prefill_tokens_per_s"] = B * w.seq / (out["prefill_ms"] / 1e3)
+        x = y_p[:, -1:, :].contiguous()
+        del ws_p, xp, y_p
+    else:
+        x = synth.activations(w.seed + synth.ACT_SEED_OFFSET, B, w.d, torch.bfloat16, device=dev).reshape(B, 1, w.d)
     y = torch.empty_like(x)
     ws = torch.empty(mmf.stack_ws_size(blocks, B, 1), dtype=torch.uint8, device=dev)
     side = torch.cuda.Stream(dev)
     side.wait_stream(torch.cuda.current_stream(dev))
-    with torch.cuda.stream(side):
+    with torch.cuda.stream(side):   # eager steps first: they also allocate the state's decode buffers
         for _ in range(3):
             mmf.stack_forward(blocks, st, x, ws=ws, out=y)
     torch.cuda.current_stream(dev).wait_stream(side)
     torch.cuda.synchronize()
+    mmf.check()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         mmf.stack_forward(blocks, st, x, ws=ws, out=y)
         x.copy_(y)
-    steps = args.decode_steps or w.decode_steps
-    for _ in range(args.warmup):
+    for _ in range(max(warmup, 3)):
         graph.replay()
     torch.cuda.synchronize()
-    clocks = ClockSampler(local)
+    clocks = ClockSampler(dev.index or 0)
     clocks.start()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for _ in range(steps):
         graph.replay()
     e1.record()
+    wait_event(e1)
     torch.cuda.synchronize()
     clk = clocks.stop()
+    del graph
+    mmf.check()
     step_ms = e0.elapsed_time(e1) / steps
     # per-kernel device time of a decode step (eager launches, outside the timed region)
     mmf.prof_reset()
@@ -719,26 +773,39 @@ def run_decode(args):
     torch.cuda.synchronize()
     mmf.prof_enable(False)
     prof = mmf.prof_collect()
-    per_kernel = {k: round(v[1] / 5, 4) for k, v in prof.items()}
-    launches_per_step = sum(v[0] for v in prof.values()) // 5
-    weights = w.layers * (4 * w.d * w.d + 3 * w.d * w.inner) / 4.0
-    state = 2.0 * w.layers * B * w.d * 4
-    gbs = (weights + state) / (step_ms / 1e3) / 1e9
+    nbytes = decode_bytes_per_step(w, B)
+    gbs = nbytes / (step_ms / 1e3) / 1e9
+    out.update({"decode_steps": steps, "ms_per_step": step_ms, "tokens_per_s": B / (step_ms / 1e3),
+                "GBps": gbs, "frac": gbs / peaks["hbm_gbs"], "bytes_per_step": nbytes,
+                "launches_per_step": sum(v[0] for v in prof.values()) // 5,
+                "per_kernel_ms_eager_step": {k: round(v[1] / 5, 4) for k, v in prof.items()}, "clocks": clk})
+    return out
+
+
+def run_decode(args):
+    _, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    dev = torch.device("cuda", local)
+    w = synth.STACK_1P3B if args.workload == "decode1p3b" else synth.STACK_2P7B
+    B = args.batch or w.batch
+    peaks, peak_kind = load_peaks()
+    steps = args.decode_steps or w.decode_steps
+    r = measure_decode(mmf, w, B, steps, args.warmup, dev, peaks, prompt=True)
     if rank == 0:
         print(json.dumps({
-            "metric": METRIC, "value": B / (step_ms / 1e3), "unit": "tokens/s", "n_gpus": 1, "steps": steps,
-            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "metric": METRIC, "value": r["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": f"{w.name}_b{B}", "batch": B, "layers": w.layers, "d": w.d, "inner": w.inner,
-                       "prompt": w.seq, "decode_steps": steps,
-                       "prefill_ms": prefill_ms, "prefill_tokens_per_s": B * w.seq / (prefill_ms / 1e3),
-                       "l2": "weight stream per step > L2"},
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "decode step (all kernels)",
-                         "bytes_per_step": weights + state, "peak_source": peak_kind,
-                         "per_kernel_ms_eager_step": per_kernel},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": launches_per_step * steps, "clocks": clk}),
-              flush=True)
+                       "prompt": w.seq, "decode_steps": steps, "prefill_ms": r["prefill_ms"],
+                       "prefill_tokens_per_s": r["prefill_tokens_per_s"], "l2": "weight stream per step > L2"},
+            "roofline": {"bound": "hbm", "achieved": r["GBps"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": r["frac"], "traffic": None, "kernel": "decode step (all kernels)",
+                         "bytes_per_step": r["bytes_per_step"], "peak_source": peak_kind,
+                         "per_kernel_ms_eager_step": r["per_kernel_ms_eager_step"]},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": r["launches_per_step"] * steps,
+            "clocks": r["clocks"]}), flush=True)
     return 0
 
 

@@ -232,24 +232,20 @@ void mmf_block_destroy(mmf_block* blk);
 
 /* Recurrent state h for L layers x B sequences x d channels, fp32, zeroed.
  * The library allocates it with cudaMalloc on the current device and frees it
- * in mmf_state_destroy. It also holds the two barrier words of the opt-in
- * one-launch decode step (environment variable MMF_DECODE_BLOCK_KERNEL=1:
- * T == 1, B <= 8, d and I multiples of 64), which must be zero between
- * launches; calls that share a state are stream-ordered anyway, since h is
- * updated in place. */
+ * in mmf_state_destroy. The first decode step (T = 1) that runs as one launch
+ * (see mmf_block_forward) also allocates, with cudaMalloc, the state's
+ * exchange buffers for that launch (2 x 4 bytes x B x (3 d + I) per layer plus
+ * a small header; again for a later call with a larger I), so make that first
+ * decode call before any stream capture. Calls that share a state must be
+ * ordered on one stream: h and the exchange buffers are updated in place. */
 mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_state** out);
 void mmf_state_destroy(mmf_state* st);
-/* Zero every layer's state and the barrier words (asynchronous on stream);
- * also the way to recover after mmf_check reported a barrier wait that gave
- * up (code 4). */
+/* Zero every layer's state and reset the decode exchange buffers
+ * (asynchronous on stream); also the way to recover after mmf_check reported
+ * a decode step whose waits gave up (codes 5 and 6). */
 mmf_status mmf_state_reset(mmf_state* st, void* stream);
 /* Device address of layer `layer`'s state, float [B, d]; NULL if out of range. */
 float* mmf_state_layer(mmf_state* st, int32_t layer);
-/* Device address of the state's 256 bytes of barrier words (counter at byte
- * 0, generation at byte 128, uint32 each), for diagnostics and tests; NULL for
- * a null state. Nonzero words between launches make the one-launch decode
- * step's barriers give up after their bounded wait (status code 4). */
-uint32_t* mmf_state_barrier(mmf_state* st);
 /* Copy the whole state [L, B, d] fp32 to / from host memory; synchronises stream. */
 mmf_status mmf_state_get(const mmf_state* st, float* host_dst, void* stream);
 mmf_status mmf_state_set(mmf_state* st, const float* host_src, void* stream);
@@ -263,20 +259,58 @@ size_t mmf_block_ws_size(const mmf_block* blk, int32_t B, int32_t T);
  * projections, recurrence and o-projection) and [DC] "Core components".
  * The MLGRU continues from the state of `layer` in `st` and leaves h_T there,
  * so T = 1 is one decode step and consecutive calls may split a prompt.
- * A decode step (T = 1) runs four contractions (f|c|g with the recurrence
- * step in its epilogue, o, gate|up, down). With MMF_DECODE_BLOCK_KERNEL=1 and
- * B <= 8, d and I multiples of 64, it runs as one cooperative launch instead,
- * with the same results; that launch uses the state's barrier words.
- * x and y must not overlap. Errors: INVALID_ARG, UNSUPPORTED_SHAPE,
- * MISALIGNED, WORKSPACE, CUDA. */
+ * A decode step (T = 1) of B <= 8 sequences (d and I multiples of 64, at
+ * most 3 x 16 rows of each matrix per SM) runs as one cooperative launch:
+ * every CTA streams its rows of the four projections through shared memory
+ * and the stages hand their outputs over through the state's exchange
+ * buffers (mmf_state_create). Each wait in that launch is bounded (about 1 s);
+ * one that runs out is reported by mmf_check (MMF_ERR_TIMEOUT, code 5 or 6),
+ * after which the state must be reset. Larger batches, other shapes, or the
+ * environment variable MMF_DECODE_STEP_KERNEL=0 run four contractions instead
+ * (f|c|g with the recurrence step in its epilogue, o, gate|up, down), with the
+ * same arithmetic. x and y must not overlap. Errors: INVALID_ARG,
+ * UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, NOMEM, CUDA. */
 mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf_state* st,
                              const void* x, void* y, int32_t B, int32_t T, mmf_dtype dtype,
                              float eps, void* ws, size_t ws_bytes, void* stream);
 
+/* Optional device outputs of one block step's stored intermediates, for
+ * checking each stage on its own (any field may be NULL; M = B * T tokens,
+ * activation dtype unless stated):
+ *   pre       [M, 3, d]: the f~, c~, g~ pre-activations as the kernels store them
+ *   og        [M, d]: o' = g * h, the input of the o projection
+ *   y1        [M, d]: x + o, the token mixer's output and the GLU's input
+ *   p         [M, I]: SiLU(gate) * up, the input of the down projection
+ *   q[i]      int8 activation codes of the i-th quantised input (0: x [M, d],
+ *             1: o' [M, d], 2: y1 [M, d], 3: p [M, I])
+ *   scale[i]  float [M]: their per-token scales s
+ * Buffers are 16-byte aligned device memory of at least the sizes above. */
+typedef struct mmf_block_debug {
+  void* pre;
+  void* og;
+  void* y1;
+  void* p;
+  int8_t* q[4];
+  float* scale[4];
+} mmf_block_debug;
+
+/* mmf_block_forward, also writing the intermediates named in `dbg` (host
+ * struct of device pointers; NULL behaves as mmf_block_forward). The stages
+ * and their results are those of mmf_block_forward; the extra copies are
+ * stream-ordered device-to-device copies, plus code outputs of the
+ * contraction kernels that quantise their own input rows.
+ * Errors: as mmf_block_forward, and MISALIGNED for a debug buffer. */
+mmf_status mmf_block_forward_debug(const mmf_block* blk, int32_t layer, mmf_state* st,
+                                   const void* x, void* y, int32_t B, int32_t T, mmf_dtype dtype,
+                                   float eps, void* ws, size_t ws_bytes, void* stream,
+                                   const mmf_block_debug* dbg);
+
 /* L blocks in sequence (block l uses state layer l): y = block_{L-1}(...block_0(x)).
  * blocks (host) array of L handles. x and y (device) [B, T, d] must not overlap;
  * intermediate activations live in the workspace (mmf_block_ws_size of the
- * largest block). Errors as mmf_block_forward. */
+ * largest block). A decode step (T = 1) that qualifies for the one-launch form
+ * (mmf_block_forward) covers up to 32 layers per launch. Errors as
+ * mmf_block_forward. */
 mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t L, mmf_state* st,
                              const void* x, void* y, int32_t B, int32_t T, mmf_dtype dtype,
                              float eps, void* ws, size_t ws_bytes, void* stream);

@@ -30,6 +30,10 @@ class BitlinearDebug(ctypes.Structure):
     _fields_ = [("q", c_vp), ("scale", c_vp), ("acc", c_vp)]
 
 
+class BlockDebug(ctypes.Structure):
+    _fields_ = [("pre", c_vp), ("og", c_vp), ("y1", c_vp), ("p", c_vp), ("q", c_vp * 4), ("scale", c_vp * 4)]
+
+
 class BlockWeights(ctypes.Structure):
     _fields_ = [(n, TLinear) for n in ("f", "c", "g", "o", "gate", "up", "down")]
 
@@ -56,12 +60,13 @@ SIGNATURES = {
     "mmf_state_destroy": (None, [c_vp]),
     "mmf_state_reset": (ctypes.c_int, [c_vp, c_vp]),
     "mmf_state_layer": (c_vp, [c_vp, c_i32]),
-    "mmf_state_barrier": (c_vp, [c_vp]),
     "mmf_state_get": (ctypes.c_int, [c_vp, c_vp, c_vp]),
     "mmf_state_set": (ctypes.c_int, [c_vp, c_vp, c_vp]),
     "mmf_block_ws_size": (c_sz, [c_vp, c_i32, c_i32]),
     "mmf_block_forward": (ctypes.c_int, [c_vp, c_i32, c_vp, c_vp, c_vp, c_i32, c_i32, ctypes.c_int, c_f, c_vp, c_sz,
                                          c_vp]),
+    "mmf_block_forward_debug": (ctypes.c_int, [c_vp, c_i32, c_vp, c_vp, c_vp, c_i32, c_i32, ctypes.c_int, c_f, c_vp,
+                                               c_sz, c_vp, ctypes.POINTER(BlockDebug)]),
     "mmf_stack_forward": (ctypes.c_int, [ctypes.POINTER(c_vp), c_i32, c_vp, c_vp, c_vp, c_i32, c_i32, ctypes.c_int,
                                          c_f, c_vp, c_sz, c_vp]),
     "mmf_bitlinear_noalloc": (ctypes.c_int, [ctypes.POINTER(TLinear), c_vp, ctypes.c_int, c_i32, c_vp, c_f, c_vp]),

@@ -199,15 +199,6 @@ class State:
     def reset(self):
         L.check(L.load().mmf_state_reset(self.handle, _stream(torch.device("cuda"))), "mmf_state_reset")
 
-    def barrier_words(self) -> torch.Tensor:
-        """uint32 view [64] of the state's barrier words (mmf_state_barrier): counter at [0], generation at [32]."""
-        ptr = L.load().mmf_state_barrier(self.handle)
-
-        class _Words:
-            __cuda_array_interface__ = {"shape": (64,), "typestr": "<u4", "data": (ptr, False), "version": 2}
-
-        return torch.as_tensor(_Words(), device="cuda")
-
     def get(self) -> torch.Tensor:
         out = torch.empty(self.L, self.B, self.d, dtype=torch.float32)
         L.check(L.load().mmf_state_get(self.handle, ctypes.c_void_p(out.data_ptr()),
@@ -244,6 +235,32 @@ def block_forward(block: Block, layer: int, state: State, x: torch.Tensor, eps: 
                                        _vp(w), w.numel() * w.element_size(), _stream(x.device)),
             "mmf_block_forward")
     return y
+
+
+def block_forward_debug(block: Block, layer: int, state: State, x: torch.Tensor, eps: float = DEFAULT_EPS,
+                        ws: Optional[torch.Tensor] = None):
+    """block_forward that also returns the stored intermediates (mmf_block_forward_debug): a dict with
+    pre [B, T, 3, d], og [B, T, d], y1 [B, T, d], p [B, T, I], and q[i] / s[i] (int8 codes [M, K] and
+    scales [M] of the i-th quantised input: 0 x, 1 o', 2 y1, 3 p)."""
+    _need_cuda(x)
+    B, T, d = x.shape
+    M, I = B * T, block.inner
+    dev = x.device
+    y = torch.empty_like(x)
+    w = _workspace(block.ws_size(B, T), dev, ws)
+    out = {"pre": torch.empty(B, T, 3, d, dtype=x.dtype, device=dev),
+           "og": torch.empty(B, T, d, dtype=x.dtype, device=dev),
+           "y1": torch.empty(B, T, d, dtype=x.dtype, device=dev),
+           "p": torch.empty(B, T, I, dtype=x.dtype, device=dev),
+           "q": [torch.empty(M, k, dtype=torch.int8, device=dev) for k in (d, d, d, I)],
+           "s": [torch.empty(M, dtype=torch.float32, device=dev) for _ in range(4)]}
+    dbg = L.BlockDebug(out["pre"].data_ptr(), out["og"].data_ptr(), out["y1"].data_ptr(), out["p"].data_ptr(),
+                       (L.c_vp * 4)(*[t.data_ptr() for t in out["q"]]),
+                       (L.c_vp * 4)(*[t.data_ptr() for t in out["s"]]))
+    L.check(L.load().mmf_block_forward_debug(block.handle, layer, state.handle, _vp(x), _vp(y), B, T, _dtype(x), eps,
+                                             _vp(w), w.numel() * w.element_size(), _stream(dev), ctypes.byref(dbg)),
+            "mmf_block_forward_debug")
+    return y, out
 
 
 def stack_ws_size(blocks: Sequence[Block], B: int, T: int) -> int:

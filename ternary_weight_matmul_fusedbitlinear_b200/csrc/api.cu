@@ -124,13 +124,10 @@ cudaError_t timed(const char* name, cudaStream_t s, F&& launch) {
   return e;
 }
 
-// Contraction dispatch: the single-SM tcgen05 kernel from 128 tokens, the
-// mma.sync kernel for decode-sized token counts and for shapes the tcgen05
-// kernels do not take. The SM-pair tcgen05 kernel (M >= 256) is selected only
-// on request: it is correct but measured slower than the single-SM kernel on
-// the 370M shapes. MMF_GEMM_PATH=mma|tc|tc1|tc2|auto (default auto; tc and tc1
-// both mean the single-SM kernel) pins one implementation; all compute the
-// same exact integer accumulators.
+// Contraction dispatch: the tcgen05 kernel from 128 tokens, the mma.sync
+// kernel for decode-sized token counts and for shapes the tcgen05 kernel does
+// not take. MMF_GEMM_PATH=mma|tc|auto (default auto) pins one implementation;
+// both compute the same exact integer accumulators.
 constexpr int kTcMinTokens = 128;
 
 int gemm_path_pref() {
@@ -138,19 +135,7 @@ int gemm_path_pref() {
   if (e == nullptr) return 0;
   if (strcmp(e, "mma") == 0) return 1;
   if (strcmp(e, "tc") == 0) return 2;
-  if (strcmp(e, "tc1") == 0) return 3;
-  if (strcmp(e, "tc2") == 0) return 4;
   return 0;
-}
-
-// The prefill token mixer as one kernel (contraction + MLGRU in the epilogue)
-// only with MMF_FUSED_MLGRU=1: it saves the pre-activation round trip through
-// HBM, but its epilogue (gates and a warp-shuffle scan per channel) takes
-// about twice as long as the contraction's main loop, and on one B200 it
-// measured 3.9 ms per 370M step against 3.0 ms for contraction + scan.
-bool fused_mlgru_enabled() {
-  const char* e = getenv("MMF_FUSED_MLGRU");
-  return e != nullptr && strcmp(e, "1") == 0;
 }
 
 bool gemm_uses_tc(const TGemmArgs& a, Epi epi) {
@@ -172,17 +157,12 @@ bool decode_fused_quant_wanted(int M) {
 
 // `what` names the projection for the launch-timing totals ("fcg", "o", ...).
 cudaError_t run_gemm(const TGemmArgs& a, Epi epi, mmf_dtype dt, cudaStream_t s, const char* what = "") {
-  const int pref = gemm_path_pref();
-  const bool tc2_ok = tgemm_tc2_supported(a, epi);
-  bool use_tc = gemm_uses_tc(a, epi);
-  const bool use_tc2 = use_tc && tc2_ok && pref == 4;
+  const bool use_tc = gemm_uses_tc(a, epi);
   char name[48];
-  snprintf(name, sizeof(name), "%s%s%s", use_tc2 ? "tgemm_tc2" : (use_tc ? "tgemm_tc" : "tgemm_mma"),
-           what[0] ? ":" : "", what);
+  snprintf(name, sizeof(name), "%s%s%s", use_tc ? "tgemm_tc" : "tgemm_mma", what[0] ? ":" : "", what);
   if (use_tc) {
     int* st = nullptr;
     if (device_status_ptr(&st) != MMF_OK) return cudaErrorUnknown;
-    if (use_tc2) return timed(name, s, [&] { return launch_tgemm_tc2(a, epi, dt, st, s); });
     return timed(name, s, [&] { return launch_tgemm_tc(a, epi, dt, st, s); });
   }
   return timed(name, s, [&] { return launch_tgemm_mma(a, epi, dt, s); });
@@ -291,20 +271,26 @@ void mmf::set_last_error(const char* msg) { g_last_error = msg; }
 // wu: one-byte codes of the seven matrices (f, c, g, o, gate, up, down) for
 // the prefill contraction: the caller's mmf_tlinear.codes, or copies made at
 // creation (owned[i]); all null when disabled.
+// ddesc: device copy of the block's decode descriptor (weights, scales,
+// biases, gains), read by the one-launch decode step.
 struct mmf_block {
   mmf_block_weights w;
   int d, I;
   const uint8_t* wu[7];
   uint8_t* owned[7];
+  DecodeLayerDesc* ddesc;
 };
 
-// bar: 256 bytes holding the counter and generation words of the one-launch
-// decode step's grid barrier, zero between launches; calls sharing a state are stream-ordered
-// anyway (h is updated in place), so one pair serves every layer.
+// xbuf: exchange buffers of the one-launch decode step, allocated by the first
+// decode step that needs them: a header of L launch-parity words and one abort
+// word (rounded up to 256 bytes), then decode_xlayer_bytes(B, d, xI) bytes per
+// layer, filled with all-ones bytes. xdt is the dtype of the last decode step.
 struct mmf_state {
   float* h;
-  unsigned* bar;
   int L, B, d;
+  uint8_t* xbuf;
+  size_t xbytes;
+  int xI, xdt;
 };
 
 // ------------------------------------------------------------------ misc
@@ -426,11 +412,7 @@ extern "C" mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B
   int* status = nullptr;
   mmf_status r = device_status_ptr(&status);
   if (r != MMF_OK) return r;
-  MMF_CUDA(timed("mlgru_scan", s,
-                 [&] {
-                   cudaError_t e = reset_mlgru_scan_ws(ws, B, T, d, s);
-                   return e != cudaSuccess ? e : launch_mlgru_scan(pre, dtype, B, T, d, h, o, ws, status, s);
-                 }),
+  MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(pre, dtype, B, T, d, h, o, status, s); }),
            "mlgru_scan");
   return MMF_OK;
 }
@@ -460,21 +442,27 @@ mmf_status check_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_t
 
 // p = SiLU(gate(x)) * up(x); y = down(p) + residual. x is quantised with the
 // gate's RMSNorm gain (gate and up share it), p with the down projection's.
+mmf_status dbg_codes(const mmf_block_debug* dbg, int i, const QAct& qa, int M, int K, cudaStream_t s);
+
 mmf_status run_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tlinear* down, const void* x,
                    const void* residual, void* y, int M, mmf_dtype dt, float eps, void* p, const QAct& qa,
-                   cudaStream_t s, const uint8_t* const* wu = nullptr /* gate, up, down one-byte codes */) {
+                   cudaStream_t s, const uint8_t* const* wu = nullptr /* gate, up, down one-byte codes */,
+                   const mmf_block_debug* dbg = nullptr) {
   const mmf_tlinear* gu[2] = {gate, up};
   TGemmArgs a = gemm_args(gu, 2, qa.q, qa.s, qa.qsum, M, p, gate->N, nullptr, nullptr);
   if (wu) {
     a.wu[0] = wu[0];
     a.wu[1] = wu[1];
   }   // otherwise the layers' own codes (if any), set by gemm_args
-  mmf_status r = quant_gemm(x, gate->gain, eps, qa, a, Epi::kGlu, dt, s, "gate_up", false);
+  mmf_status r = quant_gemm(x, gate->gain, eps, qa, a, Epi::kGlu, dt, s, "gate_up", dbg != nullptr);
+  if (r == MMF_OK) r = dbg_codes(dbg, 2, qa, M, gate->K, s);
   if (r != MMF_OK) return r;
   const mmf_tlinear* dn[1] = {down};
   TGemmArgs b = gemm_args(dn, 1, qa.q, qa.s, qa.qsum, M, y, down->N, residual, nullptr);
   if (wu) b.wu[0] = wu[2];
-  return quant_gemm(p, down->gain, eps, qa, b, Epi::kStore, dt, s, "down", false);
+  r = quant_gemm(p, down->gain, eps, qa, b, Epi::kStore, dt, s, "down", dbg != nullptr);
+  if (r == MMF_OK) r = dbg_codes(dbg, 3, qa, M, down->K, s);
+  return r;
 }
 
 }  // namespace
@@ -532,10 +520,31 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
   b->w = *w;
   b->d = d;
   b->I = I;
+  b->ddesc = nullptr;
   const mmf_tlinear* all[7] = {&w->f, &w->c, &w->g, &w->o, &w->gate, &w->up, &w->down};
   for (int i = 0; i < 7; ++i) {
     b->wu[i] = all[i]->codes;
     b->owned[i] = nullptr;
+  }
+  {   // the decode step's device descriptor of this block
+    DecodeLayerDesc h{};
+    for (int i = 0; i < 7; ++i) {
+      h.w[i] = all[i]->packed;
+      h.gamma[i] = all[i]->gamma;
+      h.bias[i] = all[i]->bias;
+    }
+    h.gain[0] = w->f.gain;
+    h.gain[1] = w->o.gain;
+    h.gain[2] = w->gate.gain;
+    h.gain[3] = w->down.gain;
+    // without it the block's decode steps take the four-contraction path
+    cudaError_t e = cudaMalloc(&b->ddesc, sizeof(DecodeLayerDesc));
+    if (e == cudaSuccess) e = cudaMemcpy(b->ddesc, &h, sizeof(h), cudaMemcpyHostToDevice);
+    if (e != cudaSuccess) {
+      (void)cudaGetLastError();
+      cudaFree(b->ddesc);
+      b->ddesc = nullptr;
+    }
   }
   if (prefill_unpacked_enabled()) {
     // copies for the matrices the caller gave no codes for; they only speed
@@ -582,6 +591,7 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
 extern "C" void mmf_block_destroy(mmf_block* blk) {
   if (!blk) return;
   for (int i = 0; i < 7; ++i) cudaFree(blk->owned[i]);
+  cudaFree(blk->ddesc);
   delete blk;
 }
 
@@ -597,23 +607,19 @@ extern "C" mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_stat
     delete st;
     return fail(MMF_ERR_NOMEM, "mmf_state_create: cudaMalloc(%zu): %s", bytes, cudaGetErrorString(e));
   }
-  e = cudaMalloc(&st->bar, 256);
-  if (e != cudaSuccess) {
-    cudaFree(st->h);
-    delete st;
-    return fail(MMF_ERR_NOMEM, "mmf_state_create: cudaMalloc(256): %s", cudaGetErrorString(e));
-  }
   e = cudaMemset(st->h, 0, bytes);
-  if (e == cudaSuccess) e = cudaMemset(st->bar, 0, 256);
   if (e != cudaSuccess) {
     cudaFree(st->h);
-    cudaFree(st->bar);
     delete st;
     return cuda_fail(e, "mmf_state_create: cudaMemset");
   }
   st->L = L;
   st->B = B;
   st->d = d;
+  st->xbuf = nullptr;
+  st->xbytes = 0;
+  st->xI = 0;
+  st->xdt = -1;
   *out = st;
   return MMF_OK;
 }
@@ -621,19 +627,58 @@ extern "C" mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_stat
 extern "C" void mmf_state_destroy(mmf_state* st) {
   if (!st) return;
   cudaFree(st->h);
-  cudaFree(st->bar);
+  cudaFree(st->xbuf);
   delete st;
 }
+
+namespace {
+
+size_t decode_header_bytes(int L) { return round_up(sizeof(uint32_t) * ((size_t)L + 1), 256); }
+
+// Launch parities all zero, abort word zero, every exchange element all-ones.
+cudaError_t reset_decode_buffers(mmf_state* st, cudaStream_t s) {
+  if (st->xbuf == nullptr) return cudaSuccess;
+  const size_t hb = decode_header_bytes(st->L);
+  cudaError_t e = cudaMemsetAsync(st->xbuf, 0, hb, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(st->xbuf + hb, 0xff, st->xbytes - hb, s);
+  return e;
+}
+
+// Exchange buffers for decode steps of blocks with inner size I in dtype dt:
+// allocated (cudaMalloc) the first time and whenever a larger I comes, and
+// reset when the dtype changes.
+mmf_status ensure_decode_buffers(mmf_state* st, int I, mmf_dtype dt, cudaStream_t s) {
+  if (st->xbuf == nullptr || I > st->xI) {
+    const size_t bytes = decode_header_bytes(st->L) + (size_t)st->L * decode_xlayer_bytes(st->B, st->d, I);
+    if (st->xbuf != nullptr) {
+      MMF_CUDA(cudaStreamSynchronize(s), "decode buffers: synchronise");
+      cudaFree(st->xbuf);
+      st->xbuf = nullptr;
+    }
+    uint8_t* p = nullptr;
+    cudaError_t e = cudaMalloc(&p, bytes);
+    if (e != cudaSuccess) return fail(MMF_ERR_NOMEM, "decode buffers: cudaMalloc(%zu): %s", bytes, cudaGetErrorString(e));
+    st->xbuf = p;
+    st->xbytes = bytes;
+    st->xI = I;
+    st->xdt = -1;
+  }
+  if (st->xdt != (int)dt) {
+    MMF_CUDA(reset_decode_buffers(st, s), "decode buffers: reset");
+    st->xdt = (int)dt;
+  }
+  return MMF_OK;
+}
+
+}  // namespace
 
 extern "C" mmf_status mmf_state_reset(mmf_state* st, void* stream) {
   if (!st) return fail(MMF_ERR_INVALID_ARG, "mmf_state_reset: null state");
   MMF_CUDA(cudaMemsetAsync(st->h, 0, sizeof(float) * (size_t)st->L * st->B * st->d, as_stream(stream)),
            "mmf_state_reset");
-  MMF_CUDA(cudaMemsetAsync(st->bar, 0, 256, as_stream(stream)), "mmf_state_reset: barrier words");
+  MMF_CUDA(reset_decode_buffers(st, as_stream(stream)), "mmf_state_reset: decode buffers");
   return MMF_OK;
 }
-
-extern "C" uint32_t* mmf_state_barrier(mmf_state* st) { return st ? st->bar : nullptr; }
 
 extern "C" float* mmf_state_layer(mmf_state* st, int32_t layer) {
   if (!st || layer < 0 || layer >= st->L) return nullptr;
@@ -668,7 +713,6 @@ struct BlockWs {
   void* p;     // [M, I] GLU product
   void* ping;  // [M, d] stack intermediates
   void* pong;
-  void* scan;  // scan scratch
   size_t bytes;
 };
 
@@ -684,112 +728,118 @@ BlockWs carve_block(void* base, int B, int T, int d, int I, mmf_dtype dt) {
   w.p = c.take<char>((size_t)M * I * e);
   w.ping = c.take<char>((size_t)M * d * e);
   w.pong = c.take<char>((size_t)M * d * e);
-  w.scan = c.take<char>(std::max(mlgru_scan_ws_bytes(B, T, d), tgemm_tc_mlgru_ws_bytes(B, T, d)));
   w.bytes = c.off + 256;
   return w;
 }
 
-// With MMF_DECODE_BLOCK_KERNEL=1 a decode step of up to 8 tokens runs as one
-// launch per block (four stages, grid barriers between them) instead of four
-// contractions; both compute the same values. Off by default: on one B200 a
-// 2.7B-shaped block step took 41.5 us that way against 29.1 us for the
-// separate kernels (each stage's row quantisation, contraction and epilogue
-// stay serial, and a grid barrier costs about as much as a kernel boundary
-// with programmatic dependent launch).
-bool decode_block_enabled() {
-  const char* e = getenv("MMF_DECODE_BLOCK_KERNEL");
-  return e != nullptr && strcmp(e, "1") == 0;
+// Decode steps (T = 1) of up to 8 sequences run as one launch over all the
+// layers of the call (decode_step.cu) unless MMF_DECODE_STEP_KERNEL=0, which
+// selects the four contractions per block instead (the same arithmetic; the
+// codes can differ only where the fp64 sum of squares rounds differently).
+bool decode_step_enabled() {
+  const char* e = getenv("MMF_DECODE_STEP_KERNEL");
+  return e == nullptr || strcmp(e, "0") != 0;
 }
 
-DecodeStage decode_stage(const mmf_tlinear* const* segs, int nseg) {
-  DecodeStage st{};
-  for (int i = 0; i < 3; ++i) {
-    const mmf_tlinear* l = segs[i < nseg ? i : 0];
-    st.w[i] = l->packed;
-    st.gamma[i] = l->gamma;
-    st.bias[i] = l->bias;
+
+bool decode_step_usable(const mmf_block* const* blocks, int L, int B, mmf_dtype dt) {
+  if (!decode_step_enabled()) return false;
+  for (int l = 0; l < L; ++l)
+    if (blocks[l]->I != blocks[0]->I || blocks[l]->d != blocks[0]->d || blocks[l]->ddesc == nullptr) return false;
+  return decode_step_supported(B, blocks[0]->d, blocks[0]->I, std::min(L, kDecodeMaxLayers), dt);
+}
+
+// One decode step of blocks[0 .. L) (state layers layer0 ..), in launches of
+// at most kDecodeMaxLayers layers; x -> y, `mid` [B, d] carries the output of
+// one launch to the next.
+mmf_status run_decode_step(const mmf_block* const* blocks, int L, int layer0, mmf_state* st, const void* x, void* y,
+                           void* mid, int B, mmf_dtype dt, float eps, cudaStream_t s, const mmf_block_debug* dbg) {
+  mmf_status r = ensure_decode_buffers(st, blocks[0]->I, dt, s);
+  if (r != MMF_OK) return r;
+  int* status = nullptr;
+  if ((r = device_status_ptr(&status)) != MMF_OK) return r;
+  const size_t hb = decode_header_bytes(st->L);
+  for (int l0 = 0; l0 < L; l0 += kDecodeMaxLayers) {
+    const int n = std::min(kDecodeMaxLayers, L - l0);
+    DecodeStepArgs a{};
+    for (int l = 0; l < n; ++l) a.layer[l] = blocks[l0 + l]->ddesc;
+    a.x = l0 == 0 ? x : mid;
+    a.y = l0 + n == L ? y : mid;
+    a.h = st->h;
+    a.xbuf = st->xbuf + hb;
+    a.parity = reinterpret_cast<unsigned*>(st->xbuf);
+    a.abort_word = reinterpret_cast<int*>(st->xbuf) + st->L;
+    a.status = status;
+    if (dbg != nullptr && n == 1) a.dbg = *dbg;
+    a.wait_cycles = wait_limit_cycles();
+    a.eps = eps;
+    a.L = n;
+    a.layer0 = layer0 + l0;
+    a.M = B;
+    a.d = blocks[0]->d;
+    a.I = blocks[0]->I;
+    a.xI = st->xI;
+    a.skip_cta = test_hook("MMF_DECODE_SKIP_CTA");   // test: CTA b never publishes its first stage
+    MMF_CUDA(timed("decode_step", s, [&] { return launch_decode_step(a, dt, s); }), "decode step");
   }
-  st.gain = segs[0]->gain;
-  st.nseg = nseg;
-  st.N = segs[0]->N;
-  st.K = segs[0]->K;
-  return st;
+  return MMF_OK;
 }
 
-mmf_status block_forward_impl(const mmf_block* blk, float* h, unsigned* bar, const void* x, void* y, int B, int T,
-                              mmf_dtype dt, float eps, const BlockWs& w, cudaStream_t s) {
+// Stream-ordered copy of the quantised input of stage i (codes, scales) into the debug outputs.
+mmf_status dbg_codes(const mmf_block_debug* dbg, int i, const QAct& qa, int M, int K, cudaStream_t s) {
+  if (dbg == nullptr) return MMF_OK;
+  if (dbg->q[i]) MMF_CUDA(cudaMemcpyAsync(dbg->q[i], qa.q, (size_t)M * K, cudaMemcpyDeviceToDevice, s), "dbg q");
+  if (dbg->scale[i])
+    MMF_CUDA(cudaMemcpyAsync(dbg->scale[i], qa.s, sizeof(float) * M, cudaMemcpyDeviceToDevice, s), "dbg scale");
+  return MMF_OK;
+}
+
+mmf_status dbg_copy(void* dst, const void* src, size_t bytes, cudaStream_t s) {
+  if (dst == nullptr) return MMF_OK;
+  MMF_CUDA(cudaMemcpyAsync(dst, src, bytes, cudaMemcpyDeviceToDevice, s), "dbg copy");
+  return MMF_OK;
+}
+
+mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, void* y, int B, int T, mmf_dtype dt,
+                              float eps, const BlockWs& w, cudaStream_t s, const mmf_block_debug* dbg = nullptr) {
   const int M = B * T, d = blk->d;
   const mmf_block_weights& W = blk->w;
   const mmf_tlinear* fcg[3] = {&W.f, &W.c, &W.g};
-  if (T == 1 && decode_block_enabled()) {
-    const mmf_tlinear* o1[1] = {&W.o};
-    const mmf_tlinear* gu[2] = {&W.gate, &W.up};
-    const mmf_tlinear* dn[1] = {&W.down};
-    DecodeBlockArgs a{};
-    a.st[0] = decode_stage(fcg, 3);
-    a.st[1] = decode_stage(o1, 1);
-    a.st[2] = decode_stage(gu, 2);
-    a.st[3] = decode_stage(dn, 1);
-    a.x = x;
-    a.og = w.og;
-    a.y1 = w.y1;
-    a.p = w.p;
-    a.y = y;
-    a.h = h;
-    a.M = M;
-    a.d = d;
-    a.I = blk->I;
-    a.eps = eps;
-    a.bar = bar;
-    a.status = status_word();
-    if (a.status != nullptr && decode_block_supported(a, dt)) {
-      MMF_CUDA(timed("decode_block", s, [&] { return launch_decode_block(a, dt, s); }), "decode block");
-      return MMF_OK;
-    }
-  }
-  TGemmArgs tm = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, nullptr);
-  for (int i = 0; i < 3; ++i) tm.wu[i] = blk->wu[i];
-  const bool fused_mixer = T > 1 && fused_mlgru_enabled() && gemm_uses_tc(tm, Epi::kStore) &&
-                           tgemm_tc_mlgru_supported(tm, T, d);
-  // prefill: the scan's scratch (all-ones before the scan) is filled by the
-  // quantiser of x as side work, so no memset sits between the kernels
-  const size_t scan_fill = fused_mixer ? tgemm_tc_mlgru_ws_bytes(B, T, d) : (T > 1 ? mlgru_scan_ws_bytes(B, T, d) : 0);
+  const bool want = dbg != nullptr;
   // token mixer: x quantised once for f, c, g (shared gain)
-  if (fused_mixer) {
-    MMF_CUDA(timed("rmsnorm_quant", s,
-                   [&] {
-                     return launch_rmsnorm_quant(x, dt, M, d, W.f.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, status_word(),
-                                                 s, w.scan, scan_fill);
-                   }),
-             "block quant x");
-    int* status = nullptr;
-    mmf_status r = device_status_ptr(&status);
-    if (r != MMF_OK) return r;
-    MMF_CUDA(timed("tgemm_tc_mlgru", s, [&] { return launch_tgemm_tc_mlgru(tm, dt, T, d, h, w.scan, status, s); }),
-             "block fcg+mlgru");
-  } else if (T == 1) {
+  if (T == 1) {
     // decode: projections and one recurrence step in one launch; h updated in place
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, h);
-    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kScanStep, dt, s, "fcg_step", false);
+    if (want) a.pre_out = dbg->pre;
+    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kScanStep, dt, s, "fcg_step", want);
+    if (r == MMF_OK) r = dbg_codes(dbg, 0, w.qa, M, d, s);
     if (r != MMF_OK) return r;
   } else {
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.pre, 3 * d, nullptr, nullptr);
     for (int i = 0; i < 3; ++i) a.wu[i] = blk->wu[i];
-    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", false, w.scan, scan_fill);
+    mmf_status r = quant_gemm(x, W.f.gain, eps, w.qa, a, Epi::kStore, dt, s, "fcg", want);
+    if (r == MMF_OK) r = dbg_codes(dbg, 0, w.qa, M, d, s);
+    if (r == MMF_OK && want) r = dbg_copy(dbg->pre, w.pre, (size_t)M * 3 * d * elem_bytes(dt), s);
     if (r != MMF_OK) return r;
     int* status = nullptr;
     r = device_status_ptr(&status);
     if (r != MMF_OK) return r;
-    MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, w.scan, status, s); }),
+    MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, status, s); }),
              "block scan");
   }
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
   b.wu[0] = blk->wu[3];
-  mmf_status r = quant_gemm(w.og, W.o.gain, eps, w.qa, b, Epi::kStore, dt, s, "o", false);
+  mmf_status r = quant_gemm(w.og, W.o.gain, eps, w.qa, b, Epi::kStore, dt, s, "o", want);
+  if (r == MMF_OK) r = dbg_codes(dbg, 1, w.qa, M, d, s);
   if (r != MMF_OK) return r;
   // channel mixer
-  return run_glu(&W.gate, &W.up, &W.down, w.y1, w.y1, y, M, dt, eps, w.p, w.qa, s, blk->wu + 4);
+  r = run_glu(&W.gate, &W.up, &W.down, w.y1, w.y1, y, M, dt, eps, w.p, w.qa, s, blk->wu + 4, dbg);
+  if (r != MMF_OK || !want) return r;
+  const size_t e = elem_bytes(dt);
+  if ((r = dbg_copy(dbg->og, w.og, (size_t)M * d * e, s)) != MMF_OK) return r;
+  if ((r = dbg_copy(dbg->y1, w.y1, (size_t)M * d * e, s)) != MMF_OK) return r;
+  return dbg_copy(dbg->p, w.p, (size_t)M * blk->I * e, s);
 }
 
 mmf_status check_forward_args(const mmf_block* blk, mmf_state* st, const void* x, void* y, int B, int T,
@@ -828,7 +878,35 @@ extern "C" mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf
   BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype);
   if (ws_bytes < mmf_block_ws_size(blk, B, T))
     return fail(MMF_ERR_WORKSPACE, "mmf_block_forward: ws_bytes=%zu < %zu", ws_bytes, mmf_block_ws_size(blk, B, T));
-  return block_forward_impl(blk, mmf_state_layer(st, layer), st->bar, x, y, B, T, dtype, eps, w, as_stream(stream));
+  if (T == 1 && decode_step_usable(&blk, 1, B, dtype))
+    return run_decode_step(&blk, 1, layer, st, x, y, nullptr, B, dtype, eps, as_stream(stream), nullptr);
+  return block_forward_impl(blk, mmf_state_layer(st, layer), x, y, B, T, dtype, eps, w, as_stream(stream));
+}
+
+extern "C" mmf_status mmf_block_forward_debug(const mmf_block* blk, int32_t layer, mmf_state* st, const void* x,
+                                              void* y, int32_t B, int32_t T, mmf_dtype dtype, float eps, void* ws,
+                                              size_t ws_bytes, void* stream, const mmf_block_debug* dbg) {
+  if (dbg != nullptr) {
+    const void* ptrs[12] = {dbg->pre, dbg->og, dbg->y1, dbg->p};
+    for (int i = 0; i < 4; ++i) {
+      ptrs[4 + i] = dbg->q[i];
+      ptrs[8 + i] = dbg->scale[i];
+    }
+    for (const void* p : ptrs)
+      if (p != nullptr && !aligned16(p)) return fail(MMF_ERR_MISALIGNED, "mmf_block_forward_debug: debug buffer");
+  }
+  mmf_status r = check_forward_args(blk, st, x, y, B, T, dtype, eps, ws, "mmf_block_forward_debug");
+  if (r != MMF_OK) return r;
+  if (layer < 0 || layer >= st->L)
+    return fail(MMF_ERR_INVALID_ARG, "mmf_block_forward_debug: layer %d of %d", layer, st->L);
+  if (T == 0) return MMF_OK;
+  BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype);
+  if (ws_bytes < mmf_block_ws_size(blk, B, T))
+    return fail(MMF_ERR_WORKSPACE, "mmf_block_forward_debug: ws_bytes=%zu < %zu", ws_bytes,
+                mmf_block_ws_size(blk, B, T));
+  if (T == 1 && decode_step_usable(&blk, 1, B, dtype))
+    return run_decode_step(&blk, 1, layer, st, x, y, nullptr, B, dtype, eps, as_stream(stream), dbg);
+  return block_forward_impl(blk, mmf_state_layer(st, layer), x, y, B, T, dtype, eps, w, as_stream(stream), dbg);
 }
 
 extern "C" mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t L, mmf_state* st, const void* x,
@@ -847,11 +925,15 @@ extern "C" mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t 
   if (T == 0) return MMF_OK;
   if (ws_bytes < need) return fail(MMF_ERR_WORKSPACE, "mmf_stack_forward: ws_bytes=%zu < %zu", ws_bytes, need);
   cudaStream_t s = as_stream(stream);
+  if (T == 1 && decode_step_usable(blocks, L, B, dtype)) {
+    BlockWs w = carve_block(ws, B, T, blocks[0]->d, blocks[0]->I, dtype);
+    return run_decode_step(blocks, L, 0, st, x, y, w.ping, B, dtype, eps, s, nullptr);
+  }
   const void* cur = x;
   for (int l = 0; l < L; ++l) {
     BlockWs w = carve_block(ws, B, T, blocks[l]->d, blocks[l]->I, dtype);
     void* dst = (l == L - 1) ? y : ((l % 2 == 0) ? w.ping : w.pong);
-    mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), st->bar, cur, dst, B, T, dtype, eps, w, s);
+    mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), cur, dst, B, T, dtype, eps, w, s);
     if (r != MMF_OK) return r;
     cur = dst;
   }

@@ -1,0 +1,667 @@
+// One decode step (T = 1) of a stack of MatMul-free blocks in one kernel
+// launch (sm_100a).
+//
+// "MatMul-free language models" (DataCamp blog), sections "Replacing MatMul
+// with ternary operations" and "Core components: MLGRU and GLU"; the hysenlabs
+// review, sections "FusedBitLinear" and "HGRN attention". A layer is four
+// FusedBitLinear stages, each of which normalises and quantises its whole
+// input rows before it accumulates against ternary weights:
+//   S0  x  -> f|c|g (3 x d rows) -> MLGRU step: h = f h + (1 - f) c, o' = g h
+//   S1  o' -> o (d rows) + x                            -> y1
+//   S2  y1 -> gate|up (2 x I rows) -> SiLU(gate) * up   -> p
+//   S3  p  -> down (d rows) + y1                        -> x of the next layer (y after the last)
+//
+// Why one launch: a decode step is a chain of 4 L dependent stages. Each
+// stage needs every element of the previous stage's output (the RMS and the
+// absmax scale are reductions over the whole row), while the weights it
+// streams (a few MB) take HBM about a microsecond. The step's time is the
+// chain's latency, so the launch is built around it:
+//   * Stage outputs travel through buffers owned by the recurrent state. Their
+//     elements are reset to all-ones bits (a NaN pattern that no stage ever
+//     stores) one launch ahead, and a consumer re-reads its input rows until no
+//     element holds that pattern: the data are their own ready flags (each
+//     element is written once, by one aligned store). There is no grid
+//     barrier, no fence and no flag round trip. Two sets of buffers alternate
+//     by a per-layer launch parity kept in the state: a launch writes set P
+//     and resets set 1 - P for the next launch.
+//   * A CTA owns the 16-row tiles b, b + G, ... of every stage's matrices. Its
+//     weight slices stream into a shared-memory ring by 1-D bulk copies
+//     (cp.async.bulk, one per packed row) several stages ahead, with L2
+//     prefetches further ahead. Weights do not depend on activations, so the
+//     HBM stream runs ahead of the chain.
+//   * Every CTA quantises the whole input rows itself with all 16 warps: the
+//     rows go to registers, the fp64 sum of squares and the max are reduced
+//     over the block in a fixed order (every CTA gets the same scale), and the
+//     codes go to shared memory with the same fp32 steps as the standalone
+//     quantiser. The contraction is mma.sync m16n8k32 (stored codes w + 1 as
+//     u8 against s8 activations; the row's code sum is subtracted after).
+// Launch: cooperative, one CTA of 512 threads per SM, so every CTA is resident
+// and every wait ends. Each wait is also bounded: on timeout a CTA records
+// status code 5 (input rows) or 6 (weight slice), raises the state's abort word
+// so that the other CTAs leave as well, lets its copies land and returns. The
+// state must then be reset before its next decode step.
+#include "kernels.cuh"
+#include "quant_row.cuh"
+#include "tma.cuh"
+
+namespace mmf {
+
+namespace {
+
+constexpr int kThreads = 512;
+constexpr int kWarps = kThreads / 32;
+constexpr int kVmax = 16;            // 16-byte input vectors per thread and stage
+constexpr int kPrefetchAhead = 6;    // L2 prefetch distance beyond the ring, in stages
+constexpr uint32_t kLow2 = 0x03030303u;
+
+struct StageGeom {
+  int nseg, N, K, mat0, gain;
+};
+__host__ __device__ __forceinline__ StageGeom stage_geom(int s, int d, int I) {
+  if (s == 0) return StageGeom{3, d, d, 0, 0};
+  if (s == 1) return StageGeom{1, d, d, 3, 1};
+  if (s == 2) return StageGeom{2, I, d, 4, 2};
+  return StageGeom{1, d, I, 6, 3};
+}
+// 16-row tiles of an N-row matrix that CTA b of G owns (tiles b, b + G, ...).
+__host__ __device__ __forceinline__ int tiles_of(int N, int b, int G) {
+  const int nt = N / 16;
+  return b < nt ? (nt - b + G - 1) / G : 0;
+}
+
+// Byte offset of region r (0: o', 1: y1, 2: p, 3: next layer's x) inside one
+// buffer set; 4 bytes per element whatever the dtype, so regions never move.
+__host__ __device__ __forceinline__ size_t region_off(int r, int M, int d, int I) {
+  const size_t md = (size_t)M * d * 4;
+  return r == 0 ? 0 : (r == 1 ? md : (r == 2 ? 2 * md : 2 * md + (size_t)M * I * 4));
+}
+
+// Regions are laid out for the inner size the buffers were allocated for (xI >= I).
+__device__ __forceinline__ uint8_t* xregion(const DecodeStepArgs& a, int l, int set, int r) {
+  return a.xbuf + (size_t)(a.layer0 + l) * a.xlayer_bytes + (size_t)set * a.xset_bytes + region_off(r, a.M, a.d, a.xI);
+}
+
+__device__ __forceinline__ void mma_u8s8(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};\n"
+      : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t u4get(const uint4& v, int i) {
+  return i == 0 ? v.x : (i == 1 ? v.y : (i == 2 ? v.z : v.w));
+}
+
+__device__ __forceinline__ uint4 ld_relaxed_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.relaxed.gpu.global.v4.b32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p)
+               : "memory");
+  return r;
+}
+__device__ __forceinline__ int ld_relaxed_i32(const int* p) {
+  int v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// One element of a stage output: published with a relaxed store (read by
+// other CTAs' relaxed loads), and the same position of the other buffer set
+// reset to all-ones bits for the next launch.
+__device__ __forceinline__ void publish(bf16* cur, bf16* next, float v) {
+  const bf16 h = from_f32<bf16>(v);
+  const unsigned short u = *reinterpret_cast<const unsigned short*>(&h);
+  asm volatile("st.relaxed.gpu.global.b16 [%0], %1;" ::"l"(cur), "h"(u) : "memory");
+  *reinterpret_cast<unsigned short*>(next) = 0xffffu;
+}
+__device__ __forceinline__ void publish(float* cur, float* next, float v) {
+  asm volatile("st.relaxed.gpu.global.b32 [%0], %1;" ::"l"(cur), "r"(__float_as_uint(v)) : "memory");
+  *reinterpret_cast<uint32_t*>(next) = 0xffffffffu;
+}
+
+// Whether a 16-byte vector of stage output still holds an unwritten element.
+template <typename T> __device__ __forceinline__ bool has_unset(const uint4& v);
+template <> __device__ __forceinline__ bool has_unset<bf16>(const uint4& v) {
+  return (__vcmpeq2(v.x, 0xffffffffu) | __vcmpeq2(v.y, 0xffffffffu) | __vcmpeq2(v.z, 0xffffffffu) |
+          __vcmpeq2(v.w, 0xffffffffu)) != 0u;
+}
+template <> __device__ __forceinline__ bool has_unset<float>(const uint4& v) {
+  return v.x == ~0u || v.y == ~0u || v.z == ~0u || v.w == ~0u;
+}
+
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
+}
+
+struct Smem {
+  int red[kDecodeTiles][3][16][8];      // per tile, segment, row, token: exact int32 partial sums
+  double red_d[kWarps];
+  uint32_t red_u[kWarps];
+  int red_i[kWarps];
+  float scale[8], rinv[8];
+  int qsum[8];
+  float res_x[kDecodeTiles * 16 * 8];   // block input x of this CTA's d-channels (S1 residual)
+  float res_y1[kDecodeTiles * 16 * 8];  // y1 of this CTA's d-channels (S3 residual)
+  float gam[kDecodeMaxLayers][7];
+  unsigned par[kDecodeMaxLayers];
+  uint64_t slot_bar[kDecodeMaxSlots];
+};
+
+// Warp 0: start the bulk copies of stage q's weight slice into its ring slot.
+__device__ void fill_slot(const DecodeStepArgs& a, const DecodeLayerDesc* desc, uint8_t* slots, Smem& sm, int q,
+                          int lane) {
+  const int l = q >> 2, s = q & 3;
+  const StageGeom g = stage_geom(s, a.d, a.I);
+  const int ntl = tiles_of(g.N, blockIdx.x, gridDim.x);
+  const int rowb = g.K / 4, pitch = rowb + 64;
+  const int slot = q % a.nslot;
+  uint8_t* dst0 = slots + (size_t)slot * a.slot_bytes;
+  const int ncopy = ntl * g.nseg * 16;
+  if (lane == 0) {
+    if (ncopy > 0) mbar_arrive_expect_tx(&sm.slot_bar[slot], (uint32_t)ncopy * rowb);
+    else mbar_arrive(&sm.slot_bar[slot]);
+  }
+  __syncwarp();
+  for (int i = lane; i < ncopy; i += 32) {
+    const int ti = i / (g.nseg * 16), rem = i - ti * g.nseg * 16;
+    const int r = rem >> 4, row = rem & 15;
+    const int n = (blockIdx.x + ti * gridDim.x) * 16 + row;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(desc[l].w[g.mat0 + r]) + (size_t)n * rowb;
+    bulk_g2s(dst0 + (size_t)((ti * g.nseg + r) * 16 + row) * pitch, src, (uint32_t)rowb, &sm.slot_bar[slot]);
+  }
+}
+
+// Warp 0: prefetch stage q's weight slice into L2.
+__device__ void prefetch_stage(const DecodeStepArgs& a, const DecodeLayerDesc* desc, int q, int lane) {
+  const int l = q >> 2, s = q & 3;
+  const StageGeom g = stage_geom(s, a.d, a.I);
+  const int ntl = tiles_of(g.N, blockIdx.x, gridDim.x);
+  const int rowb = g.K / 4;
+  for (int i = lane; i < ntl * g.nseg; i += 32) {
+    const int ti = i / g.nseg, r = i - ti * g.nseg;
+    const int t = blockIdx.x + ti * gridDim.x;
+    prefetch_l2(reinterpret_cast<const uint8_t*>(desc[l].w[g.mat0 + r]) + (size_t)t * 16 * rowb, (uint32_t)(16 * rowb));
+  }
+}
+
+// Accumulate this CTA's tiles of one stage into red[ti][r][row][token].
+template <int R>
+__device__ __forceinline__ void stage_mma(const uint4* slot, const int8_t* qs, int qpitch, int M, int K, int ntl,
+                                          int (*red)[3][16][8]) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int g = lane >> 2, t = lane & 3;
+  const int wpr = K / 16, nkseg = ceil_div(K, 256);
+  const int pitch4 = K / 64 + 4;
+  for (int item = warp; item < ntl * nkseg; item += kWarps) {
+    const int ti = item / nkseg, seg = item - ti * nkseg;
+    const int w0 = seg * 16 + 4 * t;   // first packed word of this lane
+    const bool in = w0 < wpr;          // wpr % 4 == 0: a 16-byte group is all in or all out
+    uint4 wa[R], wb[R];
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      const uint4* base = slot + (size_t)((ti * R + r) * 16) * pitch4 + (w0 >> 2);
+      wa[r] = in ? base[(size_t)g * pitch4] : make_uint4(0u, 0u, 0u, 0u);
+      wb[r] = in ? base[(size_t)(g + 8) * pitch4] : make_uint4(0u, 0u, 0u, 0u);
+    }
+    uint4 act[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const bool ok = (g < M) && (w0 + u < wpr);
+      act[u] = ok ? *reinterpret_cast<const uint4*>(qs + (size_t)g * qpitch + (w0 + u) * 16)
+                  : make_uint4(0u, 0u, 0u, 0u);
+    }
+    int acc[R][4];
+#pragma unroll
+    for (int r = 0; r < R; ++r)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[r][e] = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int u = i >> 1, sub = (i & 1) * 2;
+      const uint32_t b0 = u4get(act[u], sub), b1 = u4get(act[u], sub + 1);
+#pragma unroll
+      for (int r = 0; r < R; ++r) {
+        const uint32_t wg = u4get(wa[r], u), wg8 = u4get(wb[r], u);
+        mma_u8s8(acc[r], (wg >> (2 * sub)) & kLow2, (wg8 >> (2 * sub)) & kLow2, (wg >> (2 * sub + 2)) & kLow2,
+                 (wg8 >> (2 * sub + 2)) & kLow2, b0, b1);
+      }
+    }
+#pragma unroll
+    for (int r = 0; r < R; ++r) {
+      atomicAdd(&red[ti][r][g][2 * t], acc[r][0]);
+      atomicAdd(&red[ti][r][g][2 * t + 1], acc[r][1]);
+      atomicAdd(&red[ti][r][g + 8][2 * t], acc[r][2]);
+      atomicAdd(&red[ti][r][g + 8][2 * t + 1], acc[r][3]);
+    }
+  }
+}
+
+// Give up: record `code`, raise the abort word, let this CTA's weight copies
+// in flight land (bounded), and return.
+__device__ void give_up(const DecodeStepArgs& a, Smem& sm, int code, int q_first, int q_end) {
+  if (threadIdx.x == 0) {
+    if (a.status) atomicExch(a.status, code);
+    atomicExch(a.abort_word, 1);
+    for (int q = q_first; q < q_end; ++q) {
+      const long long t0 = clock64();
+      while (!mbar_try_wait(&sm.slot_bar[q % a.nslot], (uint32_t)(q / a.nslot) & 1u) &&
+             clock64() - t0 < a.wait_cycles) {
+      }
+    }
+  }
+  __syncthreads();
+}
+
+template <typename T, int MPAD>
+__global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_constant__ DecodeStepArgs a) {
+  extern __shared__ __align__(128) uint8_t dsm[];
+  __shared__ Smem sm;
+  using V = Vec<T>;
+  constexpr int E = V::E;
+  constexpr int kTpr = kThreads / MPAD;     // threads per token row in the quantisation
+  DecodeLayerDesc* desc = reinterpret_cast<DecodeLayerDesc*>(dsm);
+  int8_t* codes = reinterpret_cast<int8_t*>(dsm + a.desc_bytes);
+  uint8_t* slots = dsm + a.desc_bytes + a.codes_bytes;
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int b = blockIdx.x, G = gridDim.x;
+  const int M = a.M, d = a.d, I = a.I, L = a.L;
+  const int nq = 4 * L;
+  const int qpitch = a.qpitch;
+
+  if (tid == 0) {
+    for (int s = 0; s < a.nslot; ++s) mbar_init(&sm.slot_bar[s], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  {   // layer descriptors into shared memory (written before this launch)
+    constexpr int kWords = sizeof(DecodeLayerDesc) / 8;
+    for (int i = tid; i < L * kWords; i += kThreads)
+      reinterpret_cast<uint64_t*>(desc)[i] = reinterpret_cast<const uint64_t*>(a.layer[i / kWords])[i % kWords];
+  }
+  __syncthreads();
+  for (int i = tid; i < L * 7; i += kThreads) sm.gam[i / 7][i % 7] = *desc[i / 7].gamma[i % 7];
+  // the weight stream does not depend on the previous kernel: start it first
+  int q_issued = 0;   // stages whose ring fill has been issued
+  if (warp == 0) {
+    for (int q = 0; q < a.nslot && q < nq; ++q) fill_slot(a, desc, slots, sm, q, lane);
+    for (int q = a.nslot; q < a.nslot + kPrefetchAhead && q < nq; ++q) prefetch_stage(a, desc, q, lane);
+  }
+  q_issued = a.nslot < nq ? a.nslot : nq;
+  pdl_wait();
+  if (tid < L) sm.par[tid] = a.parity[a.layer0 + tid] & 1u;
+  __syncthreads();
+
+  const int m_row = tid / kTpr, lt = tid - m_row * kTpr;   // quantisation: this thread's token row
+  const bool row_ok = m_row < M;
+
+  for (int q = 0; q < nq; ++q) {
+    const int l = q >> 2, s = q & 3;
+    const StageGeom g = stage_geom(s, d, I);
+    const DecodeLayerDesc& D = desc[l];
+    const int ntl = tiles_of(g.N, b, G);
+    const int par = (int)sm.par[l];
+    const int K = g.K, N = g.N;
+    for (int i = tid; i < kDecodeTiles * 3 * 16 * 8; i += kThreads) (&sm.red[0][0][0][0])[i] = 0;
+
+    // ---------------------------------------------------- epilogue operands that need no input row
+    const int nout = ntl * 16 * M;
+    const bool has_out = tid < nout;
+    const int e_ti = tid / (16 * M), e_rem = tid - e_ti * 16 * M;
+    const int e_m = e_rem >> 4, e_row = e_rem & 15;
+    const int e_n = (b + e_ti * G) * 16 + e_row;
+    float* hp = a.h + ((size_t)(a.layer0 + l) * M + e_m) * d + e_n;
+    float hval = 0.0f, bias[3] = {0.0f, 0.0f, 0.0f};
+    if (has_out) {
+      if (s == 0) hval = *hp;
+      for (int r = 0; r < g.nseg; ++r)
+        if (D.bias[g.mat0 + r] != nullptr) bias[r] = D.bias[g.mat0 + r][e_n];
+    }
+
+    // ---------------------------------------------------- input rows -> registers
+    const uint8_t* in;
+    bool poll = true;
+    if (s == 0) {
+      if (l == 0) {
+        in = static_cast<const uint8_t*>(a.x);
+        poll = false;
+      } else {
+        in = xregion(a, l - 1, (int)sm.par[l - 1], 3);
+      }
+    } else {
+      in = xregion(a, l, par, s - 1);
+    }
+    const int nvec = K * (int)sizeof(T) / 16;
+    const uint8_t* src = in + (size_t)(row_ok ? m_row : 0) * K * sizeof(T);
+    uint4 raw[kVmax];
+    uint32_t pend = 0;
+#pragma unroll
+    for (int j = 0; j < kVmax; ++j) {
+      raw[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (row_ok && lt + kTpr * j < nvec) pend |= 1u << j;
+    }
+    const uint32_t have = pend;
+    bool failed = false;
+    if (!poll) {
+#pragma unroll
+      for (int j = 0; j < kVmax; ++j)
+        if (have & (1u << j)) raw[j] = __ldg(reinterpret_cast<const uint4*>(src) + lt + kTpr * j);
+    } else {
+      long long t0 = 0;
+      while (pend != 0u) {
+#pragma unroll
+        for (int j = 0; j < kVmax; ++j)
+          if (pend & (1u << j)) {
+            raw[j] = ld_relaxed_v4(src + (size_t)(lt + kTpr * j) * 16);
+            if (!has_unset<T>(raw[j])) pend &= ~(1u << j);
+          }
+        if (pend == 0u) break;
+        const long long now = clock64();
+        if (t0 == 0) t0 = now;
+        else if (now - t0 > a.wait_cycles || ld_relaxed_i32(a.abort_word) != 0) {
+          failed = true;
+          break;
+        }
+      }
+    }
+    if (__syncthreads_or(failed)) {
+      give_up(a, sm, 5, q, q_issued);
+      return;
+    }
+
+    // ---------------------------------------------------- RMSNorm + absmax int8 codes, whole block
+    {
+      double ss = 0.0;
+      uint32_t am = 0;
+#pragma unroll
+      for (int j = 0; j < kVmax; ++j)
+        if (have & (1u << j)) {
+#pragma unroll
+          for (int i = 0; i < E; ++i) {
+            const uint32_t mg = V::mag(raw[j], i);
+            am = max(am, mg);
+            const double xd = magbits_to_f64(mg);
+            ss = fma(xd, xd, ss);
+          }
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      am = __reduce_max_sync(0xffffffffu, am);
+      if (lane == 0) {
+        sm.red_d[warp] = ss;
+        sm.red_u[warp] = am;
+      }
+    }
+    __syncthreads();
+    const float* gain = D.gain[g.gain];
+    if (tid < M) {   // per row, warps in order: the same sum in every CTA
+      constexpr int wpr = kTpr / 32;
+      double t = 0.0;
+      uint32_t mx = 0;
+      for (int w = tid * wpr; w < (tid + 1) * wpr; ++w) {
+        t += sm.red_d[w];
+        mx = max(mx, sm.red_u[w]);
+      }
+      const float ms = (float)(t / (double)K);
+      const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, a.eps)));
+      sm.rinv[tid] = rinv;
+      if (gain == nullptr)   // rounding is monotone: fl(max|x| * rinv) = max fl(|x| * rinv)
+        sm.scale[tid] = __fdiv_rn(127.0f, fmaxf(__fmul_rn(__uint_as_float(mx), rinv), 1e-5f));
+    }
+    __syncthreads();
+    const float rinv = row_ok ? sm.rinv[m_row] : 0.0f;
+    if (gain != nullptr) {   // max |(x * rinv) * gain|
+      uint32_t hm = 0;
+#pragma unroll
+      for (int j = 0; j < kVmax; ++j)
+        if (have & (1u << j)) {
+          const int k0 = (lt + kTpr * j) * E;
+#pragma unroll
+          for (int i = 0; i < E; ++i) {
+            const float hv = __fmul_rn(__fmul_rn(V::val(raw[j], i), rinv), __ldg(gain + k0 + i));
+            hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
+          }
+        }
+      hm = __reduce_max_sync(0xffffffffu, hm);
+      if (lane == 0) sm.red_u[warp] = hm;
+      __syncthreads();
+      if (tid < M) {
+        constexpr int wpr = kTpr / 32;
+        uint32_t mx = 0;
+        for (int w = tid * wpr; w < (tid + 1) * wpr; ++w) mx = max(mx, sm.red_u[w]);
+        sm.scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx), 1e-5f));
+      }
+      __syncthreads();
+    }
+    {
+      const float sc = row_ok ? sm.scale[m_row] : 0.0f;
+      int isum = 0;
+      float* res = s == 0 ? sm.res_x : (s == 2 ? sm.res_y1 : nullptr);
+#pragma unroll
+      for (int j = 0; j < kVmax; ++j)
+        if (have & (1u << j)) {
+          const int v = lt + kTpr * j;
+          uint32_t c[E];
+#pragma unroll
+          for (int i = 0; i < E; ++i) {
+            float hv = __fmul_rn(V::val(raw[j], i), rinv);
+            if (gain != nullptr) hv = __fmul_rn(hv, __ldg(gain + v * E + i));
+            c[i] = rint_bits(__fmul_rn(hv, sc));
+          }
+          V::store_codes(codes + (size_t)m_row * qpitch + v * E, c, isum);
+          if (res != nullptr) {   // keep this CTA's channels of x (S1) / y1 (S3) for the residual
+            const int t16 = (v * E) >> 4;
+            if (t16 % G == b) {
+              const int ti = t16 / G;
+#pragma unroll
+              for (int i = 0; i < E; ++i) res[(ti * 16 + ((v * E + i) & 15)) * 8 + m_row] = V::val(raw[j], i);
+            }
+          }
+        }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+      if (lane == 0) sm.red_i[warp] = isum;
+    }
+    __syncthreads();
+    if (tid < M) {
+      constexpr int wpr = kTpr / 32;
+      int t = 0;
+      for (int w = tid * wpr; w < (tid + 1) * wpr; ++w) t += sm.red_i[w];
+      sm.qsum[tid] = t;
+    }
+    __syncthreads();
+    if (a.dbg.q[s] != nullptr && b == 0) {   // debug: this stage's codes and scales (one launch, one layer)
+      for (int i = tid; i < M * K / 16; i += kThreads) {
+        const int m = i / (K / 16), c16 = i - m * (K / 16);
+        *reinterpret_cast<uint4*>(a.dbg.q[s] + (size_t)m * K + c16 * 16) =
+            *reinterpret_cast<const uint4*>(codes + (size_t)m * qpitch + c16 * 16);
+      }
+      if (tid < M && a.dbg.scale[s] != nullptr) a.dbg.scale[s][tid] = sm.scale[tid];
+    }
+
+    // ---------------------------------------------------- this stage's weight slice, then the contraction
+    {
+      const int slot = q % a.nslot;
+      bool got = mbar_try_wait(&sm.slot_bar[slot], (uint32_t)(q / a.nslot) & 1u);
+      if (!got) {
+        const long long t0 = clock64();
+        while (!(got = mbar_try_wait(&sm.slot_bar[slot], (uint32_t)(q / a.nslot) & 1u))) {
+          if (clock64() - t0 > a.wait_cycles) break;
+        }
+      }
+      if (__syncthreads_or(!got)) {
+        give_up(a, sm, 6, q, q_issued);
+        return;
+      }
+      const uint4* sl = reinterpret_cast<const uint4*>(slots + (size_t)slot * a.slot_bytes);
+      if (g.nseg == 3) stage_mma<3>(sl, codes, qpitch, M, K, ntl, sm.red);
+      else if (g.nseg == 2) stage_mma<2>(sl, codes, qpitch, M, K, ntl, sm.red);
+      else stage_mma<1>(sl, codes, qpitch, M, K, ntl, sm.red);
+    }
+    __syncthreads();
+    if (warp == 0) {   // the slot is free: refill it `nslot` stages ahead; prefetch further ahead into L2
+      fence_proxy_async_smem();
+      if (q + a.nslot < nq) {
+        fill_slot(a, desc, slots, sm, q + a.nslot, lane);
+        q_issued = q + a.nslot + 1;
+      }
+      if (q + a.nslot + kPrefetchAhead < nq) prefetch_stage(a, desc, q + a.nslot + kPrefetchAhead, lane);
+    }
+    if (q + a.nslot < nq) q_issued = q + a.nslot + 1;
+
+    // ---------------------------------------------------- epilogue: one output element per thread
+    if (has_out) {
+      const float sc = sm.scale[e_m];
+      const int qs = sm.qsum[e_m];
+      const size_t o_idx = (size_t)e_m * N + e_n;
+      const bool skip = b == a.skip_cta && q == 0;   // test hook: one CTA never publishes its first stage
+      if (s == 0) {
+        float pre[3];
+#pragma unroll
+        for (int r = 0; r < 3; ++r) {
+          pre[r] = round_to<T>(rescale_acc(sm.red[e_ti][r][e_row][e_m] - qs, sm.gam[l][r], sc) + bias[r]);
+          if (a.dbg.pre != nullptr) static_cast<T*>(a.dbg.pre)[((size_t)e_m * 3 + r) * d + e_n] = from_f32<T>(pre[r]);
+        }
+        const float og = mlgru_step(pre[0], pre[1], pre[2], hval);
+        *hp = hval;
+        if (!skip)
+          publish(reinterpret_cast<T*>(xregion(a, l, par, 0)) + o_idx, reinterpret_cast<T*>(xregion(a, l, par ^ 1, 0)) + o_idx,
+                  og);
+        if (a.dbg.og != nullptr) static_cast<T*>(a.dbg.og)[o_idx] = from_f32<T>(og);
+      } else if (s == 2) {
+        float uv[2];
+#pragma unroll
+        for (int r = 0; r < 2; ++r) uv[r] = rescale_acc(sm.red[e_ti][r][e_row][e_m] - qs, sm.gam[l][4 + r], sc) + bias[r];
+        const float p = siluf_(uv[0]) * uv[1];
+        publish(reinterpret_cast<T*>(xregion(a, l, par, 2)) + o_idx, reinterpret_cast<T*>(xregion(a, l, par ^ 1, 2)) + o_idx, p);
+        if (a.dbg.p != nullptr) static_cast<T*>(a.dbg.p)[o_idx] = from_f32<T>(p);
+      } else {
+        const float* res = s == 1 ? sm.res_x : sm.res_y1;
+        const float v = rescale_acc(sm.red[e_ti][0][e_row][e_m] - qs, sm.gam[l][g.mat0], sc) + bias[0] +
+                        res[(e_ti * 16 + e_row) * 8 + e_m];
+        if (s == 1) {
+          publish(reinterpret_cast<T*>(xregion(a, l, par, 1)) + o_idx,
+                  reinterpret_cast<T*>(xregion(a, l, par ^ 1, 1)) + o_idx, v);
+          if (a.dbg.y1 != nullptr) static_cast<T*>(a.dbg.y1)[o_idx] = from_f32<T>(v);
+        } else if (l == L - 1) {
+          static_cast<T*>(a.y)[o_idx] = from_f32<T>(v);
+        } else {
+          publish(reinterpret_cast<T*>(xregion(a, l, par, 3)) + o_idx,
+                  reinterpret_cast<T*>(xregion(a, l, par ^ 1, 3)) + o_idx, v);
+        }
+      }
+    }
+    __syncthreads();   // red, codes and the residual slices are reused by the next stage
+  }
+  if (b == 0 && tid < L) a.parity[a.layer0 + tid] = sm.par[tid] ^ 1u;
+}
+
+struct Geom {
+  int nslot, slot_bytes, qpitch;
+  size_t desc_bytes, codes_bytes, smem;
+};
+
+constexpr size_t kDecodeSmemBudget = 214 * 1024;   // dynamic part; the static part is ~9 KB of the 227 KB
+
+bool geometry(int M, int d, int I, int L, int esize, int G, Geom& g) {
+  const int kmax = std::max(d, I);
+  g.qpitch = kmax + 16;
+  g.desc_bytes = (sizeof(DecodeLayerDesc) * (size_t)L + 127) / 128 * 128;
+  g.codes_bytes = ((size_t)M * g.qpitch + 127) / 128 * 128;
+  size_t slot = 0;
+  for (int s = 0; s < 4; ++s) {
+    const StageGeom sg = stage_geom(s, d, I);
+    slot = std::max(slot, (size_t)tiles_of(sg.N, 0, G) * sg.nseg * 16 * (sg.K / 4 + 64));
+  }
+  g.slot_bytes = (int)((slot + 127) / 128 * 128);
+  const size_t fixed = g.desc_bytes + g.codes_bytes;
+  if (fixed + g.slot_bytes > kDecodeSmemBudget) return false;
+  g.nslot = (int)std::min<size_t>(kDecodeMaxSlots, (kDecodeSmemBudget - fixed) / g.slot_bytes);
+  g.smem = fixed + (size_t)g.nslot * g.slot_bytes;
+  (void)esize;
+  return true;
+}
+
+int mpad_of(int M) { return M <= 1 ? 1 : (M <= 2 ? 2 : (M <= 4 ? 4 : 8)); }
+
+template <typename T, int MPAD>
+cudaError_t launch_typed(DecodeStepArgs a, const Geom& g, cudaStream_t stream) {
+  auto kern = decode_step_kernel<T, MPAD>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)g.smem);
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, g.smem);
+  if (e != cudaSuccess) return e;
+  if (per_sm < 1) return cudaErrorCooperativeLaunchTooLarge;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(decode_step_grid(a.d, a.I));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = g.smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, a);
+}
+
+template <typename T>
+cudaError_t launch_t(const DecodeStepArgs& a, const Geom& g, cudaStream_t stream) {
+  switch (mpad_of(a.M)) {
+    case 1: return launch_typed<T, 1>(a, g, stream);
+    case 2: return launch_typed<T, 2>(a, g, stream);
+    case 4: return launch_typed<T, 4>(a, g, stream);
+    default: return launch_typed<T, 8>(a, g, stream);
+  }
+}
+
+}  // namespace
+
+int decode_step_grid(int d, int I) { return std::min(num_sms(), std::max(d, I) / 16); }
+
+size_t decode_xlayer_bytes(int M, int d, int I) {
+  return (2 * (region_off(3, M, d, I) + (size_t)M * d * 4) + 255) / 256 * 256;
+}
+
+bool decode_step_supported(int M, int d, int I, int L, mmf_dtype dt) {
+  if (M < 1 || M > 8 || L < 1 || L > kDecodeMaxLayers) return false;
+  if (d < 64 || I < 64 || d % 64 != 0 || I % 64 != 0) return false;
+  const int G = decode_step_grid(d, I);
+  if (G < 1) return false;
+  const int esize = dt == MMF_BF16 ? 2 : 4;
+  const int mpad = mpad_of(M);
+  const int tpr = kThreads / mpad;
+  for (int s = 0; s < 4; ++s) {
+    const StageGeom sg = stage_geom(s, d, I);
+    if (tiles_of(sg.N, 0, G) > kDecodeTiles) return false;
+    if (ceil_div(sg.K * esize / 16, tpr) > kVmax) return false;   // input vectors per thread
+  }
+  Geom g;
+  return geometry(M, d, I, L, esize, G, g);
+}
+
+cudaError_t launch_decode_step(DecodeStepArgs a, mmf_dtype dt, cudaStream_t stream) {
+  if (!decode_step_supported(a.M, a.d, a.I, a.L, dt)) return cudaErrorNotSupported;
+  Geom g;
+  geometry(a.M, a.d, a.I, a.L, dt == MMF_BF16 ? 2 : 4, decode_step_grid(a.d, a.I), g);
+  a.nslot = g.nslot;
+  a.slot_bytes = g.slot_bytes;
+  a.qpitch = g.qpitch;
+  a.desc_bytes = (int)g.desc_bytes;
+  a.codes_bytes = (int)g.codes_bytes;
+  if (a.xI < a.I) return cudaErrorInvalidValue;
+  a.xlayer_bytes = decode_xlayer_bytes(a.M, a.d, a.xI);
+  a.xset_bytes = a.xlayer_bytes / 2;
+  return dt == MMF_BF16 ? launch_t<bf16>(a, g, stream) : launch_t<float>(a, g, stream);
+}
+
+}  // namespace mmf

@@ -17,6 +17,11 @@ bool tma_available();
 bool make_tma_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dt, int esize, uint64_t cols,
                  uint64_t rows, uint32_t box_cols, uint32_t box_rows, CUtensorMapSwizzle swz);
 int num_sms();
+// Bound of the kernels' device-side waits, in SM cycles: about 1 s at 2 GHz, or
+// MMF_WAIT_LIMIT_US microseconds when set (tests make waits run out quickly).
+long long wait_limit_cycles();
+// Integer test hook from the environment variable `name` (-1 when unset).
+int test_hook(const char* name);
 
 // Launch `kern` with programmatic stream serialization (the kernel must call
 // pdl_wait() before touching anything a predecessor wrote or reads).
@@ -78,6 +83,7 @@ struct TGemmArgs {
   int ldo;                  // leading dimension of out (elements)
   const void* residual;     // [M, N] in the activation dtype, or null
   float* h;                 // kScanStep: [M, N] fp32 state, updated in place
+  void* pre_out;            // kScanStep, nullable: the stored f~, c~, g~ values, [M, 3, N] (activation dtype)
   // Decode contraction only: when x is set, the kernel quantises the token
   // rows x [M, K] (activation dtype, RMSNorm gain `gain` or null, `eps`)
   // itself and q/s/qsum above are not read; q_out/s_out/qsum_out (nullable)
@@ -104,62 +110,49 @@ bool tgemm_mma_fused_quant_supported(int M, int K, int esize);
 bool tgemm_tc_supported(const TGemmArgs& a, Epi epi);
 cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
 
-// The same contraction on SM pairs (tcgen05 cta_group::2, 256-token tiles); needs M >= 256.
-bool tgemm_tc2_supported(const TGemmArgs& a, Epi epi);
-cudaError_t launch_tgemm_tc2(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* status, cudaStream_t stream);
-
-// Prefill token mixer in one kernel: the f|c|g contraction (a.nseg == 3, rows
-// of the three matrices for the same channels) with the MLGRU gates and
-// recurrence in its epilogue; writes o' [M, d] (a.out, activation dtype) and
-// updates the state h [B, d]. Needs T % 128 == 0 and d % 64 == 0. `ws` holds
-// tgemm_tc_mlgru_ws_bytes(B, T, d) bytes that reset_tgemm_tc_mlgru_ws() must
-// prepare (stream-ordered) before every launch.
-bool tgemm_tc_mlgru_supported(const TGemmArgs& a, int T, int d);
-size_t tgemm_tc_mlgru_ws_bytes(int B, int T, int d);
-cudaError_t reset_tgemm_tc_mlgru_ws(void* ws, int B, int T, int d, cudaStream_t stream);
-cudaError_t launch_tgemm_tc_mlgru(const TGemmArgs& a, mmf_dtype dt, int T, int d, float* h, void* ws, int* status,
-                                  cudaStream_t stream);
-
-// One decode step (T = 1, M <= 8 tokens) of a whole block in one cooperative
-// launch (grid = one CTA per SM): stage 0 quantises x with st[0].gain and runs
-// f|c|g (3 segments, N = d) with the MLGRU step (h in place, o' -> og); stage 1
-// quantises og and runs o (+ x) -> y1; stage 2 quantises y1 and runs gate|up
-// (2 segments, N = I) with SiLU(gate) * up -> p; stage 3 quantises p and runs
-// down (+ y1) -> y. `bar` holds 256 bytes (words 0 and 32 used) that are zero
-// between launches.
-constexpr int kDecodeMaxTiles = 4;   // 16-row weight tiles per CTA and stage
-struct DecodeStage {
-  const uint32_t* w[3];     // packed codes per segment, [N, K/16]
-  const float* gamma[3];    // per-segment scale (device scalar)
-  const float* bias[3];     // per-segment bias [N] or null
-  const float* gain;        // RMSNorm gain [K] of the stage's input, or null
-  int nseg, N, K;
+// One decode step (T = 1) of L consecutive blocks in one cooperative launch
+// (decode_step.cu). Per-block device descriptor, built at block creation:
+struct DecodeLayerDesc {
+  const uint32_t* w[7];     // packed codes: f, c, g, o, gate, up, down
+  const float* gamma[7];    // their scales (device scalars)
+  const float* bias[7];     // their biases, or null
+  const float* gain[4];     // RMSNorm gains of the four quantised inputs (x, o', y1, p), or null
 };
-struct DecodeBlockArgs {
-  DecodeStage st[4];        // f|c|g, o, gate|up, down
-  const void* x;            // [M, d] block input (activation dtype)
-  void* og;                 // [M, d] o'
-  void* y1;                 // [M, d] token-mixer output
-  void* p;                  // [M, I] GLU product
-  void* y;                  // [M, d] block output
-  float* h;                 // [M, d] recurrent state
-  int M, d, I;
+constexpr int kDecodeMaxLayers = 32;   // layers per launch
+constexpr int kDecodeTiles = 3;        // 16-row tiles per CTA and stage
+constexpr int kDecodeMaxSlots = 4;     // weight ring depth
+struct DecodeStepArgs {
+  const DecodeLayerDesc* layer[kDecodeMaxLayers];
+  const void* x;            // [M, d] input of the first layer (activation dtype)
+  void* y;                  // [M, d] output of the last layer
+  float* h;                 // state [L_state, M, d]; this launch uses layers layer0 .. layer0 + L - 1
+  uint8_t* xbuf;            // exchange buffers: per state layer decode_xlayer_bytes(M, d, I) bytes
+  unsigned* parity;         // per state layer: which buffer set the next launch writes
+  int* abort_word;          // raised by a CTA that gave up a wait; zero between launches
+  int* status;              // device status word (codes 5, 6)
+  mmf_block_debug dbg;      // L == 1 only: optional copies of the intermediates
+  size_t xlayer_bytes, xset_bytes;
+  long long wait_cycles;    // bound of every wait, in SM clock cycles
   float eps;
-  unsigned* bar;            // grid-barrier words (counter, generation)
-  int* status;              // device status word (code 4: a barrier wait gave up)
-  int slot_bytes;           // set by the launcher
+  int L, layer0, M, d, I;
+  int xI;                   // inner size the exchange buffers were allocated for (>= I)
+  int nslot, slot_bytes, qpitch, desc_bytes, codes_bytes;   // set by the launcher
+  int skip_cta;             // test hook: this CTA never publishes its first stage (-1: none)
 };
-bool decode_block_supported(const DecodeBlockArgs& a, mmf_dtype dt);
-cudaError_t launch_decode_block(DecodeBlockArgs a, mmf_dtype dt, cudaStream_t stream);
+// Bytes of exchange buffers (both sets) per state layer.
+size_t decode_xlayer_bytes(int M, int d, int I);
+bool decode_step_supported(int M, int d, int I, int L, mmf_dtype dt);
+// Grid of the launch: one CTA per SM, at most one per 16-row tile of the widest stage.
+int decode_step_grid(int d, int I);
+cudaError_t launch_decode_step(DecodeStepArgs a, mmf_dtype dt, cudaStream_t stream);
 
-// Chunk-parallel MLGRU scan; `ws` holds mlgru_scan_ws_bytes(B, T, d) bytes of
-// scratch, which reset_mlgru_scan_ws() must prepare (stream-ordered) before
-// every launch; launch_mlgru_scan() itself enqueues only the kernel (launched
-// as a programmatic dependent of the kernel before it). `status` is the device
-// status word for bounded-wait timeouts.
+// MLGRU gates + scan; one CTA per (sequence, 64 or 32 channels) walks the
+// sequence's chunks in order. Launched as a programmatic dependent of the
+// kernel before it. `status` is the device status word for bounded-wait
+// timeouts. mlgru_scan_ws_bytes() is the scratch the C ABI's workspace size
+// reports (the kernel uses none).
 size_t mlgru_scan_ws_bytes(int B, int T, int d);
-cudaError_t reset_mlgru_scan_ws(void* ws, int B, int T, int d, cudaStream_t stream);
-cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, void* ws,
-                              int* status, cudaStream_t stream);
+cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, int* status,
+                              cudaStream_t stream);
 
 }  // namespace mmf

@@ -158,3 +158,125 @@ __device__ __forceinline__ RowCode quant_row(const uint4* v, int nvec, int K, co
 }
 
 }  // namespace mmf
+
+namespace mmf {
+
+// Block-wide form of the same quantisation for a few token rows at once (at
+// most MPAD rows; NT threads, NT / MPAD >= 32 threads per row). Thread t works
+// on row t / (NT / MPAD) and holds that row's 16-byte vectors lt, lt + tpr, ...
+// (lt = t % tpr, tpr = NT / MPAD) in raw[j] for every bit j set in `have`. The
+// row's fp64 sum of squares and its max are reduced over the row's warps in a
+// fixed order, so every CTA that quantises the same rows gets the same scale;
+// the fp32 steps are those of quant_row. Codes go to codes + m * qpitch (16-byte
+// aligned rows); scale[m], qsum[m] (shared) get the row's scale and code sum.
+// `red` is shared scratch of at least NT / 32 entries of each type. Contains
+// __syncthreads(): every thread of the block calls it.
+struct BlockRed {
+  double* d;
+  uint32_t* u;
+  int* i;
+  float* rinv;   // [MPAD]
+};
+
+template <typename T, int MPAD, int NT, int VMAX>
+__device__ __forceinline__ void block_quant(const uint4 (&raw)[VMAX], uint32_t have, int M, int K,
+                                            const float* __restrict__ gain, float eps, int8_t* codes, int qpitch,
+                                            float* scale, int* qsum, const BlockRed& red) {
+  using V = Vec<T>;
+  constexpr int E = V::E;
+  constexpr int kTpr = NT / MPAD;
+  constexpr int kWpr = kTpr / 32;
+  static_assert(kTpr >= 32, "at least one warp per row");
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int m_row = tid / kTpr, lt = tid - m_row * kTpr;
+  const bool row_ok = m_row < M;
+  {   // sum of squares (fp64) and max |x|
+    double ss = 0.0;
+    uint32_t am = 0;
+#pragma unroll
+    for (int j = 0; j < VMAX; ++j)
+      if (have & (1u << j)) {
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const uint32_t mg = V::mag(raw[j], i);
+          am = max(am, mg);
+          const double xd = magbits_to_f64(mg);
+          ss = fma(xd, xd, ss);
+        }
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    am = __reduce_max_sync(0xffffffffu, am);
+    if (lane == 0) {
+      red.d[warp] = ss;
+      red.u[warp] = am;
+    }
+  }
+  __syncthreads();
+  if (tid < M) {   // per row, its warps in order
+    double t = 0.0;
+    uint32_t mx = 0;
+    for (int w = tid * kWpr; w < (tid + 1) * kWpr; ++w) {
+      t += red.d[w];
+      mx = max(mx, red.u[w]);
+    }
+    const float ms = (float)(t / (double)K);
+    const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
+    red.rinv[tid] = rinv;
+    if (gain == nullptr)   // rounding is monotone: fl(max|x| * rinv) = max fl(|x| * rinv)
+      scale[tid] = __fdiv_rn(127.0f, fmaxf(__fmul_rn(__uint_as_float(mx), rinv), 1e-5f));
+  }
+  __syncthreads();
+  const float rinv = row_ok ? red.rinv[m_row] : 0.0f;
+  if (gain != nullptr) {   // max |(x * rinv) * gain|
+    uint32_t hm = 0;
+#pragma unroll
+    for (int j = 0; j < VMAX; ++j)
+      if (have & (1u << j)) {
+        const int k0 = (lt + kTpr * j) * E;
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          const float hv = __fmul_rn(__fmul_rn(V::val(raw[j], i), rinv), __ldg(gain + k0 + i));
+          hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
+        }
+      }
+    hm = __reduce_max_sync(0xffffffffu, hm);
+    if (lane == 0) red.u[warp] = hm;
+    __syncthreads();
+    if (tid < M) {
+      uint32_t mx = 0;
+      for (int w = tid * kWpr; w < (tid + 1) * kWpr; ++w) mx = max(mx, red.u[w]);
+      scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx), 1e-5f));
+    }
+    __syncthreads();
+  }
+  {   // codes and their sum
+    const float sc = row_ok ? scale[m_row] : 0.0f;
+    int isum = 0;
+#pragma unroll
+    for (int j = 0; j < VMAX; ++j)
+      if (have & (1u << j)) {
+        const int v = lt + kTpr * j;
+        uint32_t c[E];
+#pragma unroll
+        for (int i = 0; i < E; ++i) {
+          float hv = __fmul_rn(V::val(raw[j], i), rinv);
+          if (gain != nullptr) hv = __fmul_rn(hv, __ldg(gain + v * E + i));
+          c[i] = rint_bits(__fmul_rn(hv, sc));
+        }
+        V::store_codes(codes + (size_t)m_row * qpitch + v * E, c, isum);
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
+    if (lane == 0) red.i[warp] = isum;
+  }
+  __syncthreads();
+  if (tid < M) {
+    int t = 0;
+    for (int w = tid * kWpr; w < (tid + 1) * kWpr; ++w) t += red.i[w];
+    qsum[tid] = t;
+  }
+  __syncthreads();
+}
+
+}  // namespace mmf

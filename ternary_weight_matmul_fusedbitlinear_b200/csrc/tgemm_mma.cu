@@ -81,8 +81,16 @@ __host__ __device__ __forceinline__ int wsm_pitch4(int wpr) { return wpr / 4 + 4
 // more than a row, which spreads the 8 rows of a fragment load over the banks.
 __host__ __device__ __forceinline__ int fq_pitch(int K) { return K + 16; }
 
-template <int NT, int R, Epi EPI, typename T, bool SMEMW, bool FQ>
+// FQM: how the kernel gets its activation codes. 0: from the standalone
+// quantiser (a.q, a.s, a.qsum); 1, 2, 4, 8: it quantises its token rows itself
+// with the whole block (block_quant, rows padded to FQM, at most 8 tokens);
+// 16: itself, one warp per row (up to 16 tokens).
+constexpr int kFqWarpRows = 16;
+constexpr int kFqVmax = 16;   // 16-byte vectors per thread and row in block_quant
+
+template <int NT, int R, Epi EPI, typename T, bool SMEMW, int FQM>
 __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
+  constexpr bool FQ = FQM != 0;
   __shared__ int red[R][16][NT * 8];
   __shared__ float s_sm[FQ ? NT * 8 : 1];
   __shared__ int qsum_sm[FQ ? NT * 8 : 1];
@@ -112,7 +120,40 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
   for (int i = threadIdx.x; i < R * 16 * NT * 8; i += kThreads) (&red[0][0][0])[i] = 0;
   int8_t* qs = reinterpret_cast<int8_t*>(wsm + (SMEMW ? R * 16 * pitch4 : 0));
   const int qpitch = fq_pitch(K);
-  if constexpr (FQ) {   // quantise this CTA's token rows, one warp per row
+  if constexpr (FQM >= 1 && FQM <= 8) {   // the whole block quantises the (at most 8) token rows
+    __shared__ double red_d[kWarps];
+    __shared__ uint32_t red_u[kWarps];
+    __shared__ int red_i[kWarps];
+    __shared__ float red_r[FQM];
+    constexpr int kTpr = kThreads / FQM;
+    const int m_row = threadIdx.x / kTpr, lt = threadIdx.x - m_row * kTpr;
+    const int nvec = (int)(K * sizeof(T) / 16);
+    const uint4* xg = reinterpret_cast<const uint4*>(static_cast<const T*>(a.x) + (size_t)m_row * K);
+    uint4 raw[kFqVmax];
+    uint32_t have = 0;
+#pragma unroll
+    for (int j = 0; j < kFqVmax; ++j) {
+      const int v = lt + kTpr * j;
+      raw[j] = make_uint4(0u, 0u, 0u, 0u);
+      if (m_row < M && v < nvec) {
+        have |= 1u << j;
+        raw[j] = __ldg(xg + v);
+      }
+    }
+    block_quant<T, FQM, kThreads, kFqVmax>(raw, have, M, K, a.gain, a.eps, qs, qpitch, s_sm, qsum_sm,
+                                           BlockRed{red_d, red_u, red_i, red_r});
+    if (blockIdx.x == 0 && a.q_out != nullptr) {   // one CTA also hands the codes out
+      for (int i = threadIdx.x; i < M * K / 16; i += kThreads) {
+        const int m = i / (K / 16), c16 = i - m * (K / 16);
+        *reinterpret_cast<uint4*>(a.q_out + (size_t)m * K + c16 * 16) =
+            *reinterpret_cast<const uint4*>(qs + (size_t)m * qpitch + c16 * 16);
+      }
+      if (threadIdx.x < M) {
+        if (a.s_out) a.s_out[threadIdx.x] = s_sm[threadIdx.x];
+        if (a.qsum_out) a.qsum_out[threadIdx.x] = qsum_sm[threadIdx.x];
+      }
+    }
+  } else if constexpr (FQM == kFqWarpRows) {   // quantise this CTA's token rows, one warp per row
     const int nvec = (int)(K * sizeof(T) / 16);
     const int rows = min(NT * 8, M - m0);
     uint4* xs = reinterpret_cast<uint4*>(qs + (size_t)NT * 8 * qpitch);
@@ -245,6 +286,7 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
         float v = rescale_acc(red[r][row][mc] - row_qsum(mc), *a.gamma[r], row_scale(mc));
         if (a.bias[r] != nullptr) v += a.bias[r][n];
         pre[r] = round_to<T>(v);   // the pre-activations are a storage point
+        if (a.pre_out != nullptr) static_cast<T*>(a.pre_out)[((size_t)m * 3 + r) * N + n] = from_f32<T>(pre[r]);
       }
       float* hp = a.h + (size_t)m * N + n;
       float hn = *hp;
@@ -271,9 +313,9 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
 
 constexpr size_t kFqBytes = 128 * 1024;   // fused-quantisation limit: codes + staged token rows
 
-template <int NT, int R, Epi EPI, typename T, bool SMEMW, bool FQ>
+template <int NT, int R, Epi EPI, typename T, bool SMEMW, int FQM>
 cudaError_t launch_variant(const TGemmArgs& a, dim3 grid, size_t smem, cudaStream_t stream) {
-  auto kern = tgemm_mma_kernel<NT, R, EPI, T, SMEMW, FQ>;
+  auto kern = tgemm_mma_kernel<NT, R, EPI, T, SMEMW, FQM>;
   if (smem > 0) {   // the default limit covers static + dynamic together, so opt in whenever there is any
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
@@ -294,10 +336,26 @@ cudaError_t launch_one(const TGemmArgs& a, cudaStream_t stream) {
   // the weight slice goes to shared memory when it fits next to the codes
   const bool smemw = wpr % 4 == 0 && wbytes <= 100 * 1024 && wbytes + qbytes <= 200 * 1024;
   const size_t smem = (smemw ? wbytes : 0) + qbytes;
-  if (smemw) return fq ? launch_variant<NT, R, EPI, T, true, true>(a, grid, smem, stream)
-                       : launch_variant<NT, R, EPI, T, true, false>(a, grid, smem, stream);
-  return fq ? launch_variant<NT, R, EPI, T, false, true>(a, grid, smem, stream)
-            : launch_variant<NT, R, EPI, T, false, false>(a, grid, smem, stream);
+  if (!fq) return smemw ? launch_variant<NT, R, EPI, T, true, 0>(a, grid, smem, stream)
+                        : launch_variant<NT, R, EPI, T, false, 0>(a, grid, smem, stream);
+  if constexpr (NT == 1) {   // the whole block on each row when every thread's share fits its registers
+    const int mpad = a.M <= 1 ? 1 : (a.M <= 2 ? 2 : (a.M <= 4 ? 4 : 8));
+    const int nvec = (int)(a.K * sizeof(T) / 16);
+    if (ceil_div(nvec, kThreads / mpad) <= kFqVmax) {
+      switch (mpad) {
+        case 1: return smemw ? launch_variant<NT, R, EPI, T, true, 1>(a, grid, smem, stream)
+                             : launch_variant<NT, R, EPI, T, false, 1>(a, grid, smem, stream);
+        case 2: return smemw ? launch_variant<NT, R, EPI, T, true, 2>(a, grid, smem, stream)
+                             : launch_variant<NT, R, EPI, T, false, 2>(a, grid, smem, stream);
+        case 4: return smemw ? launch_variant<NT, R, EPI, T, true, 4>(a, grid, smem, stream)
+                             : launch_variant<NT, R, EPI, T, false, 4>(a, grid, smem, stream);
+        default: return smemw ? launch_variant<NT, R, EPI, T, true, 8>(a, grid, smem, stream)
+                              : launch_variant<NT, R, EPI, T, false, 8>(a, grid, smem, stream);
+      }
+    }
+  }
+  return smemw ? launch_variant<NT, R, EPI, T, true, kFqWarpRows>(a, grid, smem, stream)
+               : launch_variant<NT, R, EPI, T, false, kFqWarpRows>(a, grid, smem, stream);
 }
 
 template <int NT, typename T>

@@ -81,6 +81,8 @@ struct TcArgs {
   TGemmArgs g;
   int m_tiles, n_tiles;
   int* status;
+  long long wait_cycles;   // bound of every wait
+  uint32_t skip_it;        // test hook: CTA 0 never loads this k-step (~0u: none)
 };
 
 // Rows of weight segment `seg` starting at `row0` feed half `h` of tile `nt`.
@@ -165,7 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         half_source(p, EPI, nt, 1, seg1, row1);
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % NS;
-          if (!mbar_wait(&sm.tma_empty[s], ((it / NS) & 1) ^ 1, abort_flag, p.status)) { ok = false; break; }
+          if (!mbar_wait(&sm.tma_empty[s], ((it / NS) & 1) ^ 1, abort_flag, p.status, p.wait_cycles)) { ok = false; break; }
+          if (it == p.skip_it && blockIdx.x == 0) continue;   // test hook: these copies are never issued
           if constexpr (UNP) {   // int8 weight rows straight into the SW128 tile of this stage
             mbar_arrive_expect_tx(&sm.tma_full[s], A_BYTES + BU_BYTES);
             tma_load_2d(sm.a[s], &map_a, kb * BK, mt * BM, &sm.tma_full[s]);
@@ -181,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // let every copy this thread issued land before the CTA can exit
       for (uint32_t j = (it > NS ? it - NS : 0); j < it; ++j)
-        mbar_wait(&sm.tma_full[j % NS], (j / NS) & 1, abort_flag, nullptr);
+        if (j != p.skip_it || blockIdx.x != 0) mbar_drain(&sm.tma_full[j % NS], (j / NS) & 1, p.wait_cycles);
     }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
@@ -191,13 +194,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x, ++tl) {
         const int acc = tl & 1;
         const uint32_t acc_ph = (tl >> 1) & 1;
-        if (!mbar_wait(&sm.tmem_empty[acc], acc_ph ^ 1, abort_flag, p.status)) break;
+        if (!mbar_wait(&sm.tmem_empty[acc], acc_ph ^ 1, abort_flag, p.status, p.wait_cycles)) break;
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * BN;
         for (int kb = 0; kb < nk; ++kb, ++it) {
           const int s = it % NS, u = UNP ? s : (int)(it % NB);
-          if ((!UNP && !mbar_wait(&sm.bu_full[u], (it / NB) & 1, abort_flag, p.status)) ||
-              !mbar_wait(&sm.tma_full[s], (it / NS) & 1, abort_flag, p.status)) {
+          if ((!UNP && !mbar_wait(&sm.bu_full[u], (it / NB) & 1, abort_flag, p.status, p.wait_cycles)) ||
+              !mbar_wait(&sm.tma_full[s], (it / NS) & 1, abort_flag, p.status, p.wait_cycles)) {
             ok = false;
             break;
           }
@@ -214,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every MMA this thread issued has finished before TMEM can be released
       umma_commit(&sm.mma_drain);
-      mbar_wait(&sm.mma_drain, 0, abort_flag, nullptr);
+      mbar_drain(&sm.mma_drain, 0, p.wait_cycles);
     }
   } else if (warp >= kUnpackWarp0) {
     // ------------------------------------------------------------ unpack 2-bit codes to int8 (idle with UNP)
@@ -228,8 +231,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < n_tiles_total && ok; tile += gridDim.x) {
       for (int kb = 0; kb < nk; ++kb, ++it) {
         const int s = it % NS, u = it % NB;
-        if (!mbar_wait(&sm.tma_full[s], (it / NS) & 1, abort_flag, p.status) ||
-            !mbar_wait(&sm.bu_empty[u], ((it / NB) & 1) ^ 1, abort_flag, p.status)) {
+        if (!mbar_wait(&sm.tma_full[s], (it / NS) & 1, abort_flag, p.status, p.wait_cycles) ||
+            !mbar_wait(&sm.bu_empty[u], ((it / NB) & 1) ^ 1, abort_flag, p.status, p.wait_cycles)) {
           ok = false;
           break;
         }
@@ -287,7 +290,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mt = tile / p.n_tiles, nt = tile % p.n_tiles;
       const int acc = tl & 1;
       const uint32_t acc_ph = (tl >> 1) & 1;
-      const bool got = mbar_wait(&sm.tmem_full[acc], acc_ph, abort_flag, p.status);
+      const bool got = mbar_wait(&sm.tmem_full[acc], acc_ph, abort_flag, p.status, p.wait_cycles);
       __syncwarp();                               // tcgen05.ld below is warp-collective
       if (!__all_sync(0xffffffffu, got)) break;
       tc_fence_after();
@@ -348,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 out[j] = v;
               }
               if (has_res) {
-                const bool ok = mbar_wait(&sm.res_full[ew], nres & 1, abort_flag, p.status);
+                const bool ok = mbar_wait(&sm.res_full[ew], nres & 1, abort_flag, p.status, p.wait_cycles);
                 ++nres;
                 if (!__all_sync(0xffffffffu, ok)) { alive = false; break; }
                 add_staged_row(buf, lane, out, (T*)nullptr);
@@ -433,6 +436,8 @@ cudaError_t launch_tgemm_tc(const TGemmArgs& a, Epi epi, mmf_dtype dt, int* stat
   TcArgs p;
   p.g = a;
   p.status = status;
+  p.wait_cycles = wait_limit_cycles();
+  p.skip_it = (uint32_t)test_hook("MMF_TC_SKIP_KSTEP");
   p.m_tiles = ceil_div(a.M, BM);
   p.n_tiles = (epi == Epi::kGlu) ? ceil_div(a.N, HALF) : ceil_div(a.nseg * a.N, BN);
   const bool b = dt == MMF_BF16;

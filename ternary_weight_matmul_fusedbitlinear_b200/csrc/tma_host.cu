@@ -2,6 +2,8 @@
 // through the runtime's driver entry point, so nothing links libcuda).
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+#include <cstdlib>
 #include <mutex>
 
 #include "kernels.cuh"
@@ -49,6 +51,17 @@ int num_sms() {
     if (n <= 0) n = 148;
   }
   return n;
+}
+
+long long wait_limit_cycles() {
+  const char* e = getenv("MMF_WAIT_LIMIT_US");
+  const long long us = e != nullptr ? atoll(e) : 1000000;
+  return std::max(1LL, us) * 2000;
+}
+
+int test_hook(const char* name) {
+  const char* e = getenv(name);
+  return e != nullptr ? atoi(e) : -1;
 }
 
 }  // namespace mmf

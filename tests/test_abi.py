@@ -94,7 +94,6 @@ def test_block_create_validation(lib):
 
 def test_state_accessors_on_null_handle(lib):
     assert lib.mmf_state_layer(None, 0) is None
-    assert lib.mmf_state_barrier(None) is None
     assert lib.mmf_state_reset(None, None) == 1
 
 

@@ -9,14 +9,14 @@ import torch
 
 import oracle as O
 import synth
-from parity import E2E_TOL, TORCH_DT, assert_close, assert_codes_close, make_block, make_layer, packed_to_np, to_np
+from parity import TORCH_DT, assert_close, assert_codes_close, check_block_stages, make_block, make_layer, packed_to_np, to_np
 
 pytestmark = pytest.mark.gpu
 
 mmf = pytest.importorskip("ternary_weight_matmul_fusedbitlinear_b200")
 
 
-@pytest.fixture(params=["tc", "tc2", "mma"])
+@pytest.fixture(params=["tc", "mma"])
 def path(request, monkeypatch):
     monkeypatch.setenv("MMF_GEMM_PATH", request.param)
     return request.param
@@ -64,12 +64,35 @@ def test_tc_glu_parity(m, d, inner, dtype, path):
 
 @pytest.mark.parametrize("dtype", ["bf16", "f32"])
 def test_tc_block_prefill_parity(dtype, path):
+    # one block with every contraction on the pinned kernel, stage by stage at TOL
     d, inner, B, T = 256, 768, 3, 100
     blk, oblk = make_block(970, d, inner)
     x = synth.activations(971, B * T, d, TORCH_DT[dtype]).reshape(B, T, d)
     st = mmf.State(1, B, d)
-    y = mmf.block_forward(blk, 0, st, x.cuda())
-    y_ref, h_ref = O.block_forward(to_np(x), oblk, np.zeros((B, d)), dtype)
-    assert_close(to_np(y), y_ref, dtype, "block y", tol=E2E_TOL)
-    assert_close(st.get()[0].numpy(), h_ref, "f32", "block h", tol=E2E_TOL)
+    y, dbg = mmf.block_forward_debug(blk, 0, st, x.cuda())
     mmf.check()
+    check_block_stages(x, np.zeros((B, d)), y, st.get()[0].numpy(), dbg, oblk, dtype, f"block ({path})")
+
+
+def test_tc_wait_gives_up_and_reports(monkeypatch):
+    # failure detection without a fault: CTA 0 never loads its second k-step,
+    # so the MMA issuer's bounded wait runs out (20 ms); every role of that CTA
+    # leaves its loop, the MMAs and copies already started are drained, tensor
+    # memory is released, and mmf_check reports code 1; the next call is exact
+    k, n, m = 1024, 1024, 512
+    _, lin, olin = make_layer(980, n, k)
+    x = synth.activations(981, m, k, torch.bfloat16).cuda()
+    monkeypatch.setenv("MMF_GEMM_PATH", "tc")
+    monkeypatch.setenv("MMF_TC_SKIP_KSTEP", "1")
+    monkeypatch.setenv("MMF_WAIT_LIMIT_US", "20000")
+    mmf.bitlinear(lin, x)
+    with pytest.raises(mmf.MMFError) as err:
+        mmf.check()
+    assert err.value.status == 6 and "code 1" in str(err.value)
+    monkeypatch.delenv("MMF_TC_SKIP_KSTEP")
+    monkeypatch.delenv("MMF_WAIT_LIMIT_US")
+    y, q, s, acc = mmf.bitlinear(lin, x, debug=True)
+    mmf.check()
+    codes = O.unpack_codes(packed_to_np(lin.packed), k)
+    np.testing.assert_array_equal(acc.cpu().numpy().astype(np.int64), O.ternary_accumulate(q.cpu().numpy(), codes))
+    assert_close(to_np(y), O.bitlinear(to_np(x.cpu()), olin), "bf16", "y after the timeout")
