@@ -147,8 +147,7 @@ struct Smem {
   double red_d[kWarps];
   uint32_t red_u[kWarps];
   int red_i[kWarps];
-  float scale[8], rinv[8];
-  int qsum[8];
+  float scale[8];
   float res_x[kDecodeTiles * 16 * 8];   // block input x of this CTA's d-channels (S1 residual)
   float res_y1[kDecodeTiles * 16 * 8];  // y1 of this CTA's d-channels (S3 residual)
   float gam[kDecodeMaxLayers][7];
@@ -156,27 +155,28 @@ struct Smem {
   uint64_t slot_bar[kDecodeMaxSlots];
 };
 
-// Warp 0: start the bulk copies of stage q's weight slice into its ring slot.
+// One warp: start the bulk copies of stage q's weight slice into its ring slot.
+// A 16-row tile of one matrix is contiguous in memory (rows of K/4 bytes), so
+// each (tile, segment) is one copy, landing as 16 dense rows.
 __device__ void fill_slot(const DecodeStepArgs& a, const DecodeLayerDesc* desc, uint8_t* slots, Smem& sm, int q,
                           int lane) {
   const int l = q >> 2, s = q & 3;
   const StageGeom g = stage_geom(s, a.d, a.I);
   const int ntl = tiles_of(g.N, blockIdx.x, gridDim.x);
-  const int rowb = g.K / 4, pitch = rowb + 64;
+  const int tile_bytes = 16 * (g.K / 4);
   const int slot = q % a.nslot;
   uint8_t* dst0 = slots + (size_t)slot * a.slot_bytes;
-  const int ncopy = ntl * g.nseg * 16;
+  const int ncopy = ntl * g.nseg;
   if (lane == 0) {
-    if (ncopy > 0) mbar_arrive_expect_tx(&sm.slot_bar[slot], (uint32_t)ncopy * rowb);
+    if (ncopy > 0) mbar_arrive_expect_tx(&sm.slot_bar[slot], (uint32_t)(ncopy * tile_bytes));
     else mbar_arrive(&sm.slot_bar[slot]);
   }
   __syncwarp();
   for (int i = lane; i < ncopy; i += 32) {
-    const int ti = i / (g.nseg * 16), rem = i - ti * g.nseg * 16;
-    const int r = rem >> 4, row = rem & 15;
-    const int n = (blockIdx.x + ti * gridDim.x) * 16 + row;
-    const uint8_t* src = reinterpret_cast<const uint8_t*>(desc[l].w[g.mat0 + r]) + (size_t)n * rowb;
-    bulk_g2s(dst0 + (size_t)((ti * g.nseg + r) * 16 + row) * pitch, src, (uint32_t)rowb, &sm.slot_bar[slot]);
+    const int ti = i / g.nseg, r = i - ti * g.nseg;
+    const int t = blockIdx.x + ti * gridDim.x;
+    const uint8_t* src = reinterpret_cast<const uint8_t*>(desc[l].w[g.mat0 + r]) + (size_t)t * tile_bytes;
+    bulk_g2s(dst0 + (size_t)i * tile_bytes, src, (uint32_t)tile_bytes, &sm.slot_bar[slot]);
   }
 }
 
@@ -200,7 +200,7 @@ __device__ __forceinline__ void stage_mma(const uint4* slot, const int8_t* qs, i
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int wpr = K / 16, nkseg = ceil_div(K, 256);
-  const int pitch4 = K / 64 + 4;
+  const int pitch4 = K / 64;   // dense rows of K/4 bytes
   for (int item = warp; item < ntl * nkseg; item += kWarps) {
     const int ti = item / nkseg, seg = item - ti * nkseg;
     const int w0 = seg * 16 + 4 * t;   // first packed word of this lane
@@ -219,11 +219,11 @@ __device__ __forceinline__ void stage_mma(const uint4* slot, const int8_t* qs, i
       act[u] = ok ? *reinterpret_cast<const uint4*>(qs + (size_t)g * qpitch + (w0 + u) * 16)
                   : make_uint4(0u, 0u, 0u, 0u);
     }
-    int acc[R][4];
+    int acc[R][2][4];   // two accumulator chains per segment (even / odd k-steps): half the MMA latency chain
 #pragma unroll
     for (int r = 0; r < R; ++r)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) acc[r][e] = 0;
+      for (int e = 0; e < 4; ++e) acc[r][0][e] = acc[r][1][e] = 0;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       const int u = i >> 1, sub = (i & 1) * 2;
@@ -231,16 +231,16 @@ __device__ __forceinline__ void stage_mma(const uint4* slot, const int8_t* qs, i
 #pragma unroll
       for (int r = 0; r < R; ++r) {
         const uint32_t wg = u4get(wa[r], u), wg8 = u4get(wb[r], u);
-        mma_u8s8(acc[r], (wg >> (2 * sub)) & kLow2, (wg8 >> (2 * sub)) & kLow2, (wg >> (2 * sub + 2)) & kLow2,
-                 (wg8 >> (2 * sub + 2)) & kLow2, b0, b1);
+        mma_u8s8(acc[r][i & 1], (wg >> (2 * sub)) & kLow2, (wg8 >> (2 * sub)) & kLow2,
+                 (wg >> (2 * sub + 2)) & kLow2, (wg8 >> (2 * sub + 2)) & kLow2, b0, b1);
       }
     }
 #pragma unroll
     for (int r = 0; r < R; ++r) {
-      atomicAdd(&red[ti][r][g][2 * t], acc[r][0]);
-      atomicAdd(&red[ti][r][g][2 * t + 1], acc[r][1]);
-      atomicAdd(&red[ti][r][g + 8][2 * t], acc[r][2]);
-      atomicAdd(&red[ti][r][g + 8][2 * t + 1], acc[r][3]);
+      atomicAdd(&red[ti][r][g][2 * t], acc[r][0][0] + acc[r][1][0]);
+      atomicAdd(&red[ti][r][g][2 * t + 1], acc[r][0][1] + acc[r][1][1]);
+      atomicAdd(&red[ti][r][g + 8][2 * t], acc[r][0][2] + acc[r][1][2]);
+      atomicAdd(&red[ti][r][g + 8][2 * t + 1], acc[r][0][3] + acc[r][1][3]);
     }
   }
 }
@@ -268,6 +268,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
   using V = Vec<T>;
   constexpr int E = V::E;
   constexpr int kTpr = kThreads / MPAD;     // threads per token row in the quantisation
+  const BlockRed red{sm.red_d, sm.red_u, sm.red_i};
   DecodeLayerDesc* desc = reinterpret_cast<DecodeLayerDesc*>(dsm);
   int8_t* codes = reinterpret_cast<int8_t*>(dsm + a.desc_bytes);
   uint8_t* slots = dsm + a.desc_bytes + a.codes_bytes;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
   for (int i = tid; i < L * 7; i += kThreads) sm.gam[i / 7][i % 7] = *desc[i / 7].gamma[i % 7];
   // the weight stream does not depend on the previous kernel: start it first
   int q_issued = 0;   // stages whose ring fill has been issued
-  if (warp == 0) {
+  if (warp == kWarps - 1) {
     for (int q = 0; q < a.nslot && q < nq; ++q) fill_slot(a, desc, slots, sm, q, lane);
     for (int q = a.nslot; q < a.nslot + kPrefetchAhead && q < nq; ++q) prefetch_stage(a, desc, q, lane);
   }
@@ -353,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
     if (!poll) {
 #pragma unroll
       for (int j = 0; j < kVmax; ++j)
-        if (have & (1u << j)) raw[j] = __ldg(reinterpret_cast<const uint4*>(src) + lt + kTpr * j);
+        if (have & (1u << j)) raw[j] = __ldcg(reinterpret_cast<const uint4*>(src) + lt + kTpr * j);
     } else {
       long long t0 = 0;
       while (pend != 0u) {
@@ -378,106 +379,22 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
     }
 
     // ---------------------------------------------------- RMSNorm + absmax int8 codes, whole block
-    {
-      double ss = 0.0;
-      uint32_t am = 0;
-#pragma unroll
-      for (int j = 0; j < kVmax; ++j)
-        if (have & (1u << j)) {
-#pragma unroll
-          for (int i = 0; i < E; ++i) {
-            const uint32_t mg = V::mag(raw[j], i);
-            am = max(am, mg);
-            const double xd = magbits_to_f64(mg);
-            ss = fma(xd, xd, ss);
-          }
-        }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      am = __reduce_max_sync(0xffffffffu, am);
-      if (lane == 0) {
-        sm.red_d[warp] = ss;
-        sm.red_u[warp] = am;
-      }
-    }
-    __syncthreads();
     const float* gain = D.gain[g.gain];
-    if (tid < M) {   // per row, warps in order: the same sum in every CTA
-      constexpr int wpr = kTpr / 32;
-      double t = 0.0;
-      uint32_t mx = 0;
-      for (int w = tid * wpr; w < (tid + 1) * wpr; ++w) {
-        t += sm.red_d[w];
-        mx = max(mx, sm.red_u[w]);
-      }
-      const float ms = (float)(t / (double)K);
-      const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, a.eps)));
-      sm.rinv[tid] = rinv;
-      if (gain == nullptr)   // rounding is monotone: fl(max|x| * rinv) = max fl(|x| * rinv)
-        sm.scale[tid] = __fdiv_rn(127.0f, fmaxf(__fmul_rn(__uint_as_float(mx), rinv), 1e-5f));
-    }
-    __syncthreads();
-    const float rinv = row_ok ? sm.rinv[m_row] : 0.0f;
-    if (gain != nullptr) {   // max |(x * rinv) * gain|
-      uint32_t hm = 0;
+    block_quant<T, MPAD, kThreads, kVmax>(raw, have, M, K, gain, a.eps, codes, qpitch, sm.scale, red);
+    if (s == 0 || s == 2) {   // keep this CTA's channels of x (S1 residual) / y1 (S3 residual)
+      float* res = s == 0 ? sm.res_x : sm.res_y1;
 #pragma unroll
-      for (int j = 0; j < kVmax; ++j)
-        if (have & (1u << j)) {
-          const int k0 = (lt + kTpr * j) * E;
+      for (int j = 0; j < kVmax; ++j) {
+        if (!(have & (1u << j))) break;
+        const int v = lt + kTpr * j;
+        const int t16 = (v * E) >> 4;
+        if (t16 % G == b) {
+          const int ti = t16 / G;
 #pragma unroll
-          for (int i = 0; i < E; ++i) {
-            const float hv = __fmul_rn(__fmul_rn(V::val(raw[j], i), rinv), __ldg(gain + k0 + i));
-            hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
-          }
+          for (int i = 0; i < E; ++i) res[(ti * 16 + ((v * E + i) & 15)) * 8 + m_row] = V::val(raw[j], i);
         }
-      hm = __reduce_max_sync(0xffffffffu, hm);
-      if (lane == 0) sm.red_u[warp] = hm;
-      __syncthreads();
-      if (tid < M) {
-        constexpr int wpr = kTpr / 32;
-        uint32_t mx = 0;
-        for (int w = tid * wpr; w < (tid + 1) * wpr; ++w) mx = max(mx, sm.red_u[w]);
-        sm.scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx), 1e-5f));
       }
-      __syncthreads();
-    }
-    {
-      const float sc = row_ok ? sm.scale[m_row] : 0.0f;
-      int isum = 0;
-      float* res = s == 0 ? sm.res_x : (s == 2 ? sm.res_y1 : nullptr);
-#pragma unroll
-      for (int j = 0; j < kVmax; ++j)
-        if (have & (1u << j)) {
-          const int v = lt + kTpr * j;
-          uint32_t c[E];
-#pragma unroll
-          for (int i = 0; i < E; ++i) {
-            float hv = __fmul_rn(V::val(raw[j], i), rinv);
-            if (gain != nullptr) hv = __fmul_rn(hv, __ldg(gain + v * E + i));
-            c[i] = rint_bits(__fmul_rn(hv, sc));
-          }
-          V::store_codes(codes + (size_t)m_row * qpitch + v * E, c, isum);
-          if (res != nullptr) {   // keep this CTA's channels of x (S1) / y1 (S3) for the residual
-            const int t16 = (v * E) >> 4;
-            if (t16 % G == b) {
-              const int ti = t16 / G;
-#pragma unroll
-              for (int i = 0; i < E; ++i) res[(ti * 16 + ((v * E + i) & 15)) * 8 + m_row] = V::val(raw[j], i);
-            }
-          }
-        }
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
-      if (lane == 0) sm.red_i[warp] = isum;
-    }
-    __syncthreads();
-    if (tid < M) {
-      constexpr int wpr = kTpr / 32;
-      int t = 0;
-      for (int w = tid * wpr; w < (tid + 1) * wpr; ++w) t += sm.red_i[w];
-      sm.qsum[tid] = t;
-    }
-    __syncthreads();
+    }   // read by the epilogue of a later stage, after several barriers
     if (a.dbg.q[s] != nullptr && b == 0) {   // debug: this stage's codes and scales (one launch, one layer)
       for (int i = tid; i < M * K / 16; i += kThreads) {
         const int m = i / (K / 16), c16 = i - m * (K / 16);
@@ -507,12 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
       else stage_mma<1>(sl, codes, qpitch, M, K, ntl, sm.red);
     }
     __syncthreads();
-    if (warp == 0) {   // the slot is free: refill it `nslot` stages ahead; prefetch further ahead into L2
-      fence_proxy_async_smem();
-      if (q + a.nslot < nq) {
-        fill_slot(a, desc, slots, sm, q + a.nslot, lane);
-        q_issued = q + a.nslot + 1;
-      }
+    if (warp == kWarps - 1) {   // the slot is free: refill it `nslot` stages ahead, prefetch further ahead
+      fence_proxy_async_smem();  // into L2; this warp has no epilogue work (at most 384 outputs per CTA)
+      if (q + a.nslot < nq) fill_slot(a, desc, slots, sm, q + a.nslot, lane);
       if (q + a.nslot + kPrefetchAhead < nq) prefetch_stage(a, desc, q + a.nslot + kPrefetchAhead, lane);
     }
     if (q + a.nslot < nq) q_issued = q + a.nslot + 1;
@@ -520,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
     // ---------------------------------------------------- epilogue: one output element per thread
     if (has_out) {
       const float sc = sm.scale[e_m];
-      const int qs = sm.qsum[e_m];
+      const int qs = block_qsum<MPAD, kThreads>(red, e_m);
       const size_t o_idx = (size_t)e_m * N + e_n;
       const bool skip = b == a.skip_cta && q == 0;   // test hook: one CTA never publishes its first stage
       if (s == 0) {
@@ -579,7 +493,7 @@ bool geometry(int M, int d, int I, int L, int esize, int G, Geom& g) {
   size_t slot = 0;
   for (int s = 0; s < 4; ++s) {
     const StageGeom sg = stage_geom(s, d, I);
-    slot = std::max(slot, (size_t)tiles_of(sg.N, 0, G) * sg.nseg * 16 * (sg.K / 4 + 64));
+    slot = std::max(slot, (size_t)tiles_of(sg.N, 0, G) * sg.nseg * 16 * (sg.K / 4));
   }
   g.slot_bytes = (int)((slot + 127) / 128 * 128);
   const size_t fixed = g.desc_bytes + g.codes_bytes;

@@ -46,6 +46,7 @@ struct ScanSmem {
   static constexpr int CPL = CC / 32;   // channels per lane
   float A[SW][CPL][32];                 // composed multiplier of each warp's steps
   float Bv[SW][CPL][32];                // composed offset
+  float hnext[CPL][32];                 // state leaving the chunk (written by the last warp)
   uint64_t full[kMaxStages];
 };
 template <int CC> constexpr size_t tiles_offset() { return (sizeof(ScanSmem<CC>) + 127) / 128 * 128; }
@@ -64,21 +65,77 @@ __device__ __forceinline__ float rcp_approx(float x) {
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kMaxExp2 = 29.0f * kLog2e;   // e^-z capped at e^29
 
-// The three logistic terms of one channel-step with one reciprocal:
-// with p_x = 1 + e^-x and r = 1 / (p_f p_c p_g),
-//   f = sigmoid(zf) = p_c p_g r,   sigmoid(zc) = p_f p_g r,   g = sigmoid(zg) = p_f p_c r,
-// and b = (1 - f) SiLU(zc) = (1 - f) zc sigmoid(zc). Each exponent is capped at
-// 29 so that the product of the three stays finite ((1 + e^29)^3 < 2^127);
-// below -29 a logistic is under 3e-13 and the cap moves it by less than that.
+// The three logistic terms of one channel-step with one reciprocal: with
+// E_x = e^-x, p_x = 1 + E_x and r = 1 / (p_f p_c p_g),
+//   f = sigmoid(zf) = p_c p_g r,   g = sigmoid(zg) = p_f p_c r,
+//   b = (1 - f) SiLU(zc) = zc (E_f / p_f)(1 / p_c) = zc E_f p_g r.
+// Each exponent is capped at 29 so that the product stays finite
+// ((1 + e^29)^3 < 2^127); below -29 a logistic is under 3e-13 and the cap
+// moves it by less than that.
 __device__ __forceinline__ void gates(float zf, float zc, float zg, float& f, float& b, float& g) {
-  const float pf = 1.0f + ex2_approx(fminf(-zf * kLog2e, kMaxExp2));
+  const float ef = ex2_approx(fminf(-zf * kLog2e, kMaxExp2));
+  const float pf = 1.0f + ef;
   const float pc = 1.0f + ex2_approx(fminf(-zc * kLog2e, kMaxExp2));
   const float pg = 1.0f + ex2_approx(fminf(-zg * kLog2e, kMaxExp2));
-  const float r = rcp_approx(pf * pc * pg);
+  const float pfc = pf * pc;
+  const float r = rcp_approx(pfc * pg);
   f = (pc * pg) * r;
-  g = (pf * pc) * r;
-  b = (1.0f - f) * (zc * ((pf * pg) * r));
+  g = pfc * r;
+  b = ((zc * ef) * pg) * r;
 }
+
+// Two channels at once in packed fp32 pairs (the f32x2 instructions of
+// sm_100a): lane values x (low word) and y (high word).
+struct F2 {
+  unsigned long long v;
+};
+__device__ __forceinline__ F2 f2(float x, float y) {
+  return F2{(unsigned long long)__float_as_uint(x) | ((unsigned long long)__float_as_uint(y) << 32)};
+}
+__device__ __forceinline__ float lo(F2 a) { return __uint_as_float((uint32_t)a.v); }
+__device__ __forceinline__ float hi(F2 a) { return __uint_as_float((uint32_t)(a.v >> 32)); }
+__device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
+  F2 d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d.v) : "l"(a.v), "l"(b.v), "l"(c.v));
+  return d;
+}
+__device__ __forceinline__ F2 mul2(F2 a, F2 b) {
+  F2 d;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ F2 add2(F2 a, F2 b) {
+  F2 d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d.v) : "l"(a.v), "l"(b.v));
+  return d;
+}
+__device__ __forceinline__ F2 ex2_capped(F2 z) {   // e^-z per lane, exponent capped as in gates()
+  const F2 t = mul2(z, f2(-kLog2e, -kLog2e));
+  return f2(ex2_approx(fminf(lo(t), kMaxExp2)), ex2_approx(fminf(hi(t), kMaxExp2)));
+}
+// gates() for a channel pair
+__device__ __forceinline__ void gates2(F2 zf, F2 zc, F2 zg, F2& f, F2& b, F2& g) {
+  const F2 one = f2(1.0f, 1.0f);
+  const F2 ef = ex2_capped(zf);
+  const F2 pf = add2(ef, one);
+  const F2 pc = add2(ex2_capped(zc), one);
+  const F2 pg = add2(ex2_capped(zg), one);
+  const F2 pfc = mul2(pf, pc);
+  const F2 pp = mul2(pfc, pg);
+  const F2 r = f2(rcp_approx(lo(pp)), rcp_approx(hi(pp)));
+  f = mul2(mul2(pc, pg), r);
+  g = mul2(pfc, r);
+  b = mul2(mul2(mul2(zc, ef), pg), r);
+}
+__device__ __forceinline__ F2 load_pair(const bf16* p) {   // two bf16 -> fp32 pair (exact)
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+  return F2{(unsigned long long)(w << 16) | ((unsigned long long)(w & 0xffff0000u) << 32)};
+}
+__device__ __forceinline__ F2 load_pair(const float* p) { return F2{*reinterpret_cast<const unsigned long long*>(p)}; }
+__device__ __forceinline__ void store_pair(bf16* p, F2 v) {
+  *reinterpret_cast<__nv_bfloat162*>(p) = __floats2bfloat162_rn(lo(v), hi(v));
+}
+__device__ __forceinline__ void store_pair(float* p, F2 v) { *reinterpret_cast<unsigned long long*>(p) = v.v; }
 
 template <int CPL> struct Lane;
 template <> struct Lane<2> {   // two adjacent channels per lane
@@ -175,75 +232,112 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     const int t0 = j * TC;
     const T(*tile)[TC][CC] = ring[s];
-
-    // 1. gates and this warp's composed map
-    float f[LS][CPL], bb[LS][CPL], gg[LS][CPL];
-    float Aa[CPL], Bb[CPL];
+    const bool full = t0 + TC <= T_;   // every step of the chunk is inside the sequence
+    T* op = o + ((size_t)b * T_ + t0 + warp * LS) * d + ch;
+    if constexpr (CPL == 2) {
+      // 1. gates and this warp's composed map, two channels per lane in packed pairs
+      F2 f[LS], bb[LS], gg[LS];
+      F2 Aa = f2(1.0f, 1.0f), Bb = f2(0.0f, 0.0f);
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      Aa[c] = 1.0f;
-      Bb[c] = 0.0f;
-    }
+      for (int k = 0; k < LS; ++k) {
+        const int tl = warp * LS + k;
+        if (full || t0 + tl < T_) {
+          gates2(load_pair(&tile[0][tl][2 * lane]), load_pair(&tile[1][tl][2 * lane]),
+                 load_pair(&tile[2][tl][2 * lane]), f[k], bb[k], gg[k]);
+        } else {   // past the end of the sequence: identity map
+          f[k] = f2(1.0f, 1.0f);
+          bb[k] = f2(0.0f, 0.0f);
+          gg[k] = f2(0.0f, 0.0f);
+        }
+        Bb = fma2(f[k], Bb, bb[k]);
+        Aa = mul2(Aa, f[k]);
+      }
+      sm.A[warp][0][lane] = lo(Aa);
+      sm.A[warp][1][lane] = hi(Aa);
+      sm.Bv[warp][0][lane] = lo(Bb);
+      sm.Bv[warp][1][lane] = hi(Bb);
+      __syncthreads();
+      // 2. this warp's entering state (the maps of the warps before it); the
+      //    last warp also gets the state leaving the chunk
+      F2 hw = f2(hin[0], hin[1]);
+      for (int w = 0; w < warp; ++w)
+        hw = fma2(f2(sm.A[w][0][lane], sm.A[w][1][lane]), hw, f2(sm.Bv[w][0][lane], sm.Bv[w][1][lane]));
+      if (warp == SW - 1) {
+        const F2 hn = fma2(Aa, hw, Bb);
+        sm.hnext[0][lane] = lo(hn);
+        sm.hnext[1][lane] = hi(hn);
+      }
+      // 3. replay this warp's steps and store o'
+      if (valid) {
 #pragma unroll
-    for (int k = 0; k < LS; ++k) {
-      const int tl = warp * LS + k;
-      if (t0 + tl < T_) {
-        float zf[CPL], zc[CPL], zg[CPL];
-        LN::load(&tile[0][tl][lane * CPL], zf);
-        LN::load(&tile[1][tl][lane * CPL], zc);
-        LN::load(&tile[2][tl][lane * CPL], zg);
+        for (int k = 0; k < LS; ++k) {
+          hw = fma2(f[k], hw, bb[k]);
+          if (full || t0 + warp * LS + k < T_) store_pair(op + (size_t)k * d, mul2(gg[k], hw));
+        }
+      }
+    } else {
+      // 1. gates and this warp's composed map
+      float f[LS][CPL], bb[LS][CPL], gg[LS][CPL];
+      float Aa[CPL], Bb[CPL];
 #pragma unroll
-        for (int c = 0; c < CPL; ++c) gates(zf[c], zc[c], zg[c], f[k][c], bb[k][c], gg[k][c]);
-      } else {   // past the end of the sequence: identity map
+      for (int c = 0; c < CPL; ++c) {
+        Aa[c] = 1.0f;
+        Bb[c] = 0.0f;
+      }
+#pragma unroll
+      for (int k = 0; k < LS; ++k) {
+        const int tl = warp * LS + k;
+        if (full || t0 + tl < T_) {
+          float zf[CPL], zc[CPL], zg[CPL];
+          LN::load(&tile[0][tl][lane * CPL], zf);
+          LN::load(&tile[1][tl][lane * CPL], zc);
+          LN::load(&tile[2][tl][lane * CPL], zg);
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) gates(zf[c], zc[c], zg[c], f[k][c], bb[k][c], gg[k][c]);
+        } else {   // past the end of the sequence: identity map
+#pragma unroll
+          for (int c = 0; c < CPL; ++c) {
+            f[k][c] = 1.0f;
+            bb[k][c] = 0.0f;
+            gg[k][c] = 0.0f;
+          }
+        }
 #pragma unroll
         for (int c = 0; c < CPL; ++c) {
-          f[k][c] = 1.0f;
-          bb[k][c] = 0.0f;
-          gg[k][c] = 0.0f;
+          Bb[c] = fmaf(f[k][c], Bb[c], bb[k][c]);
+          Aa[c] *= f[k][c];
         }
       }
 #pragma unroll
       for (int c = 0; c < CPL; ++c) {
-        Bb[c] = fmaf(f[k][c], Bb[c], bb[k][c]);
-        Aa[c] *= f[k][c];
+        sm.A[warp][c][lane] = Aa[c];
+        sm.Bv[warp][c][lane] = Bb[c];
+      }
+      __syncthreads();
+      // 2. as above, one channel per lane
+      float hw[CPL];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        float hv = hin[c];
+        for (int w = 0; w < warp; ++w) hv = fmaf(sm.A[w][c][lane], hv, sm.Bv[w][c][lane]);
+        hw[c] = hv;
+        if (warp == SW - 1) sm.hnext[c][lane] = fmaf(Aa[c], hv, Bb[c]);
+      }
+      // 3. replay this warp's steps and store o'
+#pragma unroll
+      for (int k = 0; k < LS; ++k) {
+        float out[CPL];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) {
+          hw[c] = fmaf(f[k][c], hw[c], bb[k][c]);
+          out[c] = gg[k][c] * hw[c];
+        }
+        if (valid && (full || t0 + warp * LS + k < T_)) LN::store(op + (size_t)k * d, out);
       }
     }
+    __syncthreads();   // the stage and the warps' maps are free again; hnext is written
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      sm.A[warp][c][lane] = Aa[c];
-      sm.Bv[warp][c][lane] = Bb[c];
-    }
-    __syncthreads();
-
-    // 2. this warp's entering state and the chunk's leaving state, from the chunk's entering state
-    float hw[CPL], hout[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      float hv = hin[c];
-      for (int w = 0; w < SW; ++w) {
-        if (w == warp) hw[c] = hv;
-        hv = fmaf(sm.A[w][c][lane], hv, sm.Bv[w][c][lane]);
-      }
-      hout[c] = hv;
-    }
-
-    // 3. replay this warp's steps and store o'
-    T* op = o + ((size_t)b * T_ + t0 + warp * LS) * d + ch;
-#pragma unroll
-    for (int k = 0; k < LS; ++k) {
-      const int tl = warp * LS + k;
-      float out[CPL];
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) hw[c] = fmaf(f[k][c], hw[c], bb[k][c]);
-      if (valid && t0 + tl < T_) {
-#pragma unroll
-        for (int c = 0; c < CPL; ++c) out[c] = gg[k][c] * hw[c];
-        LN::store(op + (size_t)k * d, out);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) hin[c] = hout[c];
-    __syncthreads();   // the stage and the warps' maps are free again
+    for (int c = 0; c < CPL; ++c) hin[c] = sm.hnext[c][lane];
     if (threadIdx.x == 0 && j + nst < nchunk) {
       fence_proxy_async_smem();
       issue(j + nst);

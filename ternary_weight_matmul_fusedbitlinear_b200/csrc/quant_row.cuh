@@ -165,45 +165,66 @@ namespace mmf {
 // most MPAD rows; NT threads, NT / MPAD >= 32 threads per row). Thread t works
 // on row t / (NT / MPAD) and holds that row's 16-byte vectors lt, lt + tpr, ...
 // (lt = t % tpr, tpr = NT / MPAD) in raw[j] for every bit j set in `have`. The
-// row's fp64 sum of squares and its max are reduced over the row's warps in a
-// fixed order, so every CTA that quantises the same rows gets the same scale;
-// the fp32 steps are those of quant_row. Codes go to codes + m * qpitch (16-byte
-// aligned rows); scale[m], qsum[m] (shared) get the row's scale and code sum.
-// `red` is shared scratch of at least NT / 32 entries of each type. Contains
+// row's fp64 sum of squares and its max are reduced in a fixed order (lanes by
+// an xor-shuffle tree, then the row's warps by a shuffle tree), so every CTA
+// that quantises the same rows gets the same scale; every warp of a row folds
+// the row's partials itself, so no thread waits for another's fold. The fp32
+// steps are those of quant_row. Codes go to codes + m * qpitch (16-byte aligned
+// rows) and scale[m] gets the row's scale. The code sums are left as per-warp
+// partials in red.i: block_qsum() folds them after the caller's next barrier.
+// `red` is shared scratch of NT / 32 entries of each type. Contains
 // __syncthreads(): every thread of the block calls it.
 struct BlockRed {
   double* d;
   uint32_t* u;
   int* i;
-  float* rinv;   // [MPAD]
 };
+
+// Fold a row's kWpr per-warp partials (red[w0 .. w0 + kWpr)) in a fixed tree
+// order; every lane gets the result.
+template <int kWpr, typename V, typename Op>
+__device__ __forceinline__ V fold_row(const V* red, int w0, int lane, V zero, Op op) {
+  V v = lane < kWpr ? red[w0 + lane] : zero;
+#pragma unroll
+  for (int o = kWpr / 2; o > 0; o >>= 1) {
+    const V other = __shfl_down_sync(0xffffffffu, v, o);
+    if (lane < o) v = op(v, other);
+  }
+  return __shfl_sync(0xffffffffu, v, 0);
+}
 
 template <typename T, int MPAD, int NT, int VMAX>
 __device__ __forceinline__ void block_quant(const uint4 (&raw)[VMAX], uint32_t have, int M, int K,
                                             const float* __restrict__ gain, float eps, int8_t* codes, int qpitch,
-                                            float* scale, int* qsum, const BlockRed& red) {
+                                            float* scale, const BlockRed& red) {
   using V = Vec<T>;
   constexpr int E = V::E;
   constexpr int kTpr = NT / MPAD;
   constexpr int kWpr = kTpr / 32;
-  static_assert(kTpr >= 32, "at least one warp per row");
+  static_assert(kTpr >= 32 && (kWpr & (kWpr - 1)) == 0, "a power-of-two number of warps per row");
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int m_row = tid / kTpr, lt = tid - m_row * kTpr;
+  const int w0 = m_row * kWpr;
   const bool row_ok = m_row < M;
-  {   // sum of squares (fp64) and max |x|
-    double ss = 0.0;
+  // A thread's slots are a prefix of 0..VMAX-1 (vector lt + tpr j is in the row
+  // for every j below some bound), so the unrolled loops stop at the first
+  // empty slot instead of running predicated bodies for all VMAX slots.
+  {   // sum of squares (fp64, two chains: even and odd elements) and max |x|
+    double s0 = 0.0, s1 = 0.0;
     uint32_t am = 0;
 #pragma unroll
-    for (int j = 0; j < VMAX; ++j)
-      if (have & (1u << j)) {
+    for (int j = 0; j < VMAX; ++j) {
+      if (!(have & (1u << j))) break;
 #pragma unroll
-        for (int i = 0; i < E; ++i) {
-          const uint32_t mg = V::mag(raw[j], i);
-          am = max(am, mg);
-          const double xd = magbits_to_f64(mg);
-          ss = fma(xd, xd, ss);
-        }
+      for (int i = 0; i < E; ++i) {
+        const uint32_t mg = V::mag(raw[j], i);
+        am = max(am, mg);
+        const double xd = magbits_to_f64(mg);
+        if (i & 1) s1 = fma(xd, xd, s1);
+        else s0 = fma(xd, xd, s0);
       }
+    }
+    double ss = s0 + s1;
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
     am = __reduce_max_sync(0xffffffffu, am);
@@ -213,70 +234,63 @@ __device__ __forceinline__ void block_quant(const uint4 (&raw)[VMAX], uint32_t h
     }
   }
   __syncthreads();
-  if (tid < M) {   // per row, its warps in order
-    double t = 0.0;
-    uint32_t mx = 0;
-    for (int w = tid * kWpr; w < (tid + 1) * kWpr; ++w) {
-      t += red.d[w];
-      mx = max(mx, red.u[w]);
-    }
-    const float ms = (float)(t / (double)K);
-    const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
-    red.rinv[tid] = rinv;
-    if (gain == nullptr)   // rounding is monotone: fl(max|x| * rinv) = max fl(|x| * rinv)
-      scale[tid] = __fdiv_rn(127.0f, fmaxf(__fmul_rn(__uint_as_float(mx), rinv), 1e-5f));
-  }
-  __syncthreads();
-  const float rinv = row_ok ? red.rinv[m_row] : 0.0f;
-  if (gain != nullptr) {   // max |(x * rinv) * gain|
+  const double tot = fold_row<kWpr>(red.d, w0, lane, 0.0, [](double x, double y) { return x + y; });
+  const uint32_t mx = fold_row<kWpr>(red.u, w0, lane, 0u, [](uint32_t x, uint32_t y) { return max(x, y); });
+  const float ms = (float)(tot / (double)K);
+  const float rinv = __frcp_rn(__fsqrt_rn(__fadd_rn(ms, eps)));
+  float sc;
+  if (gain == nullptr) {   // rounding is monotone: fl(max|x| * rinv) = max fl(|x| * rinv)
+    sc = __fdiv_rn(127.0f, fmaxf(__fmul_rn(__uint_as_float(mx), rinv), 1e-5f));
+  } else {   // max |(x * rinv) * gain|
     uint32_t hm = 0;
 #pragma unroll
-    for (int j = 0; j < VMAX; ++j)
-      if (have & (1u << j)) {
-        const int k0 = (lt + kTpr * j) * E;
+    for (int j = 0; j < VMAX; ++j) {
+      if (!(have & (1u << j))) break;
+      const int k0 = (lt + kTpr * j) * E;
 #pragma unroll
-        for (int i = 0; i < E; ++i) {
-          const float hv = __fmul_rn(__fmul_rn(V::val(raw[j], i), rinv), __ldg(gain + k0 + i));
-          hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
-        }
+      for (int i = 0; i < E; ++i) {
+        const float hv = __fmul_rn(__fmul_rn(V::val(raw[j], i), rinv), __ldg(gain + k0 + i));
+        hm = max(hm, __float_as_uint(hv) & 0x7fffffffu);
       }
+    }
     hm = __reduce_max_sync(0xffffffffu, hm);
+    __syncthreads();   // every warp has read the first partials
     if (lane == 0) red.u[warp] = hm;
     __syncthreads();
-    if (tid < M) {
-      uint32_t mx = 0;
-      for (int w = tid * kWpr; w < (tid + 1) * kWpr; ++w) mx = max(mx, red.u[w]);
-      scale[tid] = __fdiv_rn(127.0f, fmaxf(__uint_as_float(mx), 1e-5f));
-    }
-    __syncthreads();
+    const uint32_t gm = fold_row<kWpr>(red.u, w0, lane, 0u, [](uint32_t x, uint32_t y) { return max(x, y); });
+    sc = __fdiv_rn(127.0f, fmaxf(__uint_as_float(gm), 1e-5f));
   }
-  {   // codes and their sum
-    const float sc = row_ok ? scale[m_row] : 0.0f;
+  if (row_ok && lt == 0) scale[m_row] = sc;
+  {   // codes and this warp's part of their sum
     int isum = 0;
 #pragma unroll
-    for (int j = 0; j < VMAX; ++j)
-      if (have & (1u << j)) {
-        const int v = lt + kTpr * j;
-        uint32_t c[E];
+    for (int j = 0; j < VMAX; ++j) {
+      if (!(have & (1u << j))) break;
+      const int v = lt + kTpr * j;
+      uint32_t c[E];
 #pragma unroll
-        for (int i = 0; i < E; ++i) {
-          float hv = __fmul_rn(V::val(raw[j], i), rinv);
-          if (gain != nullptr) hv = __fmul_rn(hv, __ldg(gain + v * E + i));
-          c[i] = rint_bits(__fmul_rn(hv, sc));
-        }
-        V::store_codes(codes + (size_t)m_row * qpitch + v * E, c, isum);
+      for (int i = 0; i < E; ++i) {
+        float hv = __fmul_rn(V::val(raw[j], i), rinv);
+        if (gain != nullptr) hv = __fmul_rn(hv, __ldg(gain + v * E + i));
+        c[i] = rint_bits(__fmul_rn(hv, sc));
       }
+      V::store_codes(codes + (size_t)m_row * qpitch + v * E, c, isum);
+    }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) isum += __shfl_xor_sync(0xffffffffu, isum, o);
     if (lane == 0) red.i[warp] = isum;
   }
   __syncthreads();
-  if (tid < M) {
-    int t = 0;
-    for (int w = tid * kWpr; w < (tid + 1) * kWpr; ++w) t += red.i[w];
-    qsum[tid] = t;
-  }
-  __syncthreads();
+}
+
+// Code sum of row m from block_quant's per-warp partials (any thread, after block_quant).
+template <int MPAD, int NT>
+__device__ __forceinline__ int block_qsum(const BlockRed& red, int m) {
+  constexpr int kWpr = NT / MPAD / 32;
+  int t = 0;
+#pragma unroll
+  for (int w = 0; w < kWpr; ++w) t += red.i[m * kWpr + w];
+  return t;
 }
 
 }  // namespace mmf

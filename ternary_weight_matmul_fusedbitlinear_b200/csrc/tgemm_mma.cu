@@ -124,7 +124,6 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
     __shared__ double red_d[kWarps];
     __shared__ uint32_t red_u[kWarps];
     __shared__ int red_i[kWarps];
-    __shared__ float red_r[FQM];
     constexpr int kTpr = kThreads / FQM;
     const int m_row = threadIdx.x / kTpr, lt = threadIdx.x - m_row * kTpr;
     const int nvec = (int)(K * sizeof(T) / 16);
@@ -137,11 +136,13 @@ __global__ void __launch_bounds__(kThreads) tgemm_mma_kernel(TGemmArgs a) {
       raw[j] = make_uint4(0u, 0u, 0u, 0u);
       if (m_row < M && v < nvec) {
         have |= 1u << j;
-        raw[j] = __ldg(xg + v);
+        raw[j] = __ldcg(xg + v);   // coherent: the previous kernel may have written x while this one started
       }
     }
-    block_quant<T, FQM, kThreads, kFqVmax>(raw, have, M, K, a.gain, a.eps, qs, qpitch, s_sm, qsum_sm,
-                                           BlockRed{red_d, red_u, red_i, red_r});
+    const BlockRed red{red_d, red_u, red_i};
+    block_quant<T, FQM, kThreads, kFqVmax>(raw, have, M, K, a.gain, a.eps, qs, qpitch, s_sm, red);
+    if (threadIdx.x < M) qsum_sm[threadIdx.x] = block_qsum<FQM, kThreads>(red, threadIdx.x);
+    __syncthreads();
     if (blockIdx.x == 0 && a.q_out != nullptr) {   // one CTA also hands the codes out
       for (int i = threadIdx.x; i < M * K / 16; i += kThreads) {
         const int m = i / (K / 16), c16 = i - m * (K / 16);
