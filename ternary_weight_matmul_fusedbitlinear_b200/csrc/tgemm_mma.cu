@@ -373,12 +373,15 @@ cudaError_t launch_nt(const TGemmArgs& a, Epi epi, cudaStream_t stream) {
   return cudaErrorInvalidValue;
 }
 
+// At most 32 tokens per CTA: above that a second grid row takes the next 32
+// tokens and reads the same weight slice again (from L2). A 64-token CTA would
+// keep eight token tiles of fragments and its accumulators in registers and
+// spill (the f|c|g step needs 255 registers).
 template <typename T>
 cudaError_t launch_t(const TGemmArgs& a, Epi epi, cudaStream_t stream) {
   if (a.M <= 8) return launch_nt<1, T>(a, epi, stream);
   if (a.M <= 16) return launch_nt<2, T>(a, epi, stream);
-  if (a.M <= 32) return launch_nt<4, T>(a, epi, stream);
-  return launch_nt<8, T>(a, epi, stream);
+  return launch_nt<4, T>(a, epi, stream);
 }
 
 }  // namespace

@@ -105,7 +105,10 @@ def test_bitlinear_zero_rows():
 # ------------------------------------------------------------------ MLGRU scan
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-@pytest.mark.parametrize("b,t,d", [(2, 64, 256), (1, 3, 16), (3, 200, 264), (8, 1, 1024), (4, 517, 2048)])
+# (8, 300, 2560) has enough 64-channel blocks to fill every SM twice: the
+# 64-channel variant; the others run 32-channel CTAs, two per SM
+@pytest.mark.parametrize("b,t,d", [(2, 64, 256), (1, 3, 16), (3, 200, 264), (8, 1, 1024), (4, 517, 2048),
+                                   (8, 300, 2560)])
 def test_scan_parity(b, t, d, dtype):
     pre = synth.preacts(400 + t, b, t, d, TORCH_DT[dtype], scale=2.0)
     h0 = synth.activations(401, b, d)
