@@ -142,7 +142,18 @@ __device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
   asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
+// This CTA's share of one stage type (S0..S3 repeat in every layer), worked
+// out once at kernel start so that no integer division sits on the chain.
+struct StagePlan {
+  int ntl;                 // 16-row tiles of each segment (tiles b, b + G, ...)
+  int nk;                  // 128-column units per row
+  short a0[kWarps];        // warp w's units: segment a0, column block c0, n units (segment-major)
+  short c0[kWarps];
+  short n[kWarps];
+};
+
 struct Smem {
+  StagePlan plan[4];
   int red[kDecodeTiles][3][16][8];      // per tile, segment, row, token: exact int32 partial sums
   double red_d[kWarps];
   uint32_t red_u[kWarps];
@@ -157,12 +168,14 @@ struct Smem {
 
 // One warp: start the bulk copies of stage q's weight slice into its ring slot.
 // A 16-row tile of one matrix is contiguous in memory (rows of K/4 bytes), so
-// each (tile, segment) is one copy, landing as 16 dense rows.
+// each (tile, segment) is one copy, landing as 16 dense rows. (A copy per row,
+// to pad the rows in shared memory, floods the SM's memory pipeline with copy
+// instructions and stalls the stores and loads of the chain behind them.)
 __device__ void fill_slot(const DecodeStepArgs& a, const DecodeLayerDesc* desc, uint8_t* slots, Smem& sm, int q,
                           int lane) {
   const int l = q >> 2, s = q & 3;
   const StageGeom g = stage_geom(s, a.d, a.I);
-  const int ntl = tiles_of(g.N, blockIdx.x, gridDim.x);
+  const int ntl = sm.plan[s].ntl;
   const int tile_bytes = 16 * (g.K / 4);
   const int slot = q % a.nslot;
   uint8_t* dst0 = slots + (size_t)slot * a.slot_bytes;
@@ -172,7 +185,7 @@ __device__ void fill_slot(const DecodeStepArgs& a, const DecodeLayerDesc* desc, 
     else mbar_arrive(&sm.slot_bar[slot]);
   }
   __syncwarp();
-  for (int i = lane; i < ncopy; i += 32) {
+  for (int i = lane; i < ncopy; i += 32) {   // i = tile * nseg + segment
     const int ti = i / g.nseg, r = i - ti * g.nseg;
     const int t = blockIdx.x + ti * gridDim.x;
     const uint8_t* src = reinterpret_cast<const uint8_t*>(desc[l].w[g.mat0 + r]) + (size_t)t * tile_bytes;
@@ -180,11 +193,11 @@ __device__ void fill_slot(const DecodeStepArgs& a, const DecodeLayerDesc* desc, 
   }
 }
 
-// Warp 0: prefetch stage q's weight slice into L2.
-__device__ void prefetch_stage(const DecodeStepArgs& a, const DecodeLayerDesc* desc, int q, int lane) {
+// One warp: prefetch stage q's weight slice into L2.
+__device__ void prefetch_stage(const DecodeStepArgs& a, const DecodeLayerDesc* desc, const Smem& sm, int q, int lane) {
   const int l = q >> 2, s = q & 3;
   const StageGeom g = stage_geom(s, a.d, a.I);
-  const int ntl = tiles_of(g.N, blockIdx.x, gridDim.x);
+  const int ntl = sm.plan[s].ntl;
   const int rowb = g.K / 4;
   for (int i = lane; i < ntl * g.nseg; i += 32) {
     const int ti = i / g.nseg, r = i - ti * g.nseg;
@@ -194,53 +207,75 @@ __device__ void prefetch_stage(const DecodeStepArgs& a, const DecodeLayerDesc* d
 }
 
 // Accumulate this CTA's tiles of one stage into red[ti][r][row][token].
-template <int R>
-__device__ __forceinline__ void stage_mma(const uint4* slot, const int8_t* qs, int qpitch, int M, int K, int ntl,
-                                          int (*red)[3][16][8]) {
+//
+// The stored code c = w + 1 of column 16 j + 4 p + b sits at bits 8 b + 2 p of
+// packed word j, so word & (0x03030303 << 2 p) holds c 4^p in byte b: one
+// logic operation per 4 codes and no shift. Each field position p
+// accumulates into its own sums, which are multiples of 4^p and are scaled
+// back exactly by an arithmetic shift: acc = sum_p (chain_p >> 2 p).
+// m16n8k32 MMAs take rows g and g + 8 of a tile segment against tokens 2 t,
+// 2 t + 1. A unit is 128 columns of a segment (the lane's two packed words of
+// each of the two rows) and four MMAs, one per field position; consecutive
+// units go to two sets of chains so that two MMAs of a chain are never back to
+// back. Warp w takes the contiguous units [w U / 16, (w + 1) U / 16) of the
+// segment-major order (the stage plan), so every warp gets an equal share
+// whatever the CTA's tile count.
+__device__ __forceinline__ void mma_unit(int (&acc)[4][4], const uint8_t* wrow, int rowb, const int8_t* qrow, int c,
+                                         int K, int t, bool tok) {
+  const bool kin = c * 128 + t * 32 < K;   // K % 64 == 0: a last unit of 64 columns uses lanes t < 2
+  uint2 wa = make_uint2(0u, 0u), wb = wa;
+  uint4 x0 = make_uint4(0u, 0u, 0u, 0u), x1 = x0;
+  if (kin) {
+    wa = *reinterpret_cast<const uint2*>(wrow + c * 32);
+    wb = *reinterpret_cast<const uint2*>(wrow + (size_t)8 * rowb + c * 32);
+    if (tok) {   // token g's codes of the lane's two words
+      x0 = *reinterpret_cast<const uint4*>(qrow + c * 128);
+      x1 = *reinterpret_cast<const uint4*>(qrow + c * 128 + 16);
+    }
+  }
+#pragma unroll
+  for (int p = 0; p < 4; ++p) {
+    const uint32_t m = kLow2 << (2 * p);
+    mma_u8s8(acc[p], wa.x & m, wb.x & m, wa.y & m, wb.y & m, u4get(x0, p), u4get(x1, p));
+  }
+}
+
+// Tile of segment index a of a stage with nseg segments per tile (a < 9, nseg <= 3), without a division.
+__device__ __forceinline__ int seg_tile(int a, int nseg) { return nseg == 1 ? a : (nseg == 2 ? a >> 1 : (a * 11) >> 5); }
+
+__device__ __forceinline__ void stage_mma(const uint8_t* slot, const int8_t* qs, int qpitch, int M, int K,
+                                          const StagePlan& pl, int nseg, int (*red)[3][16][8]) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
-  const int wpr = K / 16, nkseg = ceil_div(K, 256);
-  const int pitch4 = K / 64;   // dense rows of K/4 bytes
-  for (int item = warp; item < ntl * nkseg; item += kWarps) {
-    const int ti = item / nkseg, seg = item - ti * nkseg;
-    const int w0 = seg * 16 + 4 * t;   // first packed word of this lane
-    const bool in = w0 < wpr;          // wpr % 4 == 0: a 16-byte group is all in or all out
-    uint4 wa[R], wb[R];
+  const int rowb = K / 4, nk = pl.nk;
+  const bool tok = g < M;
+  const int8_t* qrow = qs + (size_t)(tok ? g : 0) * qpitch + t * 32;
+  int left = pl.n[warp], c0 = pl.c0[warp];
+  for (int a = pl.a0[warp]; left > 0; ++a, c0 = 0) {   // the tile segments this warp's units touch
+    const int c1 = min(nk, c0 + left);
+    left -= c1 - c0;
+    const uint8_t* wrow = slot + ((size_t)a * 16 + g) * rowb + t * 8;
+    int acc0[4][4], acc1[4][4];
 #pragma unroll
-    for (int r = 0; r < R; ++r) {
-      const uint4* base = slot + (size_t)((ti * R + r) * 16) * pitch4 + (w0 >> 2);
-      wa[r] = in ? base[(size_t)g * pitch4] : make_uint4(0u, 0u, 0u, 0u);
-      wb[r] = in ? base[(size_t)(g + 8) * pitch4] : make_uint4(0u, 0u, 0u, 0u);
+    for (int p = 0; p < 4; ++p)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc0[p][e] = acc1[p][e] = 0;
+    int c = c0;
+    for (; c + 1 < c1; c += 2) {
+      mma_unit(acc0, wrow, rowb, qrow, c, K, t, tok);
+      mma_unit(acc1, wrow, rowb, qrow, c + 1, K, t, tok);
     }
-    uint4 act[4];
+    if (c < c1) mma_unit(acc0, wrow, rowb, qrow, c, K, t, tok);
+    const int ti = seg_tile(a, nseg), r = a - ti * nseg;
 #pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      const bool ok = (g < M) && (w0 + u < wpr);
-      act[u] = ok ? *reinterpret_cast<const uint4*>(qs + (size_t)g * qpitch + (w0 + u) * 16)
-                  : make_uint4(0u, 0u, 0u, 0u);
-    }
-    int acc[R][2][4];   // two accumulator chains per segment (even / odd k-steps): half the MMA latency chain
+    for (int e = 0; e < 4; ++e) {
+      const int col = 2 * t + (e & 1);
+      if (col < M) {
+        int v = 0;
 #pragma unroll
-    for (int r = 0; r < R; ++r)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[r][0][e] = acc[r][1][e] = 0;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const int u = i >> 1, sub = (i & 1) * 2;
-      const uint32_t b0 = u4get(act[u], sub), b1 = u4get(act[u], sub + 1);
-#pragma unroll
-      for (int r = 0; r < R; ++r) {
-        const uint32_t wg = u4get(wa[r], u), wg8 = u4get(wb[r], u);
-        mma_u8s8(acc[r][i & 1], (wg >> (2 * sub)) & kLow2, (wg8 >> (2 * sub)) & kLow2,
-                 (wg >> (2 * sub + 2)) & kLow2, (wg8 >> (2 * sub + 2)) & kLow2, b0, b1);
+        for (int p = 0; p < 4; ++p) v += (acc0[p][e] + acc1[p][e]) >> (2 * p);
+        atomicAdd(&red[ti][r][g + 8 * (e >> 1)][col], v);
       }
-    }
-#pragma unroll
-    for (int r = 0; r < R; ++r) {
-      atomicAdd(&red[ti][r][g][2 * t], acc[r][0][0] + acc[r][1][0]);
-      atomicAdd(&red[ti][r][g][2 * t + 1], acc[r][0][1] + acc[r][1][1]);
-      atomicAdd(&red[ti][r][g + 8][2 * t], acc[r][0][2] + acc[r][1][2]);
-      atomicAdd(&red[ti][r][g + 8][2 * t + 1], acc[r][0][3] + acc[r][1][3]);
     }
   }
 }
@@ -288,13 +323,27 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
     for (int i = tid; i < L * kWords; i += kThreads)
       reinterpret_cast<uint64_t*>(desc)[i] = reinterpret_cast<const uint64_t*>(a.layer[i / kWords])[i % kWords];
   }
+  if (tid < 4 * kWarps) {   // the stage plans: thread 16 s + w works out warp w's units of stage type s
+    const int ps = tid / kWarps, pw = tid % kWarps;
+    const StageGeom pg = stage_geom(ps, d, I);
+    const int ntl = tiles_of(pg.N, b, G), nk = ceil_div(pg.K, 128);
+    const int total = ntl * pg.nseg * nk;
+    const int u0 = pw * total / kWarps, u1 = (pw + 1) * total / kWarps;
+    sm.plan[ps].a0[pw] = (short)(u0 / nk);
+    sm.plan[ps].c0[pw] = (short)(u0 % nk);
+    sm.plan[ps].n[pw] = (short)(u1 - u0);
+    if (pw == 0) {
+      sm.plan[ps].ntl = ntl;
+      sm.plan[ps].nk = nk;
+    }
+  }
   __syncthreads();
   for (int i = tid; i < L * 7; i += kThreads) sm.gam[i / 7][i % 7] = *desc[i / 7].gamma[i % 7];
   // the weight stream does not depend on the previous kernel: start it first
   int q_issued = 0;   // stages whose ring fill has been issued
   if (warp == kWarps - 1) {
     for (int q = 0; q < a.nslot && q < nq; ++q) fill_slot(a, desc, slots, sm, q, lane);
-    for (int q = a.nslot; q < a.nslot + kPrefetchAhead && q < nq; ++q) prefetch_stage(a, desc, q, lane);
+    for (int q = a.nslot; q < a.nslot + kPrefetchAhead && q < nq; ++q) prefetch_stage(a, desc, sm, q, lane);
   }
   q_issued = a.nslot < nq ? a.nslot : nq;
   pdl_wait();
@@ -303,12 +352,16 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
 
   const int m_row = tid / kTpr, lt = tid - m_row * kTpr;   // quantisation: this thread's token row
   const bool row_ok = m_row < M;
+  // epilogue: thread tid owns output row e_row of tile e_ti for token e_m (tid < ntl 16 M)
+  const int e_ti = tid / (16 * M), e_rem = tid - e_ti * 16 * M;
+  const int e_m = e_rem >> 4, e_row = e_rem & 15;
+  const int e_n = (b + e_ti * G) * 16 + e_row;
 
   for (int q = 0; q < nq; ++q) {
     const int l = q >> 2, s = q & 3;
     const StageGeom g = stage_geom(s, d, I);
     const DecodeLayerDesc& D = desc[l];
-    const int ntl = tiles_of(g.N, b, G);
+    const int ntl = sm.plan[s].ntl;
     const int par = (int)sm.par[l];
     const int K = g.K, N = g.N;
     for (int i = tid; i < kDecodeTiles * 3 * 16 * 8; i += kThreads) (&sm.red[0][0][0][0])[i] = 0;
@@ -316,9 +369,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
     // ---------------------------------------------------- epilogue operands that need no input row
     const int nout = ntl * 16 * M;
     const bool has_out = tid < nout;
-    const int e_ti = tid / (16 * M), e_rem = tid - e_ti * 16 * M;
-    const int e_m = e_rem >> 4, e_row = e_rem & 15;
-    const int e_n = (b + e_ti * G) * 16 + e_row;
     float* hp = a.h + ((size_t)(a.layer0 + l) * M + e_m) * d + e_n;
     float hval = 0.0f, bias[3] = {0.0f, 0.0f, 0.0f};
     if (has_out) {
@@ -387,9 +437,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
       for (int j = 0; j < kVmax; ++j) {
         if (!(have & (1u << j))) break;
         const int v = lt + kTpr * j;
-        const int t16 = (v * E) >> 4;
-        if (t16 % G == b) {
-          const int ti = t16 / G;
+        const int t16 = (v * E) >> 4;   // this CTA's tiles are b, b + G, b + 2 G (d <= 48 G)
+        const int ti = t16 == b ? 0 : (t16 == b + G ? 1 : (t16 == b + 2 * G ? 2 : -1));
+        if (ti >= 0) {
 #pragma unroll
           for (int i = 0; i < E; ++i) res[(ti * 16 + ((v * E + i) & 15)) * 8 + m_row] = V::val(raw[j], i);
         }
@@ -418,16 +468,13 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
         give_up(a, sm, 6, q, q_issued);
         return;
       }
-      const uint4* sl = reinterpret_cast<const uint4*>(slots + (size_t)slot * a.slot_bytes);
-      if (g.nseg == 3) stage_mma<3>(sl, codes, qpitch, M, K, ntl, sm.red);
-      else if (g.nseg == 2) stage_mma<2>(sl, codes, qpitch, M, K, ntl, sm.red);
-      else stage_mma<1>(sl, codes, qpitch, M, K, ntl, sm.red);
+      stage_mma(slots + (size_t)slot * a.slot_bytes, codes, qpitch, M, K, sm.plan[s], g.nseg, sm.red);
     }
     __syncthreads();
     if (warp == kWarps - 1) {   // the slot is free: refill it `nslot` stages ahead, prefetch further ahead
       fence_proxy_async_smem();  // into L2; this warp has no epilogue work (at most 384 outputs per CTA)
       if (q + a.nslot < nq) fill_slot(a, desc, slots, sm, q + a.nslot, lane);
-      if (q + a.nslot + kPrefetchAhead < nq) prefetch_stage(a, desc, q + a.nslot + kPrefetchAhead, lane);
+      if (q + a.nslot + kPrefetchAhead < nq) prefetch_stage(a, desc, sm, q + a.nslot + kPrefetchAhead, lane);
     }
     if (q + a.nslot < nq) q_issued = q + a.nslot + 1;
 

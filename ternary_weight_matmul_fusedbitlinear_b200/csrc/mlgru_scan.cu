@@ -86,13 +86,13 @@ __device__ __forceinline__ F2 f2(float x, float y) {
   return r;
 }
 __device__ __forceinline__ float lo(F2 a) {
-  float x, y;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(a.v));
+  float x;
+  asm("{ .reg .f32 t; mov.b64 {%0, t}, %1; }" : "=f"(x) : "l"(a.v));
   return x;
 }
 __device__ __forceinline__ float hi(F2 a) {
-  float x, y;
-  asm("mov.b64 {%0, %1}, %2;" : "=f"(x), "=f"(y) : "l"(a.v));
+  float y;
+  asm("{ .reg .f32 t; mov.b64 {t, %0}, %1; }" : "=f"(y) : "l"(a.v));
   return y;
 }
 __device__ __forceinline__ F2 fma2(F2 a, F2 b, F2 c) {
