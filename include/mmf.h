@@ -158,7 +158,8 @@ mmf_status mmf_bitlinear(const mmf_tlinear* lin, const void* x, mmf_dtype dtype,
 /* MLGRU scan                                                                 */
 /* ------------------------------------------------------------------------- */
 
-/* Scratch bytes mmf_mlgru_scan needs for B sequences of T tokens and d channels. */
+/* Scratch bytes mmf_mlgru_scan needs for B sequences of T tokens and d channels
+ * (a small constant: the scan keeps its state on chip). */
 size_t mmf_mlgru_scan_ws_size(int32_t B, int32_t T, int32_t d);
 
 /* MLGRU gates and gated recurrence over T tokens for B sequences.
@@ -171,9 +172,10 @@ size_t mmf_mlgru_scan_ws_size(int32_t B, int32_t T, int32_t d);
  *   h   (device) float [B, d]: h_0 on entry, h_T on return (in place)
  *   o   (device) [B, T, d] in dtype: o'
  *   ws  (device) scratch of mmf_mlgru_scan_ws_size(B, T, d) bytes.
- * The sequence is split into chunks processed in parallel; a chunk takes its
- * entering state from the previous chunk through a bounded wait (a timeout is
- * reported by mmf_check as MMF_ERR_TIMEOUT).
+ * One CTA owns a block of channels of one sequence and walks the sequence's
+ * chunks in order with the state on chip; within a chunk the warps' steps are
+ * composed as affine maps. Its waits for the gate tiles it streams in are
+ * bounded (a timeout is reported by mmf_check as MMF_ERR_TIMEOUT).
  * T = 0 leaves h unchanged. Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d % 8),
  * MISALIGNED, WORKSPACE, CUDA. */
 mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,

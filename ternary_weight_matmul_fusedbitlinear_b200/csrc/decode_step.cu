@@ -26,15 +26,18 @@
 //     and resets set 1 - P for the next launch.
 //   * A CTA owns the 16-row tiles b, b + G, ... of every stage's matrices. Its
 //     weight slices stream into a shared-memory ring by 1-D bulk copies
-//     (cp.async.bulk, one per packed row) several stages ahead, with L2
-//     prefetches further ahead. Weights do not depend on activations, so the
-//     HBM stream runs ahead of the chain.
+//     (cp.async.bulk, one per tile and segment) several stages ahead. Weights
+//     do not depend on activations, so the HBM stream runs ahead of the chain.
+//     (L2 prefetches further ahead measured slower: their instructions share
+//     the SM's memory pipeline with the chain's own loads and stores.)
 //   * Every CTA quantises the whole input rows itself with all 16 warps: the
 //     rows go to registers, the fp64 sum of squares and the max are reduced
 //     over the block in a fixed order (every CTA gets the same scale), and the
 //     codes go to shared memory with the same fp32 steps as the standalone
 //     quantiser. The contraction is mma.sync m16n8k32 (stored codes w + 1 as
-//     u8 against s8 activations; the row's code sum is subtracted after).
+//     u8 against s8 activations; the row's code sum is subtracted after),
+//     its units spread evenly over the warps by a per-stage plan worked out
+//     once at kernel start.
 // Launch: cooperative, one CTA of 512 threads per SM, so every CTA is resident
 // and every wait ends. Each wait is also bounded: on timeout a CTA records
 // status code 5 (input rows) or 6 (weight slice), raises the state's abort word
@@ -51,7 +54,6 @@ namespace {
 constexpr int kThreads = 512;
 constexpr int kWarps = kThreads / 32;
 constexpr int kVmax = 16;            // 16-byte input vectors per thread and stage
-constexpr int kPrefetchAhead = 6;    // L2 prefetch distance beyond the ring, in stages
 constexpr uint32_t kLow2 = 0x03030303u;
 
 struct StageGeom {
@@ -138,9 +140,6 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
-__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
-  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
-}
 
 // This CTA's share of one stage type (S0..S3 repeat in every layer), worked
 // out once at kernel start so that no integer division sits on the chain.
@@ -190,19 +189,6 @@ __device__ void fill_slot(const DecodeStepArgs& a, const DecodeLayerDesc* desc, 
     const int t = blockIdx.x + ti * gridDim.x;
     const uint8_t* src = reinterpret_cast<const uint8_t*>(desc[l].w[g.mat0 + r]) + (size_t)t * tile_bytes;
     bulk_g2s(dst0 + (size_t)i * tile_bytes, src, (uint32_t)tile_bytes, &sm.slot_bar[slot]);
-  }
-}
-
-// One warp: prefetch stage q's weight slice into L2.
-__device__ void prefetch_stage(const DecodeStepArgs& a, const DecodeLayerDesc* desc, const Smem& sm, int q, int lane) {
-  const int l = q >> 2, s = q & 3;
-  const StageGeom g = stage_geom(s, a.d, a.I);
-  const int ntl = sm.plan[s].ntl;
-  const int rowb = g.K / 4;
-  for (int i = lane; i < ntl * g.nseg; i += 32) {
-    const int ti = i / g.nseg, r = i - ti * g.nseg;
-    const int t = blockIdx.x + ti * gridDim.x;
-    prefetch_l2(reinterpret_cast<const uint8_t*>(desc[l].w[g.mat0 + r]) + (size_t)t * 16 * rowb, (uint32_t)(16 * rowb));
   }
 }
 
@@ -343,7 +329,6 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
   int q_issued = 0;   // stages whose ring fill has been issued
   if (warp == kWarps - 1) {
     for (int q = 0; q < a.nslot && q < nq; ++q) fill_slot(a, desc, slots, sm, q, lane);
-    for (int q = a.nslot; q < a.nslot + kPrefetchAhead && q < nq; ++q) prefetch_stage(a, desc, sm, q, lane);
   }
   q_issued = a.nslot < nq ? a.nslot : nq;
   pdl_wait();
@@ -471,10 +456,9 @@ __global__ void __launch_bounds__(kThreads, 1) decode_step_kernel(const __grid_c
       stage_mma(slots + (size_t)slot * a.slot_bytes, codes, qpitch, M, K, sm.plan[s], g.nseg, sm.red);
     }
     __syncthreads();
-    if (warp == kWarps - 1) {   // the slot is free: refill it `nslot` stages ahead, prefetch further ahead
-      fence_proxy_async_smem();  // into L2; this warp has no epilogue work (at most 384 outputs per CTA)
+    if (warp == kWarps - 1) {   // the slot is free: refill it `nslot` stages ahead (this warp has
+      fence_proxy_async_smem();  // no epilogue work: at most 384 outputs per CTA)
       if (q + a.nslot < nq) fill_slot(a, desc, slots, sm, q + a.nslot, lane);
-      if (q + a.nslot + kPrefetchAhead < nq) prefetch_stage(a, desc, sm, q + a.nslot + kPrefetchAhead, lane);
     }
     if (q + a.nslot < nq) q_issued = q + a.nslot + 1;
 
