@@ -222,9 +222,11 @@ typedef struct mmf_state mmf_state;   /* opaque */
  * For the prefill contraction the block uses each matrix's codes one byte per
  * weight: the caller's mmf_tlinear.codes when given, otherwise a copy the
  * library makes (4x the packed size, e.g. 303 MB for a 24-block d=1024 /
- * I=2816 stack): it allocates them with cudaMalloc on the current device,
- * fills them with one kernel on the legacy default stream, waits for it, and
- * frees them in mmf_block_destroy. The environment variable
+ * I=2816 stack). The copy is not made here: the block's first forward call
+ * with T > 1 and at least 128 tokens allocates it with cudaMalloc on the
+ * current device and fills it with one kernel on that call's stream, so make
+ * that first prefill call outside stream capture; a decode-only block never
+ * allocates it. mmf_block_destroy frees it. The environment variable
  * MMF_PREFILL_UNPACKED=0 turns the copy off, and when the memory cannot be
  * allocated the block goes without it (the contraction then expands the packed
  * codes in shared memory; same results).

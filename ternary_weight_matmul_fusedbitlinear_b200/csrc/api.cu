@@ -211,8 +211,9 @@ mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& q
   return MMF_OK;
 }
 
-// Blocks keep one-byte copies of their codes for the prefill contraction
-// (4x the packed weight memory) unless MMF_PREFILL_UNPACKED=0.
+// Blocks make one-byte copies of their codes for the prefill contraction
+// (4x the packed weight memory), at their first prefill-sized call, unless
+// MMF_PREFILL_UNPACKED=0.
 bool prefill_unpacked_enabled() {
   const char* e = getenv("MMF_PREFILL_UNPACKED");
   return e == nullptr || strcmp(e, "0") != 0;
@@ -273,11 +274,16 @@ void mmf::set_last_error(const char* msg) { g_last_error = msg; }
 // creation (owned[i]); all null when disabled.
 // ddesc: device copy of the block's decode descriptor (weights, scales,
 // biases, gains), read by the one-launch decode step.
+// wu: the one-byte codes the prefill contraction loads (the caller's, or the
+// library's copies in owned, made by the first prefill-sized call; null: the
+// contraction expands the packed codes). codes_tried and mu guard that copy.
 struct mmf_block {
   mmf_block_weights w;
   int d, I;
-  const uint8_t* wu[7];
-  uint8_t* owned[7];
+  mutable const uint8_t* wu[7];
+  mutable uint8_t* owned[7];
+  mutable bool codes_tried;
+  mutable std::mutex mu;
   DecodeLayerDesc* ddesc;
 };
 
@@ -521,6 +527,7 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
   b->d = d;
   b->I = I;
   b->ddesc = nullptr;
+  b->codes_tried = false;
   const mmf_tlinear* all[7] = {&w->f, &w->c, &w->g, &w->o, &w->gate, &w->up, &w->down};
   for (int i = 0; i < 7; ++i) {
     b->wu[i] = all[i]->codes;
@@ -544,44 +551,6 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
       (void)cudaGetLastError();
       cudaFree(b->ddesc);
       b->ddesc = nullptr;
-    }
-  }
-  if (prefill_unpacked_enabled()) {
-    // copies for the matrices the caller gave no codes for; they only speed
-    // prefill up, so without device memory for them the block keeps using the
-    // packed codes
-    bool have = true;
-    for (int i = 0; i < 7 && have; ++i) {
-      if (b->wu[i] != nullptr) continue;
-      if (cudaMalloc(&b->owned[i], (size_t)all[i]->N * all[i]->K) != cudaSuccess) {
-        b->owned[i] = nullptr;
-        have = false;
-      }
-    }
-    if (!have) {
-      (void)cudaGetLastError();   // clear the allocation error
-      for (int i = 0; i < 7; ++i) {
-        cudaFree(b->owned[i]);
-        b->owned[i] = nullptr;
-      }
-    }
-    bool launched = false;
-    for (int i = 0; i < 7 && have; ++i) {
-      if (b->owned[i] == nullptr) continue;
-      cudaError_t e = launch_unpack_codes(all[i]->packed, all[i]->N, all[i]->K, b->owned[i], 0);
-      if (e != cudaSuccess) {
-        mmf_block_destroy(b);
-        return cuda_fail(e, "mmf_block_create: unpack codes");
-      }
-      b->wu[i] = b->owned[i];
-      launched = true;
-    }
-    if (launched) {
-      cudaError_t e = cudaStreamSynchronize(0);
-      if (e != cudaSuccess) {
-        mmf_block_destroy(b);
-        return cuda_fail(e, "mmf_block_create: synchronise");
-      }
     }
   }
   *out = b;
@@ -800,12 +769,51 @@ mmf_status dbg_copy(void* dst, const void* src, size_t bytes, cudaStream_t s) {
   return MMF_OK;
 }
 
+// The block's one-byte code copies, made once, by the first call with enough
+// tokens for the tensor-core contraction: allocated with cudaMalloc and filled
+// by one kernel on the call's stream (so the contraction, later on the same
+// stream, sees them). Without device memory for all of them the block keeps the
+// packed codes (same results).
+void ensure_prefill_codes(const mmf_block* b, cudaStream_t s) {
+  std::lock_guard<std::mutex> lock(b->mu);
+  if (b->codes_tried) return;
+  b->codes_tried = true;
+  if (!prefill_unpacked_enabled()) return;
+  const mmf_block_weights& w = b->w;
+  const mmf_tlinear* all[7] = {&w.f, &w.c, &w.g, &w.o, &w.gate, &w.up, &w.down};
+  bool have = true;
+  for (int i = 0; i < 7 && have; ++i) {
+    if (b->wu[i] != nullptr) continue;
+    if (cudaMalloc(&b->owned[i], (size_t)all[i]->N * all[i]->K) != cudaSuccess) {
+      b->owned[i] = nullptr;
+      have = false;
+    }
+  }
+  if (!have) {
+    (void)cudaGetLastError();   // clear the allocation error
+    for (int i = 0; i < 7; ++i) {
+      cudaFree(b->owned[i]);
+      b->owned[i] = nullptr;
+    }
+    return;
+  }
+  for (int i = 0; i < 7; ++i) {
+    if (b->owned[i] == nullptr) continue;
+    if (launch_unpack_codes(all[i]->packed, all[i]->N, all[i]->K, b->owned[i], s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return;   // this and later matrices keep their packed codes
+    }
+    b->wu[i] = b->owned[i];
+  }
+}
+
 mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, void* y, int B, int T, mmf_dtype dt,
                               float eps, const BlockWs& w, cudaStream_t s, const mmf_block_debug* dbg = nullptr) {
   const int M = B * T, d = blk->d;
   const mmf_block_weights& W = blk->w;
   const mmf_tlinear* fcg[3] = {&W.f, &W.c, &W.g};
   const bool want = dbg != nullptr;
+  if (T > 1 && (M >= kTcMinTokens || gemm_path_pref() >= 2)) ensure_prefill_codes(blk, s);
   // token mixer: x quantised once for f, c, g (shared gain)
   if (T == 1) {
     // decode: projections and one recurrence step in one launch; h updated in place

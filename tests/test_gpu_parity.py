@@ -263,6 +263,32 @@ def test_block_prefill_unpacked_copy_is_bit_identical(dtype, monkeypatch):
     assert torch.equal(outs[0][0], outs[1][0]) and torch.equal(outs[0][1], outs[1][1])
 
 
+def test_block_byte_copy_made_by_first_prefill_call_only():
+    # creating a block and decoding with it allocate no one-byte code copy; the
+    # first prefill-sized call makes it (7 matrices, N x K bytes each)
+    d, inner, B, T = 1024, 2816, 2, 192
+    copy_bytes = 4 * d * d + 3 * d * inner
+    x = synth.activations(7044, B * T, d, torch.bfloat16).reshape(B, T, d).cuda()
+    blk, _ = make_block(7043, d, inner)
+    st = mmf.State(1, B, d)
+    ws = torch.empty(mmf.stack_ws_size([blk], B, T), dtype=torch.uint8, device="cuda")
+    torch.cuda.synchronize()
+    free0 = torch.cuda.mem_get_info()[0]
+    mmf.block_forward(blk, 0, st, x[:, :1].contiguous(), ws=ws)   # a decode step
+    torch.cuda.synchronize()
+    free1 = torch.cuda.mem_get_info()[0]
+    mmf.block_forward(blk, 0, st, x, ws=ws)                       # first prefill: makes the copy
+    torch.cuda.synchronize()
+    free2 = torch.cuda.mem_get_info()[0]
+    mmf.block_forward(blk, 0, st, x, ws=ws)                       # second prefill: nothing new
+    torch.cuda.synchronize()
+    free3 = torch.cuda.mem_get_info()[0]
+    mmf.check()
+    assert free0 - free1 < copy_bytes // 4, (free0, free1)
+    assert free1 - free2 >= copy_bytes, (free1, free2, copy_bytes)
+    assert abs(free2 - free3) < copy_bytes // 4, (free2, free3)
+
+
 @pytest.mark.parametrize("m", [128, 300])
 def test_bitlinear_and_glu_with_byte_codes_bit_identical(m):
     # mmf_tlinear.codes (mmf_unpack_codes) lets the prefill contraction load the
