@@ -33,6 +33,9 @@ compositions ``mlgru``, ``block_forward`` and ``stack_forward`` are pinned
 through special cases only: scaled-identity weights, where every BitLinear
 reduces to alpha * q / s and the scan to its unrolled sum; zero weights; the
 prefill == decode invariant. The pages print no worked example for them.
+The g_norm output gate (``rmsnorm_swish_gate``) is pinned by a hand-worked
+two-channel case, g~ = 0 giving o' = 0, the mean-square invariant under a
+constant gate, scale invariance, and the identity-weight block.
 """
 from __future__ import annotations
 
@@ -326,9 +329,54 @@ def mlgru_scan(pf, pc, pg, h0):
     return o, h
 
 
+def rmsnorm_swish_gate(h, pg, w=None, eps: float = EPS_NORM) -> np.ndarray:
+    """g_norm output gate: RMSNorm of the recurrence state fused with a swish gate (fp64).
+
+    [HL] "HGRN attention": the token mixer's recurrence output passes g_norm,
+    a FusedRMSNormSwishGate (normalisation and swish activation in one step),
+    before o_proj. The page prints no formula; the plainest reading used here:
+        o'_t = h_t / sqrt(mean_n h_t[n]^2 + eps) * w * swish(g~_t),
+        swish(z) = z * sigmoid(z) (= SiLU),
+    normalised per token over all d channels (one head), w the gate norm's
+    gain (ones when None), eps the block's norm epsilon.
+    h, pg: [..., d]. Returns o' [..., d] fp64.
+    """
+    h = np.asarray(h, dtype=np.float64)
+    ms = np.mean(np.square(h), axis=-1, keepdims=True)
+    y = h / np.sqrt(ms + eps)
+    if w is not None:
+        y = y * np.asarray(w, dtype=np.float64)
+    return y * silu(pg)
+
+
+def mlgru_scan_gnorm(pf, pc, pg, h0, w=None, eps: float = EPS_NORM):
+    """MLGRU recurrence with the g_norm output gate in place of sigmoid(g~) * h.
+
+    The recurrence is the one of ``mlgru_scan`` (f_t = sigmoid(f~_t),
+    c_t = SiLU(c~_t), h_t = f_t h_{t-1} + (1 - f_t) c_t, carried in fp64); the
+    output is ``rmsnorm_swish_gate(h_t, g~_t, w, eps)`` at every step.
+    Returns (o' [B,T,d] fp64, h_T [B,d] fp64).
+    """
+    pf = np.asarray(pf, dtype=np.float64)
+    pc = np.asarray(pc, dtype=np.float64)
+    h = np.array(h0, dtype=np.float64, copy=True)
+    T = pf.shape[1]
+    hs = np.empty_like(pf)
+    for t in range(T):
+        f = sigmoid(pf[:, t])
+        h = f * h + (1.0 - f) * silu(pc[:, t])
+        hs[:, t] = h
+    return rmsnorm_swish_gate(hs, pg, w, eps), h
+
+
 @dataclasses.dataclass
 class Block:
-    """Ternary weights of one MatMul-free block."""
+    """Ternary weights of one MatMul-free block.
+
+    ``gnorm``: gain of the g_norm output gate ([d] fp32). None selects the
+    sigmoid output gate o' = sigmoid(g~) * h; a gain selects
+    o' = RMSNorm(h) * gnorm * swish(g~) (``rmsnorm_swish_gate``).
+    """
     f: TLinear
     c: TLinear
     g: TLinear
@@ -336,6 +384,7 @@ class Block:
     gate: TLinear
     up: TLinear
     down: TLinear
+    gnorm: Optional[np.ndarray] = None
 
     @property
     def d(self) -> int:
@@ -346,9 +395,14 @@ class Block:
         return self.gate.N
 
 
-def make_block(latents: dict, cache: bool = False) -> Block:
-    """latents: dict of name -> fp32 latent [N, K] for f, c, g, o, gate, up, down."""
-    return Block(**{k: make_tlinear(latents[k], cache=cache) for k in ("f", "c", "g", "o", "gate", "up", "down")})
+def make_block(latents: dict, cache: bool = False, gnorm=None) -> Block:
+    """latents: dict of name -> fp32 latent [N, K] for f, c, g, o, gate, up, down.
+
+    gnorm: optional [d] gain selecting the g_norm output gate.
+    """
+    lins = {k: make_tlinear(latents[k], cache=cache) for k in ("f", "c", "g", "o", "gate", "up", "down")}
+    g = None if gnorm is None else np.asarray(gnorm, dtype=np.float32).astype(np.float64)
+    return Block(**lins, gnorm=g)
 
 
 def mlgru_preacts(x, blk: Block, dtype: str, eps: float = EPS_NORM):
@@ -362,11 +416,15 @@ def mlgru_preacts(x, blk: Block, dtype: str, eps: float = EPS_NORM):
 def mlgru(x, blk: Block, h0, dtype: str, eps: float = EPS_NORM, parts: bool = False):
     """MLGRU token mixer on x [B,T,d]: projections, gated scan, output gate, o-projection.
 
-    Storage points (the kernels store these tensors): f~/c~/g~ and o' in the run
-    dtype, the state h in fp32. Returns (o [B,T,d] fp64 unrounded, h_T fp32 values).
+    The output gate is sigmoid(g~) * h, or the g_norm gate when ``blk.gnorm`` is
+    set. Storage points (the kernels store these tensors): f~/c~/g~ and o' in
+    the run dtype, the state h in fp32. Returns (o [B,T,d] fp64 unrounded, h_T fp32 values).
     """
     pf, pc, pg = mlgru_preacts(x, blk, dtype, eps)
-    o_gate, hT = mlgru_scan(pf, pc, pg, h0)
+    if blk.gnorm is None:
+        o_gate, hT = mlgru_scan(pf, pc, pg, h0)
+    else:
+        o_gate, hT = mlgru_scan_gnorm(pf, pc, pg, h0, blk.gnorm, eps)
     o_gate = store(o_gate, dtype)
     o = bitlinear(o_gate, blk.o, eps)
     hT = round_f32(hT)

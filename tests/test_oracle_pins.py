@@ -393,6 +393,62 @@ def test_scan_convex_bound_and_chunking_and_batch_independence():
     np.testing.assert_array_equal(ob[0], o[1])
 
 
+# ----------------------------------------------------------------- g_norm output gate
+
+def test_gnorm_hand_worked_two_channels():
+    # h = (3, 4): mean square 12.5, so h / rms = (3, 4) * sqrt(2) / 5; sigmoid(ln 3) = 3/4,
+    # so swish(ln 3) = 0.75 ln 3 and swish(-ln 3) = -0.25 ln 3; gain (2, 5)
+    ln3 = math.log(3.0)
+    o = O.rmsnorm_swish_gate(np.array([3.0, 4.0]), np.array([ln3, -ln3]), w=np.array([2.0, 5.0]), eps=0.0)
+    r2 = math.sqrt(2.0)
+    np.testing.assert_allclose(o, [2 * 3 * r2 / 5 * 0.75 * ln3, 5 * 4 * r2 / 5 * (-0.25 * ln3)], rtol=1e-14)
+    # eps adds to the mean square: sqrt(12.5 + 0.5) = sqrt(13)
+    o = O.rmsnorm_swish_gate(np.array([3.0, 4.0]), np.array([ln3, ln3]), eps=0.5)
+    np.testing.assert_allclose(o, np.array([3.0, 4.0]) / math.sqrt(13.0) * 0.75 * ln3, rtol=1e-14)
+    # h constant across channels, eps = 0: the norm is the sign, o' = sign(a) swish(g~)
+    g = np.array([-2.0, 0.5, 3.0])
+    np.testing.assert_allclose(O.rmsnorm_swish_gate(np.full(3, -7.5), g, eps=0.0), -O.silu(g), rtol=1e-15)
+
+
+def test_gnorm_zero_gate_scale_invariance_and_axis():
+    pf, pc, pg = _scan_inputs(38, B=2, T=20, d=16)
+    h0 = synth.activations(39, 2, 16).numpy().astype(np.float64)
+    # g~ = 0: swish(0) = 0, so o' = 0 exactly whatever the state
+    o, _ = O.mlgru_scan_gnorm(pf, pc, np.zeros_like(pg), h0)
+    assert np.all(o == 0.0)
+    # constant g~ = z and unit gain: every token's mean square is swish(z)^2 ms/(ms + eps),
+    # ms the token's mean square of h (taken from the recurrence with a unit sigmoid gate
+    # written as g~ = +inf); normalising over time instead of channels breaks it
+    z, eps = 0.8, 1e-3
+    o, _ = O.mlgru_scan_gnorm(pf, pc, np.full_like(pg, z), h0, eps=eps)
+    h, _ = O.mlgru_scan(pf, pc, np.full_like(pg, 1e4), h0)
+    ms = np.mean(h * h, axis=-1)
+    np.testing.assert_allclose(np.mean(o * o, axis=-1), O.silu(z) ** 2 * ms / (ms + eps), rtol=1e-12)
+    # with eps = 0 the output is invariant to a positive scale of the state and odd in it
+    hh = synth.activations(40, 6, 16).numpy().astype(np.float64)
+    a = O.rmsnorm_swish_gate(hh, pg[0, :6], eps=0.0)
+    np.testing.assert_allclose(O.rmsnorm_swish_gate(hh * 37.0, pg[0, :6], eps=0.0), a, rtol=1e-13)
+    np.testing.assert_allclose(O.rmsnorm_swish_gate(-hh, pg[0, :6], eps=0.0), -a, rtol=1e-13)
+
+
+def test_gnorm_scan_forget_zero_and_unrolled():
+    pf, pc, pg = _scan_inputs(56, B=2, T=12, d=8)
+    w = 0.5 + synth.activations(57, 1, 8).numpy().astype(np.float64)[0] ** 2
+    h0 = synth.activations(58, 2, 8).numpy().astype(np.float64)
+    # forget gate 0: h_t = SiLU(c~_t)
+    o, hT = O.mlgru_scan_gnorm(np.full_like(pc, -1e4), pc, pg, h0, w)
+    c = O.silu(pc)
+    ref = c / np.sqrt(np.mean(c * c, axis=-1, keepdims=True) + O.EPS_NORM) * w * O.silu(pg)
+    np.testing.assert_allclose(o, ref, rtol=1e-13)
+    np.testing.assert_allclose(hT, c[:, -1], rtol=1e-15)
+    # general gates: the state is the unrolled sum, the same one the sigmoid gate multiplies
+    o, hT = O.mlgru_scan_gnorm(pf, pc, pg, h0, w)
+    og, _ = O.mlgru_scan(pf, pc, pg, h0)
+    H = og / O.sigmoid(pg)
+    np.testing.assert_allclose(O.rmsnorm_swish_gate(H, pg, w), o, rtol=1e-12, atol=1e-15)
+    np.testing.assert_allclose(H[:, -1], hT, rtol=1e-12)
+
+
 # ----------------------------------------------------------------- GLU and block
 
 def _block(seed, d, inner):
@@ -506,6 +562,31 @@ def test_block_identity_weights_closed_form():
     assert np.max(np.abs(O.round_f32(x + _dq(blk.down, p_x)) - y)) > 1e-3
 
 
+def test_block_gnorm_identity_weights_and_zero_gate():
+    # identity weights with the g_norm gate: o' = RMSNorm(h) * w * SiLU(g~) with h the
+    # unrolled state; the sigmoid gate would give a different o'
+    d, B, T = 32, 2, 5
+    blk = _eye_block(d)
+    blk.gnorm = 0.25 + synth.activations(65, 1, d).numpy().astype(np.float64)[0] ** 2
+    x = O.round_f32(synth.activations(66, B * T, d).numpy().reshape(B, T, d))
+    h0 = synth.activations(67, B, d).numpy().astype(np.float64)
+    y, hT, parts = O.block_forward(x, blk, h0, "f32", parts=True)
+    pf, pc, pg = (O.round_f32(_dq(getattr(blk, n), x)) for n in ("f", "c", "g"))
+    H = np.stack([_unrolled_scan(O.sigmoid(pf[:, :t + 1]), O.silu(pc[:, :t + 1]),
+                                 np.ones_like(pg[:, :t + 1]), h0)[1] for t in range(T)], axis=1)
+    ms = np.mean(H * H, axis=-1, keepdims=True)
+    og = O.round_f32(H / np.sqrt(ms + O.EPS_NORM) * blk.gnorm * O.silu(pg))
+    np.testing.assert_allclose(parts["o_gate"], og, rtol=2e-7, atol=1e-12)
+    np.testing.assert_allclose(hT, O.round_f32(H[:, -1]), rtol=2e-7)
+    sig = O.round_f32(O.sigmoid(pg) * H)
+    assert np.max(np.abs(sig - og)) > 0.05 * np.max(np.abs(og))
+    # g-projection weights zero: g~ = 0, o' = 0, the o-projection of zeros is 0, y1 = x
+    blk.g = O.make_tlinear(np.zeros((d, d), np.float32))
+    _, _, parts = O.block_forward(x, blk, h0, "f32", parts=True)
+    assert np.all(parts["o_gate"] == 0.0)
+    np.testing.assert_array_equal(parts["y1"], x)
+
+
 def test_block_zero_weights_is_identity():
     d, inner, B, T = 32, 48, 2, 6
     blk = _block(43, d, inner)
@@ -520,10 +601,12 @@ def test_block_zero_weights_is_identity():
     np.testing.assert_array_equal(hT, O.round_f32(h0 * 0.5 ** T))
 
 
-@pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_block_prefill_equals_decode_steps(dtype):
+@pytest.mark.parametrize("dtype,gnorm", [("f32", False), ("bf16", False), ("bf16", True)])
+def test_block_prefill_equals_decode_steps(dtype, gnorm):
     d, inner, B, T = 32, 64, 2, 5
     blk = _block(46, d, inner)
+    if gnorm:
+        blk.gnorm = 1.0 + 0.1 * synth.activations(48, 1, d).numpy().astype(np.float64)[0]
     x = O.store(synth.activations(47, B * T, d).numpy().reshape(B, T, d), dtype)
     h0 = np.zeros((B, d))
     y, hT = O.block_forward(x, blk, h0, dtype)
