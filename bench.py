@@ -69,6 +69,8 @@ def parse_args(argv=None):
                     help="stack370m: number of blocks (default 24; fewer for short profiler captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) pass")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--gnorm", action="store_true",
+                    help="scan: the g_norm output gate (RMSNorm of the state fused with a swish gate)")
     ap.add_argument("--no-sub", action="store_true",
                     help="stack370m: skip the decode-step and GEMV-sweep sub-measurements")
     return ap.parse_args(argv)
@@ -136,7 +138,7 @@ class L2Flush:
     def __init__(self, dev):
         self.w = torch.empty(2 * L2_BYTES, dtype=torch.uint8, device=dev)
         self.r = torch.ones(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
-        self.sink = torch.empty(1, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
 
     def __call__(self):
         self.w.zero_()
@@ -525,6 +527,10 @@ def run_mmf(args):
                                                       "launches_per_step", "decode_steps", "clocks")}
         torch.cuda.empty_cache()
         sub["gemv_sweep"] = measure_gemv(mmf, dev, 2, 3, peaks)
+        for gn in (False, True):
+            m = measure_scan(mmf, dev, 10, 3, gn)
+            m["frac"] = round(m["GBps"] / peaks["hbm_gbs"], 4)
+            sub["scan_gnorm" if gn else "scan"] = m
 
     if rank == 0:
         line = {
@@ -610,42 +616,59 @@ def run_bitlinear(args):
     return 0
 
 
+def measure_scan(mmf, dev, steps: int, warmup: int, gnorm: bool, flush=None) -> dict:
+    """One MLGRU scan per step on the 370M layer shape (8 x 2048 tokens, d = 1024, bf16), L2 flushed
+    between steps. Algorithmic bytes: 8 per channel-step (6 B of pre-activations read, 2 B of o'
+    written) for either output gate; the g_norm path's own design also writes and reads v in fp32
+    (16 B per channel-step in all)."""
+    w = synth.STACK_370M
+    B, T, d = w.batch, w.seq, w.d
+    pre = synth.preacts(77, B, T, d, torch.bfloat16, scale=2.0, device=dev)
+    h = torch.zeros(B, d, device=dev)
+    gain = synth.gains(78, d, device=str(dev)) if gnorm else None
+    flush = flush or L2Flush(dev)
+    run = (lambda: mmf.mlgru_scan_gnorm(pre, h, gain)) if gnorm else (lambda: mmf.mlgru_scan(pre, h))
+    key = "mlgru_scan_gnorm" if gnorm else "mlgru_scan"
+    for _ in range(warmup):
+        run()
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    torch.cuda.synchronize()
+    for _ in range(steps):
+        flush()
+        run()
+    torch.cuda.synchronize()
+    mmf.prof_enable(False)
+    prof = mmf.prof_collect()
+    ms = prof[key][1] / prof[key][0]
+    nbytes = 8.0 * B * T * d
+    gbs = nbytes / (ms / 1e3) / 1e9
+    r = {"workload": f"mlgru_scan{'_gnorm' if gnorm else ''}_b{B}_t{T}_d{d}_bf16", "us": round(ms * 1e3, 2),
+         "GBps": round(gbs, 1), "bytes": nbytes, "launches": (2 if gnorm else 1) * prof[key][0]}
+    if gnorm:
+        r["design_bytes"] = 16.0 * B * T * d
+    return r
+
+
 def run_scan(args):
     """One MLGRU scan per step on the 370M layer shape; GB/s = 8 bytes per channel-step (bf16)."""
     _, rank, local = dist_env()
     torch.cuda.set_device(local)
     import ternary_weight_matmul_fusedbitlinear_b200 as mmf
     dev = torch.device("cuda", local)
-    w = synth.STACK_370M
-    B, T, d = w.batch, w.seq, w.d
     peaks, peak_kind = load_peaks()
-    pre = synth.preacts(77, B, T, d, torch.bfloat16, scale=2.0, device=dev)
-    h = torch.zeros(B, d, device=dev)
-    flush = L2Flush(dev)
-    for _ in range(args.warmup):
-        mmf.mlgru_scan(pre, h)
-    mmf.prof_reset()
-    mmf.prof_enable(True)
-    torch.cuda.synchronize()
-    for _ in range(args.steps):
-        flush()
-        mmf.mlgru_scan(pre, h)
-    torch.cuda.synchronize()
-    mmf.prof_enable(False)
-    prof = mmf.prof_collect()
-    ms = prof["mlgru_scan"][1] / prof["mlgru_scan"][0]
-    nbytes = 8.0 * B * T * d
-    gbs = nbytes / (ms / 1e3) / 1e9
+    m = measure_scan(mmf, dev, args.steps, args.warmup, args.gnorm)
+    gbs, ms = m["GBps"], m["us"] / 1e3
+    kernel = "mlgru_scan_gnorm (scan + row kernel)" if args.gnorm else "mlgru_scan"
     if rank == 0:
         print(json.dumps({
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
             "ms_per_step": ms, "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
-            "data": "synthetic", "config": {"workload": f"mlgru_scan_b{B}_t{T}_d{d}_bf16",
-                                            "l2": L2Flush.NOTE},
+            "data": "synthetic", "config": {"workload": m["workload"], "l2": L2Flush.NOTE},
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": "mlgru_scan (with its scratch reset)",
+                         "frac": gbs / peaks["hbm_gbs"], "traffic": None, "kernel": kernel,
                          "peak_source": peak_kind},
-            "cpu_baseline": None, "e2e": None, "gpu_launches": prof["mlgru_scan"][0]}), flush=True)
+            "cpu_baseline": None, "e2e": None, "gpu_launches": m["launches"], "detail": m}), flush=True)
     return 0
 
 

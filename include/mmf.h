@@ -181,6 +181,25 @@ size_t mmf_mlgru_scan_ws_size(int32_t B, int32_t T, int32_t d);
 mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
                           float* h, void* o, void* ws, size_t ws_bytes, void* stream);
 
+/* Scratch bytes mmf_mlgru_scan_gnorm needs: 4 x B x T x d bytes for
+ * v = swish(g~) h in fp32, 4 x B x T x ceil(d / 32) for the partial sums of
+ * h^2, and a little padding. */
+size_t mmf_mlgru_scan_gnorm_ws_size(int32_t B, int32_t T, int32_t d);
+
+/* The MLGRU recurrence of mmf_mlgru_scan with the g_norm output gate in place
+ * of sigmoid(g~) h. [HL] "HGRN attention": the recurrence output passes g_norm,
+ * a FusedRMSNormSwishGate (RMSNorm and swish activation fused). Per token t,
+ * normalising over the d channels:
+ *   o'_t = h_t / sqrt(mean_n h_t[n]^2 + eps) * gain * swish(g~_t),
+ *   swish(z) = z sigmoid(z)
+ * pre, h, o as for mmf_mlgru_scan; gain (device) float [d], not NULL (a
+ * vector of ones for an unscaled norm); eps > 0. Two launches on `stream`:
+ * the scan writes v = swish(g~) h and per-token partial sums of h^2 into ws,
+ * then a row kernel writes o'. Errors: as mmf_mlgru_scan. */
+mmf_status mmf_mlgru_scan_gnorm(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
+                                float* h, const float* gain, float eps, void* o, void* ws,
+                                size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------- */
 /* MatMul-free GLU                                                            */
 /* ------------------------------------------------------------------------- */
@@ -208,9 +227,12 @@ mmf_status mmf_glu(const mmf_tlinear* gate, const mmf_tlinear* up, const mmf_tli
 
 /* Weights of one MatMul-free block: MLGRU projections f, c, g, o (d x d) and
  * GLU gate, up (I x d) and down (d x I). f, c and g share one gain, gate and up
- * share one gain. */
+ * share one gain. gnorm (device, float [d], 16-byte aligned) selects the
+ * g_norm output gate of mmf_mlgru_scan_gnorm with that gain; NULL selects the
+ * sigmoid output gate o' = sigmoid(g~) h. */
 typedef struct mmf_block_weights {
   mmf_tlinear f, c, g, o, gate, up, down;
+  const float* gnorm;
 } mmf_block_weights;
 
 typedef struct mmf_block mmf_block;   /* opaque */
@@ -259,6 +281,7 @@ size_t mmf_block_ws_size(const mmf_block* blk, int32_t B, int32_t T);
 
 /* One MatMul-free block on x [B, T, d] -> y [B, T, d] (both device, dtype):
  *   y1 = x + o_proj(MLGRU(x)),  y = y1 + GLU(y1)
+ * with the block's output gate (sigmoid, or g_norm when its gnorm gain is set).
  * [HL] "HGRN attention" (the block input is normalised first, then f/c/g
  * projections, recurrence and o-projection) and [DC] "Core components".
  * The MLGRU continues from the state of `layer` in `st` and leaves h_T there,
@@ -272,7 +295,9 @@ size_t mmf_block_ws_size(const mmf_block* blk, int32_t B, int32_t T);
  * after which the state must be reset. Larger batches, other shapes, or the
  * environment variable MMF_DECODE_STEP_KERNEL=0 run four contractions instead
  * (f|c|g with the recurrence step in its epilogue, o, gate|up, down), with the
- * same arithmetic. x and y must not overlap. Errors: INVALID_ARG,
+ * same arithmetic. A g_norm block's decode step runs its prefill sequence
+ * (f|c|g contraction, scan and row kernel of mmf_mlgru_scan_gnorm, o, gate|up,
+ * down) with T = 1. x and y must not overlap. Errors: INVALID_ARG,
  * UNSUPPORTED_SHAPE, MISALIGNED, WORKSPACE, NOMEM, CUDA. */
 mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf_state* st,
                              const void* x, void* y, int32_t B, int32_t T, mmf_dtype dtype,
@@ -282,7 +307,7 @@ mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf_state* st,
  * checking each stage on its own (any field may be NULL; M = B * T tokens,
  * activation dtype unless stated):
  *   pre       [M, 3, d]: the f~, c~, g~ pre-activations as the kernels store them
- *   og        [M, d]: o' = g * h, the input of the o projection
+ *   og        [M, d]: o', the output-gated state, the input of the o projection
  *   y1        [M, d]: x + o, the token mixer's output and the GLU's input
  *   p         [M, I]: SiLU(gate) * up, the input of the down projection
  *   q[i]      int8 activation codes of the i-th quantised input (0: x [M, d],

@@ -67,6 +67,12 @@ def preacts(seed: int, b: int, t: int, d: int, dtype: torch.dtype = torch.float3
     return x.to(dtype)
 
 
+def gains(seed: int, d: int, spread: float = 0.1, device: str = "cpu") -> torch.Tensor:
+    """fp32 [d] norm gain ~ 1 + N(0, spread^2), for tests of a learned (non-unit) gain."""
+    g = _gen(seed, device)
+    return 1.0 + spread * torch.randn(d, generator=g, dtype=torch.float32, device=device)
+
+
 @dataclasses.dataclass(frozen=True)
 class Workload:
     """Shape of one synthetic workload (no arithmetic, only sizes)."""

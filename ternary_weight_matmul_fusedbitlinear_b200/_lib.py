@@ -35,7 +35,7 @@ class BlockDebug(ctypes.Structure):
 
 
 class BlockWeights(ctypes.Structure):
-    _fields_ = [(n, TLinear) for n in ("f", "c", "g", "o", "gate", "up", "down")]
+    _fields_ = [(n, TLinear) for n in ("f", "c", "g", "o", "gate", "up", "down")] + [("gnorm", ctypes.c_void_p)]
 
 
 # name -> (restype, argtypes)
@@ -51,6 +51,9 @@ SIGNATURES = {
                                      c_vp, ctypes.POINTER(BitlinearDebug)]),
     "mmf_mlgru_scan_ws_size": (c_sz, [c_i32, c_i32, c_i32]),
     "mmf_mlgru_scan": (ctypes.c_int, [c_vp, ctypes.c_int, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_sz, c_vp]),
+    "mmf_mlgru_scan_gnorm_ws_size": (c_sz, [c_i32, c_i32, c_i32]),
+    "mmf_mlgru_scan_gnorm": (ctypes.c_int, [c_vp, ctypes.c_int, c_i32, c_i32, c_i32, c_vp, c_vp, c_f, c_vp, c_vp, c_sz,
+                                            c_vp]),
     "mmf_glu_ws_size": (c_sz, [c_i32, c_i32, c_i32]),
     "mmf_glu": (ctypes.c_int, [ctypes.POINTER(TLinear)] * 3 + [c_vp, c_vp, c_vp, c_i32, ctypes.c_int, c_f, c_vp,
                                                              c_sz, c_vp]),

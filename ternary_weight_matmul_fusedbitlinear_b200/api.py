@@ -142,6 +142,29 @@ def mlgru_scan(pre: torch.Tensor, h: torch.Tensor, ws: Optional[torch.Tensor] = 
     return o
 
 
+def mlgru_scan_gnorm(pre: torch.Tensor, h: torch.Tensor, gain: torch.Tensor, eps: float = DEFAULT_EPS,
+                     ws: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """The scan with the g_norm output gate: o' = RMSNorm(h) * gain * swish(g~).
+
+    pre [B, T, 3, d] -> o' [B, T, d]; h [B, d] fp32 is updated in place to h_T;
+    gain float32 [d].
+    """
+    _need_cuda(pre, h, gain)
+    if pre.dim() != 4 or pre.shape[2] != 3:
+        raise ValueError("pre must be [B, T, 3, d]")
+    B, T, _, d = pre.shape
+    if h.dtype != torch.float32 or tuple(h.shape) != (B, d):
+        raise ValueError("h must be float32 [B, d]")
+    if gain.dtype != torch.float32 or tuple(gain.shape) != (d,):
+        raise ValueError("gain must be float32 [d]")
+    o = torch.empty(B, T, d, dtype=pre.dtype, device=pre.device)
+    lib = L.load()
+    w = _workspace(lib.mmf_mlgru_scan_gnorm_ws_size(B, T, d), pre.device, ws)
+    L.check(lib.mmf_mlgru_scan_gnorm(_vp(pre), _dtype(pre), B, T, d, _vp(h), _vp(gain), eps, _vp(o), _vp(w),
+                                     w.numel() * w.element_size(), _stream(pre.device)), "mmf_mlgru_scan_gnorm")
+    return o
+
+
 def glu(gate: TLinear, up: TLinear, down: TLinear, x: torch.Tensor, residual: Optional[torch.Tensor] = None,
         eps: float = DEFAULT_EPS, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """y = down(SiLU(gate(x)) * up(x)) (+ residual) for x [..., d]."""
@@ -162,11 +185,17 @@ class Block:
 
     NAMES = ("f", "c", "g", "o", "gate", "up", "down")
 
-    def __init__(self, lins: dict):
+    def __init__(self, lins: dict, gnorm: Optional[torch.Tensor] = None):
+        """lins: name -> TLinear for NAMES; gnorm: float32 [d] gain selecting the g_norm output gate."""
         self.lins = dict(lins)
         self.d = self.lins["f"].K
         self.inner = self.lins["gate"].N
-        bw = L.BlockWeights(*[self.lins[n].c() for n in self.NAMES])
+        if gnorm is not None:
+            _need_cuda(gnorm)
+            if gnorm.dtype != torch.float32 or tuple(gnorm.shape) != (self.d,) or not gnorm.is_contiguous():
+                raise ValueError("gnorm must be a contiguous float32 [d] tensor")
+        self.gnorm = gnorm
+        bw = L.BlockWeights(*[self.lins[n].c() for n in self.NAMES], _vp(gnorm))
         h = ctypes.c_void_p()
         lib = L.load()
         L.check(lib.mmf_block_create(ctypes.byref(bw), self.d, self.inner, ctypes.byref(h)), "mmf_block_create")

@@ -423,6 +423,35 @@ extern "C" mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B
   return MMF_OK;
 }
 
+extern "C" size_t mmf_mlgru_scan_gnorm_ws_size(int32_t B, int32_t T, int32_t d) {
+  if (B < 0 || T < 0 || d < 0) return 0;
+  return mlgru_scan_gnorm_ws_bytes(B, T, d);
+}
+
+extern "C" mmf_status mmf_mlgru_scan_gnorm(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
+                                           float* h, const float* gain, float eps, void* o, void* ws,
+                                           size_t ws_bytes, void* stream) {
+  if (!dtype_ok(dtype)) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_gnorm: bad dtype");
+  if (B < 0 || T < 0 || d < 1) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_gnorm: B=%d T=%d d=%d", B, T, d);
+  if (!(eps > 0.0f)) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_gnorm: eps must be > 0");
+  if (d % 8 != 0) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_mlgru_scan_gnorm: d=%d %% 8 != 0", d);
+  if (B == 0 || T == 0) return MMF_OK;
+  if (!pre || !h || !gain || !o || !ws) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_gnorm: null pointer");
+  if (!aligned16(pre) || !aligned16(h) || !aligned16(gain) || !aligned16(o) || !aligned16(ws))
+    return fail(MMF_ERR_MISALIGNED, "mmf_mlgru_scan_gnorm");
+  if (ws_bytes < mlgru_scan_gnorm_ws_bytes(B, T, d))
+    return fail(MMF_ERR_WORKSPACE, "mmf_mlgru_scan_gnorm: ws_bytes=%zu < %zu", ws_bytes,
+                mlgru_scan_gnorm_ws_bytes(B, T, d));
+  cudaStream_t s = as_stream(stream);
+  int* status = nullptr;
+  mmf_status r = device_status_ptr(&status);
+  if (r != MMF_OK) return r;
+  MMF_CUDA(timed("mlgru_scan_gnorm", s,
+                 [&] { return launch_mlgru_scan_gnorm(pre, dtype, B, T, d, h, gain, eps, o, ws, status, s); }),
+           "mlgru_scan_gnorm");
+  return MMF_OK;
+}
+
 // ------------------------------------------------------------------ GLU
 
 namespace {
@@ -519,6 +548,7 @@ extern "C" mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, in
   }
   if (w->f.gain != w->c.gain || w->f.gain != w->g.gain)
     return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_block_create: f, c and g must share one gain");
+  if (w->gnorm != nullptr && !aligned16(w->gnorm)) return fail(MMF_ERR_MISALIGNED, "mmf_block_create: gnorm");
   if ((st = check_glu(&w->gate, &w->up, &w->down, d)) != MMF_OK) return st;
   if (w->gate.N != I) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_block_create: gate N=%d != I=%d", w->gate.N, I);
   mmf_block* b = new (std::nothrow) mmf_block;
@@ -677,7 +707,8 @@ namespace {
 struct BlockWs {
   QAct qa;     // quantised activations, [M, max(d, I)]
   void* pre;   // [M, 3, d] pre-activations (prefill only)
-  void* og;    // [M, d] o' = g * h
+  void* og;    // [M, d] o' (the scan's output gate applied)
+  void* gn;    // g_norm blocks: the scan's scratch (mlgru_scan_gnorm_ws_bytes), else null
   void* y1;    // [M, d] after the token mixer
   void* p;     // [M, I] GLU product
   void* ping;  // [M, d] stack intermediates
@@ -685,7 +716,7 @@ struct BlockWs {
   size_t bytes;
 };
 
-BlockWs carve_block(void* base, int B, int T, int d, int I, mmf_dtype dt) {
+BlockWs carve_block(void* base, int B, int T, int d, int I, mmf_dtype dt, bool gnorm) {
   const int M = B * T;
   Carver c(base);
   BlockWs w;
@@ -697,6 +728,7 @@ BlockWs carve_block(void* base, int B, int T, int d, int I, mmf_dtype dt) {
   w.p = c.take<char>((size_t)M * I * e);
   w.ping = c.take<char>((size_t)M * d * e);
   w.pong = c.take<char>((size_t)M * d * e);
+  w.gn = gnorm ? c.take<char>(mlgru_scan_gnorm_ws_bytes(B, T, d)) : nullptr;
   w.bytes = c.off + 256;
   return w;
 }
@@ -714,7 +746,9 @@ bool decode_step_enabled() {
 bool decode_step_usable(const mmf_block* const* blocks, int L, int B, mmf_dtype dt) {
   if (!decode_step_enabled()) return false;
   for (int l = 0; l < L; ++l)
-    if (blocks[l]->I != blocks[0]->I || blocks[l]->d != blocks[0]->d || blocks[l]->ddesc == nullptr) return false;
+    if (blocks[l]->I != blocks[0]->I || blocks[l]->d != blocks[0]->d || blocks[l]->ddesc == nullptr ||
+        blocks[l]->w.gnorm != nullptr)
+      return false;
   return decode_step_supported(B, blocks[0]->d, blocks[0]->I, std::min(L, kDecodeMaxLayers), dt);
 }
 
@@ -813,9 +847,10 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   const mmf_block_weights& W = blk->w;
   const mmf_tlinear* fcg[3] = {&W.f, &W.c, &W.g};
   const bool want = dbg != nullptr;
+  const bool gnorm = W.gnorm != nullptr;
   if (T > 1 && (M >= kTcMinTokens || gemm_path_pref() >= 2)) ensure_prefill_codes(blk, s);
   // token mixer: x quantised once for f, c, g (shared gain)
-  if (T == 1) {
+  if (T == 1 && !gnorm) {
     // decode: projections and one recurrence step in one launch; h updated in place
     TGemmArgs a = gemm_args(fcg, 3, w.qa.q, w.qa.s, w.qa.qsum, M, w.og, d, nullptr, h);
     if (want) a.pre_out = dbg->pre;
@@ -832,8 +867,13 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
     int* status = nullptr;
     r = device_status_ptr(&status);
     if (r != MMF_OK) return r;
-    MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, status, s); }),
-             "block scan");
+    if (gnorm)
+      MMF_CUDA(timed("mlgru_scan_gnorm", s,
+                     [&] { return launch_mlgru_scan_gnorm(w.pre, dt, B, T, d, h, W.gnorm, eps, w.og, w.gn, status, s); }),
+               "block scan");
+    else
+      MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, status, s); }),
+               "block scan");
   }
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
@@ -873,7 +913,7 @@ mmf_status check_forward_args(const mmf_block* blk, mmf_state* st, const void* x
 
 extern "C" size_t mmf_block_ws_size(const mmf_block* blk, int32_t B, int32_t T) {
   if (!blk || B < 0 || T < 0) return 0;
-  return carve_block(nullptr, B, T, blk->d, blk->I, MMF_F32).bytes;
+  return carve_block(nullptr, B, T, blk->d, blk->I, MMF_F32, blk->w.gnorm != nullptr).bytes;
 }
 
 extern "C" mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf_state* st, const void* x, void* y,
@@ -883,7 +923,7 @@ extern "C" mmf_status mmf_block_forward(const mmf_block* blk, int32_t layer, mmf
   if (r != MMF_OK) return r;
   if (layer < 0 || layer >= st->L) return fail(MMF_ERR_INVALID_ARG, "mmf_block_forward: layer %d of %d", layer, st->L);
   if (T == 0) return MMF_OK;
-  BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype);
+  BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype, blk->w.gnorm != nullptr);
   if (ws_bytes < mmf_block_ws_size(blk, B, T))
     return fail(MMF_ERR_WORKSPACE, "mmf_block_forward: ws_bytes=%zu < %zu", ws_bytes, mmf_block_ws_size(blk, B, T));
   if (T == 1 && decode_step_usable(&blk, 1, B, dtype))
@@ -908,7 +948,7 @@ extern "C" mmf_status mmf_block_forward_debug(const mmf_block* blk, int32_t laye
   if (layer < 0 || layer >= st->L)
     return fail(MMF_ERR_INVALID_ARG, "mmf_block_forward_debug: layer %d of %d", layer, st->L);
   if (T == 0) return MMF_OK;
-  BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype);
+  BlockWs w = carve_block(ws, B, T, blk->d, blk->I, dtype, blk->w.gnorm != nullptr);
   if (ws_bytes < mmf_block_ws_size(blk, B, T))
     return fail(MMF_ERR_WORKSPACE, "mmf_block_forward_debug: ws_bytes=%zu < %zu", ws_bytes,
                 mmf_block_ws_size(blk, B, T));
@@ -934,12 +974,12 @@ extern "C" mmf_status mmf_stack_forward(const mmf_block* const* blocks, int32_t 
   if (ws_bytes < need) return fail(MMF_ERR_WORKSPACE, "mmf_stack_forward: ws_bytes=%zu < %zu", ws_bytes, need);
   cudaStream_t s = as_stream(stream);
   if (T == 1 && decode_step_usable(blocks, L, B, dtype)) {
-    BlockWs w = carve_block(ws, B, T, blocks[0]->d, blocks[0]->I, dtype);
+    BlockWs w = carve_block(ws, B, T, blocks[0]->d, blocks[0]->I, dtype, false);
     return run_decode_step(blocks, L, 0, st, x, y, w.ping, B, dtype, eps, s, nullptr);
   }
   const void* cur = x;
   for (int l = 0; l < L; ++l) {
-    BlockWs w = carve_block(ws, B, T, blocks[l]->d, blocks[l]->I, dtype);
+    BlockWs w = carve_block(ws, B, T, blocks[l]->d, blocks[l]->I, dtype, blocks[l]->w.gnorm != nullptr);
     void* dst = (l == L - 1) ? y : ((l % 2 == 0) ? w.ping : w.pong);
     mmf_status r = block_forward_impl(blocks[l], mmf_state_layer(st, l), cur, dst, B, T, dtype, eps, w, s);
     if (r != MMF_OK) return r;

@@ -154,5 +154,13 @@ cudaError_t launch_decode_step(DecodeStepArgs a, mmf_dtype dt, cudaStream_t stre
 size_t mlgru_scan_ws_bytes(int B, int T, int d);
 cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, int* status,
                               cudaStream_t stream);
+// The same recurrence with the g_norm output gate: the scan writes
+// v = swish(g~) h (fp32) and per-(token, channel block) sums of h^2 into `ws`
+// (mlgru_scan_gnorm_ws_bytes), then a row kernel writes
+// o' = v / sqrt(mean h^2 + eps) * gain in dtype. Two launches, each a
+// programmatic dependent of the one before.
+size_t mlgru_scan_gnorm_ws_bytes(int B, int T, int d);
+cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, const float* gain,
+                                    float eps, void* o, void* ws, int* status, cudaStream_t stream);
 
 }  // namespace mmf

@@ -10,6 +10,14 @@
 // The gates live only in registers: the kernel reads the three pre-activation
 // rows once and writes o' and the final state, nothing else.
 //
+// g_norm output gate (the hysenlabs review, same section: g_norm is a
+// FusedRMSNormSwishGate). o'_t = h_t / sqrt(mean_n h_t^2 + eps) * w * swish(g~_t)
+// needs the whole token row of h, which no CTA holds, so it takes two
+// kernels: the scan (GN = true) computes swish(g~) in place of sigmoid(g~),
+// writes v_t = swish(g~_t) h_t in fp32 and, per token and channel block, the
+// partial sum of h_t^2; gnorm_apply_kernel adds a row's partials and writes
+// o' = v * (1 / sqrt(sum / d + eps)) * w in the storage type.
+//
 // Work split. A CTA owns CC channels of one sequence and walks that
 // sequence's chunks of TC = 128 steps in order, carrying the state from one
 // chunk to the next, so no CTA ever waits for another. A TMA ring keeps the
@@ -34,6 +42,8 @@
 // reads it). Every wait on the ring is bounded: on timeout the kernel records
 // status code 2 and returns (its output is then invalid; mmf_check reports
 // MMF_ERR_TIMEOUT).
+#include <type_traits>
+
 #include "kernels.cuh"
 #include "tma.cuh"
 
@@ -141,6 +151,8 @@ __device__ __forceinline__ F2 exp_neg(F2 z) {   // e^-z per lane (z >= -29, so a
 // Every z is at least -29 (see load_z), so the product stays finite
 // ((1 + e^29)^3 < 2^127); below -29 a logistic is under 3e-13 and the floor
 // moves it by less than that.
+// With SWISH the third term is the swish gate g = zg sigmoid(zg) = zg p_f p_c r.
+template <bool SWISH>
 __device__ __forceinline__ void gates2(F2 zf, F2 zc, F2 zg, F2& f, F2& b, F2& g) {
   const F2 one = f2(1.0f, 1.0f);
   const F2 ef = exp_neg(zf);
@@ -151,8 +163,32 @@ __device__ __forceinline__ void gates2(F2 zf, F2 zc, F2 zg, F2& f, F2& b, F2& g)
   const F2 pp = mul2(pfc, pg);
   const F2 r = f2(rcp_approx(lo(pp)), rcp_approx(hi(pp)));
   f = mul2(mul2(pc, pg), r);
-  g = mul2(pfc, r);
+  g = SWISH ? mul2(zg, mul2(pfc, r)) : mul2(pfc, r);
   b = mul2(mul2(mul2(zc, ef), pg), r);
+}
+
+// Sums of q[k] (one value per step k of the lane) over the NP lanes of the
+// lane's step group. Reduce-scatter by halving: at offset NP/2 a lane keeps the
+// half of its steps picked by that lane bit and adds its partner's copy of it,
+// and so on down to one value at offset NP/LS; plain xor-adds over the lower
+// offsets finish the sum. Returns the total of step (lane % NP) / (NP / LS),
+// log2(LS) + log2(NP / LS) rounds and LS - 1 + log2(NP / LS) shuffles.
+template <int NP, int LS>
+__device__ __forceinline__ float group_step_sum(float (&q)[LS], int lane) {
+#pragma unroll
+  for (int n = LS, o = NP / 2; n > 1; n >>= 1, o >>= 1) {
+    const bool up = (lane & o) != 0;
+#pragma unroll
+    for (int i = 0; i < n / 2; ++i) {
+      const float keep = up ? q[i + n / 2] : q[i];
+      const float send = up ? q[i] : q[i + n / 2];
+      q[i] = keep + __shfl_xor_sync(0xffffffffu, send, o);
+    }
+  }
+  float t = q[0];
+#pragma unroll
+  for (int o = NP / LS / 2; o > 0; o >>= 1) t += __shfl_xor_sync(0xffffffffu, t, o);
+  return t;
 }
 
 
@@ -165,10 +201,15 @@ __device__ void drain_stage(uint64_t* bar, uint32_t parity, long long limit) {
 }
 
 // CC = 32 keeps at most 64 registers per thread so that two CTAs share an SM.
-template <typename T, int CC>
+// GN: g_norm mode; `o` receives v = swish(g~) h in fp32 and `ss` [B*T_][n_cb]
+// the partial sums of h^2 (see the file comment). Otherwise `o` receives o'.
+template <typename T, int CC, bool GN>
 __global__ void __launch_bounds__(kThreads, 64 / CC)
     mlgru_scan_kernel(const __grid_constant__ CUtensorMap map, int B, int T_, int d, int n_cb, int nst,
-                      float* __restrict__ h, T* __restrict__ o, int* status, long long wait_cycles, int skip_chunk) {
+                      float* __restrict__ h, void* __restrict__ out, float* __restrict__ ss, int* status,
+                      long long wait_cycles, int skip_chunk) {
+  using OT = std::conditional_t<GN, float, T>;
+  OT* __restrict__ o = static_cast<OT*>(out);
   using S = ScanSmem<CC>;
   constexpr int NP = S::NP;         // channel pairs: lanes per step group
   constexpr int H = 32 / NP;        // lane groups splitting the warp's steps (1 or 2)
@@ -225,8 +266,8 @@ __global__ void __launch_bounds__(kThreads, 64 / CC)
     for (int k = 0; k < LS; ++k) {
       const int tl = tw + k;
       if (full || t0 + tl < T_) {
-        gates2(load_z(&tile[0][tl][2 * pr]), load_z(&tile[1][tl][2 * pr]), load_z(&tile[2][tl][2 * pr]), f[k], bb[k],
-               gg[k]);
+        gates2<GN>(load_z(&tile[0][tl][2 * pr]), load_z(&tile[1][tl][2 * pr]), load_z(&tile[2][tl][2 * pr]), f[k],
+                   bb[k], gg[k]);
       } else {   // past the end of the sequence: identity map
         f[k] = f2(1.0f, 1.0f);
         bb[k] = f2(0.0f, 0.0f);
@@ -270,14 +311,28 @@ __global__ void __launch_bounds__(kThreads, 64 / CC)
     if constexpr (H == 2) {
       if (grp == 1) hw = fma2(A0, hw, B0);
     }
-    // 3. replay this lane's steps and store o'
+    // 3. replay this lane's steps and store o' (GN: v and the squares' partial sums)
+    float sq[LS];
     if (valid) {
-      T* op = o + ((size_t)b * T_ + t0 + tw) * d + ch;
+      OT* op = o + ((size_t)b * T_ + t0 + tw) * d + ch;
 #pragma unroll
       for (int k = 0; k < LS; ++k) {
         hw = fma2(f[k], hw, bb[k]);
         if (full || t0 + tw + k < T_) store_pair(op + (size_t)k * d, mul2(gg[k], hw));
+        if constexpr (GN) {
+          const F2 h2 = mul2(hw, hw);
+          sq[k] = lo(h2) + hi(h2);
+        }
       }
+    } else {
+#pragma unroll
+      for (int k = 0; k < LS; ++k) sq[k] = 0.0f;
+    }
+    if constexpr (GN) {
+      const float tot = group_step_sum<NP, LS>(sq, lane);
+      const int k = (lane % NP) / (NP / LS);   // the step whose total this lane holds
+      if (lane % (NP / LS) == 0 && (full || t0 + tw + k < T_))
+        ss[((size_t)b * T_ + t0 + tw + k) * n_cb + cb] = tot;
     }
   }
   __syncthreads();   // the last warp has written the state leaving the last chunk
@@ -287,9 +342,9 @@ __global__ void __launch_bounds__(kThreads, 64 / CC)
   }
 }
 
-template <typename T, int CC>
-cudaError_t launch_typed(const void* pre, int B, int T_, int d, float* h, void* o, int* status, long long wait_cycles,
-                         int skip_chunk, cudaStream_t stream) {
+template <typename T, int CC, bool GN>
+cudaError_t launch_typed(const void* pre, int B, int T_, int d, float* h, void* o, float* ss, int* status,
+                         long long wait_cycles, int skip_chunk, cudaStream_t stream) {
   CUtensorMap map;
   const CUtensorMapDataType dt = sizeof(T) == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
   // box = one gate of one chunk (CC channels x TC steps); a stage holds 3 boxes
@@ -301,12 +356,50 @@ cudaError_t launch_typed(const void* pre, int B, int T_, int d, float* h, void* 
   const size_t budget = CC == 32 ? 96 * 1024 : 192 * 1024;   // two CTAs per SM with CC = 32
   const int nst = (int)std::max<size_t>(2, std::min<size_t>(kMaxStages, budget / stage_bytes));
   const size_t smem = 128 + tiles_offset<CC>() + nst * stage_bytes;
-  auto kern = mlgru_scan_kernel<T, CC>;
+  auto kern = mlgru_scan_kernel<T, CC, GN>;
   const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
-  return launch_pdl(kern, dim3(B * n_cb), dim3(kThreads), smem, stream, map, B, T_, d, n_cb, nst, h,
-                    static_cast<T*>(o), status, wait_cycles, skip_chunk);
+  return launch_pdl(kern, dim3(B * n_cb), dim3(kThreads), smem, stream, map, B, T_, d, n_cb, nst, h, o, ss, status,
+                    wait_cycles, skip_chunk);
 }
+
+// o'[m, :] = v[m, :] * (1 / sqrt(sum_c ss[m, c] / d + eps)) * gain, one warp per
+// token row, four channels per lane per step (16-byte loads of v and gain).
+template <typename T>
+__global__ void __launch_bounds__(256) gnorm_apply_kernel(const float* __restrict__ v, const float* __restrict__ ss,
+                                                          int n_cb, const float* __restrict__ gain, float eps, int M,
+                                                          int d, T* __restrict__ o) {
+  const int lane = threadIdx.x & 31;
+  const int nw = gridDim.x * (blockDim.x >> 5);
+  pdl_trigger();
+  pdl_wait();   // v and ss are the scan's output
+  for (int m = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); m < M; m += nw) {
+    float t = 0.0f;
+    for (int c = lane; c < n_cb; c += 32) t += ss[(size_t)m * n_cb + c];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    const float rinv = __frsqrt_rn(__fadd_rn(__fdiv_rn(t, (float)d), eps));
+    const float4* vr = reinterpret_cast<const float4*>(v + (size_t)m * d);
+    const float4* gr = reinterpret_cast<const float4*>(gain);
+    T* orow = o + (size_t)m * d;
+    for (int k = lane; k < d / 4; k += 32) {
+      const float4 x = vr[k], g = gr[k];
+      const float y0 = x.x * rinv * g.x, y1 = x.y * rinv * g.y, y2 = x.z * rinv * g.z, y3 = x.w * rinv * g.w;
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(y0, y1), b = __floats2bfloat162_rn(y2, y3);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&a);
+        w.y = *reinterpret_cast<const uint32_t*>(&b);
+        *reinterpret_cast<uint2*>(orow + 4 * k) = w;
+      } else {
+        *reinterpret_cast<float4*>(orow + 4 * k) = make_float4(y0, y1, y2, y3);
+      }
+    }
+  }
+}
+
+// 64 channels per CTA when that gives enough CTAs to cover the GPU, else 32
+bool scan_wide(int B, int d) { return (size_t)B * ceil_div(d, 64) >= (size_t)num_sms() * 3 / 4; }
 
 }  // namespace
 
@@ -318,14 +411,45 @@ cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d
   if (!tma_available()) return cudaErrorNotSupported;
   const long long wait = wait_limit_cycles();
   const int skip = test_hook("MMF_SCAN_SKIP_CHUNK");
-  // 32 channels per CTA (two CTAs per SM) unless 64-channel CTAs alone fill every SM twice
-  // 64 channels per CTA when that gives enough CTAs to cover the GPU, else 32
-  const bool wide = (size_t)B * ceil_div(d, 64) >= (size_t)num_sms() * 3 / 4;
+  const bool wide = scan_wide(B, d);
   if (dt == MMF_BF16)
-    return wide ? launch_typed<bf16, 64>(pre, B, T, d, h, o, status, wait, skip, stream)
-                : launch_typed<bf16, 32>(pre, B, T, d, h, o, status, wait, skip, stream);
-  return wide ? launch_typed<float, 64>(pre, B, T, d, h, o, status, wait, skip, stream)
-              : launch_typed<float, 32>(pre, B, T, d, h, o, status, wait, skip, stream);
+    return wide ? launch_typed<bf16, 64, false>(pre, B, T, d, h, o, nullptr, status, wait, skip, stream)
+                : launch_typed<bf16, 32, false>(pre, B, T, d, h, o, nullptr, status, wait, skip, stream);
+  return wide ? launch_typed<float, 64, false>(pre, B, T, d, h, o, nullptr, status, wait, skip, stream)
+              : launch_typed<float, 32, false>(pre, B, T, d, h, o, nullptr, status, wait, skip, stream);
+}
+
+size_t mlgru_scan_gnorm_ws_bytes(int B, int T, int d) {
+  const size_t M = (size_t)B * T;
+  return (M * d * sizeof(float) + 255) / 256 * 256 + M * ceil_div(d, 32) * sizeof(float) + 256;
+}
+
+cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, const float* gain,
+                                    float eps, void* o, void* ws, int* status, cudaStream_t stream) {
+  if (B == 0 || T == 0) return cudaSuccess;
+  if (!tma_available()) return cudaErrorNotSupported;
+  const size_t M = (size_t)B * T;
+  float* v = static_cast<float*>(ws);
+  float* ss = reinterpret_cast<float*>(static_cast<char*>(ws) + (M * d * sizeof(float) + 255) / 256 * 256);
+  const long long wait = wait_limit_cycles();
+  const int skip = test_hook("MMF_SCAN_SKIP_CHUNK");
+  const bool wide = scan_wide(B, d);
+  const int n_cb = ceil_div(d, wide ? 64 : 32);
+  cudaError_t e;
+  if (dt == MMF_BF16)
+    e = wide ? launch_typed<bf16, 64, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream)
+             : launch_typed<bf16, 32, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream);
+  else
+    e = wide ? launch_typed<float, 64, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream)
+             : launch_typed<float, 32, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream);
+  if (e != cudaSuccess) return e;
+  constexpr int kWarpsA = 8;
+  const int grid = (int)std::max<size_t>(1, std::min<size_t>((M + kWarpsA - 1) / kWarpsA, (size_t)num_sms() * 8));
+  if (dt == MMF_BF16)
+    return launch_pdl(gnorm_apply_kernel<bf16>, dim3(grid), dim3(32 * kWarpsA), 0, stream, (const float*)v,
+                      (const float*)ss, n_cb, gain, eps, (int)M, d, static_cast<bf16*>(o));
+  return launch_pdl(gnorm_apply_kernel<float>, dim3(grid), dim3(32 * kWarpsA), 0, stream, (const float*)v,
+                    (const float*)ss, n_cb, gain, eps, (int)M, d, static_cast<float*>(o));
 }
 
 }  // namespace mmf

@@ -109,8 +109,8 @@ def record_drift(name: str, data) -> None:
             json.dump(data, f, indent=1)
 
 
-def make_block(seed: int, d: int, inner: int, layer: int = 0, cache: bool = False):
-    """GPU Block + oracle Block from the same latents."""
+def make_block(seed: int, d: int, inner: int, layer: int = 0, cache: bool = False, gnorm: bool = False):
+    """GPU Block + oracle Block from the same latents (gnorm: with a seeded g_norm gain)."""
     from ternary_weight_matmul_fusedbitlinear_b200 import Block, quantize_weights
     shapes = {"f": (d, d), "c": (d, d), "g": (d, d), "o": (d, d), "gate": (inner, d), "up": (inner, d),
               "down": (d, inner)}
@@ -119,7 +119,16 @@ def make_block(seed: int, d: int, inner: int, layer: int = 0, cache: bool = Fals
         W = synth.latent_weight(synth.sub_seed(seed, layer, i), *shapes[name])
         lat[name] = W.numpy()
         lins[name] = quantize_weights(W.cuda())
-    return Block(lins), O.make_block(lat, cache=cache)
+    gain = synth.gains(synth.sub_seed(seed, layer, 7), d) if gnorm else None
+    return (Block(lins, None if gain is None else gain.cuda()),
+            O.make_block(lat, cache=cache, gnorm=None if gain is None else gain.numpy()))
+
+
+def scan_ref(pf, pc, pg, h0, oblk):
+    """The oracle's scan with the block's output gate (sigmoid, or g_norm when the block has a gain)."""
+    if oblk.gnorm is None:
+        return O.mlgru_scan(pf, pc, pg, h0)
+    return O.mlgru_scan_gnorm(pf, pc, pg, h0, oblk.gnorm)
 
 
 def check_block_stages(x, h0, y, hT, dbg, oblk, dtype: str, what: str = "", seqs=None) -> dict:
@@ -166,7 +175,7 @@ def check_block_stages(x, h0, y, hT, dbg, oblk, dtype: str, what: str = "", seqs
         errs[name] = assert_close(pre[:, :, j], _forced_bitlinear(xn, lin, qg[0], tag + "codes of x"), dtype,
                                   tag + name)
     # 2. gates and scan on the stored pre-activations
-    o_ref, h_ref = O.mlgru_scan(pre[:, :, 0], pre[:, :, 1], pre[:, :, 2], h0)
+    o_ref, h_ref = scan_ref(pre[:, :, 0], pre[:, :, 1], pre[:, :, 2], h0, oblk)
     errs["o'"] = assert_close(og, o_ref, dtype, tag + "o'")
     errs["h_T"] = assert_close(hg, h_ref, "f32", tag + "h_T")
     # 3. o projection + residual on the stored o'
@@ -215,7 +224,7 @@ def check_block_tie_forced(x, h0, y, hT, dbg, oblk, dtype: str, what: str = "", 
     pf = O.store(_forced_bitlinear(xn, oblk.f, q0, tag + "codes of x"), dtype)
     pc = O.store(_forced_bitlinear(xn, oblk.c, q0, tag + "codes of x"), dtype)
     pg = O.store(_forced_bitlinear(xn, oblk.g, q0, tag + "codes of x"), dtype)
-    og, h_ref = O.mlgru_scan(pf, pc, pg, h0)
+    og, h_ref = scan_ref(pf, pc, pg, h0, oblk)
     og = O.store(og, dtype)
     y1 = O.store(xn + _forced_bitlinear(og, oblk.o, q_of(1, d), tag + "codes of o'"), dtype)
     q2 = q_of(2, d)

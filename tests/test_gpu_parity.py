@@ -137,6 +137,46 @@ def test_scan_closed_forms_on_gpu():
     assert_close(to_np(o), g * 7.0, "f32", "f=1")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("b,t,d", [(2, 64, 256), (1, 3, 16), (3, 200, 264), (8, 1, 1024), (4, 517, 2048),
+                                   (8, 300, 2560)])
+def test_scan_gnorm_parity(b, t, d, dtype):
+    # the g_norm output gate: both CTA widths, ragged chunks and channel blocks, T = 1
+    pre = synth.preacts(420 + t, b, t, d, TORCH_DT[dtype], scale=2.0)
+    h0 = synth.activations(421, b, d)
+    gain = synth.gains(422, d)
+    h = h0.cuda().clone()
+    o = mmf.mlgru_scan_gnorm(pre.cuda(), h, gain.cuda())
+    mmf.check()
+    p = to_np(pre)
+    o_ref, h_ref = O.mlgru_scan_gnorm(p[:, :, 0], p[:, :, 1], p[:, :, 2], h0.numpy().astype(np.float64),
+                                      gain.numpy())
+    assert_close(to_np(o), o_ref, dtype, "o' (g_norm)")
+    assert_close(to_np(h), h_ref, "f32", "h_T (g_norm)")
+
+
+def test_scan_gnorm_closed_forms_on_gpu():
+    b, t, d = 2, 150, 64
+    pre = synth.preacts(423, b, t, d)
+    ones = torch.ones(d, device="cuda")
+    # g~ = 0: swish(0) = 0, so o' = 0 exactly whatever the state
+    z0 = pre.clone()
+    z0[:, :, 2] = 0.0
+    o = mmf.mlgru_scan_gnorm(z0.cuda(), torch.full((b, d), 3.0, device="cuda"), ones)
+    assert torch.all(o == 0)
+    # constant g~ = z, unit gain: each token's mean of o'^2 is swish(z)^2 ms / (ms + eps), ms the
+    # mean square of that token's state, read from the sigmoid-gate scan with g~ = 1e4 (o' = h)
+    z, eps = 0.8, 1e-3
+    zc = pre.clone()
+    zc[:, :, 2] = z
+    o = mmf.mlgru_scan_gnorm(zc.cuda(), torch.zeros(b, d, device="cuda"), ones, eps=eps)
+    zh = pre.clone()
+    zh[:, :, 2] = 1e4
+    hs = to_np(mmf.mlgru_scan(zh.cuda(), torch.zeros(b, d, device="cuda")))
+    ms = np.mean(hs * hs, axis=-1)
+    np.testing.assert_allclose(np.mean(to_np(o) ** 2, axis=-1), O.silu(z) ** 2 * ms / (ms + eps), rtol=1e-5)
+
+
 def test_scan_wait_gives_up_and_reports(monkeypatch):
     # failure detection without a fault: chunk 1 of CTA 0 is never loaded, so
     # its bounded wait runs out (20 ms); the kernel lets its other copies land

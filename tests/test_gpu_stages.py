@@ -112,3 +112,39 @@ def test_block_stages_with_gains_and_biases():
         y, hT, dbg = _run(blk, x, h0, "bf16")
         check_block_stages(x, h0, y, hT, dbg, oblk, "bf16", f"gains and biases T={T}")
         check_block_tie_forced(x, h0, y, hT, dbg, oblk, "bf16", f"gains and biases T={T}")
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("B,T", [(3, 100), (1, 5), (4, 1), (9, 1)])
+def test_block_gnorm_stages(B, T, dtype):
+    # the g_norm output gate (seeded non-unit gain): prefill on the tensor-core
+    # (M = 300) and warp-MMA (M = 5) contractions, and decode steps, which run
+    # the prefill sequence with T = 1; every stage teacher-forced at TOL
+    d, inner = 256, 768
+    blk, oblk = make_block(8500 + T + B, d, inner, gnorm=True)
+    x = synth.activations(8501 + T, B * T, d, TORCH_DT[dtype]).reshape(B, T, d)
+    h0 = synth.activations(8502, B, d).numpy().astype(np.float64) * 0.5
+    y, hT, dbg = _run(blk, x, h0, dtype)
+    check_block_stages(x, h0, y, hT, dbg, oblk, dtype, f"g_norm B={B} T={T}")
+    check_block_tie_forced(x, h0, y, hT, dbg, oblk, dtype, f"g_norm B={B} T={T}")
+
+
+def test_block_gnorm_prefill_then_decode():
+    # a g_norm block: a 40-token prompt, then 8 decode steps from the GPU's
+    # state, each step teacher-forced; the whole run against the oracle's
+    # block at the composite tolerance
+    d, inner, B, T, S = 256, 768, 2, 40, 8
+    blk, oblk = make_block(8600, d, inner, gnorm=True)
+    x = synth.activations(8601, B * (T + S), d, torch.bfloat16).reshape(B, T + S, d)
+    st = mmf.State(1, B, d)
+    ys = [mmf.block_forward(blk, 0, st, x[:, :T].contiguous().cuda())]
+    for t in range(T, T + S):
+        h_prev = st.get()[0].numpy().astype(np.float64)
+        xt = x[:, t:t + 1].contiguous()
+        y, dbg = mmf.block_forward_debug(blk, 0, st, xt.cuda())
+        check_block_stages(xt, h_prev, y, st.get()[0].numpy(), dbg, oblk, "bf16", f"g_norm step {t}")
+        ys.append(y)
+    mmf.check()
+    y_ref, h_ref = O.block_forward(x.float().numpy(), oblk, np.zeros((B, d)), "bf16")
+    assert_close(to_np(torch.cat(ys, 1)), y_ref, "bf16", "g_norm prompt + decode y", tol=E2E_TOL)
+    assert_close(st.get()[0].numpy(), h_ref, "f32", "g_norm prompt + decode h_T", tol=E2E_TOL)
