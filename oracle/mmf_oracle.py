@@ -36,6 +36,9 @@ prefill == decode invariant. The pages print no worked example for them.
 The g_norm output gate (``rmsnorm_swish_gate``) is pinned by a hand-worked
 two-channel case, g~ = 0 giving o' = 0, the mean-square invariant under a
 constant gate, scale invariance, and the identity-weight block.
+The model ends (``embed``, ``lm_logits``, ``greedy_token``, ``model_forward``,
+``generate_greedy``) are pinned by brute force on small tables, ties, and a
+generation that follows a known permutation (zero blocks, identity head).
 """
 from __future__ import annotations
 
@@ -476,3 +479,72 @@ def stack_forward(x, blocks, h0s, dtype: str, eps: float = EPS_NORM):
         x, h = block_forward(x, blk, h0s[l], dtype, eps)
         hs.append(h)
     return x, np.stack(hs)
+
+
+# ---------------------------------------------------------------------------
+# Model ends: embedding lookup, LM head, greedy next token
+# ---------------------------------------------------------------------------
+
+
+def embed(ids, table, dtype: str) -> np.ndarray:
+    """Token embedding: x[m] = E[ids[m]], stored in the run dtype.
+
+    [HL] "Install and model initialisation": the default configuration has an
+    embedding of 32000 entries at hidden size 2048. A lookup is a row copy;
+    an id outside [0, V) is an error (IndexError).
+    """
+    ids = np.asarray(ids, dtype=np.int64)
+    E = np.asarray(table, dtype=np.float64)
+    if ids.size and (ids.min() < 0 or ids.max() >= E.shape[0]):
+        raise IndexError("token id outside [0, V)")
+    return store(E[ids], dtype)
+
+
+def lm_logits(x, head: TLinear, dtype: str, eps: float = EPS_NORM) -> np.ndarray:
+    """Logits of the language-model head, stored in the run dtype.
+
+    [HL] "FusedBitLinear": every linear projection of the model is a
+    FusedBitLinear. Reading: so is the head, logits = BitLinear_head(x)
+    ([d] -> [V]); its own RMSNorm is the final norm.
+    """
+    return store(bitlinear(x, head, eps), dtype)
+
+
+def greedy_token(logits) -> np.ndarray:
+    """Index of the largest logit of each row, the lowest index on ties.
+
+    [HL] "Official generation example" samples the next token (top-p 0.4,
+    temperature 0.6); the deterministic reading taken for the on-device loop
+    is greedy decoding, the argmax of the stored logits.
+    """
+    L = np.asarray(logits, dtype=np.float64)
+    return np.argmax(L, axis=-1).astype(np.int64)   # first occurrence of the maximum
+
+
+def model_forward(ids, table, blocks, head: TLinear, h0s, dtype: str, eps: float = EPS_NORM):
+    """Embedding -> L blocks -> LM head on the last token of each sequence.
+
+    ids [B, T] -> (logits [B, V] of token T-1, h_T [L, B, d]).
+    """
+    x = embed(ids, table, dtype)
+    y, hs = stack_forward(x, blocks, h0s, dtype, eps)
+    return lm_logits(y[:, -1], head, dtype, eps), hs
+
+
+def generate_greedy(prompt, n: int, table, blocks, head: TLinear, dtype: str, eps: float = EPS_NORM):
+    """Greedy generation of n tokens after a prompt [B, T0] (T0 >= 1), state carried.
+
+    The prompt runs as one prefill; each new token is the greedy token of the
+    previous step's logits and is fed back as a one-token step.
+    Returns (tokens [B, n], h_T [L, B, d]).
+    """
+    prompt = np.asarray(prompt, dtype=np.int64)
+    B = prompt.shape[0]
+    d = blocks[0].d
+    logits, hs = model_forward(prompt, table, blocks, head, np.zeros((len(blocks), B, d)), dtype, eps)
+    out = []
+    for _ in range(n):
+        tok = greedy_token(logits)
+        out.append(tok)
+        logits, hs = model_forward(tok[:, None], table, blocks, head, hs, dtype, eps)
+    return np.stack(out, axis=1) if out else np.zeros((B, 0), np.int64), hs

@@ -634,3 +634,87 @@ def test_stack_composes_blocks():
         z, h = O.block_forward(z, blocks[l], h0s[l], "f32")
         np.testing.assert_array_equal(h, hs[l])
     np.testing.assert_array_equal(z, y)
+
+
+# ----------------------------------------------------------------- model ends
+
+def test_embed_brute_force_and_range():
+    E = synth.activations(70, 7, 5).numpy()
+    ids = np.array([[3, 0, 6], [6, 6, 1]])
+    x = O.embed(ids, E, "bf16")
+    for b in range(2):
+        for t in range(3):
+            for k in range(5):
+                assert x[b, t, k] == O.round_bf16(float(E[ids[b, t], k]))
+    np.testing.assert_array_equal(O.embed(ids, E, "f32"), O.round_f32(E[ids]))
+    for bad in ([[-1]], [[7]]):
+        with pytest.raises(IndexError):
+            O.embed(np.array(bad), E, "f32")
+
+
+def test_greedy_token_brute_force_and_ties():
+    rng = np.random.default_rng(71)
+    L = rng.integers(-3, 4, size=(40, 9)).astype(np.float64)   # many ties
+    tok = O.greedy_token(L)
+    for r in range(40):
+        best = 0
+        for j in range(1, 9):
+            if L[r, j] > L[r, best]:
+                best = j
+        assert tok[r] == best
+    assert O.greedy_token(np.array([[-5.0, -5.0, -7.0]]))[0] == 0
+    assert O.greedy_token(np.array([[1.0]]))[0] == 0
+
+
+def test_lm_logits_identity_head_closed_form():
+    d = 32
+    head = _scaled_eye(d, 1.5)
+    x = synth.activations(72, 6, d).numpy()
+    np.testing.assert_array_equal(O.lm_logits(x, head, "bf16"), O.round_bf16(_dq(head, x)))
+
+
+def _zero_block(d, inner):
+    z = {n: np.zeros(s, np.float32) for n, s in (("f", (d, d)), ("c", (d, d)), ("g", (d, d)), ("o", (d, d)),
+                                                  ("gate", (inner, d)), ("up", (inner, d)), ("down", (d, inner)))}
+    return O.make_block(z)
+
+
+def test_generation_follows_a_permutation():
+    # zero blocks are the identity and the head is the identity, so the next
+    # token is the position of the largest entry of the current token's
+    # embedding row: a table whose row i peaks at perm[i] makes greedy
+    # generation follow the permutation
+    V = d = 16
+    perm = np.random.default_rng(73).permutation(V)
+    E = 0.1 * synth.activations(74, V, d).numpy()
+    E[np.arange(V), perm] = 3.0
+    blocks = [_zero_block(d, 24) for _ in range(2)]
+    head = _scaled_eye(d, 1.0)
+    prompt = np.array([[5, 2, 9], [0, 0, 3]])
+    toks, hs = O.generate_greedy(prompt, 6, E, blocks, head, "bf16")
+    for b in range(2):
+        t = prompt[b, -1]
+        for k in range(6):
+            t = perm[t]
+            assert toks[b, k] == t
+    assert np.all(hs == 0.0)
+
+
+def test_generation_matches_prefill_of_the_grown_sequence():
+    # each generated token is also the greedy token of one prefill over the
+    # prompt and the tokens before it (state carried vs recomputed, fp32 runs)
+    V, d, inner = 40, 32, 48
+    blocks = [_block(75 + l, d, inner) for l in range(2)]
+    head = O.make_tlinear(synth.latent_weight(77, V, d).numpy())
+    E = synth.activations(78, V, d).numpy()
+    prompt = np.array([[3, 17, 8, 8]])
+    toks, hs = O.generate_greedy(prompt, 3, E, blocks, head, "f32")
+    for k in range(3):
+        seq = np.concatenate([prompt, toks[:, :k]], axis=1)
+        logits, _ = O.model_forward(seq, E, blocks, head, np.zeros((2, 1, d)), "f32")
+        assert O.greedy_token(logits)[0] == toks[0, k]
+        srt = np.sort(logits[0])
+        assert srt[-1] - srt[-2] > 1e-3   # no near-tie that rounding could flip
+    # the carried state after the last fed-back token is the prefill's state over everything
+    _, h_all = O.model_forward(np.concatenate([prompt, toks], axis=1), E, blocks, head, np.zeros((2, 1, d)), "f32")
+    np.testing.assert_allclose(hs, h_all, rtol=1e-5, atol=1e-6)
