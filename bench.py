@@ -52,14 +52,17 @@ def parse_args(argv=None):
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["mmf", "reference"], default="mmf")
-    ap.add_argument("--workload", choices=["stack370m", "bitlinear", "scan", "gemv", "decode1p3b", "decode2p7b"],
+    ap.add_argument("--workload", choices=["stack370m", "bitlinear", "scan", "gemv", "decode1p3b", "decode2p7b",
+                                           "model2p7b"],
                     default="stack370m",
                     help="stack370m: the 370M-shaped 24-block prefill (default); bitlinear: one prefill "
                          "BitLinear of the 370M gate|up shape (16384 tokens, 1024 -> 5632); scan: one MLGRU "
                          "scan of the 370M layer shape (8 x 2048 tokens, d=1024); gemv: the decode BitLinear "
                          "sweep (2048->2048, 2048->5632, 5632->2048 at 1/4/16 tokens) over a weight pool > L2; "
                          "decode1p3b / decode2p7b: the 1.3B / 2.7B-shaped stacks, prompt prefill then decode "
-                         "steps (output fed back, state carried), each step one CUDA graph")
+                         "steps (output fed back, state carried), each step one CUDA graph; model2p7b: greedy "
+                         "generation through the 2.7B-shaped model (embedding, 32 blocks, 32000-entry head, "
+                         "argmax), one CUDA graph per token")
     ap.add_argument("--batch", type=int, default=None, help="decode2p7b: concurrent sequences (1, 8 or 64)")
     ap.add_argument("--decode-steps", type=int, default=None,
                     help="decode1p3b/decode2p7b: timed decode steps (default: the workload's own count)")
@@ -522,9 +525,14 @@ def run_mmf(args):
         torch.cuda.empty_cache()
         sub = {"kernels_in_step": others}
         w27 = synth.STACK_2P7B
-        d27 = measure_decode(mmf, w27, 1, 128, 3, dev, peaks, prompt=False)
+        blocks27 = build_stack(w27, dev)
+        d27 = measure_decode(mmf, w27, 1, 128, 3, dev, peaks, prompt=False, blocks=blocks27)
         sub["decode_2p7b_b1"] = {k: d27[k] for k in ("ms_per_step", "tokens_per_s", "GBps", "frac", "bytes_per_step",
                                                       "launches_per_step", "decode_steps", "clocks")}
+        m27 = measure_model_decode(mmf, w27, 1, 128, 3, dev, peaks, blocks=blocks27)
+        sub["model_2p7b_greedy_b1"] = {k: m27[k] for k in ("ms_per_step", "tokens_per_s", "GBps", "frac",
+                                                            "bytes_per_step", "launches_per_step", "vocab")}
+        del blocks27
         torch.cuda.empty_cache()
         sub["gemv_sweep"] = measure_gemv(mmf, dev, 2, 3, peaks)
         for gn in (False, True):
@@ -822,6 +830,96 @@ def measure_decode(mmf, w, B: int, steps: int, warmup: int, dev, peaks, prompt: 
     return out
 
 
+VOCAB = 32000   # the embedding size of the default configuration (hysenlabs review, "Install and model initialisation")
+
+
+def measure_model_decode(mmf, w, B: int, steps: int, warmup: int, dev, peaks, blocks=None) -> dict:
+    """Greedy generation through the whole model: per token the embedding lookup, every block's decode
+    step, the LM head (BitLinear d -> 32000) and the argmax, the token fed back on the device; one CUDA
+    graph replay per token. Algorithmic bytes per token: the packed weights of the blocks and the head,
+    the state read and written, the embedding rows and the logits written and read."""
+    blocks = blocks if blocks is not None else build_stack(w, dev)
+    head = mmf.quantize_weights(synth.latent_weight(synth.sub_seed(w.seed, w.layers, 7), VOCAB, w.d, device=dev))
+    table = synth.activations(w.seed + 7, VOCAB, w.d, torch.bfloat16, device=str(dev))
+    st = mmf.State(w.layers, B, w.d)
+    ids = torch.randint(0, VOCAB, (B,), dtype=torch.int32, device=dev)
+    x = torch.empty(B, 1, w.d, dtype=torch.bfloat16, device=dev)
+    y = torch.empty_like(x)
+    ws = torch.empty(mmf.stack_ws_size(blocks, B, 1), dtype=torch.uint8, device=dev)
+    ws_h = torch.empty(mmf.load().mmf_bitlinear_ws_size(B, w.d), dtype=torch.uint8, device=dev)
+
+    def token():
+        mmf.embed(table, ids, out=x.view(B, w.d))
+        mmf.stack_forward(blocks, st, x, ws=ws, out=y)
+        logits = mmf.bitlinear(head, y.view(B, w.d), ws=ws_h)
+        mmf.argmax(logits, out=ids)
+
+    side = torch.cuda.Stream(dev)
+    side.wait_stream(torch.cuda.current_stream(dev))
+    with torch.cuda.stream(side):   # eager tokens first: they also allocate the state's decode buffers
+        for _ in range(3):
+            token()
+    torch.cuda.current_stream(dev).wait_stream(side)
+    torch.cuda.synchronize()
+    mmf.check()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        token()
+    for _ in range(max(warmup, 3)):
+        graph.replay()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(steps):
+        graph.replay()
+    e1.record()
+    wait_event(e1)
+    torch.cuda.synchronize()
+    del graph
+    mmf.check()
+    step_ms = e0.elapsed_time(e1) / steps
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    for _ in range(5):
+        token()
+    torch.cuda.synchronize()
+    mmf.prof_enable(False)
+    prof = mmf.prof_collect()
+    nbytes = decode_bytes_per_step(w, B) + VOCAB * w.d / 4.0 + B * w.d * 2 + 2.0 * B * VOCAB * 2
+    gbs = nbytes / (step_ms / 1e3) / 1e9
+    return {"batch": B, "layers": w.layers, "d": w.d, "inner": w.inner, "vocab": VOCAB, "decode_steps": steps,
+            "ms_per_step": step_ms, "tokens_per_s": B / (step_ms / 1e3), "GBps": gbs, "frac": gbs / peaks["hbm_gbs"],
+            "bytes_per_step": nbytes, "launches_per_step": sum(v[0] for v in prof.values()) // 5,
+            "per_kernel_ms_eager_step": {k: round(v[1] / 5, 4) for k, v in prof.items()}}
+
+
+def run_model(args):
+    """Greedy generation tokens/s of the 2.7B-shaped model (embedding, 32 blocks, head, argmax)."""
+    _, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    import ternary_weight_matmul_fusedbitlinear_b200 as mmf
+    dev = torch.device("cuda", local)
+    w = synth.STACK_2P7B
+    B = args.batch or w.batch
+    peaks, peak_kind = load_peaks()
+    steps = args.decode_steps or w.decode_steps
+    r = measure_model_decode(mmf, w, B, steps, args.warmup, dev, peaks)
+    if rank == 0:
+        print(json.dumps({
+            "metric": METRIC, "value": r["tokens_per_s"], "unit": "tokens/s", "n_gpus": 1, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": f"model2p7b_greedy_v{VOCAB}_b{B}", "batch": B, "layers": w.layers, "d": w.d,
+                       "inner": w.inner, "vocab": VOCAB, "decode_steps": steps,
+                       "l2": "weight stream per token > L2"},
+            "roofline": {"bound": "hbm", "achieved": r["GBps"], "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": r["frac"], "traffic": None, "kernel": "greedy token (all kernels)",
+                         "bytes_per_step": r["bytes_per_step"], "peak_source": peak_kind,
+                         "per_kernel_ms_eager_step": r["per_kernel_ms_eager_step"]},
+            "cpu_baseline": None, "e2e": None, "gpu_launches": r["launches_per_step"] * steps}), flush=True)
+    return 0
+
+
 def run_decode(args):
     _, rank, local = dist_env()
     torch.cuda.set_device(local)
@@ -859,6 +957,8 @@ def main(argv=None):
         return run_bitlinear(args)
     if args.workload == "scan":
         return run_scan(args)
+    if args.workload == "model2p7b":
+        return run_model(args)
     if args.workload == "gemv":
         return run_gemv(args)
     if args.workload in ("decode1p3b", "decode2p7b"):

@@ -65,7 +65,8 @@ const char* mmf_version(void);
 /* Message of the last failed call on this host thread ("" if none). */
 const char* mmf_last_error(void);
 
-/* Synchronise `stream`, then return MMF_ERR_CUDA for a pending CUDA error or
+/* Synchronise `stream`, then return MMF_ERR_CUDA for a pending CUDA error,
+ * MMF_ERR_INVALID_ARG if mmf_embed met a token id outside [0, V), or
  * MMF_ERR_TIMEOUT if a kernel recorded a bounded-wait timeout since the last
  * check (the status word is cleared), else MMF_OK. */
 mmf_status mmf_check(void* stream);
@@ -199,6 +200,34 @@ size_t mmf_mlgru_scan_gnorm_ws_size(int32_t B, int32_t T, int32_t d);
 mmf_status mmf_mlgru_scan_gnorm(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
                                 float* h, const float* gain, float eps, void* o, void* ws,
                                 size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------- */
+/* Model ends: embedding lookup and greedy next token                         */
+/* ------------------------------------------------------------------------- */
+
+/* Token embedding lookup. [HL] "Install and model initialisation": the default
+ * configuration has an embedding of 32000 entries at hidden size 2048.
+ *   x[m, :] = table[ids[m], :]   for m < M
+ *   ids   (device) int32 [M]; table (device) [V, d] in dtype (caller-owned,
+ *         16-byte aligned); x (device) [M, d] in dtype, 16-byte aligned.
+ * A row copy, bit-exact. An id outside [0, V) writes a zero row and is
+ * reported by the next mmf_check (MMF_ERR_INVALID_ARG); the kernel does not
+ * read outside the table. M = 0 does nothing. The same call gathers any rows
+ * of a [V, d] tensor, e.g. the last token of each sequence of a block's output.
+ * Errors: INVALID_ARG, UNSUPPORTED_SHAPE (d % 16), MISALIGNED, CUDA. */
+mmf_status mmf_embed(const int32_t* ids, int32_t M, const void* table, int32_t V, int32_t d,
+                     mmf_dtype dtype, void* x, void* stream);
+
+/* Greedy next token over the LM head's logits. [HL] "Official generation
+ * example" samples; greedy decoding is the deterministic choice taken here:
+ *   ids[m] = the index of the largest of logits[m, 0..V), the lowest index on
+ *            ties (a NaN counts as larger than every number)
+ *   logits (device) [M, V] in dtype; ids (device) int32 [M].
+ * The head itself is a BitLinear d -> V (mmf_bitlinear; [HL] "FusedBitLinear":
+ * every linear projection is one). One CTA per row. M = 0 does nothing.
+ * Errors: INVALID_ARG, CUDA. */
+mmf_status mmf_argmax(const void* logits, mmf_dtype dtype, int32_t M, int32_t V, int32_t* ids,
+                      void* stream);
 
 /* ------------------------------------------------------------------------- */
 /* MatMul-free GLU                                                            */

@@ -310,6 +310,67 @@ def stack_forward(blocks: Sequence[Block], state: State, x: torch.Tensor, eps: f
     return y
 
 
+# ---------------------------------------------------------------- model ends
+
+def embed(table: torch.Tensor, ids: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """x[..., :] = table[ids[...], :] (mmf_embed); table [V, d], ids int32 on the device."""
+    _need_cuda(table, ids)
+    if table.dim() != 2 or ids.dtype != torch.int32 or not ids.is_contiguous() or not table.is_contiguous():
+        raise ValueError("table must be a contiguous [V, d] tensor and ids contiguous int32")
+    V, d = table.shape
+    x = out if out is not None else torch.empty(*ids.shape, d, dtype=table.dtype, device=table.device)
+    L.check(L.load().mmf_embed(_vp(ids), ids.numel(), _vp(table), V, d, _dtype(table), _vp(x),
+                               _stream(table.device)), "mmf_embed")
+    return x
+
+
+def argmax(logits: torch.Tensor, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Greedy next token of each row of logits [..., V] (mmf_argmax): int32, lowest index on ties."""
+    _need_cuda(logits)
+    if not logits.is_contiguous():
+        raise ValueError("logits must be contiguous")
+    V = logits.shape[-1]
+    ids = out if out is not None else torch.empty(logits.shape[:-1], dtype=torch.int32, device=logits.device)
+    L.check(L.load().mmf_argmax(_vp(logits), _dtype(logits), logits.numel() // V, V, _vp(ids),
+                                _stream(logits.device)), "mmf_argmax")
+    return ids
+
+
+class Model:
+    """Embedding -> blocks -> LM head (a BitLinear d -> V) -> greedy next token.
+
+    table: [V, d] embedding in the run dtype; blocks: Block handles; head: TLinear with K = d.
+    Every step is a library call; the torch tensors here are buffers only.
+    """
+
+    def __init__(self, table: torch.Tensor, blocks: Sequence[Block], head: TLinear):
+        if head.K != table.shape[1] or any(b.d != table.shape[1] for b in blocks):
+            raise ValueError("embedding width, block width and head input must agree")
+        self.table, self.blocks, self.head = table, list(blocks), head
+        self.V, self.d = table.shape
+
+    def forward(self, state: State, ids: torch.Tensor, eps: float = DEFAULT_EPS) -> torch.Tensor:
+        """ids [B, T] int32 -> logits [B, V] of each sequence's last token; the state is carried."""
+        B, T = ids.shape
+        x = embed(self.table, ids)
+        y = stack_forward(self.blocks, state, x, eps)
+        if T > 1:   # the last token of each sequence: a row lookup into y viewed as [B*T, d]
+            last = torch.arange(T - 1, B * T, T, dtype=torch.int32, device=ids.device)
+            y = embed(y.reshape(B * T, self.d), last)
+        return bitlinear(self.head, y.reshape(B, self.d), eps)
+
+    def generate(self, state: State, prompt: torch.Tensor, n: int, eps: float = DEFAULT_EPS) -> torch.Tensor:
+        """Greedy generation of n tokens after prompt [B, T0]: int32 [B, n]."""
+        logits = self.forward(state, prompt, eps)
+        out = []
+        for _ in range(n):
+            tok = argmax(logits)
+            out.append(tok)
+            logits = self.forward(state, tok.reshape(-1, 1), eps)
+        return torch.stack(out, 1) if out else torch.empty(prompt.shape[0], 0, dtype=torch.int32,
+                                                              device=prompt.device)
+
+
 # ---------------------------------------------------------------- launch timing
 
 def prof_enable(on: bool = True) -> None:

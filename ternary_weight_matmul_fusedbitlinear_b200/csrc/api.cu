@@ -315,6 +315,8 @@ extern "C" mmf_status mmf_check(void* stream) {
   MMF_CUDA(cudaMemcpy(&v, st, sizeof(int), cudaMemcpyDeviceToHost), "mmf_check: read status");
   if (v != 0) {
     MMF_CUDA(cudaMemset(st, 0, sizeof(int)), "mmf_check: clear status");
+    if (v == 8)
+      return fail(MMF_ERR_INVALID_ARG, "a token id was outside [0, V); its embedding row was written as zeros");
     return fail(MMF_ERR_TIMEOUT, "a device-side bounded wait gave up (code %d)", v);
   }
   return MMF_OK;
@@ -449,6 +451,35 @@ extern "C" mmf_status mmf_mlgru_scan_gnorm(const void* pre, mmf_dtype dtype, int
   MMF_CUDA(timed("mlgru_scan_gnorm", s,
                  [&] { return launch_mlgru_scan_gnorm(pre, dtype, B, T, d, h, gain, eps, o, ws, status, s); }),
            "mlgru_scan_gnorm");
+  return MMF_OK;
+}
+
+// ------------------------------------------------------------------ model ends
+
+extern "C" mmf_status mmf_embed(const int32_t* ids, int32_t M, const void* table, int32_t V, int32_t d,
+                                mmf_dtype dtype, void* x, void* stream) {
+  if (!dtype_ok(dtype)) return fail(MMF_ERR_INVALID_ARG, "mmf_embed: bad dtype");
+  if (M < 0 || V < 1 || d < 1) return fail(MMF_ERR_INVALID_ARG, "mmf_embed: M=%d V=%d d=%d", M, V, d);
+  if (d % 16 != 0) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_embed: d=%d %% 16 != 0", d);
+  if (M == 0) return MMF_OK;
+  if (!ids || !table || !x) return fail(MMF_ERR_INVALID_ARG, "mmf_embed: null pointer");
+  if (!aligned16(table) || !aligned16(x)) return fail(MMF_ERR_MISALIGNED, "mmf_embed");
+  int* status = nullptr;
+  mmf_status r = device_status_ptr(&status);
+  if (r != MMF_OK) return r;
+  cudaStream_t s = as_stream(stream);
+  MMF_CUDA(timed("embed", s, [&] { return launch_embed(ids, M, table, V, d, dtype, x, status, s); }), "embed");
+  return MMF_OK;
+}
+
+extern "C" mmf_status mmf_argmax(const void* logits, mmf_dtype dtype, int32_t M, int32_t V, int32_t* ids,
+                                 void* stream) {
+  if (!dtype_ok(dtype)) return fail(MMF_ERR_INVALID_ARG, "mmf_argmax: bad dtype");
+  if (M < 0 || V < 1) return fail(MMF_ERR_INVALID_ARG, "mmf_argmax: M=%d V=%d", M, V);
+  if (M == 0) return MMF_OK;
+  if (!logits || !ids) return fail(MMF_ERR_INVALID_ARG, "mmf_argmax: null pointer");
+  cudaStream_t s = as_stream(stream);
+  MMF_CUDA(timed("argmax", s, [&] { return launch_argmax(logits, dtype, M, V, ids, s); }), "argmax");
   return MMF_OK;
 }
 

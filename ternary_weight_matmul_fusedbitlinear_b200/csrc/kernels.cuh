@@ -163,4 +163,11 @@ size_t mlgru_scan_gnorm_ws_bytes(int B, int T, int d);
 cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, const float* gain,
                                     float eps, void* o, void* ws, int* status, cudaStream_t stream);
 
+// Model ends: token embedding lookup (one warp per row; an id outside [0, V)
+// writes zeros and records status code 8) and the greedy next token (one CTA
+// per logit row, lowest index on ties). Both are programmatic dependents.
+cudaError_t launch_embed(const int32_t* ids, int M, const void* table, int V, int d, mmf_dtype dt, void* x,
+                         int* status, cudaStream_t stream);
+cudaError_t launch_argmax(const void* logits, mmf_dtype dt, int M, int V, int32_t* ids, cudaStream_t stream);
+
 }  // namespace mmf
