@@ -148,11 +148,15 @@ bool gemm_uses_tc(const TGemmArgs& a, Epi epi) {
 // the standalone quantiser plus one kernel boundary only for single-token
 // calls (1.3B decode at 4 tokens: 0.69 ms per step fused, 0.59 ms split).
 // MMF_DECODE_FUSED_QUANT=1 fuses whenever the shapes allow, =0 never.
-bool decode_fused_quant_wanted(int M) {
+// Single-token calls quantise inside the contraction unless the projection is
+// so wide (more than 4 16-row CTAs per SM, e.g. a 32000-entry LM head) that
+// every CTA quantising the same row costs more than one quantiser launch
+// (2560 -> 32000: 32.8 us fused, 19.5 us with the quantiser).
+bool decode_fused_quant_wanted(int M, int N) {
   const char* e = getenv("MMF_DECODE_FUSED_QUANT");
   if (e != nullptr && strcmp(e, "1") == 0) return true;
   if (e != nullptr && strcmp(e, "0") == 0) return false;
-  return M == 1;
+  return M == 1 && ceil_div(N, 16) <= 4 * num_sms();
 }
 
 // `what` names the projection for the launch-timing totals ("fcg", "o", ...).
@@ -189,7 +193,7 @@ struct QAct {
 mmf_status quant_gemm(const void* x, const float* gain, float eps, const QAct& qa, TGemmArgs a, Epi epi,
                       mmf_dtype dt, cudaStream_t s, const char* what, bool want_codes, void* fill = nullptr,
                       size_t fill_bytes = 0) {
-  if (!gemm_uses_tc(a, epi) && decode_fused_quant_wanted(a.M) &&
+  if (!gemm_uses_tc(a, epi) && decode_fused_quant_wanted(a.M, a.N) &&
       tgemm_mma_fused_quant_supported(a.M, a.K, elem_bytes(dt))) {
     if (fill_bytes) MMF_CUDA(cudaMemsetAsync(fill, 0xff, fill_bytes, s), "scratch fill");
     a.x = x;
