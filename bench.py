@@ -73,7 +73,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) pass")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
     ap.add_argument("--gnorm", action="store_true",
-                    help="scan: the g_norm output gate (RMSNorm of the state fused with a swish gate)")
+                    help="scan / stack370m: the g_norm output gate (RMSNorm of the state fused with a swish gate)")
     ap.add_argument("--no-sub", action="store_true",
                     help="stack370m: skip the decode-step and GEMV-sweep sub-measurements")
     return ap.parse_args(argv)
@@ -286,7 +286,8 @@ def gemm_ops_per_step(w) -> float:
     return 2.0 * M * per_layer * w.layers
 
 
-def build_stack(w, device):
+def build_stack(w, device, gnorm: bool = False):
+    """The workload's blocks (weights from the seeded recipe); gnorm: with a seeded g_norm gain each."""
     import ternary_weight_matmul_fusedbitlinear_b200 as mmf
     shapes = {"f": (w.d, w.d), "c": (w.d, w.d), "g": (w.d, w.d), "o": (w.d, w.d),
               "gate": (w.inner, w.d), "up": (w.inner, w.d), "down": (w.d, w.inner)}
@@ -297,7 +298,8 @@ def build_stack(w, device):
             W = synth.latent_weight(synth.sub_seed(w.seed, layer, i), *shapes[name], device=device)
             lins[name] = mmf.quantize_weights(W)
             del W
-        blocks.append(mmf.Block(lins))
+        gain = synth.gains(synth.sub_seed(w.seed, layer, 7), w.d, device=str(device)) if gnorm else None
+        blocks.append(mmf.Block(lins, gain))
     torch.cuda.synchronize()
     return blocks
 
@@ -375,7 +377,7 @@ def run_mmf(args):
     w = stack_workload(args.layers)
     peaks, peak_kind = load_peaks()
 
-    blocks = build_stack(w, dev)
+    blocks = build_stack(w, dev, gnorm=args.gnorm)
     st = mmf.State(w.layers, w.batch, w.d)
     x_host = synth.activations(w.seed + synth.ACT_SEED_OFFSET + rank, w.batch * w.seq, w.d,
                                torch.bfloat16).reshape(w.batch, w.seq, w.d)
@@ -455,6 +457,12 @@ def run_mmf(args):
         gbs = 8.0 * M * w.d / (scan_ms / 1e3) / 1e9   # 6 B read + 2 B written per channel-step (bf16)
         others["mlgru_scan"] = {"us_per_layer": round(scan_ms * 1e3, 2), "GBps": round(gbs, 1),
                                 "frac": round(gbs / hbm, 4), "bytes_per_layer": 8.0 * M * w.d}
+    if "mlgru_scan_gnorm" in prof:   # scan + the row kernel that forms o' and quantises it
+        g_ms = prof["mlgru_scan_gnorm"][1] / prof["mlgru_scan_gnorm"][0]
+        gbs = 8.0 * M * w.d / (g_ms / 1e3) / 1e9
+        others["mlgru_scan_gnorm"] = {"us_per_layer": round(g_ms * 1e3, 2), "GBps": round(gbs, 1),
+                                      "frac": round(gbs / hbm, 4), "bytes_per_layer": 8.0 * M * w.d,
+                                      "note": "both launches; the o projection's quantiser is folded in"}
     if "rmsnorm_quant" in prof:
         q_ms = prof["rmsnorm_quant"][1] / args.steps
         qbytes = 3.0 * M * (3 * w.d + w.inner) * w.layers   # 2 B read + 1 B written per element (bf16)
@@ -545,7 +553,8 @@ def run_mmf(args):
             "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": w.name, "d": w.d, "inner": w.inner, "layers": w.layers, "batch": w.batch,
+            "config": {"workload": w.name + ("_gnorm" if args.gnorm else ""), "d": w.d, "inner": w.inner,
+                       "layers": w.layers, "batch": w.batch,
                        "seq": w.seq, "global_batch": w.batch * world, "seq_len": w.seq,
                        "parallelism": f"replicas x{world} (independent sequences)",
                        "l2": L2Flush.NOTE},

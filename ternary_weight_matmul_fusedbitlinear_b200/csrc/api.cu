@@ -902,9 +902,12 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
     int* status = nullptr;
     r = device_status_ptr(&status);
     if (r != MMF_OK) return r;
-    if (gnorm)
+    if (gnorm)   // scan, then o' formed and quantised for the o projection in one row kernel
       MMF_CUDA(timed("mlgru_scan_gnorm", s,
-                     [&] { return launch_mlgru_scan_gnorm(w.pre, dt, B, T, d, h, W.gnorm, eps, w.og, w.gn, status, s); }),
+                     [&] {
+                       return launch_mlgru_scan_gnorm_quant(w.pre, dt, B, T, d, h, W.gnorm, eps, want ? w.og : nullptr,
+                                                            w.gn, status, W.o.gain, eps, w.qa.q, w.qa.s, w.qa.qsum, s);
+                     }),
                "block scan");
     else
       MMF_CUDA(timed("mlgru_scan", s, [&] { return launch_mlgru_scan(w.pre, dt, B, T, d, h, w.og, status, s); }),
@@ -913,7 +916,12 @@ mmf_status block_forward_impl(const mmf_block* blk, float* h, const void* x, voi
   const mmf_tlinear* op[1] = {&W.o};
   TGemmArgs b = gemm_args(op, 1, w.qa.q, w.qa.s, w.qa.qsum, M, w.y1, d, x, nullptr);
   b.wu[0] = blk->wu[3];
-  mmf_status r = quant_gemm(w.og, W.o.gain, eps, w.qa, b, Epi::kStore, dt, s, "o", want);
+  mmf_status r = MMF_OK;
+  if (gnorm) {   // the codes of o' are already in w.qa
+    MMF_CUDA(run_gemm(b, Epi::kStore, dt, s, "o"), "contraction");
+  } else {
+    r = quant_gemm(w.og, W.o.gain, eps, w.qa, b, Epi::kStore, dt, s, "o", want);
+  }
   if (r == MMF_OK) r = dbg_codes(dbg, 1, w.qa, M, d, s);
   if (r != MMF_OK) return r;
   // channel mixer

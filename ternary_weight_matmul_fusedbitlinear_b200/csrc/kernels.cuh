@@ -162,6 +162,14 @@ cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d
 size_t mlgru_scan_gnorm_ws_bytes(int B, int T, int d);
 cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, const float* gain,
                                     float eps, void* o, void* ws, int* status, cudaStream_t stream);
+// Inside a block: the same scan, then one row kernel that forms o' and
+// quantises it for the o projection (RMSNorm gain qgain, eps) into q / scale /
+// qsum with the standalone quantiser's row routine; o' is written only when
+// `o` is not null.
+cudaError_t launch_mlgru_scan_gnorm_quant(const void* pre, mmf_dtype dt, int B, int T, int d, float* h,
+                                          const float* gain, float eps_g, void* o, void* ws, int* status,
+                                          const float* qgain, float eps, int8_t* q, float* scale, int32_t* qsum,
+                                          cudaStream_t stream);
 
 // Model ends: token embedding lookup (one warp per row; an id outside [0, V)
 // writes zeros and records status code 8) and the greedy next token (one CTA

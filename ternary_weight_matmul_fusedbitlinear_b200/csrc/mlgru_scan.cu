@@ -16,7 +16,11 @@
 // kernels: the scan (GN = true) computes swish(g~) in place of sigmoid(g~),
 // writes v_t = swish(g~_t) h_t in fp32 and, per token and channel block, the
 // partial sum of h_t^2; gnorm_apply_kernel adds a row's partials and writes
-// o' = v * (1 / sqrt(sum / d + eps)) * w in the storage type.
+// o' = v * (1 / sqrt(sum / d + eps)) * w in the storage type. Inside a block
+// the o projection's quantiser is folded into that row kernel
+// (gnorm_apply_quant_kernel): each warp forms its token's o' row in shared
+// memory and quantises it with the standalone quantiser's row routine, so the
+// codes are the same and o' never goes to HBM.
 //
 // Work split. A CTA owns CC channels of one sequence and walks that
 // sequence's chunks of TC = 128 steps in order, carrying the state from one
@@ -45,6 +49,7 @@
 #include <type_traits>
 
 #include "kernels.cuh"
+#include "quant_row.cuh"
 #include "tma.cuh"
 
 namespace mmf {
@@ -398,8 +403,93 @@ __global__ void __launch_bounds__(256) gnorm_apply_kernel(const float* __restric
   }
 }
 
+// gnorm_apply_kernel's o' row, then the o projection's RMSNorm + absmax
+// quantisation of it (quant_row, the standalone quantiser's routine and fp32
+// steps) from a per-warp shared-memory copy of the row; o' itself goes to HBM
+// only when `o` is given. One warp per token row.
+constexpr int kApplyWarps = 8;
+template <typename T, bool GAIN>
+__global__ void __launch_bounds__(kApplyWarps * 32)
+    gnorm_apply_quant_kernel(const float* __restrict__ v, const float* __restrict__ ss, int n_cb,
+                             const float* __restrict__ gain, float eps_g, int M, int d, T* __restrict__ o,
+                             const float* __restrict__ qgain, float eps, int8_t* __restrict__ q,
+                             float* __restrict__ scale, int32_t* __restrict__ qsum, int pitch) {
+  extern __shared__ uint4 rows[];   // [kApplyWarps][pitch / 16]
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  T* row_sm = reinterpret_cast<T*>(reinterpret_cast<uint8_t*>(rows) + (size_t)warp * pitch);
+  const int nw = gridDim.x * kApplyWarps;
+  const int nvec = d * (int)sizeof(T) / 16;
+  pdl_trigger();
+  pdl_wait();   // v and ss are the scan's output
+  for (int m = blockIdx.x * kApplyWarps + warp; m < M; m += nw) {
+    float t = 0.0f;
+    for (int c = lane; c < n_cb; c += 32) t += ss[(size_t)m * n_cb + c];
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) t += __shfl_xor_sync(0xffffffffu, t, off);
+    const float rinv = __frsqrt_rn(__fadd_rn(__fdiv_rn(t, (float)d), eps_g));
+    const float4* vr = reinterpret_cast<const float4*>(v + (size_t)m * d);
+    const float4* gr = reinterpret_cast<const float4*>(gain);
+#pragma unroll 4
+    for (int k = lane; k < d / 4; k += 32) {
+      const float4 x = vr[k], g = gr[k];
+      const float y0 = x.x * rinv * g.x, y1 = x.y * rinv * g.y, y2 = x.z * rinv * g.z, y3 = x.w * rinv * g.w;
+      if constexpr (sizeof(T) == 2) {
+        const __nv_bfloat162 a = __floats2bfloat162_rn(y0, y1), b = __floats2bfloat162_rn(y2, y3);
+        uint2 w;
+        w.x = *reinterpret_cast<const uint32_t*>(&a);
+        w.y = *reinterpret_cast<const uint32_t*>(&b);
+        *reinterpret_cast<uint2*>(row_sm + 4 * k) = w;
+        if (o) *reinterpret_cast<uint2*>(o + (size_t)m * d + 4 * k) = w;
+      } else {
+        const float4 w = make_float4(y0, y1, y2, y3);
+        *reinterpret_cast<float4*>(row_sm + 4 * k) = w;
+        if (o) *reinterpret_cast<float4*>(o + (size_t)m * d + 4 * k) = w;
+      }
+    }
+    __syncwarp();
+    const RowCode rc = quant_row<T, GAIN, false>(reinterpret_cast<const uint4*>(row_sm), nvec, d, qgain, eps,
+                                                 q + (size_t)m * d, lane);
+    if (lane == 0) {
+      scale[m] = rc.scale;
+      qsum[m] = rc.qsum;
+    }
+    __syncwarp();   // the row buffer is rewritten for the next row
+  }
+}
+
 // 64 channels per CTA when that gives enough CTAs to cover the GPU, else 32
 bool scan_wide(int B, int d) { return (size_t)B * ceil_div(d, 64) >= (size_t)num_sms() * 3 / 4; }
+
+// The scan in g_norm mode: v and the partial sums into ws; n_cb = channel blocks.
+cudaError_t launch_scan_gnorm_part(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* ws,
+                                   int* status, cudaStream_t stream, float*& v, float*& ss, int& n_cb) {
+  const size_t M = (size_t)B * T;
+  v = static_cast<float*>(ws);
+  ss = reinterpret_cast<float*>(static_cast<char*>(ws) + (M * d * sizeof(float) + 255) / 256 * 256);
+  const long long wait = wait_limit_cycles();
+  const int skip = test_hook("MMF_SCAN_SKIP_CHUNK");
+  const bool wide = scan_wide(B, d);
+  n_cb = ceil_div(d, wide ? 64 : 32);
+  if (dt == MMF_BF16)
+    return wide ? launch_typed<bf16, 64, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream)
+                : launch_typed<bf16, 32, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream);
+  return wide ? launch_typed<float, 64, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream)
+              : launch_typed<float, 32, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream);
+}
+
+template <typename T, bool GAIN>
+cudaError_t launch_apply_quant(const float* v, const float* ss, int n_cb, const float* gain, float eps_g, int M,
+                               int d, void* o, const float* qgain, float eps, int8_t* q, float* scale, int32_t* qsum,
+                               cudaStream_t stream) {
+  const int pitch = (d * (int)sizeof(T) + 127) / 128 * 128;
+  const size_t smem = (size_t)kApplyWarps * pitch;
+  auto kern = gnorm_apply_quant_kernel<T, GAIN>;
+  const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  if (e != cudaSuccess) return e;
+  const int grid = std::max(1, std::min(ceil_div(M, kApplyWarps), num_sms() * 8));
+  return launch_pdl(kern, dim3(grid), dim3(kApplyWarps * 32), smem, stream, v, ss, n_cb, gain, eps_g, M, d,
+                    static_cast<T*>(o), qgain, eps, q, scale, qsum, pitch);
+}
 
 }  // namespace
 
@@ -429,19 +519,9 @@ cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T,
   if (B == 0 || T == 0) return cudaSuccess;
   if (!tma_available()) return cudaErrorNotSupported;
   const size_t M = (size_t)B * T;
-  float* v = static_cast<float*>(ws);
-  float* ss = reinterpret_cast<float*>(static_cast<char*>(ws) + (M * d * sizeof(float) + 255) / 256 * 256);
-  const long long wait = wait_limit_cycles();
-  const int skip = test_hook("MMF_SCAN_SKIP_CHUNK");
-  const bool wide = scan_wide(B, d);
-  const int n_cb = ceil_div(d, wide ? 64 : 32);
-  cudaError_t e;
-  if (dt == MMF_BF16)
-    e = wide ? launch_typed<bf16, 64, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream)
-             : launch_typed<bf16, 32, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream);
-  else
-    e = wide ? launch_typed<float, 64, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream)
-             : launch_typed<float, 32, true>(pre, B, T, d, h, v, ss, status, wait, skip, stream);
+  float *v, *ss;
+  int n_cb;
+  cudaError_t e = launch_scan_gnorm_part(pre, dt, B, T, d, h, ws, status, stream, v, ss, n_cb);
   if (e != cudaSuccess) return e;
   constexpr int kWarpsA = 8;
   const int grid = (int)std::max<size_t>(1, std::min<size_t>((M + kWarpsA - 1) / kWarpsA, (size_t)num_sms() * 8));
@@ -450,6 +530,26 @@ cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T,
                       (const float*)ss, n_cb, gain, eps, (int)M, d, static_cast<bf16*>(o));
   return launch_pdl(gnorm_apply_kernel<float>, dim3(grid), dim3(32 * kWarpsA), 0, stream, (const float*)v,
                     (const float*)ss, n_cb, gain, eps, (int)M, d, static_cast<float*>(o));
+}
+
+cudaError_t launch_mlgru_scan_gnorm_quant(const void* pre, mmf_dtype dt, int B, int T, int d, float* h,
+                                          const float* gain, float eps_g, void* o, void* ws, int* status,
+                                          const float* qgain, float eps, int8_t* q, float* scale, int32_t* qsum,
+                                          cudaStream_t stream) {
+  if (B == 0 || T == 0) return cudaSuccess;
+  if (!tma_available()) return cudaErrorNotSupported;
+  float *v, *ss;
+  int n_cb;
+  cudaError_t e = launch_scan_gnorm_part(pre, dt, B, T, d, h, ws, status, stream, v, ss, n_cb);
+  if (e != cudaSuccess) return e;
+  const int M = B * T;
+  if (dt == MMF_BF16)
+    return qgain ? launch_apply_quant<bf16, true>(v, ss, n_cb, gain, eps_g, M, d, o, qgain, eps, q, scale, qsum, stream)
+                 : launch_apply_quant<bf16, false>(v, ss, n_cb, gain, eps_g, M, d, o, qgain, eps, q, scale, qsum,
+                                                   stream);
+  return qgain ? launch_apply_quant<float, true>(v, ss, n_cb, gain, eps_g, M, d, o, qgain, eps, q, scale, qsum, stream)
+               : launch_apply_quant<float, false>(v, ss, n_cb, gain, eps_g, M, d, o, qgain, eps, q, scale, qsum,
+                                                  stream);
 }
 
 }  // namespace mmf

@@ -127,6 +127,10 @@ def test_block_gnorm_stages(B, T, dtype):
     y, hT, dbg = _run(blk, x, h0, dtype)
     check_block_stages(x, h0, y, hT, dbg, oblk, dtype, f"g_norm B={B} T={T}")
     check_block_tie_forced(x, h0, y, hT, dbg, oblk, dtype, f"g_norm B={B} T={T}")
+    # the o projection's codes come from the row kernel that forms o': the
+    # standalone quantiser on the same stored o' gives the same codes and scales
+    _, q, sc, _ = mmf.bitlinear(blk.lins["o"], dbg["og"].reshape(B * T, d), debug=True)
+    assert torch.equal(q, dbg["q"][1]) and torch.equal(sc, dbg["s"][1])
 
 
 def test_block_gnorm_prefill_then_decode():
