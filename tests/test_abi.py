@@ -101,3 +101,46 @@ def test_workspace_sizes_grow_with_size(lib):
     assert lib.mmf_bitlinear_ws_size(16, 2048) < lib.mmf_bitlinear_ws_size(64, 2048)
     assert lib.mmf_glu_ws_size(4, 1024, 2816) > 4 * 2816
     assert lib.mmf_quantize_weights_ws_size(2048, 2048) >= 8
+
+
+def test_gnorm_scan_validation(lib):
+    p = ctypes.c_void_p(4096)
+    ws = lib.mmf_mlgru_scan_gnorm_ws_size(2, 300, 64)
+    assert ws >= 4 * 2 * 300 * 64 + 4 * 2 * 300 * 2
+    assert lib.mmf_mlgru_scan_gnorm(p, 0, 2, 3, 12, p, p, 1e-6, p, p, 1 << 20, None) == 2       # d % 8
+    assert lib.mmf_mlgru_scan_gnorm(p, 0, 2, 3, 16, p, p, 0.0, p, p, 1 << 20, None) == 1        # eps
+    assert lib.mmf_mlgru_scan_gnorm(p, 0, 2, 3, 16, p, None, 1e-6, p, p, 1 << 20, None) == 1    # gain
+    assert lib.mmf_mlgru_scan_gnorm(p, 0, 2, 3, 16, p, ctypes.c_void_p(4100), 1e-6, p, p, 1 << 20, None) == 3
+    assert lib.mmf_mlgru_scan_gnorm(p, 0, 2, 300, 64, p, p, 1e-6, p, p, ws - 1, None) == 4      # workspace
+    assert lib.mmf_mlgru_scan_gnorm(None, 0, 0, 3, 16, None, None, 1e-6, None, None, 0, None) == 0  # B = 0
+
+
+def test_model_end_validation(lib):
+    p = ctypes.c_void_p(4096)
+    assert lib.mmf_embed(p, 4, p, 100, 24, 1, p, None) == 2                # d % 16
+    assert lib.mmf_embed(p, -1, p, 100, 32, 1, p, None) == 1
+    assert lib.mmf_embed(p, 4, p, 0, 32, 1, p, None) == 1                  # V
+    assert lib.mmf_embed(p, 4, ctypes.c_void_p(4098), 100, 32, 1, p, None) == 3
+    assert lib.mmf_embed(None, 4, p, 100, 32, 1, p, None) == 1
+    assert lib.mmf_embed(None, 0, None, 100, 32, 1, None, None) == 0       # M = 0
+    assert lib.mmf_argmax(p, 1, 2, 0, p, None) == 1                        # V
+    assert lib.mmf_argmax(None, 1, 2, 10, p, None) == 1
+    assert lib.mmf_argmax(None, 1, 0, 10, None, None) == 0                 # M = 0
+    assert lib.mmf_argmax(p, 5, 2, 10, p, None) == 1                       # dtype
+
+
+def test_block_gnorm_gain_validation_and_workspace(lib):
+    d, I = 32, 64
+    sq = lambda: _tl(d, d)
+    w = L.BlockWeights(sq(), sq(), sq(), sq(), _tl(I, d), _tl(I, d), _tl(d, I), None)
+    h = ctypes.c_void_p()
+    assert lib.mmf_block_create(ctypes.byref(w), d, I, ctypes.byref(h)) == 0
+    plain = lib.mmf_block_ws_size(h, 2, 8)
+    lib.mmf_block_destroy(h)
+    w.gnorm = 4104   # not 16-byte aligned
+    assert lib.mmf_block_create(ctypes.byref(w), d, I, ctypes.byref(h)) == 3
+    w.gnorm = 4096
+    assert lib.mmf_block_create(ctypes.byref(w), d, I, ctypes.byref(h)) == 0
+    # the g_norm scan's scratch (v in fp32 and the partial sums) comes on top
+    assert lib.mmf_block_ws_size(h, 2, 8) >= plain + lib.mmf_mlgru_scan_gnorm_ws_size(2, 8, d) - 256
+    lib.mmf_block_destroy(h)
