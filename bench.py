@@ -266,7 +266,7 @@ class ClockSampler:
 # DRAM bytes (read + write) per launch of the dominant kernel, measured by an ncu capture of the same
 # kernel (mean over the four contraction launches of one 370M block, one-byte weight codes). Reported as
 # the `traffic` of the headline line with the capture named in `traffic_source`; None elsewhere.
-STACK370M_CONTRACTION_TRAFFIC = 69.38e6
+STACK370M_CONTRACTION_TRAFFIC = 69.53e6
 STACK370M_TRAFFIC_SOURCE = "ncu capture, tgemm_tc at the four 370M block shapes (dram__bytes read + write)"
 
 

@@ -119,3 +119,23 @@ def test_greedy_generation_teacher_forced():
     st2 = mmf.State(2, B, d)
     gen = model.generate(st2, prompt.cuda(), n)
     np.testing.assert_array_equal(gen.cpu().numpy(), torch.stack(toks, 1).cpu().numpy())
+
+
+def test_argmax_nan_and_infinities():
+    # a NaN counts as the largest value (first NaN wins), -inf rows pick index 0,
+    # +inf beats every finite value; the same decisions as the oracle's argmax
+    V = 300
+    rows = torch.full((5, V), -float("inf"))
+    rows[1, 7] = 1.0
+    rows[1, 200] = float("inf")
+    rows[2, 50] = float("nan")
+    rows[2, 60] = float("nan")
+    rows[2, 70] = float("inf")
+    rows[3] = synth.activations(907, 1, V)[0]
+    rows[3, 299] = float("inf")
+    rows[4] = synth.activations(908, 1, V)[0]
+    for dtype in ("bf16", "f32"):
+        lg = rows.to(TORCH_DT[dtype])
+        ids = mmf.argmax(lg.cuda()).cpu().numpy()
+        np.testing.assert_array_equal(ids, O.greedy_token(to_np(lg)))
+    assert list(ids[:4]) == [0, 200, 50, 299]
