@@ -152,3 +152,31 @@ def test_block_gnorm_prefill_then_decode():
     y_ref, h_ref = O.block_forward(x.float().numpy(), oblk, np.zeros((B, d)), "bf16")
     assert_close(to_np(torch.cat(ys, 1)), y_ref, "bf16", "g_norm prompt + decode y", tol=E2E_TOL)
     assert_close(st.get()[0].numpy(), h_ref, "f32", "g_norm prompt + decode h_T", tol=E2E_TOL)
+
+
+@pytest.mark.parametrize("gnorm", [False, True])
+def test_checkpoint_resume_matches_one_prefill(gnorm):
+    # prefill half a prompt, save the state to the host, restore it into a
+    # fresh state handle and prefill the rest: the second half's output and
+    # the final state equal those of one prefill over the whole prompt
+    # (recurrent state and outputs are exact; save/restore is a bit copy)
+    d, inner, B, T, L = 256, 768, 2, 256, 2
+    pairs = [make_block(8700 + l, d, inner, layer=l, gnorm=gnorm) for l in range(L)]
+    blocks = [p_[0] for p_ in pairs]
+    x = synth.activations(8710, B * T, d, torch.bfloat16).reshape(B, T, d).cuda()
+    st = mmf.State(L, B, d)
+    y_all = mmf.stack_forward(blocks, st, x)
+    h_all = st.get()
+    st1 = mmf.State(L, B, d)
+    mmf.stack_forward(blocks, st1, x[:, :T // 2].contiguous())
+    saved = st1.get()
+    st2 = mmf.State(L, B, d)
+    st2.set(saved)
+    assert torch.equal(st2.get(), saved)   # the round trip is a bit copy
+    y2 = mmf.stack_forward(blocks, st2, x[:, T // 2:].contiguous())
+    mmf.check()
+    # the scan composes its chunks' maps in a different grouping when the
+    # sequence is cut, so the state may differ by fp32 rounding; the stored
+    # outputs then agree up to the storage rounding that carries into codes
+    torch.testing.assert_close(st2.get(), h_all, rtol=1e-5, atol=1e-6)
+    assert_close(to_np(y2), to_np(y_all[:, T // 2:]), "bf16", "resumed prefill", tol=E2E_TOL)
