@@ -173,7 +173,9 @@ namespace mmf {
 // rows) and scale[m] gets the row's scale. The code sums are left as per-warp
 // partials in red.i: block_qsum() folds them after the caller's next barrier.
 // `red` is shared scratch of NT / 32 entries of each type. Contains
-// __syncthreads(): every thread of the block calls it.
+// __syncthreads(): every thread of the block calls it. `fail` (any thread)
+// makes every thread return false right after the first barrier, with
+// nothing written; the barrier doubles as the caller's vote on giving up.
 struct BlockRed {
   double* d;
   uint32_t* u;
@@ -194,9 +196,9 @@ __device__ __forceinline__ V fold_row(const V* red, int w0, int lane, V zero, Op
 }
 
 template <typename T, int MPAD, int NT, int VMAX>
-__device__ __forceinline__ void block_quant(const uint4 (&raw)[VMAX], uint32_t have, int M, int K,
+__device__ __forceinline__ bool block_quant(const uint4 (&raw)[VMAX], uint32_t have, int M, int K,
                                             const float* __restrict__ gain, float eps, int8_t* codes, int qpitch,
-                                            float* scale, const BlockRed& red) {
+                                            float* scale, const BlockRed& red, bool fail = false) {
   using V = Vec<T>;
   constexpr int E = V::E;
   constexpr int kTpr = NT / MPAD;
@@ -233,7 +235,7 @@ __device__ __forceinline__ void block_quant(const uint4 (&raw)[VMAX], uint32_t h
       red.u[warp] = am;
     }
   }
-  __syncthreads();
+  if (__syncthreads_or(fail)) return false;
   const double tot = fold_row<kWpr>(red.d, w0, lane, 0.0, [](double x, double y) { return x + y; });
   const uint32_t mx = fold_row<kWpr>(red.u, w0, lane, 0u, [](uint32_t x, uint32_t y) { return max(x, y); });
   const float ms = (float)(tot / (double)K);
@@ -281,6 +283,7 @@ __device__ __forceinline__ void block_quant(const uint4 (&raw)[VMAX], uint32_t h
     if (lane == 0) red.i[warp] = isum;
   }
   __syncthreads();
+  return true;
 }
 
 // Code sum of row m from block_quant's per-warp partials (any thread, after block_quant).
