@@ -180,3 +180,19 @@ def test_checkpoint_resume_matches_one_prefill(gnorm):
     # outputs then agree up to the storage rounding that carries into codes
     torch.testing.assert_close(st2.get(), h_all, rtol=1e-5, atol=1e-6)
     assert_close(to_np(y2), to_np(y_all[:, T // 2:]), "bf16", "resumed prefill", tol=E2E_TOL)
+
+
+@pytest.mark.parametrize("gnorm", [False, True])
+@pytest.mark.parametrize("T", [150, 1])
+def test_block_stages_ragged_widths(T, gnorm):
+    # d = 272 and I = 400 are multiples of 16 but not of 64: the tensor-core
+    # contraction does not take them (prefill runs the mma.sync kernel at 300
+    # tokens) and the one-launch decode step does not either (decode runs the
+    # four contractions); every stage teacher-forced at TOL
+    d, inner, B = 272, 400, 2
+    blk, oblk = make_block(8800 + T, d, inner, gnorm=gnorm)
+    x = synth.activations(8801 + T, B * T, d, torch.bfloat16).reshape(B, T, d)
+    h0 = synth.activations(8802, B, d).numpy().astype(np.float64) * 0.5
+    y, hT, dbg = _run(blk, x, h0, "bf16")
+    check_block_stages(x, h0, y, hT, dbg, oblk, "bf16", f"ragged widths T={T}")
+    check_block_tie_forced(x, h0, y, hT, dbg, oblk, "bf16", f"ragged widths T={T}")
