@@ -138,9 +138,20 @@ int gemm_path_pref() {
   return 0;
 }
 
+// Below 128 tokens the tcgen05 kernel still wins on wide projections, whose
+// 128 x 256 tiles (one, half empty, per 256 output columns) keep enough SMs
+// busy: 2.7B decode at 64 sequences, gate|up (54 tiles) 1.31 -> 0.66 ms per
+// step, at 32 sequences 0.78 -> 0.65 ms; the o and down projections (10
+// tiles) and anything at 16 sequences stay faster on the mma.sync kernel.
+constexpr int kTcMinTokensWide = 32;
+constexpr int kTcMinTilesWide = 48;
+
 bool gemm_uses_tc(const TGemmArgs& a, Epi epi) {
   const int pref = gemm_path_pref();
-  return tgemm_tc_supported(a, epi) && (pref >= 2 || (pref == 0 && a.M >= kTcMinTokens));
+  if (!tgemm_tc_supported(a, epi) || pref == 1) return false;
+  if (pref >= 2 || a.M >= kTcMinTokens) return true;
+  const int cols = epi == Epi::kGlu ? a.N / 128 : ceil_div(a.nseg * a.N, 256);
+  return a.M >= kTcMinTokensWide && cols >= kTcMinTilesWide;
 }
 
 // Whether the decode contraction quantises its own token rows (both ways give

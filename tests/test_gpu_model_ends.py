@@ -76,9 +76,10 @@ def test_argmax_unaligned_rows_take_the_scalar_path():
     np.testing.assert_array_equal(mmf.argmax(lg2).cpu().numpy(), O.greedy_token(to_np(lg)))
 
 
-@pytest.mark.parametrize("M", [1, 4, 16, 300])
+@pytest.mark.parametrize("M", [1, 4, 16, 64, 300])
 def test_lm_head_logits(M):
-    # the head of the 2.7B shape: BitLinear 2560 -> 32000
+    # the head of the 2.7B shape: BitLinear 2560 -> 32000 (M = 64 and 300: the
+    # tcgen05 kernel, the others the mma.sync kernel)
     _, lin, olin = make_layer(905, 32000, 2560)
     x = synth.activations(906 + M, M, 2560, torch.bfloat16)
     y = mmf.bitlinear(lin, x.cuda())

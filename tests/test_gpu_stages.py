@@ -196,3 +196,16 @@ def test_block_stages_ragged_widths(T, gnorm):
     y, hT, dbg = _run(blk, x, h0, "bf16")
     check_block_stages(x, h0, y, hT, dbg, oblk, "bf16", f"ragged widths T={T}")
     check_block_tie_forced(x, h0, y, hT, dbg, oblk, "bf16", f"ragged widths T={T}")
+
+
+def test_block_decode_step_stages_wide_batch():
+    # 40 sequences: above the one-launch decode step's batch, and the GLU's
+    # gate|up (I = 6912: 54 tiles) takes the tcgen05 kernel at 40 tokens while
+    # the other projections stay on mma.sync; every stage teacher-forced
+    d, inner, B = 256, 6912, 40
+    blk, oblk = make_block(8900, d, inner)
+    x = synth.activations(8901, B, d, torch.bfloat16).reshape(B, 1, d)
+    h0 = synth.activations(8902, B, d).numpy().astype(np.float64) * 0.5
+    y, hT, dbg = _run(blk, x, h0, "bf16")
+    check_block_stages(x, h0, y, hT, dbg, oblk, "bf16", "decode B=40")
+    check_block_tie_forced(x, h0, y, hT, dbg, oblk, "bf16", "decode B=40")
