@@ -285,6 +285,16 @@ typedef struct mmf_state mmf_state;   /* opaque */
 mmf_status mmf_block_create(const mmf_block_weights* w, int32_t d, int32_t I, mmf_block** out);
 void mmf_block_destroy(mmf_block* blk);
 
+/* Free the one-byte code copy that the block's first prefill-sized call made
+ * (see mmf_block_create), e.g. before a long decode-only phase, where only the
+ * packed codes are read: the block returns to its packed size (plus the
+ * caller's own one-byte codes, if it gave any). The next forward call with
+ * T > 1 and at least 128 tokens makes the copy again. Synchronises the device
+ * first when there is a copy to free, so call it between forward calls; it
+ * must not run concurrently with a forward call on the same block.
+ * Results are unchanged either way. Errors: INVALID_ARG (null), CUDA. */
+mmf_status mmf_block_release_codes(mmf_block* blk);
+
 /* Recurrent state h for L layers x B sequences x d channels, fp32, zeroed.
  * The library allocates it with cudaMalloc on the current device and frees it
  * in mmf_state_destroy. The first decode step (T = 1) that runs as one launch

@@ -61,6 +61,7 @@ SIGNATURES = {
                                                              c_sz, c_vp]),
     "mmf_block_create": (ctypes.c_int, [ctypes.POINTER(BlockWeights), c_i32, c_i32, ctypes.POINTER(c_vp)]),
     "mmf_block_destroy": (None, [c_vp]),
+    "mmf_block_release_codes": (ctypes.c_int, [c_vp]),
     "mmf_state_create": (ctypes.c_int, [c_i32, c_i32, c_i32, ctypes.POINTER(c_vp)]),
     "mmf_state_destroy": (None, [c_vp]),
     "mmf_state_reset": (ctypes.c_int, [c_vp, c_vp]),

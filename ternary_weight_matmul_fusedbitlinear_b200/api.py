@@ -204,6 +204,10 @@ class Block:
     def ws_size(self, B: int, T: int) -> int:
         return int(L.load().mmf_block_ws_size(self.handle, B, T))
 
+    def release_codes(self) -> None:
+        """Free the one-byte code copy made by the first prefill call (mmf_block_release_codes)."""
+        L.check(L.load().mmf_block_release_codes(self.handle), "mmf_block_release_codes")
+
     def close(self):
         if getattr(self, "handle", None) is not None and self.handle.value:
             L.load().mmf_block_destroy(self.handle)

@@ -640,6 +640,22 @@ extern "C" void mmf_block_destroy(mmf_block* blk) {
   delete blk;
 }
 
+extern "C" mmf_status mmf_block_release_codes(mmf_block* blk) {
+  if (!blk) return fail(MMF_ERR_INVALID_ARG, "mmf_block_release_codes: null block");
+  std::lock_guard<std::mutex> lock(blk->mu);
+  bool any = false;
+  for (int i = 0; i < 7; ++i) any = any || blk->owned[i] != nullptr;
+  if (any) MMF_CUDA(cudaDeviceSynchronize(), "mmf_block_release_codes: synchronize");
+  const mmf_tlinear* all[7] = {&blk->w.f, &blk->w.c, &blk->w.g, &blk->w.o, &blk->w.gate, &blk->w.up, &blk->w.down};
+  for (int i = 0; i < 7; ++i) {
+    if (blk->owned[i] != nullptr) MMF_CUDA(cudaFree(blk->owned[i]), "mmf_block_release_codes: cudaFree");
+    blk->owned[i] = nullptr;
+    blk->wu[i] = all[i]->codes;   // the caller's own one-byte codes, if it gave any
+  }
+  blk->codes_tried = false;   // the next prefill-sized call makes the copy again
+  return MMF_OK;
+}
+
 extern "C" mmf_status mmf_state_create(int32_t L, int32_t B, int32_t d, mmf_state** out) {
   if (!out) return fail(MMF_ERR_INVALID_ARG, "mmf_state_create: null out");
   *out = nullptr;

@@ -329,6 +329,37 @@ def test_block_byte_copy_made_by_first_prefill_call_only():
     assert abs(free2 - free3) < copy_bytes // 4, (free2, free3)
 
 
+def test_block_release_codes_frees_the_copy_and_changes_no_result():
+    # release the one-byte copy after a prefill: the memory comes back, a
+    # decode step afterwards and the next prefill (which makes the copy again)
+    # give bit-identical results to a block that kept its copy
+    d, inner, B, T = 1024, 2816, 2, 192
+    copy_bytes = 4 * d * d + 3 * d * inner
+    x = synth.activations(7046, B * T, d, torch.bfloat16).reshape(B, T, d).cuda()
+    blk, _ = make_block(7045, d, inner)
+    ref, _ = make_block(7045, d, inner)
+    st, st_ref = mmf.State(1, B, d), mmf.State(1, B, d)
+    ws = torch.empty(mmf.stack_ws_size([blk], B, T), dtype=torch.uint8, device="cuda")
+    y0 = mmf.block_forward(blk, 0, st, x, ws=ws)
+    r0 = mmf.block_forward(ref, 0, st_ref, x, ws=ws)
+    torch.cuda.synchronize()
+    free_before = torch.cuda.mem_get_info()[0]
+    blk.release_codes()
+    free_after = torch.cuda.mem_get_info()[0]
+    assert free_after - free_before >= copy_bytes, (free_before, free_after, copy_bytes)
+    blk.release_codes()   # nothing left to free: a no-op
+    xd = x[:, :1].contiguous()
+    y1 = mmf.block_forward(blk, 0, st, xd, ws=ws)
+    r1 = mmf.block_forward(ref, 0, st_ref, xd, ws=ws)
+    y2 = mmf.block_forward(blk, 0, st, x, ws=ws)    # makes the copy again
+    r2 = mmf.block_forward(ref, 0, st_ref, x, ws=ws)
+    mmf.check()
+    assert torch.cuda.mem_get_info()[0] <= free_after - copy_bytes + copy_bytes // 4
+    for a, b in ((y0, r0), (y1, r1), (y2, r2)):
+        assert torch.equal(a, b)
+    assert torch.equal(st.get(), st_ref.get())
+
+
 @pytest.mark.parametrize("m", [128, 300])
 def test_bitlinear_and_glu_with_byte_codes_bit_identical(m):
     # mmf_tlinear.codes (mmf_unpack_codes) lets the prefill contraction load the
