@@ -39,6 +39,9 @@ constant gate, scale invariance, and the identity-weight block.
 The model ends (``embed``, ``lm_logits``, ``greedy_token``, ``model_forward``,
 ``generate_greedy``) are pinned by brute force on small tables, ties, and a
 generation that follows a known permutation (zero blocks, identity head).
+``mlgru_scan_backward`` is pinned by central finite differences of the
+forward oracle in every input, and by special cases (no upstream gradient,
+forget gate 0, only a final-state gradient).
 """
 from __future__ import annotations
 
@@ -548,3 +551,49 @@ def generate_greedy(prompt, n: int, table, blocks, head: TLinear, dtype: str, ep
         out.append(tok)
         logits, hs = model_forward(tok[:, None], table, blocks, head, hs, dtype, eps)
     return np.stack(out, axis=1) if out else np.zeros((B, 0), np.int64), hs
+
+
+# ---------------------------------------------------------------------------
+# Training: the MLGRU recurrence backward
+# ---------------------------------------------------------------------------
+
+
+def mlgru_scan_backward(pf, pc, pg, h0, do, dhT=None):
+    """Gradients of the MLGRU scan (``mlgru_scan``) for upstream gradients do = dL/do' [B,T,d]
+    and dhT = dL/dh_T [B,d] (zero when None), in fp64.
+
+    [DC] "Memory efficiency" / "From optimised GPU to custom FPGA design": the
+    models are trained with fused GPU kernels; the pages give no backward
+    formula, so this is the exact derivative of the forward reading
+        f = sigmoid(f~), c = SiLU(c~), g = sigmoid(g~),
+        h_t = f_t h_{t-1} + (1 - f_t) c_t,  o'_t = g_t h_t.
+    With lambda_t = dL/dh_t (through o'_t and h_{t+1}):
+        lambda_T = do_T g_T + dhT,  lambda_t = do_t g_t + f_{t+1} lambda_{t+1}
+        dg~_t = do_t h_t g_t (1 - g_t)
+        df~_t = lambda_t (h_{t-1} - c_t) f_t (1 - f_t)
+        dc~_t = lambda_t (1 - f_t) SiLU'(c~_t),  SiLU'(z) = s (1 + z (1 - s)), s = sigmoid(z)
+        dh0 = f_1 lambda_1
+    Returns (dpf, dpc, dpg [B,T,d], dh0 [B,d]).
+    """
+    pf = np.asarray(pf, dtype=np.float64)
+    pc = np.asarray(pc, dtype=np.float64)
+    pg = np.asarray(pg, dtype=np.float64)
+    do = np.asarray(do, dtype=np.float64)
+    B, T, d = pf.shape
+    f, g = sigmoid(pf), sigmoid(pg)
+    sc = sigmoid(pc)
+    c = pc * sc
+    hs = np.empty((B, T + 1, d))
+    hs[:, 0] = np.asarray(h0, dtype=np.float64)
+    for t in range(T):
+        hs[:, t + 1] = f[:, t] * hs[:, t] + (1.0 - f[:, t]) * c[:, t]
+    lam = np.zeros((B, d)) if dhT is None else np.array(dhT, dtype=np.float64, copy=True)
+    dpf, dpc, dpg = np.empty_like(pf), np.empty_like(pf), np.empty_like(pf)
+    for t in range(T - 1, -1, -1):
+        lam = lam + do[:, t] * g[:, t]                 # lambda_t
+        h, hp = hs[:, t + 1], hs[:, t]
+        dpg[:, t] = do[:, t] * h * g[:, t] * (1.0 - g[:, t])
+        dpf[:, t] = lam * (hp - c[:, t]) * f[:, t] * (1.0 - f[:, t])
+        dpc[:, t] = lam * (1.0 - f[:, t]) * sc[:, t] * (1.0 + pc[:, t] * (1.0 - sc[:, t]))
+        lam = f[:, t] * lam                             # the part of lambda_{t-1} through h_t
+    return dpf, dpc, dpg, lam

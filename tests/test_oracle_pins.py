@@ -718,3 +718,61 @@ def test_generation_matches_prefill_of_the_grown_sequence():
     # the carried state after the last fed-back token is the prefill's state over everything
     _, h_all = O.model_forward(np.concatenate([prompt, toks], axis=1), E, blocks, head, np.zeros((2, 1, d)), "f32")
     np.testing.assert_allclose(hs, h_all, rtol=1e-5, atol=1e-6)
+
+
+# ----------------------------------------------------------------- scan backward
+
+def _scan_loss(pf, pc, pg, h0, do, dhT):
+    o, hT = O.mlgru_scan(pf, pc, pg, h0)
+    return float(np.sum(o * do) + np.sum(hT * dhT))
+
+
+def test_scan_backward_matches_central_differences():
+    # every gradient against (L(x + e) - L(x - e)) / 2e of the forward oracle
+    B, T, d = 2, 7, 3
+    pf, pc, pg = (1.5 * a for a in _scan_inputs(90, B, T, d))
+    h0 = synth.activations(91, B, d).numpy().astype(np.float64)
+    do = synth.activations(92, B * T, d).numpy().astype(np.float64).reshape(B, T, d)
+    dhT = synth.activations(93, B, d).numpy().astype(np.float64)
+    dpf, dpc, dpg, dh0 = O.mlgru_scan_backward(pf, pc, pg, h0, do, dhT)
+    eps = 1e-6
+    for arr, grad in ((pf, dpf), (pc, dpc), (pg, dpg)):
+        num = np.empty_like(arr)
+        for idx in np.ndindex(arr.shape):
+            old = arr[idx]
+            arr[idx] = old + eps
+            lp = _scan_loss(pf, pc, pg, h0, do, dhT)
+            arr[idx] = old - eps
+            lm = _scan_loss(pf, pc, pg, h0, do, dhT)
+            arr[idx] = old
+            num[idx] = (lp - lm) / (2 * eps)
+        np.testing.assert_allclose(grad, num, rtol=1e-6, atol=1e-8)
+    num = np.empty_like(h0)
+    for idx in np.ndindex(h0.shape):
+        old = h0[idx]
+        h0[idx] = old + eps
+        lp = _scan_loss(pf, pc, pg, h0, do, dhT)
+        h0[idx] = old - eps
+        lm = _scan_loss(pf, pc, pg, h0, do, dhT)
+        h0[idx] = old
+        num[idx] = (lp - lm) / (2 * eps)
+    np.testing.assert_allclose(dh0, num, rtol=1e-6, atol=1e-8)
+
+
+def test_scan_backward_special_cases():
+    pf, pc, pg = _scan_inputs(94, B=2, T=9, d=4)
+    h0 = synth.activations(95, 2, 4).numpy().astype(np.float64)
+    do = synth.activations(96, 18, 4).numpy().astype(np.float64).reshape(2, 9, 4)
+    # no upstream gradient: every gradient is zero
+    z = O.mlgru_scan_backward(pf, pc, pg, h0, np.zeros_like(do))
+    assert all(np.all(a == 0.0) for a in z)
+    # forget gate ~0 (f~ = -40): h_t = c_t, so dc~_t = do_t g_t SiLU'(c~_t), dh0 ~ 0
+    pf0 = np.full_like(pf, -40.0)
+    dpf, dpc, dpg, dh0 = O.mlgru_scan_backward(pf0, pc, pg, h0, do)
+    s = O.sigmoid(pc)
+    np.testing.assert_allclose(dpc, do * O.sigmoid(pg) * s * (1 + pc * (1 - s)), rtol=1e-12, atol=1e-15)
+    assert np.max(np.abs(dh0)) < 1e-15
+    # only dhT: lambda is the product of the forget gates from the end
+    dpf, dpc, dpg, dh0 = O.mlgru_scan_backward(pf, pc, pg, h0, np.zeros_like(do), np.ones((2, 4)))
+    np.testing.assert_allclose(dh0, np.prod(O.sigmoid(pf), axis=1), rtol=1e-12)
+    assert np.all(dpg == 0.0)
