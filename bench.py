@@ -72,6 +72,8 @@ def parse_args(argv=None):
                     help="stack370m: number of blocks (default 24; fewer for short profiler captures)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the end-to-end (host buffers) pass")
     ap.add_argument("--no-cpu-baseline", action="store_true", help="skip timing the CPU oracle")
+    ap.add_argument("--backward", action="store_true",
+                    help="scan: the scan's backward (training gradients) instead of its forward")
     ap.add_argument("--gnorm", action="store_true",
                     help="scan / stack370m: the g_norm output gate (RMSNorm of the state fused with a swish gate)")
     ap.add_argument("--no-sub", action="store_true",
@@ -667,6 +669,37 @@ def measure_scan(mmf, dev, steps: int, warmup: int, gnorm: bool, flush=None) -> 
     return r
 
 
+def measure_scan_backward(mmf, dev, steps: int, warmup: int) -> dict:
+    """The scan's backward on the 370M layer shape (8 x 2048 tokens, d = 1024, bf16), L2 flushed between
+    steps. Algorithmic bytes: 14 per channel-step (pre-activations 6 and dL/do' 2 read, the three
+    gradients 6 written); the design also recomputes the forward states (6 B read, 4 B written) and
+    reads them back (4 B): 28 B per channel-step."""
+    w = synth.STACK_370M
+    B, T, d = w.batch, w.seq, w.d
+    pre = synth.preacts(77, B, T, d, torch.bfloat16, scale=2.0, device=dev)
+    dout = synth.activations(79, B * T, d, torch.bfloat16, device=str(dev)).reshape(B, T, d)
+    h0 = torch.zeros(B, d, device=dev)
+    ws = torch.empty(mmf.load().mmf_mlgru_scan_backward_ws_size(B, T, d), dtype=torch.uint8, device=dev)
+    flush = L2Flush(dev)
+    for _ in range(warmup):
+        mmf.mlgru_scan_backward(pre, h0, dout, ws=ws)
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    torch.cuda.synchronize()
+    for _ in range(steps):
+        flush()
+        mmf.mlgru_scan_backward(pre, h0, dout, ws=ws)
+    torch.cuda.synchronize()
+    mmf.prof_enable(False)
+    prof = mmf.prof_collect()
+    key = "mlgru_scan_backward"
+    ms = prof[key][1] / prof[key][0]
+    nbytes = 14.0 * B * T * d
+    gbs = nbytes / (ms / 1e3) / 1e9
+    return {"workload": f"mlgru_scan_backward_b{B}_t{T}_d{d}_bf16", "us": round(ms * 1e3, 2), "GBps": round(gbs, 1),
+            "bytes": nbytes, "design_bytes": 28.0 * B * T * d, "launches": 2 * prof[key][0]}
+
+
 def run_scan(args):
     """One MLGRU scan per step on the 370M layer shape; GB/s = 8 bytes per channel-step (bf16)."""
     _, rank, local = dist_env()
@@ -674,9 +707,11 @@ def run_scan(args):
     import ternary_weight_matmul_fusedbitlinear_b200 as mmf
     dev = torch.device("cuda", local)
     peaks, peak_kind = load_peaks()
-    m = measure_scan(mmf, dev, args.steps, args.warmup, args.gnorm)
+    m = (measure_scan_backward(mmf, dev, args.steps, args.warmup) if args.backward
+         else measure_scan(mmf, dev, args.steps, args.warmup, args.gnorm))
     gbs, ms = m["GBps"], m["us"] / 1e3
-    kernel = "mlgru_scan_gnorm (scan + row kernel)" if args.gnorm else "mlgru_scan"
+    kernel = ("mlgru_scan_backward (forward states + reverse scan)" if args.backward
+              else "mlgru_scan_gnorm (scan + row kernel)" if args.gnorm else "mlgru_scan")
     if rank == 0:
         print(json.dumps({
             "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,

@@ -182,6 +182,33 @@ size_t mmf_mlgru_scan_ws_size(int32_t B, int32_t T, int32_t d);
 mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
                           float* h, void* o, void* ws, size_t ws_bytes, void* stream);
 
+/* Scratch bytes mmf_mlgru_scan_backward needs: the forward states, 4 x B x T x d. */
+size_t mmf_mlgru_scan_backward_ws_size(int32_t B, int32_t T, int32_t d);
+
+/* Training: gradients of mmf_mlgru_scan (sigmoid output gate) for the
+ * upstream gradients dout = dL/do' and dhT = dL/dh_T. The pages give no
+ * backward formula ([DC] "Memory efficiency": the models are trained with
+ * fused GPU kernels); this is the exact derivative of the forward recurrence.
+ * With lambda_t = dL/dh_t and mu_t = f_t lambda_t:
+ *   lambda_t = dout_t g_t + mu_{t+1},  mu_T = dhT
+ *   dg~_t = dout_t h_t g_t (1 - g_t)
+ *   df~_t = lambda_t (h_{t-1} - c_t) f_t (1 - f_t)
+ *   dc~_t = lambda_t (1 - f_t) sigmoid(c~_t) (1 + c~_t (1 - sigmoid(c~_t)))
+ *   dh0 = mu_0
+ *   pre  (device) [B, T, 3, d] in dtype: the forward's pre-activations
+ *   h0   (device) float [B, d]: the forward's initial state (read only)
+ *   dout (device) [B, T, d] in dtype; dhT (device) float [B, d] or NULL (zero)
+ *   dpre (device) [B, T, 3, d] in dtype: dL/df~, dL/dc~, dL/dg~ per token
+ *   dh0  (device) float [B, d]: dL/dh0; must not overlap h0
+ *   ws   (device) scratch of mmf_mlgru_scan_backward_ws_size(B, T, d) bytes.
+ * Two launches: the forward scan writing the states h_t into ws, then a
+ * reverse chunked scan (one CTA per sequence x 64 channels, chunks from the
+ * last to the first, the backward maps mu -> f mu + f dout g composed like
+ * the forward ones). T = 0 does nothing. Errors: as mmf_mlgru_scan. */
+mmf_status mmf_mlgru_scan_backward(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
+                                   const float* h0, const void* dout, const float* dhT, void* dpre,
+                                   float* dh0, void* ws, size_t ws_bytes, void* stream);
+
 /* Scratch bytes mmf_mlgru_scan_gnorm needs: 4 x B x T x d bytes for
  * v = swish(g~) h in fp32, 4 x B x T x ceil(d / 32) for the partial sums of
  * h^2, and a little padding. */

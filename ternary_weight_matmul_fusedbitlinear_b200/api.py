@@ -165,6 +165,24 @@ def mlgru_scan_gnorm(pre: torch.Tensor, h: torch.Tensor, gain: torch.Tensor, eps
     return o
 
 
+def mlgru_scan_backward(pre: torch.Tensor, h0: torch.Tensor, dout: torch.Tensor,
+                        dhT: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+    """Gradients of mlgru_scan: (dpre [B, T, 3, d] in pre's dtype, dh0 [B, d] fp32) for
+    dout = dL/do' [B, T, d] and dhT = dL/dh_T [B, d] (zero when None)."""
+    _need_cuda(pre, h0, dout, dhT)
+    B, T, _, d = pre.shape
+    if dout.shape != (B, T, d) or dout.dtype != pre.dtype:
+        raise ValueError("dout must be [B, T, d] in pre's dtype")
+    dpre = torch.empty_like(pre)
+    dh0 = torch.empty(B, d, dtype=torch.float32, device=pre.device)
+    lib = L.load()
+    w = _workspace(lib.mmf_mlgru_scan_backward_ws_size(B, T, d), pre.device, ws)
+    L.check(lib.mmf_mlgru_scan_backward(_vp(pre), _dtype(pre), B, T, d, _vp(h0), _vp(dout), _vp(dhT), _vp(dpre),
+                                        _vp(dh0), _vp(w), w.numel() * w.element_size(), _stream(pre.device)),
+            "mmf_mlgru_scan_backward")
+    return dpre, dh0
+
+
 def glu(gate: TLinear, up: TLinear, down: TLinear, x: torch.Tensor, residual: Optional[torch.Tensor] = None,
         eps: float = DEFAULT_EPS, ws: Optional[torch.Tensor] = None) -> torch.Tensor:
     """y = down(SiLU(gate(x)) * up(x)) (+ residual) for x [..., d]."""

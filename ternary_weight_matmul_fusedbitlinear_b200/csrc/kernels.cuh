@@ -162,6 +162,14 @@ cudaError_t launch_mlgru_scan(const void* pre, mmf_dtype dt, int B, int T, int d
 size_t mlgru_scan_gnorm_ws_bytes(int B, int T, int d);
 cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, const float* gain,
                                     float eps, void* o, void* ws, int* status, cudaStream_t stream);
+// Backward of the scan (training): the forward states h_t (fp32, into `ws`,
+// mlgru_scan_bwd_ws_bytes), then a reverse chunked scan writing dL/d(f~, c~, g~)
+// [B, T, 3, d] in dtype and dL/dh0 [B, d] (also the forward's carried-state
+// scratch until the reverse scan overwrites it).
+size_t mlgru_scan_bwd_ws_bytes(int B, int T, int d);
+cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, int d, const float* h0,
+                                  const void* dout, const float* dhT, void* dpre, float* dh0, void* ws, int* status,
+                                  cudaStream_t stream);
 // Inside a block: the same scan, then one row kernel that forms o' and
 // quantises it for the o projection (RMSNorm gain qgain, eps) into q / scale /
 // qsum with the standalone quantiser's row routine; o' is written only when

@@ -207,13 +207,14 @@ __device__ void drain_stage(uint64_t* bar, uint32_t parity, long long limit) {
 
 // CC = 32 keeps at most 64 registers per thread so that two CTAs share an SM.
 // GN: g_norm mode; `o` receives v = swish(g~) h in fp32 and `ss` [B*T_][n_cb]
-// the partial sums of h^2 (see the file comment). Otherwise `o` receives o'.
-template <typename T, int CC, bool GN>
+// the partial sums of h^2 (see the file comment). HS: `o` receives the states
+// h_t themselves in fp32 (what the backward pass reads). Otherwise `o` receives o'.
+template <typename T, int CC, bool GN, bool HS = false>
 __global__ void __launch_bounds__(kThreads, 64 / CC)
     mlgru_scan_kernel(const __grid_constant__ CUtensorMap map, int B, int T_, int d, int n_cb, int nst,
                       float* __restrict__ h, void* __restrict__ out, float* __restrict__ ss, int* status,
                       long long wait_cycles, int skip_chunk) {
-  using OT = std::conditional_t<GN, float, T>;
+  using OT = std::conditional_t<GN || HS, float, T>;
   OT* __restrict__ o = static_cast<OT*>(out);
   using S = ScanSmem<CC>;
   constexpr int NP = S::NP;         // channel pairs: lanes per step group
@@ -323,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 64 / CC)
 #pragma unroll
       for (int k = 0; k < LS; ++k) {
         hw = fma2(f[k], hw, bb[k]);
-        if (full || t0 + tw + k < T_) store_pair(op + (size_t)k * d, mul2(gg[k], hw));
+        if (full || t0 + tw + k < T_) store_pair(op + (size_t)k * d, HS ? hw : mul2(gg[k], hw));
         if constexpr (GN) {
           const F2 h2 = mul2(hw, hw);
           sq[k] = lo(h2) + hi(h2);
@@ -347,7 +348,7 @@ __global__ void __launch_bounds__(kThreads, 64 / CC)
   }
 }
 
-template <typename T, int CC, bool GN>
+template <typename T, int CC, bool GN, bool HS = false>
 cudaError_t launch_typed(const void* pre, int B, int T_, int d, float* h, void* o, float* ss, int* status,
                          long long wait_cycles, int skip_chunk, cudaStream_t stream) {
   CUtensorMap map;
@@ -361,7 +362,7 @@ cudaError_t launch_typed(const void* pre, int B, int T_, int d, float* h, void* 
   const size_t budget = CC == 32 ? 96 * 1024 : 192 * 1024;   // two CTAs per SM with CC = 32
   const int nst = (int)std::max<size_t>(2, std::min<size_t>(kMaxStages, budget / stage_bytes));
   const size_t smem = 128 + tiles_offset<CC>() + nst * stage_bytes;
-  auto kern = mlgru_scan_kernel<T, CC, GN>;
+  auto kern = mlgru_scan_kernel<T, CC, GN, HS>;
   const cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   return launch_pdl(kern, dim3(B * n_cb), dim3(kThreads), smem, stream, map, B, T_, d, n_cb, nst, h, o, ss, status,
@@ -457,6 +458,159 @@ __global__ void __launch_bounds__(kApplyWarps * 32)
   }
 }
 
+// ---------------------------------------------------------------- backward
+// The exact derivative of the recurrence above for upstream gradients
+// do = dL/do' and dhT = dL/dh_T. With lambda_t = dL/dh_t and mu_t = f_t lambda_t
+// (the part of lambda_t that reaches h_{t-1}):
+//   lambda_t = do_t g_t + mu_{t+1},   mu_t = f_t lambda_t,   mu_T = dhT
+//   dg~_t = do_t h_t g_t (1 - g_t)
+//   df~_t = lambda_t (h_{t-1} - c_t) f_t (1 - f_t)
+//   dc~_t = lambda_t (1 - f_t) sigmoid(c~_t) (1 + c~_t (1 - sigmoid(c~_t)))
+//   dh0 = mu_0
+// mu runs backwards through affine maps mu -> f_t mu + f_t do_t g_t, which
+// compose like the forward maps. One CTA per (sequence, 64 channels) walks the
+// chunks from the last to the first; within a chunk each lane composes its 8
+// steps, the warps' maps meet in shared memory (one barrier per chunk, double
+// buffered by chunk parity), each warp folds the maps of the warps after it
+// onto the mu entering the chunk's end, then replays its steps backwards and
+// stores the three gradients. The states h_t come from the forward scan in its
+// HS mode (fp32).
+constexpr int kBwdCC = 64;
+struct BwdSmem {
+  F2 A[2][SW][kBwdCC / 2];
+  F2 Bv[2][SW][kBwdCC / 2];
+  F2 mu_prev[2][kBwdCC / 2];   // mu leaving the chunk at its start (written by warp 0)
+};
+
+__device__ __forceinline__ F2 load_zr(const bf16* p) {   // raw value pair (no floor)
+  const uint32_t w = *reinterpret_cast<const uint32_t*>(p);
+  return f2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+}
+__device__ __forceinline__ F2 load_zr(const float* p) { return F2{*reinterpret_cast<const unsigned long long*>(p)}; }
+
+// sigmoid of a pair, with the exponent argument floored as in the forward pass
+__device__ __forceinline__ F2 sigmoid2(F2 z) {
+  const F2 zc = f2(fmaxf(lo(z), kMinZ), fmaxf(hi(z), kMinZ));
+  const F2 p = add2(exp_neg(zc), f2(1.0f, 1.0f));
+  return f2(rcp_approx(lo(p)), rcp_approx(hi(p)));
+}
+
+// L2 prefetch of chunk j's rows of this CTA's channels (pre-activations, dL/do',
+// states): one 128-byte line per thread and step of the loop.
+template <typename T>
+__device__ __forceinline__ void bwd_prefetch(const T* pre, const float* hs, const T* dout, size_t row0, int T_, int d,
+                                             int ch0, int j) {
+  constexpr int kLineEl = 128 / sizeof(T);        // elements of T per line
+  constexpr int kPerRowT = kBwdCC / kLineEl;      // lines per row of T (1 or 2)
+  constexpr int kPerRowH = kBwdCC * 4 / 128;      // lines per row of fp32 states (2)
+  constexpr int kLines = TC * (4 * kPerRowT + kPerRowH);
+  for (int l = threadIdx.x; l < kLines; l += kThreads) {
+    int r, idx = l;
+    const void* addr;
+    if (idx < TC * 3 * kPerRowT) {   // pre-activations: row, gate, part
+      r = idx / (3 * kPerRowT);
+      const int rem = idx - r * 3 * kPerRowT, g = rem / kPerRowT, part = rem - g * kPerRowT;
+      if (j * TC + r >= T_ || ch0 + part * kLineEl >= d) continue;   // the line starts inside the row
+      addr = pre + ((row0 + j * TC + r) * 3 + g) * (size_t)d + ch0 + part * kLineEl;
+    } else if ((idx -= TC * 3 * kPerRowT) < TC * kPerRowT) {   // dL/do'
+      r = idx / kPerRowT;
+      if (j * TC + r >= T_ || ch0 + (idx - r * kPerRowT) * kLineEl >= d) continue;
+      addr = dout + (row0 + j * TC + r) * (size_t)d + ch0 + (idx - r * kPerRowT) * kLineEl;
+    } else {   // states
+      idx -= TC * kPerRowT;
+      r = idx / kPerRowH;
+      if (j * TC + r >= T_ || ch0 + (idx - r * kPerRowH) * 32 >= d) continue;
+      addr = hs + (row0 + j * TC + r) * (size_t)d + ch0 + (idx - r * kPerRowH) * 32;
+    }
+    asm volatile("prefetch.global.L2 [%0];" ::"l"(addr));
+  }
+}
+
+template <typename T>
+__global__ void __launch_bounds__(kThreads, 1)
+    mlgru_scan_bwd_kernel(const T* __restrict__ pre, const float* __restrict__ hs, const float* __restrict__ h0,
+                          const T* __restrict__ dout, const float* __restrict__ dhT, int B, int T_, int d, int n_cb,
+                          T* __restrict__ dpre, float* __restrict__ dh0) {
+  __shared__ BwdSmem sm;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x / n_cb, cb = blockIdx.x - b * n_cb;
+  const int ch = cb * kBwdCC + 2 * lane;
+  const bool valid = ch < d;
+  const int nchunk = ceil_div(T_, TC);
+  const int tw = warp * WS;
+  pdl_trigger();
+  pdl_wait();   // the states are the forward scan's output
+  F2 mu_end = f2(0.0f, 0.0f);   // mu entering the current chunk's end
+  if (valid && dhT != nullptr) mu_end = load_h(dhT + (size_t)b * d + ch);
+  const size_t row0 = (size_t)b * T_;
+  const int ch0 = cb * kBwdCC;
+  bwd_prefetch(pre, hs, dout, row0, T_, d, ch0, nchunk - 1);
+  for (int j = nchunk - 1; j >= 0; --j) {
+    const int par = j & 1;
+    const int t0 = j * TC;
+    if (j > 0) bwd_prefetch(pre, hs, dout, row0, T_, d, ch0, j - 1);   // the next chunk, into L2
+    // 1. f_t and a_t = do_t g_t of this lane's steps, composed backwards
+    F2 f[WS], a[WS];
+    F2 Aa = f2(1.0f, 1.0f), Bb = f2(0.0f, 0.0f);
+#pragma unroll
+    for (int k = WS - 1; k >= 0; --k) {
+      const int t = t0 + tw + k;
+      if (valid && t < T_) {
+        const T* pr = pre + (row0 + t) * 3 * (size_t)d + ch;
+        f[k] = sigmoid2(load_zr(pr));
+        const F2 g = sigmoid2(load_zr(pr + 2 * (size_t)d));
+        a[k] = mul2(load_zr(dout + (row0 + t) * (size_t)d + ch), g);
+      } else {   // past the end of the sequence (or channel): identity map
+        f[k] = f2(1.0f, 1.0f);
+        a[k] = f2(0.0f, 0.0f);
+      }
+      // step k after the steps behind it: mu -> f (a + (A mu + B))
+      Bb = mul2(f[k], add2(a[k], Bb));
+      Aa = mul2(f[k], Aa);
+    }
+    sm.A[par][warp][lane] = Aa;
+    sm.Bv[par][warp][lane] = Bb;
+    __syncthreads();
+    // 2. mu entering this warp's last step: the maps of the warps after it,
+    //    applied to the mu entering the chunk's end; warp 0 also gets the mu
+    //    leaving the chunk's start
+    if (j < nchunk - 1) mu_end = sm.mu_prev[par ^ 1][lane];
+    F2 mu = mu_end;
+    for (int w = SW - 1; w > warp; --w) mu = fma2(sm.A[par][w][lane], mu, sm.Bv[par][w][lane]);
+    if (warp == 0) sm.mu_prev[par][lane] = fma2(Aa, mu, Bb);
+    // 3. replay backwards: lambda, the three gradients, mu for the step before
+#pragma unroll
+    for (int k = WS - 1; k >= 0; --k) {
+      const int t = t0 + tw + k;
+      const F2 lam = add2(a[k], mu);
+      if (valid && t < T_) {
+        const T* pr = pre + (row0 + t) * 3 * (size_t)d + ch;
+        const F2 zc = load_zr(pr + d);
+        const F2 g = sigmoid2(load_zr(pr + 2 * (size_t)d));
+        const F2 sc = sigmoid2(zc);
+        const F2 one = f2(1.0f, 1.0f);
+        const F2 c = mul2(zc, sc);
+        const F2 ht = load_h(hs + (row0 + t) * (size_t)d + ch);
+        const F2 hp = t > 0 ? load_h(hs + (row0 + t - 1) * (size_t)d + ch) : load_h(h0 + (size_t)b * d + ch);
+        const F2 dov = load_zr(dout + (row0 + t) * (size_t)d + ch);
+        const F2 omf = add2(one, mul2(f[k], f2(-1.0f, -1.0f)));
+        const F2 omg = add2(one, mul2(g, f2(-1.0f, -1.0f)));
+        const F2 dzg = mul2(mul2(dov, ht), mul2(g, omg));
+        const F2 dzf = mul2(mul2(lam, add2(hp, mul2(c, f2(-1.0f, -1.0f)))), mul2(f[k], omf));
+        const F2 silu_p = mul2(sc, fma2(zc, add2(one, mul2(sc, f2(-1.0f, -1.0f))), one));
+        const F2 dzc = mul2(mul2(lam, omf), silu_p);
+        T* out = dpre + (row0 + t) * 3 * (size_t)d + ch;
+        store_pair(out, dzf);
+        store_pair(out + d, dzc);
+        store_pair(out + 2 * (size_t)d, dzg);
+      }
+      mu = mul2(f[k], lam);
+    }
+  }
+  __syncthreads();   // warp 0 has written the mu leaving the first chunk
+  if (valid && warp == 0) store_pair(dh0 + (size_t)b * d + ch, sm.mu_prev[0][lane]);
+}
+
 // 64 channels per CTA when that gives enough CTAs to cover the GPU, else 32
 bool scan_wide(int B, int d) { return (size_t)B * ceil_div(d, 64) >= (size_t)num_sms() * 3 / 4; }
 
@@ -530,6 +684,38 @@ cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T,
                       (const float*)ss, n_cb, gain, eps, (int)M, d, static_cast<bf16*>(o));
   return launch_pdl(gnorm_apply_kernel<float>, dim3(grid), dim3(32 * kWarpsA), 0, stream, (const float*)v,
                     (const float*)ss, n_cb, gain, eps, (int)M, d, static_cast<float*>(o));
+}
+
+size_t mlgru_scan_bwd_ws_bytes(int B, int T, int d) { return ((size_t)B * T * d * sizeof(float) + 255) / 256 * 256; }
+
+cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, int d, const float* h0,
+                                  const void* dout, const float* dhT, void* dpre, float* dh0, void* ws, int* status,
+                                  cudaStream_t stream) {
+  if (B == 0 || T == 0) return cudaSuccess;
+  if (!tma_available()) return cudaErrorNotSupported;
+  // 1. the forward states h_t (fp32) into ws; the state buffer starts from h0
+  float* hsv = static_cast<float*>(ws);
+  float* hcur = dh0;   // scratch for the forward scan's carried state: dh0 is written last
+  cudaError_t e = cudaMemcpyAsync(hcur, h0, sizeof(float) * (size_t)B * d, cudaMemcpyDeviceToDevice, stream);
+  if (e != cudaSuccess) return e;
+  const long long wait = wait_limit_cycles();
+  const bool wide = scan_wide(B, d);
+  if (dt == MMF_BF16)
+    e = wide ? launch_typed<bf16, 64, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream)
+             : launch_typed<bf16, 32, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream);
+  else
+    e = wide ? launch_typed<float, 64, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream)
+             : launch_typed<float, 32, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream);
+  if (e != cudaSuccess) return e;
+  // 2. the reverse scan
+  const int n_cb = ceil_div(d, kBwdCC);
+  if (dt == MMF_BF16)
+    return launch_pdl(mlgru_scan_bwd_kernel<bf16>, dim3(B * n_cb), dim3(kThreads), 0, stream,
+                      static_cast<const bf16*>(pre), (const float*)hsv, h0, static_cast<const bf16*>(dout), dhT, B, T,
+                      d, n_cb, static_cast<bf16*>(dpre), dh0);
+  return launch_pdl(mlgru_scan_bwd_kernel<float>, dim3(B * n_cb), dim3(kThreads), 0, stream,
+                    static_cast<const float*>(pre), (const float*)hsv, h0, static_cast<const float*>(dout), dhT, B, T, d,
+                    n_cb, static_cast<float*>(dpre), dh0);
 }
 
 cudaError_t launch_mlgru_scan_gnorm_quant(const void* pre, mmf_dtype dt, int B, int T, int d, float* h,

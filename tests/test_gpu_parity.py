@@ -177,6 +177,27 @@ def test_scan_gnorm_closed_forms_on_gpu():
     np.testing.assert_allclose(np.mean(to_np(o) ** 2, axis=-1), O.silu(z) ** 2 * ms / (ms + eps), rtol=1e-5)
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("b,t,d,with_dhT", [(2, 64, 256, True), (1, 3, 16, False), (3, 200, 264, True),
+                                            (8, 1, 1024, True), (4, 517, 2048, False), (8, 300, 2560, True)])
+def test_scan_backward_parity(b, t, d, with_dhT, dtype):
+    # training: the scan's gradients against the oracle's exact derivative,
+    # ragged chunks and channel blocks, T = 1, with and without dL/dh_T
+    pre = synth.preacts(440 + t, b, t, d, TORCH_DT[dtype], scale=2.0)
+    h0 = synth.activations(441, b, d)
+    dout = synth.activations(442 + t, b * t, d, TORCH_DT[dtype]).reshape(b, t, d)
+    dhT = synth.activations(443, b, d) if with_dhT else None
+    dpre, dh0 = mmf.mlgru_scan_backward(pre.cuda(), h0.cuda(), dout.cuda(), None if dhT is None else dhT.cuda())
+    mmf.check()
+    p = to_np(pre)
+    ref = O.mlgru_scan_backward(p[:, :, 0], p[:, :, 1], p[:, :, 2], h0.numpy().astype(np.float64), to_np(dout),
+                                None if dhT is None else dhT.numpy().astype(np.float64))
+    g = to_np(dpre)
+    for j, name in enumerate(("df~", "dc~", "dg~")):
+        assert_close(g[:, :, j], ref[j], dtype, name)
+    assert_close(to_np(dh0), ref[3], "f32", "dh0")
+
+
 def test_scan_wait_gives_up_and_reports(monkeypatch):
     # failure detection without a fault: chunk 1 of CTA 0 is never loaded, so
     # its bounded wait runs out (20 ms); the kernel lets its other copies land
