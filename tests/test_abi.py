@@ -144,3 +144,16 @@ def test_block_gnorm_gain_validation_and_workspace(lib):
     # the g_norm scan's scratch (v in fp32 and the partial sums) comes on top
     assert lib.mmf_block_ws_size(h, 2, 8) >= plain + lib.mmf_mlgru_scan_gnorm_ws_size(2, 8, d) - 256
     lib.mmf_block_destroy(h)
+
+
+def test_scan_backward_validation(lib):
+    p = ctypes.c_void_p(4096)
+    q = ctypes.c_void_p(1 << 20)
+    ws = lib.mmf_mlgru_scan_backward_ws_size(2, 300, 64)
+    assert ws >= 4 * 2 * 300 * 64
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 12, p, p, None, p, q, p, 1 << 20, None) == 2      # d % 8
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, None, p, None, p, q, p, 1 << 20, None) == 1   # null h0
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, p, p, None, p, p, p, 1 << 20, None) == 1      # h0 = dh0
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, p, p, ctypes.c_void_p(4104), p, q, p, 1 << 20, None) == 3
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 300, 64, p, p, None, p, q, p, ws - 1, None) == 4      # workspace
+    assert lib.mmf_mlgru_scan_backward(None, 0, 0, 3, 16, None, None, None, None, None, None, 0, None) == 0
