@@ -611,6 +611,136 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (valid && warp == 0) store_pair(dh0 + (size_t)b * d + ch, sm.mu_prev[0][lane]);
 }
 
+// The same backward for bf16 with its inputs staged by TMA: each chunk's
+// pre-activation, dL/do' and state tiles (96 KB) land in one of two stages, so
+// phases 1 and 3 read shared memory; a stage is refilled with the chunk two
+// ahead at the next chunk's barrier, when every warp has finished its replay.
+// Every wait is bounded (status code 2 on timeout, as in the forward scan).
+struct BwdTile {
+  bf16 pre[3][TC][kBwdCC];
+  bf16 dout[TC][kBwdCC];
+  float h[TC][kBwdCC];
+};
+constexpr uint32_t kBwdTileBytes = sizeof(BwdTile);
+
+__global__ void __launch_bounds__(kThreads, 1)
+    mlgru_scan_bwd_tma_kernel(const __grid_constant__ CUtensorMap map_pre, const __grid_constant__ CUtensorMap map_do,
+                              const __grid_constant__ CUtensorMap map_h, const float* __restrict__ hs,
+                              const float* __restrict__ h0, const float* __restrict__ dhT, int B, int T_, int d,
+                              int n_cb, bf16* __restrict__ dpre, float* __restrict__ dh0, int* status,
+                              long long wait_cycles, int skip_chunk) {
+  __shared__ BwdSmem sm;
+  __shared__ uint64_t full[2];
+  extern __shared__ uint8_t smem_raw[];
+  BwdTile* ring = reinterpret_cast<BwdTile*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int b = blockIdx.x / n_cb, cb = blockIdx.x - b * n_cb;
+  const int ch = cb * kBwdCC + 2 * lane;
+  const bool valid = ch < d;
+  const int nchunk = ceil_div(T_, TC);
+  const int tw = warp * WS;
+  const size_t row0 = (size_t)b * T_;
+  auto issue = [&](int j) {   // thread 0: chunk j into stage (nchunk - 1 - j) & 1
+    const int s = (nchunk - 1 - j) & 1;
+    const int y = (int)row0 + j * TC;
+    if (j == skip_chunk && blockIdx.x == 0) return;   // test hook: this copy is never issued
+    mbar_arrive_expect_tx(&full[s], kBwdTileBytes);
+    for (int g = 0; g < 3; ++g) tma_load_2d(&ring[s].pre[g][0][0], &map_pre, g * d + cb * kBwdCC, y, &full[s]);
+    tma_load_2d(&ring[s].dout[0][0], &map_do, cb * kBwdCC, y, &full[s]);
+    tma_load_2d(&ring[s].h[0][0], &map_h, cb * kBwdCC, y, &full[s]);
+  };
+  if (threadIdx.x == 0) {
+    mbar_init(&full[0], 1);
+    mbar_init(&full[1], 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  __syncthreads();
+  pdl_trigger();
+  pdl_wait();   // the states are the forward scan's output
+  if (threadIdx.x == 0) {
+    issue(nchunk - 1);
+    if (nchunk > 1) issue(nchunk - 2);
+  }
+  F2 mu_end = f2(0.0f, 0.0f);
+  if (valid && dhT != nullptr) mu_end = load_h(dhT + (size_t)b * d + ch);
+  for (int j = nchunk - 1; j >= 0; --j) {
+    const int q = nchunk - 1 - j, s = q & 1, par = j & 1;
+    const int t0 = j * TC;
+    bool got = mbar_try_wait(&full[s], (uint32_t)(q >> 1) & 1u);
+    if (!got) {
+      const long long t_start = clock64();
+      while (!(got = mbar_try_wait(&full[s], (uint32_t)(q >> 1) & 1u)) && clock64() - t_start < wait_cycles) {
+      }
+    }
+    const BwdTile& tile = ring[s];
+    // 1. f_t and a_t = do_t g_t, composed backwards
+    F2 f[WS], a[WS];
+    F2 Aa = f2(1.0f, 1.0f), Bb = f2(0.0f, 0.0f);
+#pragma unroll
+    for (int k = WS - 1; k >= 0; --k) {
+      const int tl = tw + k;
+      if (valid && t0 + tl < T_) {
+        f[k] = sigmoid2(load_zr(&tile.pre[0][tl][2 * lane]));
+        a[k] = mul2(load_zr(&tile.dout[tl][2 * lane]), sigmoid2(load_zr(&tile.pre[2][tl][2 * lane])));
+      } else {
+        f[k] = f2(1.0f, 1.0f);
+        a[k] = f2(0.0f, 0.0f);
+      }
+      Bb = mul2(f[k], add2(a[k], Bb));
+      Aa = mul2(f[k], Aa);
+    }
+    sm.A[par][warp][lane] = Aa;
+    sm.Bv[par][warp][lane] = Bb;
+    if (__syncthreads_or(!got)) {   // give up: let the copies in flight land (bounded), then leave
+      if (threadIdx.x == 0) {
+        if (status) atomicExch(status, 2);
+        for (int qq = q; qq < q + 2 && qq < nchunk; ++qq) drain_stage(&full[qq & 1], (uint32_t)(qq >> 1) & 1u, wait_cycles);
+      }
+      return;
+    }
+    // the stage of the chunk before (q - 1) is free: every warp has replayed it
+    if (threadIdx.x == 0 && q >= 1 && j - 1 >= 0) {
+      fence_proxy_async_smem();
+      issue(j - 1);
+    }
+    // 2. mu entering this warp's last step; warp 0 also the mu leaving the chunk
+    if (j < nchunk - 1) mu_end = sm.mu_prev[par ^ 1][lane];
+    F2 mu = mu_end;
+    for (int w = SW - 1; w > warp; --w) mu = fma2(sm.A[par][w][lane], mu, sm.Bv[par][w][lane]);
+    if (warp == 0) sm.mu_prev[par][lane] = fma2(Aa, mu, Bb);
+    // 3. replay backwards
+#pragma unroll
+    for (int k = WS - 1; k >= 0; --k) {
+      const int tl = tw + k, t = t0 + tl;
+      const F2 lam = add2(a[k], mu);
+      if (valid && t < T_) {
+        const F2 zc = load_zr(&tile.pre[1][tl][2 * lane]);
+        const F2 g = sigmoid2(load_zr(&tile.pre[2][tl][2 * lane]));
+        const F2 sc = sigmoid2(zc);
+        const F2 one = f2(1.0f, 1.0f), neg = f2(-1.0f, -1.0f);
+        const F2 c = mul2(zc, sc);
+        const F2 ht = load_h(&tile.h[tl][2 * lane]);
+        const F2 hp = tl > 0 ? load_h(&tile.h[tl - 1][2 * lane])
+                             : (t > 0 ? load_h(hs + (row0 + t - 1) * (size_t)d + ch) : load_h(h0 + (size_t)b * d + ch));
+        const F2 dov = load_zr(&tile.dout[tl][2 * lane]);
+        const F2 omf = add2(one, mul2(f[k], neg));
+        const F2 omg = add2(one, mul2(g, neg));
+        const F2 dzg = mul2(mul2(dov, ht), mul2(g, omg));
+        const F2 dzf = mul2(mul2(lam, add2(hp, mul2(c, neg))), mul2(f[k], omf));
+        const F2 silu_p = mul2(sc, fma2(zc, add2(one, mul2(sc, neg)), one));
+        const F2 dzc = mul2(mul2(lam, omf), silu_p);
+        bf16* out = dpre + (row0 + t) * 3 * (size_t)d + ch;
+        store_pair(out, dzf);
+        store_pair(out + d, dzc);
+        store_pair(out + 2 * (size_t)d, dzg);
+      }
+      mu = mul2(f[k], lam);
+    }
+  }
+  __syncthreads();
+  if (valid && warp == 0) store_pair(dh0 + (size_t)b * d + ch, sm.mu_prev[0][lane]);
+}
+
 // 64 channels per CTA when that gives enough CTAs to cover the GPU, else 32
 bool scan_wide(int B, int d) { return (size_t)B * ceil_div(d, 64) >= (size_t)num_sms() * 3 / 4; }
 
@@ -707,8 +837,24 @@ cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, i
     e = wide ? launch_typed<float, 64, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream)
              : launch_typed<float, 32, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream);
   if (e != cudaSuccess) return e;
-  // 2. the reverse scan
+  // 2. the reverse scan (bf16: inputs staged by TMA)
   const int n_cb = ceil_div(d, kBwdCC);
+  if (dt == MMF_BF16) {
+    CUtensorMap mp, md, mh;
+    if (!make_tma_2d(&mp, pre, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)3 * d, (uint64_t)B * T, kBwdCC, TC,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tma_2d(&md, dout, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, (uint64_t)d, (uint64_t)B * T, kBwdCC, TC,
+                     CU_TENSOR_MAP_SWIZZLE_NONE) ||
+        !make_tma_2d(&mh, hsv, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, (uint64_t)d, (uint64_t)B * T, kBwdCC, TC,
+                     CU_TENSOR_MAP_SWIZZLE_NONE))
+      return cudaErrorInvalidValue;
+    const size_t smem = 2 * sizeof(BwdTile) + 128;
+    e = cudaFuncSetAttribute(mlgru_scan_bwd_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    return launch_pdl(mlgru_scan_bwd_tma_kernel, dim3(B * n_cb), dim3(kThreads), smem, stream, mp, md, mh,
+                      (const float*)hsv, h0, dhT, B, T, d, n_cb, static_cast<bf16*>(dpre), dh0, status, wait,
+                      test_hook("MMF_SCAN_SKIP_CHUNK"));
+  }
   if (dt == MMF_BF16)
     return launch_pdl(mlgru_scan_bwd_kernel<bf16>, dim3(B * n_cb), dim3(kThreads), 0, stream,
                       static_cast<const bf16*>(pre), (const float*)hsv, h0, static_cast<const bf16*>(dout), dhT, B, T,

@@ -221,6 +221,31 @@ def test_scan_wait_gives_up_and_reports(monkeypatch):
     assert_close(to_np(h), h_ref, "f32", "h_T after the timeout")
 
 
+def test_scan_backward_wait_gives_up_and_reports(monkeypatch):
+    # chunk 1 of CTA 0 is never loaded by the backward's TMA ring (the forward
+    # states pass runs normally): its bounded wait runs out, the kernel lets its
+    # other copies land and returns, mmf_check reports code 2, and the next
+    # call is correct
+    b, t, d = 2, 300, 256
+    pre = synth.preacts(450, b, t, d, torch.bfloat16).cuda()
+    dout = synth.activations(451, b * t, d, torch.bfloat16).reshape(b, t, d).cuda()
+    h0 = torch.zeros(b, d, device="cuda")
+    monkeypatch.setenv("MMF_SCAN_SKIP_CHUNK", "1")
+    monkeypatch.setenv("MMF_WAIT_LIMIT_US", "20000")
+    mmf.mlgru_scan_backward(pre, h0, dout)
+    with pytest.raises(mmf.MMFError) as err:
+        mmf.check()
+    assert err.value.status == 6 and "code 2" in str(err.value)
+    monkeypatch.delenv("MMF_SCAN_SKIP_CHUNK")
+    monkeypatch.delenv("MMF_WAIT_LIMIT_US")
+    dpre, dh0 = mmf.mlgru_scan_backward(pre, h0, dout)
+    mmf.check()
+    p = to_np(pre)
+    ref = O.mlgru_scan_backward(p[:, :, 0], p[:, :, 1], p[:, :, 2], np.zeros((b, d)), to_np(dout))
+    assert_close(to_np(dpre)[:, :, 1], ref[1], "bf16", "dc~ after the timeout")
+    assert_close(to_np(dh0), ref[3], "f32", "dh0 after the timeout")
+
+
 def test_scan_chunked_equals_whole():
     b, t, d = 2, 96, 64
     pre = synth.preacts(403, b, t, d).cuda()
