@@ -696,8 +696,34 @@ def measure_scan_backward(mmf, dev, steps: int, warmup: int) -> dict:
     ms = prof[key][1] / prof[key][0]
     nbytes = 14.0 * B * T * d
     gbs = nbytes / (ms / 1e3) / 1e9
+    # a training step instead keeps the states of its forward (mmf_mlgru_scan_states): time that
+    # forward and the backward given its states
+    hsb = torch.empty(B, T, d, dtype=torch.float32, device=dev)
+    hcur = torch.zeros(B, d, device=dev)
+    lib = mmf.load()
+    for _ in range(warmup):
+        mmf.mlgru_scan_states(pre, hcur)
+    _, hsb = mmf.mlgru_scan_states(pre, torch.zeros(B, d, device=dev))
+    for _ in range(warmup):
+        mmf.mlgru_scan_backward(pre, h0, dout, hs=hsb)
+    mmf.prof_reset()
+    mmf.prof_enable(True)
+    torch.cuda.synchronize()
+    for _ in range(steps):
+        flush()
+        mmf.mlgru_scan_states(pre, hcur)
+        flush()
+        mmf.mlgru_scan_backward(pre, h0, dout, hs=hsb)
+    torch.cuda.synchronize()
+    mmf.prof_enable(False)
+    p2 = mmf.prof_collect()
+    fwd_us = p2["mlgru_scan_states"][1] / p2["mlgru_scan_states"][0] * 1e3
+    bwd_us = p2[key][1] / p2[key][0] * 1e3
     return {"workload": f"mlgru_scan_backward_b{B}_t{T}_d{d}_bf16", "us": round(ms * 1e3, 2), "GBps": round(gbs, 1),
-            "bytes": nbytes, "design_bytes": 28.0 * B * T * d, "launches": 2 * prof[key][0]}
+            "bytes": nbytes, "design_bytes": 28.0 * B * T * d, "launches": 2 * prof[key][0],
+            "with_stored_states": {"forward_states_us": round(fwd_us, 2), "backward_us": round(bwd_us, 2),
+                                   "backward_GBps": round((14.0 + 4.0) * B * T * d / (bwd_us / 1e6) / 1e9, 1),
+                                   "note": "backward reads the stored states (4 B per channel-step more)"}}
 
 
 def run_scan(args):

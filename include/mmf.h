@@ -182,8 +182,17 @@ size_t mmf_mlgru_scan_ws_size(int32_t B, int32_t T, int32_t d);
 mmf_status mmf_mlgru_scan(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
                           float* h, void* o, void* ws, size_t ws_bytes, void* stream);
 
-/* Scratch bytes mmf_mlgru_scan_backward needs: the forward states, 4 x B x T x d. */
+/* Scratch bytes mmf_mlgru_scan_backward needs when it is not given the
+ * forward states: 4 x B x T x d (0 needed when hs is given). */
 size_t mmf_mlgru_scan_backward_ws_size(int32_t B, int32_t T, int32_t d);
+
+/* Training forward: mmf_mlgru_scan (sigmoid output gate) that also stores the
+ * states h_t, for mmf_mlgru_scan_backward.
+ *   pre, h (in place: h_0 -> h_T) as for mmf_mlgru_scan; o (device) [B, T, d]
+ *   in dtype: o', or NULL to skip it; hs (device) float [B, T, d]: h_t.
+ * No scratch. Errors: as mmf_mlgru_scan. */
+mmf_status mmf_mlgru_scan_states(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
+                                 float* h, void* o, float* hs, void* stream);
 
 /* Training: gradients of mmf_mlgru_scan (sigmoid output gate) for the
  * upstream gradients dout = dL/do' and dhT = dL/dh_T. The pages give no
@@ -198,16 +207,19 @@ size_t mmf_mlgru_scan_backward_ws_size(int32_t B, int32_t T, int32_t d);
  *   pre  (device) [B, T, 3, d] in dtype: the forward's pre-activations
  *   h0   (device) float [B, d]: the forward's initial state (read only)
  *   dout (device) [B, T, d] in dtype; dhT (device) float [B, d] or NULL (zero)
+ *   hs   (device) float [B, T, d]: the forward states (mmf_mlgru_scan_states),
+ *        or NULL: then they are recomputed into ws first (one more launch)
  *   dpre (device) [B, T, 3, d] in dtype: dL/df~, dL/dc~, dL/dg~ per token
  *   dh0  (device) float [B, d]: dL/dh0; must not overlap h0
- *   ws   (device) scratch of mmf_mlgru_scan_backward_ws_size(B, T, d) bytes.
- * Two launches: the forward scan writing the states h_t into ws, then a
+ *   ws   (device) scratch of mmf_mlgru_scan_backward_ws_size(B, T, d) bytes
+ *        (may be NULL when hs is given).
+ * Without hs, two launches: the forward scan writing the states h_t into ws, then a
  * reverse chunked scan (one CTA per sequence x 64 channels, chunks from the
  * last to the first, the backward maps mu -> f mu + f dout g composed like
  * the forward ones). T = 0 does nothing. Errors: as mmf_mlgru_scan. */
 mmf_status mmf_mlgru_scan_backward(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
-                                   const float* h0, const void* dout, const float* dhT, void* dpre,
-                                   float* dh0, void* ws, size_t ws_bytes, void* stream);
+                                   const float* h0, const void* dout, const float* dhT, const float* hs,
+                                   void* dpre, float* dh0, void* ws, size_t ws_bytes, void* stream);
 
 /* Scratch bytes mmf_mlgru_scan_gnorm needs: 4 x B x T x d bytes for
  * v = swish(g~) h in fp32, 4 x B x T x ceil(d / 32) for the partial sums of

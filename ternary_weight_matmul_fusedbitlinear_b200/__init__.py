@@ -7,7 +7,7 @@ there is no CPU fallback.
 """
 from .api import (  # noqa: F401
     DEFAULT_EPS, Block, State, TLinear, bitlinear, block_forward, block_forward_debug, check, glu, mlgru_scan,
-    mlgru_scan_gnorm, mlgru_scan_backward, quantize_weights, unpack_codes, embed, argmax, Model,
+    mlgru_scan_gnorm, mlgru_scan_states, mlgru_scan_backward, quantize_weights, unpack_codes, embed, argmax, Model,
     stack_forward, stack_ws_size, version, prof_enable, prof_reset, prof_collect,
 )
 from ._lib import LIB_PATH, MMFError, load  # noqa: F401

@@ -54,7 +54,8 @@ SIGNATURES = {
     "mmf_mlgru_scan_gnorm_ws_size": (c_sz, [c_i32, c_i32, c_i32]),
     "mmf_mlgru_scan_backward_ws_size": (c_sz, [c_i32, c_i32, c_i32]),
     "mmf_mlgru_scan_backward": (ctypes.c_int, [c_vp, ctypes.c_int, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp, c_vp,
-                                               c_vp, c_sz, c_vp]),
+                                               c_vp, c_vp, c_sz, c_vp]),
+    "mmf_mlgru_scan_states": (ctypes.c_int, [c_vp, ctypes.c_int, c_i32, c_i32, c_i32, c_vp, c_vp, c_vp, c_vp]),
     "mmf_mlgru_scan_gnorm": (ctypes.c_int, [c_vp, ctypes.c_int, c_i32, c_i32, c_i32, c_vp, c_vp, c_f, c_vp, c_vp, c_sz,
                                             c_vp]),
     "mmf_embed": (ctypes.c_int, [c_vp, c_i32, c_vp, c_i32, c_i32, ctypes.c_int, c_vp, c_vp]),

@@ -165,20 +165,34 @@ def mlgru_scan_gnorm(pre: torch.Tensor, h: torch.Tensor, gain: torch.Tensor, eps
     return o
 
 
+def mlgru_scan_states(pre: torch.Tensor, h: torch.Tensor, want_o: bool = True):
+    """Training forward: (o' [B, T, d] or None, hs [B, T, d] fp32); h [B, d] is updated in place to h_T."""
+    _need_cuda(pre, h)
+    B, T, _, d = pre.shape
+    o = torch.empty(B, T, d, dtype=pre.dtype, device=pre.device) if want_o else None
+    hs = torch.empty(B, T, d, dtype=torch.float32, device=pre.device)
+    L.check(L.load().mmf_mlgru_scan_states(_vp(pre), _dtype(pre), B, T, d, _vp(h), _vp(o), _vp(hs),
+                                           _stream(pre.device)), "mmf_mlgru_scan_states")
+    return o, hs
+
+
 def mlgru_scan_backward(pre: torch.Tensor, h0: torch.Tensor, dout: torch.Tensor,
-                        dhT: Optional[torch.Tensor] = None, ws: Optional[torch.Tensor] = None):
+                        dhT: Optional[torch.Tensor] = None, hs: Optional[torch.Tensor] = None,
+                        ws: Optional[torch.Tensor] = None):
     """Gradients of mlgru_scan: (dpre [B, T, 3, d] in pre's dtype, dh0 [B, d] fp32) for
-    dout = dL/do' [B, T, d] and dhT = dL/dh_T [B, d] (zero when None)."""
-    _need_cuda(pre, h0, dout, dhT)
+    dout = dL/do' [B, T, d] and dhT = dL/dh_T [B, d] (zero when None); hs: the forward states
+    from mlgru_scan_states (recomputed when None)."""
+    _need_cuda(pre, h0, dout, dhT, hs)
     B, T, _, d = pre.shape
     if dout.shape != (B, T, d) or dout.dtype != pre.dtype:
         raise ValueError("dout must be [B, T, d] in pre's dtype")
     dpre = torch.empty_like(pre)
     dh0 = torch.empty(B, d, dtype=torch.float32, device=pre.device)
     lib = L.load()
-    w = _workspace(lib.mmf_mlgru_scan_backward_ws_size(B, T, d), pre.device, ws)
-    L.check(lib.mmf_mlgru_scan_backward(_vp(pre), _dtype(pre), B, T, d, _vp(h0), _vp(dout), _vp(dhT), _vp(dpre),
-                                        _vp(dh0), _vp(w), w.numel() * w.element_size(), _stream(pre.device)),
+    w = None if hs is not None else _workspace(lib.mmf_mlgru_scan_backward_ws_size(B, T, d), pre.device, ws)
+    L.check(lib.mmf_mlgru_scan_backward(_vp(pre), _dtype(pre), B, T, d, _vp(h0), _vp(dout), _vp(dhT), _vp(hs),
+                                        _vp(dpre), _vp(dh0), _vp(w), 0 if w is None else w.numel() * w.element_size(),
+                                        _stream(pre.device)),
             "mmf_mlgru_scan_backward")
     return dpre, dh0
 

@@ -445,19 +445,38 @@ extern "C" size_t mmf_mlgru_scan_backward_ws_size(int32_t B, int32_t T, int32_t 
   return mlgru_scan_bwd_ws_bytes(B, T, d);
 }
 
+extern "C" mmf_status mmf_mlgru_scan_states(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
+                                            float* h, void* o, float* hs, void* stream) {
+  if (!dtype_ok(dtype)) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_states: bad dtype");
+  if (B < 0 || T < 0 || d < 1) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_states: B=%d T=%d d=%d", B, T, d);
+  if (d % 8 != 0) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_mlgru_scan_states: d=%d %% 8 != 0", d);
+  if (B == 0 || T == 0) return MMF_OK;
+  if (!pre || !h || !hs) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_states: null pointer");
+  if (!aligned16(pre) || !aligned16(h) || !aligned16(hs) || (o && !aligned16(o)))
+    return fail(MMF_ERR_MISALIGNED, "mmf_mlgru_scan_states");
+  cudaStream_t s = as_stream(stream);
+  int* status = nullptr;
+  mmf_status r = device_status_ptr(&status);
+  if (r != MMF_OK) return r;
+  MMF_CUDA(timed("mlgru_scan_states", s,
+                 [&] { return launch_mlgru_scan_states(pre, dtype, B, T, d, h, o, hs, status, s); }),
+           "mlgru_scan_states");
+  return MMF_OK;
+}
+
 extern "C" mmf_status mmf_mlgru_scan_backward(const void* pre, mmf_dtype dtype, int32_t B, int32_t T, int32_t d,
-                                              const float* h0, const void* dout, const float* dhT, void* dpre,
-                                              float* dh0, void* ws, size_t ws_bytes, void* stream) {
+                                              const float* h0, const void* dout, const float* dhT, const float* hs,
+                                              void* dpre, float* dh0, void* ws, size_t ws_bytes, void* stream) {
   if (!dtype_ok(dtype)) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_backward: bad dtype");
   if (B < 0 || T < 0 || d < 1) return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_backward: B=%d T=%d d=%d", B, T, d);
   if (d % 8 != 0) return fail(MMF_ERR_UNSUPPORTED_SHAPE, "mmf_mlgru_scan_backward: d=%d %% 8 != 0", d);
   if (B == 0 || T == 0) return MMF_OK;
-  if (!pre || !h0 || !dout || !dpre || !dh0 || !ws)
+  if (!pre || !h0 || !dout || !dpre || !dh0 || (!hs && !ws))
     return fail(MMF_ERR_INVALID_ARG, "mmf_mlgru_scan_backward: null pointer");
   if (!aligned16(pre) || !aligned16(h0) || !aligned16(dout) || !aligned16(dpre) || !aligned16(dh0) ||
-      !aligned16(ws) || (dhT && !aligned16(dhT)))
+      (ws && !aligned16(ws)) || (dhT && !aligned16(dhT)) || (hs && !aligned16(hs)))
     return fail(MMF_ERR_MISALIGNED, "mmf_mlgru_scan_backward");
-  if (ws_bytes < mlgru_scan_bwd_ws_bytes(B, T, d))
+  if (!hs && ws_bytes < mlgru_scan_bwd_ws_bytes(B, T, d))
     return fail(MMF_ERR_WORKSPACE, "mmf_mlgru_scan_backward: ws_bytes=%zu < %zu", ws_bytes,
                 mlgru_scan_bwd_ws_bytes(B, T, d));
   const char* hb = reinterpret_cast<const char*>(h0);
@@ -469,7 +488,7 @@ extern "C" mmf_status mmf_mlgru_scan_backward(const void* pre, mmf_dtype dtype, 
   mmf_status r = device_status_ptr(&status);
   if (r != MMF_OK) return r;
   MMF_CUDA(timed("mlgru_scan_backward", s,
-                 [&] { return launch_mlgru_scan_bwd(pre, dtype, B, T, d, h0, dout, dhT, dpre, dh0, ws, status, s); }),
+                 [&] { return launch_mlgru_scan_bwd(pre, dtype, B, T, d, h0, dout, dhT, hs, dpre, dh0, ws, status, s); }),
            "mlgru_scan_backward");
   return MMF_OK;
 }

@@ -168,8 +168,12 @@ cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T,
 // scratch until the reverse scan overwrites it).
 size_t mlgru_scan_bwd_ws_bytes(int B, int T, int d);
 cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, int d, const float* h0,
-                                  const void* dout, const float* dhT, void* dpre, float* dh0, void* ws, int* status,
-                                  cudaStream_t stream);
+                                  const void* dout, const float* dhT, const float* hs, void* dpre, float* dh0,
+                                  void* ws, int* status, cudaStream_t stream);
+// The forward scan (sigmoid gate) that also stores the states h_t in fp32 into
+// hs [B, T, d] for a later backward; o (o') may be null.
+cudaError_t launch_mlgru_scan_states(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, float* hs,
+                                     int* status, cudaStream_t stream);
 // Inside a block: the same scan, then one row kernel that forms o' and
 // quantises it for the o projection (RMSNorm gain qgain, eps) into q / scale /
 // qsum with the standalone quantiser's row routine; o' is written only when

@@ -207,14 +207,15 @@ __device__ void drain_stage(uint64_t* bar, uint32_t parity, long long limit) {
 
 // CC = 32 keeps at most 64 registers per thread so that two CTAs share an SM.
 // GN: g_norm mode; `o` receives v = swish(g~) h in fp32 and `ss` [B*T_][n_cb]
-// the partial sums of h^2 (see the file comment). HS: `o` receives the states
-// h_t themselves in fp32 (what the backward pass reads). Otherwise `o` receives o'.
+// the partial sums of h^2 (see the file comment). Otherwise `o` receives o'.
+// HS: `ss` receives the states h_t themselves in fp32 (what the backward pass
+// reads), and `o` (o') may be null.
 template <typename T, int CC, bool GN, bool HS = false>
 __global__ void __launch_bounds__(kThreads, 64 / CC)
     mlgru_scan_kernel(const __grid_constant__ CUtensorMap map, int B, int T_, int d, int n_cb, int nst,
                       float* __restrict__ h, void* __restrict__ out, float* __restrict__ ss, int* status,
                       long long wait_cycles, int skip_chunk) {
-  using OT = std::conditional_t<GN || HS, float, T>;
+  using OT = std::conditional_t<GN, float, T>;
   OT* __restrict__ o = static_cast<OT*>(out);
   using S = ScanSmem<CC>;
   constexpr int NP = S::NP;         // channel pairs: lanes per step group
@@ -320,11 +321,14 @@ __global__ void __launch_bounds__(kThreads, 64 / CC)
     // 3. replay this lane's steps and store o' (GN: v and the squares' partial sums)
     float sq[LS];
     if (valid) {
-      OT* op = o + ((size_t)b * T_ + t0 + tw) * d + ch;
+      const size_t e0 = ((size_t)b * T_ + t0 + tw) * d + ch;
 #pragma unroll
       for (int k = 0; k < LS; ++k) {
         hw = fma2(f[k], hw, bb[k]);
-        if (full || t0 + tw + k < T_) store_pair(op + (size_t)k * d, HS ? hw : mul2(gg[k], hw));
+        if (full || t0 + tw + k < T_) {
+          if (!HS || o != nullptr) store_pair(o + e0 + (size_t)k * d, mul2(gg[k], hw));
+          if constexpr (HS) store_pair(ss + e0 + (size_t)k * d, hw);
+        }
         if constexpr (GN) {
           const F2 h2 = mul2(hw, hw);
           sq[k] = lo(h2) + hi(h2);
@@ -818,25 +822,35 @@ cudaError_t launch_mlgru_scan_gnorm(const void* pre, mmf_dtype dt, int B, int T,
 
 size_t mlgru_scan_bwd_ws_bytes(int B, int T, int d) { return ((size_t)B * T * d * sizeof(float) + 255) / 256 * 256; }
 
-cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, int d, const float* h0,
-                                  const void* dout, const float* dhT, void* dpre, float* dh0, void* ws, int* status,
-                                  cudaStream_t stream) {
+cudaError_t launch_mlgru_scan_states(const void* pre, mmf_dtype dt, int B, int T, int d, float* h, void* o, float* hs,
+                                     int* status, cudaStream_t stream) {
   if (B == 0 || T == 0) return cudaSuccess;
   if (!tma_available()) return cudaErrorNotSupported;
-  // 1. the forward states h_t (fp32) into ws; the state buffer starts from h0
-  float* hsv = static_cast<float*>(ws);
-  float* hcur = dh0;   // scratch for the forward scan's carried state: dh0 is written last
-  cudaError_t e = cudaMemcpyAsync(hcur, h0, sizeof(float) * (size_t)B * d, cudaMemcpyDeviceToDevice, stream);
-  if (e != cudaSuccess) return e;
   const long long wait = wait_limit_cycles();
   const bool wide = scan_wide(B, d);
   if (dt == MMF_BF16)
-    e = wide ? launch_typed<bf16, 64, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream)
-             : launch_typed<bf16, 32, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream);
-  else
-    e = wide ? launch_typed<float, 64, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream)
-             : launch_typed<float, 32, false, true>(pre, B, T, d, hcur, hsv, nullptr, status, wait, -1, stream);
-  if (e != cudaSuccess) return e;
+    return wide ? launch_typed<bf16, 64, false, true>(pre, B, T, d, h, o, hs, status, wait, -1, stream)
+                : launch_typed<bf16, 32, false, true>(pre, B, T, d, h, o, hs, status, wait, -1, stream);
+  return wide ? launch_typed<float, 64, false, true>(pre, B, T, d, h, o, hs, status, wait, -1, stream)
+              : launch_typed<float, 32, false, true>(pre, B, T, d, h, o, hs, status, wait, -1, stream);
+}
+
+cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, int d, const float* h0,
+                                  const void* dout, const float* dhT, const float* hs_in, void* dpre, float* dh0,
+                                  void* ws, int* status, cudaStream_t stream) {
+  if (B == 0 || T == 0) return cudaSuccess;
+  if (!tma_available()) return cudaErrorNotSupported;
+  cudaError_t e = cudaSuccess;
+  const long long wait = wait_limit_cycles();
+  const float* hsv = hs_in;
+  if (hsv == nullptr) {   // 1. the forward states h_t (fp32) into ws, the carried state starting from h0
+    float* hcur = dh0;    // scratch for the forward scan's carried state: dh0 is written last
+    e = cudaMemcpyAsync(hcur, h0, sizeof(float) * (size_t)B * d, cudaMemcpyDeviceToDevice, stream);
+    if (e != cudaSuccess) return e;
+    e = launch_mlgru_scan_states(pre, dt, B, T, d, hcur, nullptr, static_cast<float*>(ws), status, stream);
+    if (e != cudaSuccess) return e;
+    hsv = static_cast<const float*>(ws);
+  }
   // 2. the reverse scan (bf16: inputs staged by TMA)
   const int n_cb = ceil_div(d, kBwdCC);
   if (dt == MMF_BF16) {
@@ -852,15 +866,15 @@ cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, i
     e = cudaFuncSetAttribute(mlgru_scan_bwd_tma_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     return launch_pdl(mlgru_scan_bwd_tma_kernel, dim3(B * n_cb), dim3(kThreads), smem, stream, mp, md, mh,
-                      (const float*)hsv, h0, dhT, B, T, d, n_cb, static_cast<bf16*>(dpre), dh0, status, wait,
+                      hsv, h0, dhT, B, T, d, n_cb, static_cast<bf16*>(dpre), dh0, status, wait,
                       test_hook("MMF_SCAN_SKIP_CHUNK"));
   }
   if (dt == MMF_BF16)
     return launch_pdl(mlgru_scan_bwd_kernel<bf16>, dim3(B * n_cb), dim3(kThreads), 0, stream,
-                      static_cast<const bf16*>(pre), (const float*)hsv, h0, static_cast<const bf16*>(dout), dhT, B, T,
+                      static_cast<const bf16*>(pre), hsv, h0, static_cast<const bf16*>(dout), dhT, B, T,
                       d, n_cb, static_cast<bf16*>(dpre), dh0);
   return launch_pdl(mlgru_scan_bwd_kernel<float>, dim3(B * n_cb), dim3(kThreads), 0, stream,
-                    static_cast<const float*>(pre), (const float*)hsv, h0, static_cast<const float*>(dout), dhT, B, T, d,
+                    static_cast<const float*>(pre), hsv, h0, static_cast<const float*>(dout), dhT, B, T, d,
                     n_cb, static_cast<float*>(dpre), dh0);
 }
 

@@ -151,9 +151,13 @@ def test_scan_backward_validation(lib):
     q = ctypes.c_void_p(1 << 20)
     ws = lib.mmf_mlgru_scan_backward_ws_size(2, 300, 64)
     assert ws >= 4 * 2 * 300 * 64
-    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 12, p, p, None, p, q, p, 1 << 20, None) == 2      # d % 8
-    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, None, p, None, p, q, p, 1 << 20, None) == 1   # null h0
-    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, p, p, None, p, p, p, 1 << 20, None) == 1      # h0 = dh0
-    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, p, p, ctypes.c_void_p(4104), p, q, p, 1 << 20, None) == 3
-    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 300, 64, p, p, None, p, q, p, ws - 1, None) == 4      # workspace
-    assert lib.mmf_mlgru_scan_backward(None, 0, 0, 3, 16, None, None, None, None, None, None, 0, None) == 0
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 12, p, p, None, None, p, q, p, 1 << 20, None) == 2      # d % 8
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, None, p, None, None, p, q, p, 1 << 20, None) == 1   # null h0
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, p, p, None, None, p, p, p, 1 << 20, None) == 1      # h0 = dh0
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 16, p, p, ctypes.c_void_p(4104), None, p, q, p, 1 << 20, None) == 3
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 300, 64, p, p, None, None, p, q, p, ws - 1, None) == 4      # workspace
+    assert lib.mmf_mlgru_scan_backward(None, 0, 0, 3, 16, None, None, None, None, None, None, None, 0, None) == 0
+    # with the forward states given no scratch is needed; a wrong-size workspace is then not an error
+    assert lib.mmf_mlgru_scan_backward(p, 0, 2, 3, 12, p, p, None, p, p, q, None, 0, None) == 2          # d % 8 still
+    assert lib.mmf_mlgru_scan_states(p, 0, 2, 3, 16, p, None, None, None) == 1                          # null hs
+    assert lib.mmf_mlgru_scan_states(p, 0, 2, 3, 16, p, ctypes.c_void_p(4100), p, None) == 3            # misaligned o

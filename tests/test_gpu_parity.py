@@ -221,6 +221,31 @@ def test_scan_wait_gives_up_and_reports(monkeypatch):
     assert_close(to_np(h), h_ref, "f32", "h_T after the timeout")
 
 
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("b,t,d", [(3, 200, 264), (8, 300, 2560)])
+def test_scan_states_then_backward(b, t, d, dtype):
+    # the training forward stores the states: o' equals the plain scan's bit for
+    # bit, the states match the oracle's, and the backward given them equals the
+    # backward that recomputes them, bit for bit
+    pre = synth.preacts(460 + t, b, t, d, TORCH_DT[dtype], scale=2.0).cuda()
+    h0 = synth.activations(461, b, d).cuda()
+    dout = synth.activations(462, b * t, d, TORCH_DT[dtype]).reshape(b, t, d).cuda()
+    h1, h2 = h0.clone(), h0.clone()
+    o_plain = mmf.mlgru_scan(pre, h1)
+    o, hs = mmf.mlgru_scan_states(pre, h2)
+    mmf.check()
+    assert torch.equal(o, o_plain) and torch.equal(h1, h2)
+    p = to_np(pre)
+    og, _ = O.mlgru_scan(p[:, :, 0], p[:, :, 1], p[:, :, 2], to_np(h0))
+    h_ref = og / O.sigmoid(p[:, :, 2])
+    assert_close(to_np(hs), h_ref, "f32", "states")
+    d1, dh1 = mmf.mlgru_scan_backward(pre, h0, dout)
+    d2, dh2 = mmf.mlgru_scan_backward(pre, h0, dout, hs=hs)
+    _, hs_only = mmf.mlgru_scan_states(pre, h0.clone(), want_o=False)
+    mmf.check()
+    assert torch.equal(d1, d2) and torch.equal(dh1, dh2) and torch.equal(hs_only, hs)
+
+
 def test_scan_backward_wait_gives_up_and_reports(monkeypatch):
     # chunk 1 of CTA 0 is never loaded by the backward's TMA ring (the forward
     # states pass runs normally): its bounded wait runs out, the kernel lets its
