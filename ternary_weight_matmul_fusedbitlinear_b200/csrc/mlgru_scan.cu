@@ -478,7 +478,9 @@ __global__ void __launch_bounds__(kApplyWarps * 32)
 // buffered by chunk parity), each warp folds the maps of the warps after it
 // onto the mu entering the chunk's end, then replays its steps backwards and
 // stores the three gradients. The states h_t come from the forward scan in its
-// HS mode (fp32).
+// HS mode (fp32). This form reads its inputs with plain loads and an L2
+// prefetch of the next chunk (fp32 runs, whose tiles would not fit twice in
+// shared memory); bf16 runs take the TMA-staged form below.
 constexpr int kBwdCC = 64;
 struct BwdSmem {
   F2 A[2][SW][kBwdCC / 2];
@@ -869,10 +871,6 @@ cudaError_t launch_mlgru_scan_bwd(const void* pre, mmf_dtype dt, int B, int T, i
                       hsv, h0, dhT, B, T, d, n_cb, static_cast<bf16*>(dpre), dh0, status, wait,
                       test_hook("MMF_SCAN_SKIP_CHUNK"));
   }
-  if (dt == MMF_BF16)
-    return launch_pdl(mlgru_scan_bwd_kernel<bf16>, dim3(B * n_cb), dim3(kThreads), 0, stream,
-                      static_cast<const bf16*>(pre), hsv, h0, static_cast<const bf16*>(dout), dhT, B, T,
-                      d, n_cb, static_cast<bf16*>(dpre), dh0);
   return launch_pdl(mlgru_scan_bwd_kernel<float>, dim3(B * n_cb), dim3(kThreads), 0, stream,
                     static_cast<const float*>(pre), hsv, h0, static_cast<const float*>(dout), dhT, B, T, d,
                     n_cb, static_cast<float*>(dpre), dh0);
