@@ -162,12 +162,16 @@ bool gemm_uses_tc(const TGemmArgs& a, Epi epi) {
 // Single-token calls quantise inside the contraction unless the projection is
 // so wide (more than 4 16-row CTAs per SM, e.g. a 32000-entry LM head) that
 // every CTA quantising the same row costs more than one quantiser launch
-// (2560 -> 32000: 32.8 us fused, 19.5 us with the quantiser).
+// (2560 -> 32000: 32.8 us fused, 19.5 us with the quantiser). Up to 4 tokens
+// they do so when the projection is one wave of CTAs (single calls 2048 ->
+// 2048 at 4 tokens: 3.90 vs 4.54 us; 5632 -> 2048: 6.78 vs 7.47 us); at 16
+// tokens, or on wider outputs (2048 -> 5632), the separate quantiser is faster.
 bool decode_fused_quant_wanted(int M, int N) {
   const char* e = getenv("MMF_DECODE_FUSED_QUANT");
   if (e != nullptr && strcmp(e, "1") == 0) return true;
   if (e != nullptr && strcmp(e, "0") == 0) return false;
-  return M == 1 && ceil_div(N, 16) <= 4 * num_sms();
+  if (M == 1) return ceil_div(N, 16) <= 4 * num_sms();
+  return M <= 4 && ceil_div(N, 16) <= num_sms();
 }
 
 // `what` names the projection for the launch-timing totals ("fcg", "o", ...).
